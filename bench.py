@@ -1,0 +1,394 @@
+"""Benchmark of the HATA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+One step = one hata_decode_step: append the step's key code (and K/V rows),
+hash the queries, Hamming-score every cached code, select the top-k per
+query head, gather the selected K/V rows and run softmax attention over them.
+Each step appends one token, so step t attends over N + t + 1 keys.
+
+Timing: W untimed warm-up steps, then exactly K timed steps bracketed by a
+barrier and torch.cuda.synchronize(); every step is timed on the launching
+stream with CUDA events (recorded by the library between its kernels), and L2
+is flushed (a 256 MiB write, outside the timed intervals) before every step.
+Multi-GPU: one process per GPU (torchrun), each rank decodes its own batch
+(weak scaling, no collective on the data path); rank 0 prints the max over
+ranks.  `--impl reference` times the CPU oracle instead, on a bounded sample
+of heads of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hash_aware_top_hata_b200 import hata as H  # noqa: E402
+from hash_aware_top_hata_b200 import workloads as wl  # noqa: E402
+
+METRIC = "µs per decode step & achieved HBM GB/s (score+top-k+sparse attn) vs roofline"
+UNIT = "us/step"
+DEFAULT_CONFIG = "llama31_8b_gqa_128k"
+FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: report no samples
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set() and self._nv is not None:
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons - {"gpu_idle"})}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "hata" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ oracle (CPU) --
+
+def oracle_sample(cfg, w, n_heads: int, n_len: int):
+    """Time the CPU oracle on `n_heads` query heads of the workload at
+    context n_len; returns (seconds per head, description)."""
+    import numpy as np
+    import oracle
+    G = cfg.G
+    heads = [(b, hq) for b in range(cfg.B) for hq in range(cfg.H_q)][:: max(1, cfg.B * cfg.H_q
+                                                                          // n_heads)][:n_heads]
+    Wn = w.W_H.cpu().numpy()
+    slabs, codes = {}, {}
+    for b, hq in heads:
+        h = hq // G
+        if (b, h) not in slabs:
+            K = wl.to_numpy_kv(w.K[b, h, :n_len])
+            V = wl.to_numpy_kv(w.V[b, h, :n_len])
+            slabs[(b, h)] = (K, V)
+            codes[(b, h)] = oracle.hash_keys(K[None, None], Wn[h][None])[0, 0]
+    qs = {(b, hq): w.q[0, b, hq].cpu().numpy() for b, hq in heads}
+    t0 = time.perf_counter()
+    for b, hq in heads:
+        h = hq // G
+        K, V = slabs[(b, h)]
+        oracle.decode_head(qs[(b, hq)], Wn[h], codes[(b, h)], K, V, n_len, cfg.topk,
+                           1.0 / math.sqrt(128))
+    el = time.perf_counter() - t0
+    desc = (f"oracle decode (hash q, Hamming over {n_len} codes, sorted top-{cfg.topk}, fp64 "
+            f"attention) on {len(heads)} of {cfg.B * cfg.H_q} query heads, scaled to a full step")
+    return el / len(heads), desc
+
+
+def bench_config(args):
+    """The named workload, optionally at another context / batch (profiling
+    and sweeps; the default run uses the named workload unchanged)."""
+    cfg = wl.CONFIGS[args.config]
+    if args.context or args.batch:
+        cfg = wl.scaled(cfg, N=args.context or cfg.N, B=args.batch or cfg.B,
+                        topk=max(1, round(cfg.topk * (args.context or cfg.N) / cfg.N)))
+    return cfg
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the CPU oracle, single-threaded, on the host cores."""
+    if rank != 0:
+        return
+    cfg = bench_config(args)
+    w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config), device="cpu"
+                         if not torch.cuda.is_available() else "cuda", steps=1)
+    per_head, desc = oracle_sample(cfg, w, n_heads=2, n_len=cfg.N)
+    heads_total = cfg.B * cfg.H_q
+    # each "step" re-times a bounded sample (two heads) and scales to the full step
+    import oracle  # noqa: F401
+    for _ in range(args.warmup):
+        oracle_sample(cfg, w, n_heads=1, n_len=cfg.N)
+    times = []
+    for _ in range(args.steps):
+        ph, _ = oracle_sample(cfg, w, n_heads=2, n_len=cfg.N)
+        times.append(ph * heads_total)
+    us = statistics.mean(times) * 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(us / 1e3, 3), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, "none (CPU)"),
+        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(cfg, l2: str) -> dict:
+    return {"workload": cfg.name, "B": cfg.B, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
+            "context": cfg.N, "topk": cfg.topk, "head_dim": 128, "rbit": 128,
+            "kv_dtype": cfg.kv_dtype, "tokens_appended_per_step": 1, "l2": l2}
+
+
+# ---------------------------------------------------------------- GPU arm --
+
+def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, world):
+    """e2e (host buffers in, host result out, through the same C ABI) and the
+    dense decode attention at the same shape."""
+    dev = out.device
+    B, Hq, Hkv, N = cfg.B, cfg.H_q, cfg.H_kv, cfg.N
+    scale = 1.0 / math.sqrt(128)
+    kv_elt = 2 if cfg.kv_dtype == "bf16" else 4
+    t0 = W_steps + K_steps
+    q_h = w.q[t0:t0 + K_steps].cpu().pin_memory()
+    kn_h = w.k_new[t0:t0 + K_steps].cpu().pin_memory()
+    vn_h = w.v_new[t0:t0 + K_steps].cpu().pin_memory()
+    out_h = torch.empty((K_steps, B, Hq, 128)).pin_memory()
+    q_d, kn_d, vn_d = (torch.empty_like(x[0], device=dev) for x in (q_h, kn_h, vn_h))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K_steps)]
+    for i in range(K_steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        q_d.copy_(q_h[i], non_blocking=True)
+        kn_d.copy_(kn_h[i], non_blocking=True)
+        vn_d.copy_(vn_h[i], non_blocking=True)
+        H.hata_decode_step(q_d, w.W_H, codes, w.K, w.V, seq[t0 + i], w.n_cap, cfg.topk, scale,
+                           ws, out, k_new=kn_d, v_new=vn_d)
+        out_h[i].copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, statistics.mean(a.elapsed_time(b) for a, b in e2e_ev))
+    h2d = q_d.numel() * 4 + (kn_d.numel() + vn_d.numel()) * kv_elt
+    d2h = out.numel() * 4
+
+    # ---- dense decode attention at the same shape (context for the speedup) ----
+    dws = torch.empty(H.hata_dense_workspace_size(B, Hq, Hkv, w.n_cap), dtype=torch.uint8,
+                      device=dev)
+    dout = torch.empty_like(out)
+    dseq = torch.full((B,), N, dtype=torch.int32, device=dev)
+    dense_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(10)]
+    for i in range(13):
+        flush.zero_()
+        if i >= 3:
+            dense_ev[i - 3][0].record(stream)
+        H.hata_dense_decode(w.q[0], w.K, w.V, dseq, N, scale, dws, dout)
+        if i >= 3:
+            dense_ev[i - 3][1].record(stream)
+    torch.cuda.synchronize()
+    dense_ms = statistics.median(a.elapsed_time(b) for a, b in dense_ev)
+
+    return e2e_ms, h2d, d2h, dense_ms
+
+
+def run_hata(args, world, rank, local):
+    cfg = bench_config(args)
+    K_steps, W_steps = args.steps, args.warmup
+    total_steps = W_steps + 2 * K_steps
+    seed = wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config) + 1000 * rank
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = wl.make_workload(cfg, seed, device=dev, steps=total_steps)
+    B, Hq, Hkv, N = cfg.B, cfg.H_q, cfg.H_kv, cfg.N
+    scale = 1.0 / math.sqrt(128)
+    codes = torch.zeros((B, Hkv, w.n_cap, 4), dtype=torch.int32, device=dev)
+    H.hata_hash_keys(w.K, w.W_H, codes, 0, N)
+    ws = torch.empty(H.hata_decode_workspace_size(B, Hq, Hkv, w.n_cap, cfg.topk),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty((B, Hq, 128), device=dev)
+    seq = (N + 1 + torch.arange(total_steps, dtype=torch.int32, device=dev))[:, None] \
+        .expand(total_steps, B).contiguous()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    kv_elt = 2 if cfg.kv_dtype == "bf16" else 4
+
+    def step(t, events=None):
+        H.hata_decode_step(w.q[t], w.W_H, codes, w.K, w.V, seq[t], w.n_cap, cfg.topk, scale,
+                           ws, out, k_new=w.k_new[t], v_new=w.v_new[t], events=events)
+
+    for t in range(W_steps):
+        flush.zero_()
+        step(t)
+    torch.cuda.synchronize()
+    H.hata_workspace_check(ws)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
+    for e4 in evs:  # torch creates the CUDA event on first record; the library needs handles
+        for e in e4:
+            e.record(stream)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        for i in range(K_steps):
+            flush.zero_()
+            step(W_steps + i, evs[i])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+        barrier(world)
+    H.hata_workspace_check(ws)
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    prep_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    score_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    attend_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    ms = statistics.mean(step_ms)
+    ms_max = max_over_ranks(world, ms)
+
+    e2e_ms, h2d, d2h, dense_ms = float("nan"), 0, 0, float("nan")
+    if not args.no_extras:
+        e2e_ms, h2d, d2h, dense_ms = extras(args, cfg, w, codes, ws, out, seq, flush, stream,
+                                            W_steps, K_steps, world)
+    # ---- roofline ----
+    peak, peak_kind = measured_peaks()
+    kv_row = 128 * kv_elt
+    attend_bytes = B * Hq * cfg.topk * 2 * kv_row           # selected K and V rows
+    code_bytes = B * Hkv * (N + W_steps + K_steps // 2) * 16  # every code once per KV head
+    attend_s = statistics.mean(attend_ms) / 1e3
+    score_s = statistics.mean(score_ms) / 1e3
+    achieved = attend_bytes / attend_s / 1e9
+    step_bytes = attend_bytes + code_bytes
+    line = {
+        "metric": METRIC, "value": round(ms_max * 1e3, 2), "unit": UNIT, "n_gpus": world,
+        "steps": K_steps, "warmup": W_steps, "ms_per_step": round(ms_max, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian q/K/V, 2% planted keys, N(0,1/128) W_H)",
+        "config": config_dict(cfg, "flushed before every timed step (256 MiB write)"),
+        "roofline": {"bound": "hbm", "kernel": "attend (select + gather + softmax)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": attend_bytes},
+        "step_roofline": {"bytes": step_bytes, "achieved_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
+                          "frac_of_measured": round(step_bytes / (ms / 1e3) / 1e9 / peak, 4),
+                          "frac_of_8000": round(step_bytes / (ms / 1e3) / 1e9 / 8000.0, 4)},
+        "kernels_us": {"prep": round(statistics.mean(prep_ms) * 1e3, 2),
+                       "score": round(score_s * 1e6, 2),
+                       "attend": round(attend_s * 1e6, 2),
+                       "score_gbs": round(code_bytes / score_s / 1e9, 1)},
+        "dense_us": round(dense_ms * 1e3, 1),
+        "speedup_vs_dense": round(dense_ms / ms, 2),
+        "e2e": {"value": round(e2e_ms * 1e3, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * K_steps,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": round(wall, 4),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_head, desc = oracle_sample(cfg, w, n_heads=args.cpu_heads, n_len=N)
+        line["cpu_baseline"] = {"value": round(per_head * B * Hq * 1e6, 1), "unit": UNIT,
+                                "cores": 1, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=wl.CONFIG_ORDER)
+    ap.add_argument("--impl", default="hata", choices=["hata", "reference"])
+    ap.add_argument("--cpu-heads", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--context", type=int, default=0, help="override the context length")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the e2e, dense and CPU legs (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_hata(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,376 @@
+// hata_abi.cu -- the extern "C" boundary of libhata: argument checks on the
+// host, workspace carving, and the launch sequence of each entry point on the
+// caller's stream.  Every check runs before anything is enqueued.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "hata_internal.cuh"
+
+using namespace hata;
+
+namespace {
+
+thread_local char g_err[512];
+
+hata_status_t fail(hata_status_t st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+hata_status_t ok()
+{
+    g_err[0] = '\0';
+    return HATA_OK;
+}
+
+hata_status_t cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(HATA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_dtype(hata_dtype_t t) { return t == HATA_DT_BF16 || t == HATA_DT_F32; }
+
+hata_status_t check_dims(int d, int r)
+{
+    if (d != kD) return fail(HATA_ERR_UNSUPPORTED, "head_dim d=%d: only %d is supported", d, kD);
+    if (r != kRbit) return fail(HATA_ERR_UNSUPPORTED, "hash bits r=%d: only %d is supported", r, kRbit);
+    return HATA_OK;
+}
+
+hata_status_t check_heads(int B, int H_q, int H_kv)
+{
+    if (B <= 0 || H_q <= 0 || H_kv <= 0)
+        return fail(HATA_ERR_INVALID_ARG, "B=%d H_q=%d H_kv=%d must be positive", B, H_q, H_kv);
+    if (H_q % H_kv != 0)
+        return fail(HATA_ERR_UNSUPPORTED, "H_q=%d is not a multiple of H_kv=%d", H_q, H_kv);
+    if (int64_t(B) * H_q > 65535 || int64_t(B) * H_kv > 65535)
+        return fail(HATA_ERR_UNSUPPORTED, "B*H_q=%lld exceeds 65535",
+                    (long long)(int64_t(B) * H_q));
+    return HATA_OK;
+}
+
+struct Events {
+    void *const *ev;
+    cudaStream_t s;
+    cudaError_t record(int i) const
+    {
+        return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+int hata_abi_version(void) { return 1; }
+
+const char *hata_status_string(int status)
+{
+    switch (status) {
+    case HATA_OK: return "HATA_OK";
+    case HATA_ERR_INVALID_ARG: return "HATA_ERR_INVALID_ARG";
+    case HATA_ERR_UNSUPPORTED: return "HATA_ERR_UNSUPPORTED";
+    case HATA_ERR_CUDA: return "HATA_ERR_CUDA";
+    case HATA_ERR_DEVICE_CHECK: return "HATA_ERR_DEVICE_CHECK";
+    default: return "HATA_ERR_UNKNOWN";
+    }
+}
+
+const char *hata_last_error(void) { return g_err; }
+
+hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t n_cap,
+                             const float *W_H, uint32_t *codes, int B, int H_kv, int64_t pos0,
+                             int64_t n, int d, int r, void *stream)
+{
+    if (hata_status_t st = check_dims(d, r)) return st;
+    if (!K || !W_H || !codes) return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (!valid_dtype(kv_dtype)) return fail(HATA_ERR_INVALID_ARG, "bad kv_dtype %d", int(kv_dtype));
+    if (B <= 0 || H_kv <= 0 || B > 65535 || H_kv > 65535)
+        return fail(HATA_ERR_INVALID_ARG, "B=%d H_kv=%d out of range", B, H_kv);
+    if (n_cap <= 0 || pos0 < 0 || n < 0 || pos0 > n_cap || n > n_cap - pos0)
+        return fail(HATA_ERR_INVALID_ARG, "positions [%lld, %lld) outside the cache of %lld",
+                    (long long)pos0, (long long)(pos0 + n), (long long)n_cap);
+    if (!aligned(K, 16) || !aligned(codes, 16) || !aligned(W_H, 4))
+        return fail(HATA_ERR_INVALID_ARG, "K and codes must be 16-byte aligned");
+    if (n == 0) return ok();
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = launch_hash_prefill(K, kv_dtype == HATA_DT_BF16, n_cap, W_H, codes, B,
+                                              H_kv, pos0, n, s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "hash_keys launch");
+}
+
+hata_status_t hata_append_code(const void *k_new, hata_dtype_t kv_dtype, const float *W_H,
+                               uint32_t *codes, int64_t n_cap, const int32_t *pos, int B,
+                               int H_kv, int d, int r, uint32_t *err_flags, void *stream)
+{
+    if (hata_status_t st = check_dims(d, r)) return st;
+    if (!k_new || !W_H || !codes || !pos) return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (!valid_dtype(kv_dtype)) return fail(HATA_ERR_INVALID_ARG, "bad kv_dtype %d", int(kv_dtype));
+    if (B <= 0 || H_kv <= 0 || int64_t(B) * H_kv > (int64_t(1) << 24) || H_kv > 65535)
+        return fail(HATA_ERR_INVALID_ARG, "B=%d H_kv=%d out of range", B, H_kv);
+    if (n_cap <= 0) return fail(HATA_ERR_INVALID_ARG, "n_cap=%lld", (long long)n_cap);
+    if (!aligned(k_new, 4) || !aligned(codes, 16) || !aligned(pos, 4) ||
+        (err_flags && !aligned(err_flags, 4)))
+        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer");
+    PrepArgs a{};
+    a.k_new = k_new;
+    a.W = W_H;
+    a.codes = codes;
+    a.pos = pos;
+    a.err_word = err_flags;
+    a.n_cap = n_cap;
+    a.max_seq_len = n_cap;
+    a.B = B;
+    a.H_q = H_kv;
+    a.H_kv = H_kv;
+    a.G = 1;
+    a.zgroups = 1;
+    a.kv_bf16 = kv_dtype == HATA_DT_BF16;
+    const cudaError_t e = launch_prep(a, B, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "append_code launch");
+}
+
+size_t hata_decode_workspace_size(int B, int H_q, int H_kv, int64_t max_seq_len, int topk)
+{
+    DecodeLayout L;
+    return decode_layout(B, H_q, H_kv, max_seq_len, topk, &L) ? L.total : 0;
+}
+
+int64_t hata_dist_row_bytes(int64_t max_seq_len)
+{
+    return max_seq_len <= 0 ? 0 : ceil_div(max_seq_len, kChunk) * kChunk;
+}
+
+hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
+                               void *V, hata_dtype_t kv_dtype, int64_t n_cap,
+                               const int32_t *seq_len, int64_t max_seq_len, const void *k_new,
+                               const void *v_new, int B, int H_q, int H_kv, int d, int r,
+                               int topk, float scale, void *workspace, size_t workspace_bytes,
+                               float *out, int32_t *sel_idx, uint32_t *q_codes, uint8_t *dist,
+                               int64_t dist_row_bytes, void *const *events, void *stream)
+{
+    if (hata_status_t st = check_dims(d, r)) return st;
+    if (hata_status_t st = check_heads(B, H_q, H_kv)) return st;
+    if (!q || !W_H || !codes || !K || !V || !seq_len || !workspace || !out)
+        return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (!valid_dtype(kv_dtype)) return fail(HATA_ERR_INVALID_ARG, "bad kv_dtype %d", int(kv_dtype));
+    if (v_new && !k_new) return fail(HATA_ERR_INVALID_ARG, "v_new given without k_new");
+    if (topk <= 0) return fail(HATA_ERR_INVALID_ARG, "topk=%d must be >= 1", topk);
+    if (n_cap <= 0 || n_cap >= (int64_t(1) << 31))
+        return fail(HATA_ERR_INVALID_ARG, "n_cap=%lld out of range", (long long)n_cap);
+    if (max_seq_len <= 0 || max_seq_len > n_cap)
+        return fail(HATA_ERR_INVALID_ARG, "max_seq_len=%lld must be in [1, n_cap=%lld]",
+                    (long long)max_seq_len, (long long)n_cap);
+    if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
+        return fail(HATA_ERR_INVALID_ARG, "scale must be finite");
+    if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(codes, 16) ||
+        !aligned(out, 16) || !aligned(W_H, 4) || !aligned(seq_len, 4) ||
+        (k_new && !aligned(k_new, 4)) || (v_new && !aligned(v_new, 4)) ||
+        (sel_idx && !aligned(sel_idx, 4)) || (q_codes && !aligned(q_codes, 16)))
+        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer (q, K, V, codes, out, q_codes: 16 B)");
+    if (!aligned(workspace, 256)) return fail(HATA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    DecodeLayout L;
+    if (!decode_layout(B, H_q, H_kv, max_seq_len, topk, &L))
+        return fail(HATA_ERR_INVALID_ARG, "sizes out of range");
+    if (workspace_bytes < L.total)
+        return fail(HATA_ERR_INVALID_ARG, "workspace of %zu bytes < required %zu", workspace_bytes,
+                    L.total);
+    if (dist) {
+        if (!aligned(dist, 16) || dist_row_bytes % 16 || dist_row_bytes < L.dist_row)
+            return fail(HATA_ERR_INVALID_ARG,
+                        "dist must be 16-byte aligned with dist_row_bytes >= %lld, multiple of 16",
+                        (long long)L.dist_row);
+    }
+
+    char *ws = static_cast<char *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int G = H_q / H_kv;
+    uint32_t *qc = q_codes ? q_codes : reinterpret_cast<uint32_t *>(ws + L.off_qcodes);
+    uint8_t *dst = dist ? dist : reinterpret_cast<uint8_t *>(ws + L.off_dist);
+    const int64_t drow = dist ? dist_row_bytes : L.dist_row;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(ws + L.off_hist);
+    uint32_t *cnt_score = reinterpret_cast<uint32_t *>(ws + L.off_cnt_score);
+    uint32_t *cnt_attn = reinterpret_cast<uint32_t *>(ws + L.off_cnt_attn);
+    PlanHead *plan_head = reinterpret_cast<PlanHead *>(ws + L.off_plan_head);
+    PlanChunk *plan_chunk = reinterpret_cast<PlanChunk *>(ws + L.off_plan_chunk);
+    const Events ev{events, s};
+    cudaError_t e;
+
+    if ((e = ev.record(0)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    PrepArgs p{};
+    p.q = q;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.W = W_H;
+    p.codes = codes;
+    p.K = K;
+    p.V = V;
+    p.seq_len = seq_len;
+    p.q_out = qc;
+    p.flags = reinterpret_cast<uint32_t *>(ws + L.off_flags);
+    p.hist_total = hist;
+    p.cnt_attn = cnt_attn;
+    p.cnt_score = cnt_score;
+    p.ws_header = reinterpret_cast<uint32_t *>(ws);
+    p.n_cap = n_cap;
+    p.max_seq_len = max_seq_len;
+    p.B = B;
+    p.H_q = H_q;
+    p.H_kv = H_kv;
+    p.G = G;
+    p.zgroups = L.zgroups;
+    p.kv_bf16 = kv_dtype == HATA_DT_BF16;
+    if ((e = launch_prep(p, B * G + (k_new ? B : 0), s)) != cudaSuccess)
+        return cuda_fail(e, "prep launch");
+    if ((e = ev.record(1)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    ScoreArgs sa{};
+    sa.qcodes = qc;
+    sa.codes = codes;
+    sa.seq_len = seq_len;
+    sa.dist = dst;
+    sa.dist_row = drow;
+    sa.cum = reinterpret_cast<uint32_t *>(ws + L.off_cum);
+    sa.hist_total = hist;
+    sa.plan_head = plan_head;
+    sa.plan_chunk = plan_chunk;
+    sa.cnt_score = cnt_score;
+    sa.sel_idx = sel_idx;
+    sa.n_cap = n_cap;
+    sa.max_seq_len = max_seq_len;
+    sa.n_chunks = L.n_chunks;
+    sa.B = B;
+    sa.H_q = H_q;
+    sa.H_kv = H_kv;
+    sa.G = G;
+    sa.zgroups = L.zgroups;
+    sa.topk = topk;
+    if ((e = launch_score(sa, s)) != cudaSuccess) return cuda_fail(e, "score launch");
+    if ((e = ev.record(2)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    AttendArgs aa{};
+    aa.q = q;
+    aa.K = K;
+    aa.V = V;
+    aa.seq_len = seq_len;
+    aa.dist = dst;
+    aa.dist_row = drow;
+    aa.plan_head = plan_head;
+    aa.plan_chunk = plan_chunk;
+    aa.part = reinterpret_cast<float *>(ws + L.off_part);
+    aa.cnt_attn = cnt_attn;
+    aa.out = out;
+    aa.sel_idx = sel_idx;
+    aa.n_cap = n_cap;
+    aa.max_seq_len = max_seq_len;
+    aa.n_chunks = L.n_chunks;
+    aa.B = B;
+    aa.H_q = H_q;
+    aa.H_kv = H_kv;
+    aa.G = G;
+    aa.topk = topk;
+    aa.scale_log2 = scale * 1.4426950408889634f;
+    if ((e = launch_attend(aa, kv_dtype == HATA_DT_BF16, s)) != cudaSuccess)
+        return cuda_fail(e, "attend launch");
+    if ((e = ev.record(3)) != cudaSuccess) return cuda_fail(e, "event record");
+    return ok();
+}
+
+hata_status_t hata_workspace_check(void *workspace, size_t workspace_bytes, uint32_t *flags,
+                                   void *stream)
+{
+    if (flags) *flags = 0;
+    if (!workspace || workspace_bytes < 512 || !aligned(workspace, 256))
+        return fail(HATA_ERR_INVALID_ARG, "bad workspace");
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t hdr[2] = {0, 0};
+    cudaError_t e = cudaMemcpyAsync(hdr, workspace, sizeof hdr, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace header read");
+    if (hdr[0] != kWsMagic) return ok();  // no decode step has run on it
+    const uint32_t B = hdr[1];
+    if (B == 0 || 256 + 4 * size_t(B) > workspace_bytes)
+        return fail(HATA_ERR_INVALID_ARG, "workspace header does not match its size");
+    uint32_t acc = 0;
+    char *fl = static_cast<char *>(workspace) + 256;
+    for (uint32_t b0 = 0; b0 < B; b0 += 256) {
+        uint32_t buf[256];
+        const uint32_t cnt = B - b0 < 256 ? B - b0 : 256;
+        e = cudaMemcpyAsync(buf, fl + 4 * size_t(b0), 4 * size_t(cnt), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_fail(e, "workspace flag read");
+        for (uint32_t i = 0; i < cnt; ++i) acc |= buf[i];
+    }
+    e = cudaMemsetAsync(fl, 0, 4 * size_t(B), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace flag clear");
+    if (flags) *flags = acc;
+    if (acc) return fail(HATA_ERR_DEVICE_CHECK, "device-side check flags 0x%x", acc);
+    return ok();
+}
+
+size_t hata_dense_workspace_size(int B, int H_q, int H_kv, int64_t max_seq_len)
+{
+    int64_t nch;
+    size_t op, oc, tot;
+    return dense_layout(B, H_q, H_kv, max_seq_len, &nch, &op, &oc, &tot) ? tot : 0;
+}
+
+hata_status_t hata_dense_decode(const float *q, const void *K, const void *V,
+                                hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                                int64_t max_seq_len, int B, int H_q, int H_kv, int d,
+                                float scale, void *workspace, size_t workspace_bytes, float *out,
+                                void *stream)
+{
+    if (hata_status_t st = check_dims(d, kRbit)) return st;
+    if (hata_status_t st = check_heads(B, H_q, H_kv)) return st;
+    if (!q || !K || !V || !seq_len || !workspace || !out)
+        return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (!valid_dtype(kv_dtype)) return fail(HATA_ERR_INVALID_ARG, "bad kv_dtype %d", int(kv_dtype));
+    if (n_cap <= 0 || n_cap >= (int64_t(1) << 31) || max_seq_len <= 0 || max_seq_len > n_cap)
+        return fail(HATA_ERR_INVALID_ARG, "max_seq_len=%lld n_cap=%lld out of range",
+                    (long long)max_seq_len, (long long)n_cap);
+    if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 4) ||
+        !aligned(seq_len, 4) || !aligned(workspace, 256))
+        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer");
+    int64_t nch;
+    size_t off_part, off_cnt, total;
+    if (!dense_layout(B, H_q, H_kv, max_seq_len, &nch, &off_part, &off_cnt, &total))
+        return fail(HATA_ERR_INVALID_ARG, "sizes out of range");
+    if (workspace_bytes < total)
+        return fail(HATA_ERR_INVALID_ARG, "workspace of %zu bytes < required %zu", workspace_bytes,
+                    total);
+    char *ws = static_cast<char *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DenseArgs a{};
+    a.q = q;
+    a.K = K;
+    a.V = V;
+    a.seq_len = seq_len;
+    a.part = reinterpret_cast<float *>(ws + off_part);
+    a.cnt = reinterpret_cast<uint32_t *>(ws + off_cnt);
+    a.out = out;
+    a.n_cap = n_cap;
+    a.max_seq_len = max_seq_len;
+    a.n_chunks = nch;
+    a.B = B;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.G = H_q / H_kv;
+    a.zgroups = int(ceil_div(a.G, kDenseHeads));
+    a.scale_log2 = scale * 1.4426950408889634f;
+    cudaError_t e = cudaMemsetAsync(a.cnt, 0, total - off_cnt, s);
+    if (e != cudaSuccess) return cuda_fail(e, "dense counter clear");
+    e = launch_dense(a, kv_dtype == HATA_DT_BF16, s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "dense launch");
+}
+
+}  // extern "C"

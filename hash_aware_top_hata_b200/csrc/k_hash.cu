@@ -1,0 +1,274 @@
+// k_hash.cu -- the HATA hash h(x) = sign(x W_H) on sm_100a.
+//
+// HATA review page (arXiv 2506.02572): "Assumptions & free parameters"
+// (h(x) = sign(x W_H), per-head W_H, rbit = 128), "What carries the
+// argument" (queries and keys are hashed; the key codes are cached) and the
+// Figure 2 caption (Algorithm 1: HashEncode(K) fills the code cache, rbit/32
+// words per token).
+//
+// One CTA of 128 threads hashes a group of rows against one KV head's W_H:
+// thread j owns output bit j, keeps column j of W_H in registers and runs
+// the fp32 chain acc = fmaf(x_i, W[i][j], acc), i = 0..127 ascending, for
+// every row of the group (rows staged in shared memory, read as broadcast
+// float4s).  A warp ballot packs bits 32w..32w+31 into code word w.  The
+// chain order is fixed, so codes are reproducible bit for bit by any
+// implementation that follows the same order (the CPU oracle does).
+//
+// The projection is 16K FMAs per row: on the FP32 pipes, not the tensor
+// cores, whose accumulation order is unspecified and would break bit-exact
+// codes.  At decode time the kernel also appends the new key's code (and
+// optionally its K/V rows) and clears the per-step counters the scoring
+// kernel accumulates into.
+#include "hata_internal.cuh"
+
+namespace hata {
+namespace {
+
+constexpr int kPrefillRowsPerCta = 128;
+
+template <bool BF16>
+__device__ __forceinline__ float load_x(const void *base, int64_t i)
+{
+    if (BF16) {
+        const uint16_t u = reinterpret_cast<const uint16_t *>(base)[i];
+        return __uint_as_float(uint32_t(u) << 16);
+    }
+    return reinterpret_cast<const float *>(base)[i];
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store_x(void *base, int64_t i, const void *src, int64_t si)
+{
+    if (BF16)
+        reinterpret_cast<uint16_t *>(base)[i] = reinterpret_cast<const uint16_t *>(src)[si];
+    else
+        reinterpret_cast<float *>(base)[i] = reinterpret_cast<const float *>(src)[si];
+}
+
+// Column j of one head's W_H into registers.
+__device__ __forceinline__ void load_w_column(const float *__restrict__ Wh, int j, float (&w)[kD])
+{
+#pragma unroll
+    for (int i = 0; i < kD; ++i) w[i] = __ldg(Wh + i * kRbit + j);
+}
+
+// One head's W_H [kD][kRbit] into shared memory (all loads in flight at once).
+__device__ __forceinline__ void stage_w(const float *__restrict__ Wh, float *__restrict__ ws)
+{
+    constexpr int kVec = kD * kRbit / 4;
+    const float4 *src = reinterpret_cast<const float4 *>(Wh);
+    float4 *dst = reinterpret_cast<float4 *>(ws);
+    float4 v[kVec / kD];
+#pragma unroll
+    for (int m = 0; m < kVec / kD; ++m) v[m] = __ldg(src + m * kD + threadIdx.x);
+#pragma unroll
+    for (int m = 0; m < kVec / kD; ++m) dst[m * kD + threadIdx.x] = v[m];
+}
+
+// xs: [kD][R] floats (row r of the group in column r); ws: W_H in shared
+// memory.  Returns, for every row, the ballot of this warp's 32 bits = code
+// word (threadIdx.x / 32).
+template <int R>
+__device__ __forceinline__ void hash_group_smem(const float *__restrict__ xs,
+                                                const float *__restrict__ ws,
+                                                uint32_t (&words)[R])
+{
+    const int j = threadIdx.x;
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.0f;
+#pragma unroll 8
+    for (int i = 0; i < kD; ++i) {
+        const float w = ws[i * kRbit + j];
+#pragma unroll
+        for (int r4 = 0; r4 < R / 4; ++r4) {
+            const float4 x = reinterpret_cast<const float4 *>(xs + i * R)[r4];
+            acc[4 * r4 + 0] = __fmaf_rn(x.x, w, acc[4 * r4 + 0]);
+            acc[4 * r4 + 1] = __fmaf_rn(x.y, w, acc[4 * r4 + 1]);
+            acc[4 * r4 + 2] = __fmaf_rn(x.z, w, acc[4 * r4 + 2]);
+            acc[4 * r4 + 3] = __fmaf_rn(x.w, w, acc[4 * r4 + 3]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) words[r] = __ballot_sync(0xffffffffu, acc[r] > 0.0f);
+}
+
+// Same with column j of W_H held in registers (prefill: many row groups per CTA).
+template <int R>
+__device__ __forceinline__ void hash_group(const float *__restrict__ xs, const float (&w)[kD],
+                                           uint32_t (&words)[R])
+{
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kD; ++i) {
+#pragma unroll
+        for (int r4 = 0; r4 < R / 4; ++r4) {
+            const float4 x = reinterpret_cast<const float4 *>(xs + i * R)[r4];
+            acc[4 * r4 + 0] = __fmaf_rn(x.x, w[i], acc[4 * r4 + 0]);
+            acc[4 * r4 + 1] = __fmaf_rn(x.y, w[i], acc[4 * r4 + 1]);
+            acc[4 * r4 + 2] = __fmaf_rn(x.z, w[i], acc[4 * r4 + 2]);
+            acc[4 * r4 + 3] = __fmaf_rn(x.w, w[i], acc[4 * r4 + 3]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) words[r] = __ballot_sync(0xffffffffu, acc[r] > 0.0f);
+}
+
+// -------------------------------------------------------------- prefill --
+template <bool BF16>
+__global__ void __launch_bounds__(kD) hash_prefill_kernel(const void *__restrict__ K,
+                                                          int64_t n_cap,
+                                                          const float *__restrict__ W,
+                                                          uint32_t *__restrict__ codes,
+                                                          int H_kv, int64_t pos0, int64_t n)
+{
+    constexpr int R = kPrepRows;
+    const int h = blockIdx.y, b = blockIdx.z, j = threadIdx.x;
+    const int64_t g_begin = int64_t(blockIdx.x) * kPrefillRowsPerCta;
+    const int64_t g_end = min(g_begin + kPrefillRowsPerCta, n);
+    const int64_t slab = (int64_t(b) * H_kv + h) * n_cap;  // row index of token 0
+
+    float w[kD];
+    load_w_column(W + size_t(h) * kD * kRbit, j, w);
+    __shared__ __align__(16) float xs[kD * R];
+
+    for (int64_t g0 = g_begin; g0 < g_end; g0 += R) {
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int64_t t = g0 + r;
+            xs[j * R + r] = (t < g_end) ? load_x<BF16>(K, (slab + pos0 + t) * kD + j) : 0.0f;
+        }
+        __syncthreads();
+        uint32_t words[R];
+        hash_group<R>(xs, w, words);
+        if ((j & 31) == 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (g0 + r < g_end) codes[(slab + pos0 + g0 + r) * kWords + (j >> 5)] = words[r];
+        }
+    }
+}
+
+// --------------------------------------------------------- decode prep --
+// Rows of KV head h: B*G query rows (b-major), then B appended-key rows.
+template <bool BF16>
+__global__ void __launch_bounds__(kD) prep_kernel(PrepArgs a)
+{
+    constexpr int R = kPrepRows;
+    const int h = blockIdx.y, j = threadIdx.x;
+    const int nq = a.q ? a.B * a.G : 0;
+    const int nk = a.k_new ? a.B : 0;
+    const int rows = nq + nk;
+    const int r0 = blockIdx.x * R;
+
+    if (blockIdx.x == 0) {
+        if (a.cnt_score)
+            for (int i = j; i < a.B * a.zgroups; i += kD) {
+                const int b = i / a.zgroups, z = i % a.zgroups;
+                a.cnt_score[(size_t(b) * a.H_kv + h) * a.zgroups + z] = 0u;
+            }
+        if (a.ws_header && h == 0 && j == 0) {
+            a.ws_header[0] = kWsMagic;
+            a.ws_header[1] = uint32_t(a.B);
+        }
+    }
+    if (r0 >= rows) return;
+
+    extern __shared__ __align__(16) float smem[];
+    float *ws = smem;                 // [kD][kRbit]
+    float *xs = smem + kD * kRbit;    // [kD][R]
+    stage_w(a.W + size_t(h) * kD * kRbit, ws);
+
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int row = r0 + r;
+        float x = 0.0f;
+        if (row < nq) {
+            const int b = row / a.G, g = row % a.G, hq = h * a.G + g;
+            const size_t bh = size_t(b) * a.H_q + hq;
+            x = a.q[bh * kD + j];
+            if (a.hist_total)
+                for (int t = j; t < kHistStride; t += kD) a.hist_total[bh * kHistStride + t] = 0u;
+            if (a.cnt_attn && j == 0) a.cnt_attn[bh] = 0u;
+            if (a.flags && h == 0 && g == 0 && j == 0) {
+                const int64_t sl = a.seq_len[b];
+                uint32_t f = 0;
+                if (sl < 0 || sl > a.max_seq_len || sl > a.n_cap) f |= HATA_FLAG_SEQ_LEN_RANGE;
+                if (a.k_new && (sl - 1 < 0 || sl - 1 >= a.n_cap)) f |= HATA_FLAG_POS_RANGE;
+                a.flags[b] = f;
+            }
+        } else if (row < rows) {
+            const int b = row - nq;
+            x = load_x<BF16>(a.k_new, (int64_t(b) * a.H_kv + h) * kD + j);
+        }
+        xs[j * R + r] = x;
+    }
+    __syncthreads();
+    uint32_t words[R];
+    hash_group_smem<R>(xs, ws, words);
+
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int row = r0 + r;
+        if (row < nq) {
+            if ((j & 31) == 0) {
+                const int b = row / a.G, g = row % a.G;
+                const size_t bh = size_t(b) * a.H_q + h * a.G + g;
+                a.q_out[bh * kWords + (j >> 5)] = words[r];
+            }
+        } else if (row < rows) {
+            const int b = row - nq;
+            const int64_t pos = a.pos ? int64_t(a.pos[b]) : int64_t(a.seq_len[b]) - 1;
+            if (pos >= 0 && pos < a.n_cap) {
+                const int64_t crow = (int64_t(b) * a.H_kv + h) * a.n_cap + pos;
+                if ((j & 31) == 0) a.codes[crow * kWords + (j >> 5)] = words[r];
+                if (a.v_new) {
+                    const int64_t src = (int64_t(b) * a.H_kv + h) * kD + j;
+                    store_x<BF16>(a.K, crow * kD + j, a.k_new, src);
+                    store_x<BF16>(a.V, crow * kD + j, a.v_new, src);
+                }
+            } else if (a.err_word && j == 0) {
+                atomicOr(a.err_word, HATA_FLAG_POS_RANGE);
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const float *W,
+                                uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
+                                cudaStream_t s)
+{
+    const dim3 grid(unsigned(ceil_div(n, kPrefillRowsPerCta)), unsigned(H_kv), unsigned(B));
+    if (bf16)
+        hash_prefill_kernel<true><<<grid, kD, 0, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
+    else
+        hash_prefill_kernel<false><<<grid, kD, 0, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s)
+{
+    constexpr size_t kSmem = sizeof(float) * (kD * kRbit + kD * kPrepRows);
+    static const cudaError_t attr_err = [] {
+        cudaError_t e = cudaFuncSetAttribute(prep_kernel<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prep_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+        return e;
+    }();
+    if (attr_err != cudaSuccess) return attr_err;
+    const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRows)), unsigned(a.H_kv));
+    if (a.kv_bf16)
+        prep_kernel<true><<<grid, kD, kSmem, s>>>(a);
+    else
+        prep_kernel<false><<<grid, kD, kSmem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace hata

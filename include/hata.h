@@ -1,0 +1,181 @@
+/*
+ * hata.h -- C ABI of the B200 (sm_100a) hash-aware top-k attention (HATA)
+ * decode path.
+ *
+ * The method (HATA review page, arXiv 2506.02572):
+ *   "What carries the argument": every query and key is hashed per attention
+ *     head to r = 128 bits; the query code is XOR-ed with every cached key
+ *     code and a popcount gives the Hamming score; the top-k keys are
+ *     gathered and attention runs over them only ("fused gather-attention").
+ *   "Assumptions & free parameters": inference hash h(x) = sign(x W_H),
+ *     W_H per head, rbit = 128.
+ *   Figure 2 caption, Algorithm 1 (prefill): HashEncode(K) fills the key code
+ *     cache Kcache_H, rbit/32 32-bit words per token; K and V fill the KV cache.
+ *   Referee report, major comment 1 (Algorithm 3): top-k over 129 possible
+ *     Hamming values; the choice inside the boundary bucket is left open.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, allocated and owned by the
+ *     caller; the library never allocates, frees or keeps them.  Work is
+ *     enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and the call returns without synchronising, except where noted.
+ *   - d (head_dim) and r (hash bits) must both be 128 (HATA_ERR_UNSUPPORTED
+ *     otherwise).
+ *   - Layouts are dense row-major:
+ *       W_H    [H_kv][d][r]        fp32; bit j of a code is [sum_i x_i W_H[i][j] > 0]
+ *       K, V   [B][H_kv][n_cap][d] bf16 or fp32 (kv_dtype), 16-byte aligned
+ *       codes  [B][H_kv][n_cap][r/32] uint32, bit j in word j/32 at bit j%32
+ *                                   (least significant first), 16-byte aligned
+ *       q, out [B][H_q][d] fp32, 16-byte aligned
+ *     Query head h_q uses KV head h_q / (H_q / H_kv) (grouped-query attention);
+ *     its code is made with that KV head's W_H so that codes are comparable.
+ *   - Hash arithmetic: the projection of bit j is the fp32 chain
+ *     acc = fmaf(x_i, W_H[i][j], acc) over i = 0..127 ascending from acc = +0;
+ *     bf16 inputs are widened exactly.  A projection of exactly 0 (or NaN)
+ *     gives bit 0.
+ *   - Argument checks run on the host before anything is launched; a failed
+ *     check returns HATA_ERR_INVALID_ARG / HATA_ERR_UNSUPPORTED and enqueues
+ *     nothing.  A failed launch returns HATA_ERR_CUDA.  Device-side range
+ *     checks (a seq_len beyond max_seq_len or n_cap, an append position
+ *     outside the cache) never fault: the kernel clamps or skips, records a
+ *     flag, and hata_workspace_check / the err_flags word reports it.
+ *   - Nothing throws across the ABI.  Calls are thread-safe; calls that share
+ *     a workspace must be ordered on one stream.
+ */
+#ifndef HATA_H
+#define HATA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hata_status {
+    HATA_OK = 0,
+    HATA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, small workspace */
+    HATA_ERR_UNSUPPORTED = 2,   /* d != 128, r != 128, H_q not a multiple of H_kv */
+    HATA_ERR_CUDA = 3,          /* a CUDA launch or copy failed */
+    HATA_ERR_DEVICE_CHECK = 4   /* a device-side range check fired (see the flags) */
+} hata_status_t;
+
+typedef enum hata_dtype {
+    HATA_DT_BF16 = 0,
+    HATA_DT_F32 = 1
+} hata_dtype_t;
+
+/* Device-side check flags (OR-ed into the error word). */
+#define HATA_FLAG_SEQ_LEN_RANGE 1u  /* seq_len[b] < 0, > max_seq_len or > n_cap: clamped */
+#define HATA_FLAG_POS_RANGE     2u  /* an append position outside [0, n_cap): skipped  */
+
+/* ABI revision; bumps whenever a signature below changes. */
+int hata_abi_version(void);
+
+/* Static text for a status code. */
+const char *hata_status_string(int status);
+
+/* Text describing the most recent failed call on this host thread
+ * (thread-local; "" if none). */
+const char *hata_last_error(void);
+
+/* ------------------------------------------------------------------------
+ * hata_hash_keys -- prefill (Algorithm 1: KH <- HashEncode(K); Kcache_H <- KH).
+ * Hashes the keys of positions [pos0, pos0 + n) of every (b, h_kv) of the
+ * key cache K with W_H[h_kv] and writes codes[b][h_kv][pos0 .. pos0+n).
+ *   K      [B][H_kv][n_cap][d] (kv_dtype)   read
+ *   W_H    [H_kv][d][r] fp32                read
+ *   codes  [B][H_kv][n_cap][r/32] uint32    written at the hashed positions only
+ * Requires 0 <= pos0, n >= 0, pos0 + n <= n_cap.  n == 0 enqueues nothing. */
+hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t n_cap,
+                             const float *W_H, uint32_t *codes, int B, int H_kv,
+                             int64_t pos0, int64_t n, int d, int r, void *stream);
+
+/* ------------------------------------------------------------------------
+ * hata_append_code -- decode-time growth of the key code cache (the decode
+ * stage extends Kcache_H by one token per step): hashes k_new[b][h] with
+ * W_H[h] and writes it to codes[b][h][pos[b]].
+ *   k_new     [B][H_kv][d] (kv_dtype)   read
+ *   pos       [B] int32, device         read; a position outside [0, n_cap)
+ *                                       is skipped and flagged
+ *   err_flags optional device uint32    HATA_FLAG_POS_RANGE is OR-ed in
+ */
+hata_status_t hata_append_code(const void *k_new, hata_dtype_t kv_dtype, const float *W_H,
+                               uint32_t *codes, int64_t n_cap, const int32_t *pos, int B,
+                               int H_kv, int d, int r, uint32_t *err_flags, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Workspace of hata_decode_step: device memory of at least this many bytes,
+ * 256-byte aligned, owned by the caller.  It needs no initialisation and
+ * carries no state between calls.  Returns 0 for invalid sizes. */
+size_t hata_decode_workspace_size(int B, int H_q, int H_kv, int64_t max_seq_len, int topk);
+
+/* Row length (bytes) that an optional caller-provided distance buffer must
+ * have at least: max_seq_len rounded up to the scoring chunk (4096). */
+int64_t hata_dist_row_bytes(int64_t max_seq_len);
+
+/* ------------------------------------------------------------------------
+ * hata_decode_step -- one decode step of HATA for every (b, h_q) (Figure 2):
+ *   0. optional append: if k_new != NULL its rows are hashed into
+ *      codes[b][h][seq_len[b]-1]; if v_new (and k_new) are given, k_new and
+ *      v_new are also copied into K/V at that position;
+ *   1. q_code[b][h_q] = h(q[b][h_q]) with W_H of its KV head;
+ *   2. dist[b][h_q][n] = popcount(q_code XOR codes[b][h_kv][n]), n < seq_len[b];
+ *   3. S = the min(topk, seq_len[b]) keys of smallest distance, ties in the
+ *      boundary bucket to the lower token index;
+ *   4. out[b][h_q] = sum_{n in S} softmax_n(scale * q.K[n]) V[n]  (fp32
+ *      accumulation, exact softmax over S only).  seq_len[b] == 0 gives 0.
+ * Arguments:
+ *   q         [B][H_q][d] fp32
+ *   W_H       [H_kv][d][r] fp32
+ *   codes     [B][H_kv][n_cap][r/32]; written only by the optional append
+ *   K, V      [B][H_kv][n_cap][d] kv_dtype; written only when v_new is given
+ *   seq_len   [B] int32, device: keys 0 .. seq_len[b]-1 take part
+ *   max_seq_len  host upper bound of every seq_len[b] (sizes the grids;
+ *                1 <= max_seq_len <= n_cap)
+ *   topk      >= 1 (k >= seq_len[b] selects every key)
+ *   scale     softmax scale (1/sqrt(d) for standard attention)
+ *   workspace, workspace_bytes   see hata_decode_workspace_size
+ *   out       [B][H_q][d] fp32, written
+ *   sel_idx   optional [B][H_q][topk] int32: S in ascending token order,
+ *             slots past |S| set to -1
+ *   q_codes   optional [B][H_q][r/32] uint32: the query codes
+ *   dist, dist_row_bytes  optional [B][H_q][dist_row_bytes] uint8: the
+ *             Hamming distances (0..128); positions seq_len[b] ..
+ *             hata_dist_row_bytes(max_seq_len)-1 hold 255;
+ *             dist_row_bytes >= hata_dist_row_bytes(max_seq_len), multiple of 16
+ *   events    optional array of 4 cudaEvent_t recorded on `stream` before the
+ *             first kernel and after each of the three kernels (profiling)
+ */
+hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
+                               void *V, hata_dtype_t kv_dtype, int64_t n_cap,
+                               const int32_t *seq_len, int64_t max_seq_len, const void *k_new,
+                               const void *v_new, int B, int H_q, int H_kv, int d, int r,
+                               int topk, float scale, void *workspace, size_t workspace_bytes,
+                               float *out, int32_t *sel_idx, uint32_t *q_codes, uint8_t *dist,
+                               int64_t dist_row_bytes, void *const *events, void *stream);
+
+/* ------------------------------------------------------------------------
+ * hata_workspace_check -- synchronises `stream`, reads and clears the
+ * device-side check flags of a decode workspace.  Returns HATA_OK if none
+ * fired, HATA_ERR_DEVICE_CHECK otherwise (flags, if non-NULL, receives them). */
+hata_status_t hata_workspace_check(void *workspace, size_t workspace_bytes, uint32_t *flags,
+                                   void *stream);
+
+/* ------------------------------------------------------------------------
+ * hata_dense_decode -- dense decode attention over all keys 0..seq_len[b]-1
+ * (the full-attention baseline HATA is compared with; with topk >= seq_len
+ * hata_decode_step must agree with it).  Same layouts as hata_decode_step.
+ * workspace: hata_dense_workspace_size bytes, 256-byte aligned. */
+size_t hata_dense_workspace_size(int B, int H_q, int H_kv, int64_t max_seq_len);
+hata_status_t hata_dense_decode(const float *q, const void *K, const void *V,
+                                hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                                int64_t max_seq_len, int B, int H_q, int H_kv, int d,
+                                float scale, void *workspace, size_t workspace_bytes,
+                                float *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HATA_H */

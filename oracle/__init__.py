@@ -33,13 +33,23 @@ DT_BF16 = 0
 DT_F32 = 1
 
 
+def _cpu_has_fma() -> bool:
+    try:
+        with open("/proc/cpuinfo") as f:
+            return any(line.startswith("flags") and " fma" in line for line in f)
+    except OSError:
+        return False
+
+
 def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
     """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
     if (not force and os.path.exists(out)
             and os.path.getmtime(out) >= os.path.getmtime(src)):
         return out
-    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+    cmd = ["gcc", "-O3", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
            "-fPIC", "-shared", "-o", out + ".tmp", src, "-lm"]
+    if _cpu_has_fma():
+        cmd.insert(1, "-mfma")
     subprocess.check_call(cmd)
     os.replace(out + ".tmp", out)
     return out

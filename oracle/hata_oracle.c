@@ -34,8 +34,9 @@
  *     here in fp64 from the stored (bf16 or fp32) K and V values;
  *   - attention over an empty key set returns the zero vector.
  *
- * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC (see build.py).
- * fmaf() is the correctly rounded C99 fused multiply-add.
+ * Build: gcc -O3 -ffp-contract=off -fno-fast-math -shared -fPIC, plus -mfma
+ * where the host CPU has it (see __init__.py).  fmaf() is the correctly
+ * rounded C99 fused multiply-add with or without -mfma.
  */
 #include <math.h>
 #include <stdint.h>
@@ -65,15 +66,21 @@ static float load_elem(const void *base, int dtype, int64_t i)
  * h(x) = sign(x W_H): one bit per column j of W_H. */
 void oracle_hash_f32(const float *x, const float *W, int d, int r, uint32_t *code)
 {
+    /* acc[j] is bit j's projection; every acc[j] runs its own chain over
+     * i = 0, 1, ..., d-1 (the loops are nested i-outer only so that the r
+     * independent chains advance side by side). */
+    float *acc = (float *)malloc(sizeof(float) * (size_t)r);
+    for (int j = 0; j < r; ++j)
+        acc[j] = 0.0f;
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < r; ++j)
+            acc[j] = fmaf(x[i], W[(int64_t)i * r + j], acc[j]);
     for (int w = 0; w < r / 32; ++w)
         code[w] = 0u;
-    for (int j = 0; j < r; ++j) {
-        float acc = 0.0f;
-        for (int i = 0; i < d; ++i)
-            acc = fmaf(x[i], W[(int64_t)i * r + j], acc);
-        if (acc > 0.0f)
+    for (int j = 0; j < r; ++j)
+        if (acc[j] > 0.0f)
             code[j / 32] |= 1u << (j % 32);
-    }
+    free(acc);
 }
 
 /* Same hash for a vector stored in bf16 or fp32 (widened exactly first). */

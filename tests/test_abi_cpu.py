@@ -1,0 +1,127 @@
+"""The C-ABI library without a GPU: it loads, exports every function that
+include/hata.h declares, sizes workspaces, and rejects bad arguments on the
+host before anything is enqueued (so no call here reaches the GPU)."""
+import ctypes
+
+import pytest
+import torch
+
+from hash_aware_top_hata_b200 import hata as H
+
+pytestmark = pytest.mark.skipif(
+    torch.cuda.is_available(),
+    reason="uses fake device addresses; the GPU suite checks the same cases with real tensors")
+
+FAKE = 1 << 20          # 256-byte aligned fake device address (never dereferenced)
+NULL = None
+
+
+def test_library_exports_every_header_function():
+    names = H.header_functions()
+    assert len(names) >= 10
+    lib = H.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert H.hata_abi_version() == 1
+
+
+def test_status_strings():
+    assert H.hata_status_string(0) == "HATA_OK"
+    assert H.hata_status_string(1) == "HATA_ERR_INVALID_ARG"
+    assert H.hata_status_string(4) == "HATA_ERR_DEVICE_CHECK"
+    assert H.hata_status_string(99) == "HATA_ERR_UNKNOWN"
+
+
+def test_workspace_sizes():
+    s = H.hata_decode_workspace_size(4, 32, 8, 131072, 2048)
+    assert s > 4 * 32 * 131072  # holds the u8 distance rows at least
+    assert H.hata_decode_workspace_size(1, 1, 1, 4096, 64) > 0
+    assert H.hata_decode_workspace_size(0, 1, 1, 4096, 64) == 0
+    assert H.hata_decode_workspace_size(1, 3, 2, 4096, 64) == 0     # H_q % H_kv
+    assert H.hata_decode_workspace_size(1, 1, 1, 0, 64) == 0
+    assert H.hata_decode_workspace_size(1, 1, 1, 4096, 0) == 0
+    assert H.hata_dist_row_bytes(1) == 4096
+    assert H.hata_dist_row_bytes(4096) == 4096
+    assert H.hata_dist_row_bytes(4097) == 8192
+    assert H.hata_dense_workspace_size(1, 32, 8, 1 << 20) > 0
+
+
+def decode(**over):
+    """hata_decode_step through raw ctypes with fake (never touched) pointers."""
+    args = dict(q=FAKE, W=FAKE, codes=FAKE, K=FAKE, V=FAKE, dt=0, n_cap=8192, seq_len=FAKE,
+                max_len=4096, k_new=NULL, v_new=NULL, B=1, H_q=4, H_kv=2, d=128, r=128, topk=64,
+                scale=0.088, ws=FAKE, ws_bytes=1 << 40, out=FAKE, sel=NULL, qc=NULL, dist=NULL,
+                drow=0, ev=NULL, stream=NULL)
+    args.update(over)
+    return H.lib().hata_decode_step(*args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(codes=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(seq_len=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(ws=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(d=64), H.HATA_ERR_UNSUPPORTED),
+    (dict(r=64), H.HATA_ERR_UNSUPPORTED),
+    (dict(H_q=3), H.HATA_ERR_UNSUPPORTED),
+    (dict(B=0), H.HATA_ERR_INVALID_ARG),
+    (dict(topk=0), H.HATA_ERR_INVALID_ARG),
+    (dict(max_len=0), H.HATA_ERR_INVALID_ARG),
+    (dict(max_len=8193), H.HATA_ERR_INVALID_ARG),
+    (dict(n_cap=1 << 31), H.HATA_ERR_INVALID_ARG),
+    (dict(dt=7), H.HATA_ERR_INVALID_ARG),
+    (dict(v_new=FAKE), H.HATA_ERR_INVALID_ARG),
+    (dict(q=FAKE + 4), H.HATA_ERR_INVALID_ARG),
+    (dict(codes=FAKE + 8), H.HATA_ERR_INVALID_ARG),
+    (dict(K=FAKE + 2), H.HATA_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 16), H.HATA_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), H.HATA_ERR_INVALID_ARG),
+    (dict(dist=FAKE, drow=100), H.HATA_ERR_INVALID_ARG),
+    (dict(dist=FAKE, drow=4080), H.HATA_ERR_INVALID_ARG),
+    (dict(B=4096, H_q=32, H_kv=8), H.HATA_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), H.HATA_ERR_INVALID_ARG),
+])
+def test_decode_step_rejects_on_host(over, status):
+    assert decode(**over) == status
+    assert H.lib().hata_last_error().decode() != ""
+
+
+def test_hash_and_append_reject_on_host():
+    L = H.lib()
+    ok_args = [FAKE, 0, 4096, FAKE, FAKE, 1, 2, 0, 4096, 128, 128, NULL]
+    bad = list(ok_args); bad[10] = 96
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_UNSUPPORTED
+    bad = list(ok_args); bad[8] = 4097
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[7] = -1
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[4] = FAKE + 4
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[0] = NULL
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    # n == 0 is a valid no-op that enqueues nothing
+    zero = list(ok_args); zero[8] = 0
+    assert L.hata_hash_keys(*zero) == H.HATA_OK
+    app = [FAKE, 0, FAKE, FAKE, 4096, FAKE, 1, 2, 128, 128, NULL, NULL]
+    bad = list(app); bad[5] = NULL
+    assert L.hata_append_code(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(app); bad[8] = 64
+    assert L.hata_append_code(*bad) == H.HATA_ERR_UNSUPPORTED
+
+
+def test_dense_rejects_on_host():
+    L = H.lib()
+    args = [FAKE, FAKE, FAKE, 0, 8192, FAKE, 4096, 1, 4, 2, 128, 0.1, FAKE, 1 << 40, FAKE, NULL]
+    bad = list(args); bad[10] = 64
+    assert L.hata_dense_decode(*bad) == H.HATA_ERR_UNSUPPORTED
+    bad = list(args); bad[13] = 16
+    assert L.hata_dense_decode(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(args); bad[6] = 9000
+    assert L.hata_dense_decode(*bad) == H.HATA_ERR_INVALID_ARG
+
+
+def test_workspace_check_rejects_bad_workspace():
+    flags = ctypes.c_uint32(7)
+    assert H.lib().hata_workspace_check(NULL, 4096, ctypes.byref(flags), NULL) == \
+        H.HATA_ERR_INVALID_ARG
+    assert flags.value == 0

@@ -14,13 +14,14 @@ from tests import test_oracle_pins as pins
 SRC = os.path.join(os.path.dirname(oracle.__file__), "hata_oracle.c")
 
 MUTANTS = {
-    "W_H transposed": ("W[(int64_t)i * r + j]", "W[(int64_t)j * d + i]"),
-    "sign test >= 0": ("if (acc > 0.0f)", "if (acc >= 0.0f)"),
+    "W_H transposed": ("fmaf(x[i], W[(int64_t)i * r + j], acc[j])",
+                       "fmaf(x[i], W[(int64_t)j * d + i], acc[j])"),
+    "sign test >= 0": ("if (acc[j] > 0.0f)", "if (acc[j] >= 0.0f)"),
     "bits packed MSB first": ("code[j / 32] |= 1u << (j % 32);",
                               "code[j / 32] |= 1u << (31 - j % 32);"),
     "projection in descending order": (
-        "for (int i = 0; i < d; ++i)\n            acc = fmaf",
-        "for (int i = d - 1; i >= 0; --i)\n            acc = fmaf"),
+        "for (int i = 0; i < d; ++i)\n        for (int j = 0; j < r; ++j)",
+        "for (int i = d - 1; i >= 0; --i)\n        for (int j = 0; j < r; ++j)"),
     "hamming counts equal bits": ("uint32_t x = a[j / 32] ^ b[j / 32];",
                                   "uint32_t x = ~(a[j / 32] ^ b[j / 32]);"),
     "ties go to the higher index": ("return a->i < b->i ? -1 : 1;",

@@ -1,0 +1,323 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bar: codes, distances and selected indices bit-exact; attention outputs
+within 2e-3 max abs error (bf16 K/V, fp32 accumulation).  Inputs are the
+seeded synthetic workloads of hash_aware_top_hata_b200.workloads."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hash_aware_top_hata_b200 import hata as H
+from hash_aware_top_hata_b200 import workloads as wl
+from tests.gpu_cases import (ATOL, SCALE, GpuDecoder, compare_head, host_append, host_slabs,
+                             oracle_head, to_np_codes)
+
+pytestmark = pytest.mark.gpu
+
+
+def _kv(dtype, shape, gen, scale=1.0):
+    t = torch.randn(shape, generator=gen, device="cuda") * scale
+    return t.to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+
+
+# ------------------------------------------------------------------ hash --
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_hash_keys_bit_exact(dtype):
+    g = torch.Generator(device="cuda").manual_seed(11)
+    B, Hkv, n_cap, pos0, n = 2, 3, 5003, 3, 4997
+    K = _kv(dtype, (B, Hkv, n_cap, 128), g)
+    W = torch.randn((Hkv, 128, 128), generator=g, device="cuda") / math.sqrt(128)
+    # adversarial rows: a zero key, a key whose projections hit exact zeros
+    K[0, 0, 10] = 0
+    W[1, :, 77] = 0
+    K[1, 2, 20] = -K[1, 2, 21]
+    codes = torch.full((B, Hkv, n_cap, 4), -1, dtype=torch.int32, device="cuda")
+    H.hata_hash_keys(K, W, codes, pos0, n)
+    got = to_np_codes(codes)
+    Kh = wl.to_numpy_kv(K)
+    want = oracle.hash_keys(Kh, W.cpu().numpy(), pos0=pos0, n=n)
+    assert np.array_equal(got[:, :, pos0:pos0 + n], want[:, :, pos0:pos0 + n])
+    assert np.all(got[:, :, :pos0] == 0xFFFFFFFF) and np.all(got[:, :, pos0 + n:] == 0xFFFFFFFF)
+    assert np.all(got[0, 0, 10] == 0)
+    assert np.all((got[:, 1, pos0:pos0 + n, 2] >> 13) & 1 == 0)  # bit 77 = word 2, bit 13
+
+
+def test_append_code_and_position_check():
+    g = torch.Generator(device="cuda").manual_seed(12)
+    B, Hkv, n_cap = 3, 2, 100
+    k_new = _kv("bf16", (B, Hkv, 128), g)
+    W = torch.randn((Hkv, 128, 128), generator=g, device="cuda") / math.sqrt(128)
+    codes = torch.zeros((B, Hkv, n_cap, 4), dtype=torch.int32, device="cuda")
+    pos = torch.tensor([0, 99, 100], dtype=torch.int32, device="cuda")   # last one out of range
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    H.hata_append_code(k_new, W, codes, pos, err_flags=err)
+    got = to_np_codes(codes)
+    kn = wl.to_numpy_kv(k_new)
+    Wh = W.cpu().numpy()
+    for b, p in ((0, 0), (1, 99)):
+        for h in range(Hkv):
+            assert np.array_equal(got[b, h, p], oracle.hash_vec(kn[b, h], Wh[h]))
+    assert np.all(got[2] == 0)
+    assert int(err.item()) == H.HATA_FLAG_POS_RANGE
+
+
+# ---------------------------------------------------------------- decode --
+
+def run_and_check(cfg, seed, steps, topk=None, heads=None, n_cap=None):
+    """Decode `steps` steps (each appends one token) on the GPU and compare
+    the given heads (default: all) with the oracle after every step."""
+    topk = cfg.topk if topk is None else topk
+    w = wl.make_workload(cfg, seed, device="cuda", steps=steps, n_cap=n_cap)
+    G = cfg.G
+    if heads is None:
+        heads = [(b, hq) for b in range(cfg.B) for hq in range(cfg.H_q)]
+    pairs = sorted({(b, hq // G) for b, hq in heads})
+    slabs = host_slabs(w, pairs)
+    Wn = w.W_H.cpu().numpy()
+    dec = GpuDecoder(w, topk)
+    worst = 0.0
+    for t in range(steps):
+        pos = [cfg.N + t] * cfg.B
+        host_append(slabs, w, t, pos)
+        n = cfg.N + t + 1
+        got = dec.step(w.q[t], [n] * cfg.B, k_new=w.k_new[t], v_new=w.v_new[t])
+        codes_cache = {}
+        gcodes = to_np_codes(dec.codes)
+        for b, hq in heads:
+            h = hq // G
+            codes = codes_cache.get((b, h))
+            want = oracle_head(slabs[(b, h)], Wn[h], w.q[t, b, hq].cpu().numpy(), n, topk, codes)
+            if codes is None:
+                codes_cache[(b, h)] = want[0]
+                assert np.array_equal(gcodes[b, h, :n], want[0]), ("key codes", b, h)
+            worst = max(worst, compare_head(got, want, b, hq, n, dec.drow))
+        # the K/V rows appended by the step match the generator's
+        for (b, h), s in slabs.items():
+            p = pos[b]
+            assert np.array_equal(wl.to_numpy_kv(w.K[b, h, p]), s.K[p])
+            assert np.array_equal(wl.to_numpy_kv(w.V[b, h, p]), s.V[p])
+    return worst
+
+
+SCALED = {
+    "tiny_mha_4k": dict(N=4096),
+    "llama2_7b_mha_32k": dict(N=9000, topk=140),
+    "llama31_8b_gqa_128k": dict(N=10000, topk=156, B=2),
+    "qwen_gqa_b32_32k": dict(N=6000, topk=94, B=3),
+    "needle_gqa_1m": dict(N=12289, topk=192),
+}
+
+
+@pytest.mark.parametrize("name", wl.CONFIG_ORDER)
+def test_decode_scaled_configs(name):
+    kw = SCALED[name]
+    cfg = wl.scaled(wl.CONFIGS[name], **kw)
+    if cfg.needles:
+        cfg = wl.dataclasses.replace(cfg, needles=16)
+    run_and_check(cfg, seed=wl.SEED_BASE + wl.CONFIG_ORDER.index(name), steps=2)
+
+
+def test_decode_tiny_config_full_size():
+    cfg = wl.CONFIGS["tiny_mha_4k"]
+    w_err = run_and_check(cfg, seed=wl.SEED_BASE, steps=1)
+    assert w_err <= ATOL
+
+
+@pytest.mark.parametrize("N,topk", [(1, 1), (1, 5), (7, 3), (31, 31), (31, 64), (100, 1),
+                                    (4095, 4095), (4096, 2), (4097, 4097), (8192, 300),
+                                    (9000, 9000), (12345, 20000)])
+def test_decode_edge_sizes(N, topk):
+    cfg = wl.Config("edge", 1, 4, 2, N, topk, "bf16", 0.0, 0.0, 0, 1)
+    run_and_check(cfg, seed=31 + N, steps=1)
+
+
+def test_decode_ragged_batch_lengths():
+    """Sequences of one batch at different lengths, including an empty one."""
+    cfg = wl.Config("ragged", 4, 4, 2, 9000, 70, "bf16", 0.0, 0.0, 0, 1)
+    w = wl.make_workload(cfg, 41, device="cuda", steps=1)
+    lens = [0, 1, 4096, 8999]
+    pairs = [(b, h) for b in range(4) for h in range(2)]
+    slabs = host_slabs(w, pairs)
+    dec = GpuDecoder(w, cfg.topk, max_seq_len=9000)
+    got = dec.step(w.q[0], lens)
+    Wn = w.W_H.cpu().numpy()
+    for b in range(4):
+        for hq in range(4):
+            n = lens[b]
+            if n == 0:
+                assert np.all(got[0][b, hq] == 0) and np.all(got[1][b, hq] == -1)
+                assert np.all(got[3][b, hq] == 255)
+                continue
+            want = oracle_head(slabs[(b, hq // 2)], Wn[hq // 2], w.q[0, b, hq].cpu().numpy(), n,
+                               cfg.topk)
+            compare_head(got, want, b, hq, n, dec.drow)
+
+
+def test_all_equal_distances_take_lowest_indices():
+    """Identical keys: every distance ties, so S = {0 .. k-1}."""
+    cfg = wl.Config("ties", 1, 2, 1, 10000, 5000, "bf16", 0.0, 0.0, 0, 1)
+    w = wl.make_workload(cfg, 51, device="cuda", steps=1)
+    w.K[0, 0, :] = w.K[0, 0, 0].clone()
+    dec = GpuDecoder(w, cfg.topk)
+    out, sel, qc, dist = dec.step(w.q[0], [cfg.N])
+    assert np.all(sel[0, :, :] == np.arange(5000)[None, :])
+    assert np.all(dist[0, :, :cfg.N] == dist[0, :, :1])
+
+
+def test_tie_bucket_spanning_chunk_boundaries():
+    """A run of identical keys across chunk boundaries forms the boundary
+    bucket; the lower-index ties must win, chunk by chunk."""
+    cfg = wl.Config("tie-span", 1, 3, 1, 20000, 3000, "bf16", 0.0, 0.0, 0, 1)
+    w = wl.make_workload(cfg, 52, device="cuda", steps=1)
+    w.K[0, 0, 3000:14000] = w.K[0, 0, 7].clone()
+    slabs = host_slabs(w, [(0, 0)])
+    dec = GpuDecoder(w, cfg.topk)
+    got = dec.step(w.q[0], [cfg.N])
+    Wn = w.W_H.cpu().numpy()
+    for hq in range(3):
+        want = oracle_head(slabs[(0, 0)], Wn[0], w.q[0, 0, hq].cpu().numpy(), cfg.N, cfg.topk)
+        compare_head(got, want, 0, hq, cfg.N, dec.drow)
+
+
+def test_full_budget_equals_dense():
+    """k >= seq_len selects every key: the sparse output equals dense softmax
+    attention (the GPU dense kernel and the oracle's)."""
+    cfg = wl.Config("dense", 2, 8, 2, 7000, 8000, "bf16", 0.0, 0.0, 0, 1)
+    w = wl.make_workload(cfg, 61, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk)
+    out, sel, _, _ = dec.step(w.q[0], [cfg.N, 5000])
+    dws = torch.empty(H.hata_dense_workspace_size(2, 8, 2, cfg.N), dtype=torch.uint8,
+                      device="cuda")
+    dout = torch.empty((2, 8, 128), device="cuda")
+    sl = torch.tensor([cfg.N, 5000], dtype=torch.int32, device="cuda")
+    H.hata_dense_decode(w.q[0], w.K, w.V, sl, cfg.N, SCALE, dws, dout)
+    dout = dout.cpu().numpy()
+    for b, n in ((0, cfg.N), (1, 5000)):
+        assert np.all(sel[b, :, :n] == np.arange(n)[None, :]) and np.all(sel[b, :, n:] == -1)
+        for hq in range(8):
+            K = wl.to_numpy_kv(w.K[b, hq // 4, :n])
+            V = wl.to_numpy_kv(w.V[b, hq // 4, :n])
+            ref = oracle.dense(w.q[0, b, hq].cpu().numpy(), K, V, n, SCALE)
+            assert np.max(np.abs(out[b, hq] - ref)) <= ATOL
+            assert np.max(np.abs(dout[b, hq] - ref)) <= ATOL
+
+
+def test_dense_kernel_matches_oracle_all_shapes():
+    for (B, Hq, Hkv, N, dt) in ((1, 1, 1, 4096, "f32"), (2, 28, 4, 5000, "bf16"),
+                                (1, 32, 32, 3001, "bf16"), (1, 12, 1, 100, "bf16")):
+        cfg = wl.Config("dense", B, Hq, Hkv, N, 1, dt, 0.0, 0.0, 0, 1)
+        w = wl.make_workload(cfg, 62, device="cuda", steps=1)
+        dws = torch.empty(H.hata_dense_workspace_size(B, Hq, Hkv, N), dtype=torch.uint8,
+                          device="cuda")
+        dout = torch.empty((B, Hq, 128), device="cuda")
+        sl = torch.full((B,), N, dtype=torch.int32, device="cuda")
+        H.hata_dense_decode(w.q[0], w.K, w.V, sl, N, SCALE, dws, dout)
+        dout = dout.cpu().numpy()
+        G = Hq // Hkv
+        for b in range(B):
+            for hq in range(Hq):
+                K = wl.to_numpy_kv(w.K[b, hq // G, :N])
+                V = wl.to_numpy_kv(w.V[b, hq // G, :N])
+                ref = oracle.dense(w.q[0, b, hq].cpu().numpy(), K, V, N, SCALE)
+                assert np.max(np.abs(dout[b, hq] - ref)) <= ATOL, (B, Hq, Hkv, N, b, hq)
+
+
+def test_repeatable_bitwise():
+    """Two identical calls give bitwise identical results (no races)."""
+    cfg = wl.scaled(wl.CONFIGS["qwen_gqa_b32_32k"], N=9000, topk=140, B=4)
+    w = wl.make_workload(cfg, 71, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk)
+    a = dec.step(w.q[0], [cfg.N] * 4)
+    b = dec.step(w.q[0], [cfg.N] * 4)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_seq_len_beyond_max_is_flagged_and_clamped():
+    cfg = wl.Config("flag", 2, 2, 1, 5000, 50, "bf16", 0.0, 0.0, 0, 1)
+    w = wl.make_workload(cfg, 81, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk, max_seq_len=4000)
+    out = torch.empty((2, 2, 128), device="cuda")
+    sl = torch.tensor([4000, 4500], dtype=torch.int32, device="cuda")
+    H.hata_decode_step(w.q[0], w.W_H, dec.codes, w.K, w.V, sl, 4000, cfg.topk, SCALE, dec.ws,
+                       out)
+    with pytest.raises(H.HataError) as e:
+        H.hata_workspace_check(dec.ws)
+    assert e.value.status == H.HATA_ERR_DEVICE_CHECK
+    # flags are cleared by the check and recomputed by the next step
+    sl = torch.tensor([4000, 3999], dtype=torch.int32, device="cuda")
+    H.hata_decode_step(w.q[0], w.W_H, dec.codes, w.K, w.V, sl, 4000, cfg.topk, SCALE, dec.ws,
+                       out)
+    assert H.hata_workspace_check(dec.ws) == 0
+
+
+def test_invalid_arguments_with_real_tensors():
+    cfg = wl.Config("bad", 1, 4, 2, 5000, 50, "bf16", 0.0, 0.0, 0, 1)
+    w = wl.make_workload(cfg, 82, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk)
+    out = torch.empty((1, 4, 128), device="cuda")
+    sl = torch.tensor([cfg.N], dtype=torch.int32, device="cuda")
+    cases = [
+        dict(topk=0),
+        dict(max_seq_len=0),
+        dict(max_seq_len=w.n_cap + 1),
+        dict(workspace=dec.ws[:1024]),
+        dict(workspace=dec.ws[16:]),
+    ]
+    for over in cases:
+        args = dict(q=w.q[0], W_H=w.W_H, codes=dec.codes, K=w.K, V=w.V, seq_len=sl,
+                    max_seq_len=dec.max_seq_len, topk=cfg.topk, scale=SCALE,
+                    workspace=dec.ws, out=out)
+        args.update(over)
+        with pytest.raises(H.HataError) as e:
+            H.hata_decode_step(**args)
+        assert e.value.status == H.HATA_ERR_INVALID_ARG
+    with pytest.raises(H.HataError) as e:
+        H.hata_decode_step(w.q[0][:, :3], w.W_H, dec.codes, w.K, w.V, sl, dec.max_seq_len,
+                           cfg.topk, SCALE, dec.ws, out[:, :3])
+    assert e.value.status == H.HATA_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------ full-size configs --
+
+FULL = {
+    "llama2_7b_mha_32k": [(0, 0), (0, 31)],
+    "llama31_8b_gqa_128k": [(0, 0), (3, 29)],
+    "qwen_gqa_b32_32k": [(0, 0), (31, 27)],
+    "needle_gqa_1m": [(0, 0), (0, 1)],
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size_sampled_heads(name):
+    """Full-size workloads in the launch configuration bench.py times; the
+    oracle recomputes sampled heads one by one.  For the needle workload the
+    needles of the group's first query head must all be selected."""
+    cfg = wl.CONFIGS[name]
+    heads = FULL[name]
+    w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(name), device="cuda",
+                         steps=1)
+    pairs = sorted({(b, hq // cfg.G) for b, hq in heads})
+    slabs = host_slabs(w, pairs)
+    pos = [cfg.N] * cfg.B
+    host_append(slabs, w, 0, pos)
+    dec = GpuDecoder(w, cfg.topk)
+    n = cfg.N + 1
+    got = dec.step(w.q[0], [n] * cfg.B, k_new=w.k_new[0], v_new=w.v_new[0])
+    Wn = w.W_H.cpu().numpy()
+    cache = {}
+    for b, hq in heads:
+        h = hq // cfg.G
+        want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n, cfg.topk,
+                           cache.get((b, h)))
+        cache[(b, h)] = want[0]
+        compare_head(got, want, b, hq, n, dec.drow)
+        if cfg.needles and hq % cfg.G == 0:
+            needles = set(w.planted[b, h].tolist())
+            assert needles <= set(got[1][b, hq].tolist())
+    del w, dec
+    torch.cuda.empty_cache()
