@@ -4,6 +4,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "hata_internal.cuh"
 
@@ -67,6 +69,25 @@ struct Events {
 
 }  // namespace
 
+namespace hata {
+
+cudaError_t ensure_smem_attr(const void *func, size_t bytes)
+{
+    static std::mutex mu;
+    static std::unordered_map<const void *, uint64_t> done;  // bit d: set on device d
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev)) return e;
+    const uint64_t bit = dev < 64 ? uint64_t(1) << dev : 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (bit && (done[func] & bit)) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    if (e == cudaSuccess) done[func] |= bit;
+    return e;
+}
+
+}  // namespace hata
+
 extern "C" {
 
 int hata_abi_version(void) { return 1; }
@@ -116,7 +137,7 @@ hata_status_t hata_append_code(const void *k_new, hata_dtype_t kv_dtype, const f
     if (B <= 0 || H_kv <= 0 || int64_t(B) * H_kv > (int64_t(1) << 24) || H_kv > 65535)
         return fail(HATA_ERR_INVALID_ARG, "B=%d H_kv=%d out of range", B, H_kv);
     if (n_cap <= 0) return fail(HATA_ERR_INVALID_ARG, "n_cap=%lld", (long long)n_cap);
-    if (!aligned(k_new, 4) || !aligned(codes, 16) || !aligned(pos, 4) ||
+    if (!aligned(k_new, 4) || !aligned(codes, 16) || !aligned(pos, 4) || !aligned(W_H, 16) ||
         (err_flags && !aligned(err_flags, 4)))
         return fail(HATA_ERR_INVALID_ARG, "misaligned pointer");
     PrepArgs a{};
@@ -131,7 +152,6 @@ hata_status_t hata_append_code(const void *k_new, hata_dtype_t kv_dtype, const f
     a.H_q = H_kv;
     a.H_kv = H_kv;
     a.G = 1;
-    a.zgroups = 1;
     a.kv_bf16 = kv_dtype == HATA_DT_BF16;
     const cudaError_t e = launch_prep(a, B, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "append_code launch");
@@ -171,10 +191,11 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
         return fail(HATA_ERR_INVALID_ARG, "scale must be finite");
     if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(codes, 16) ||
-        !aligned(out, 16) || !aligned(W_H, 4) || !aligned(seq_len, 4) ||
+        !aligned(out, 16) || !aligned(W_H, 16) || !aligned(seq_len, 4) ||
         (k_new && !aligned(k_new, 4)) || (v_new && !aligned(v_new, 4)) ||
         (sel_idx && !aligned(sel_idx, 4)) || (q_codes && !aligned(q_codes, 16)))
-        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer (q, K, V, codes, out, q_codes: 16 B)");
+        return fail(HATA_ERR_INVALID_ARG,
+                    "misaligned pointer (q, W_H, K, V, codes, out, q_codes: 16 B)");
     if (!aligned(workspace, 256)) return fail(HATA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     DecodeLayout L;
     if (!decode_layout(B, H_q, H_kv, max_seq_len, topk, &L))
@@ -195,11 +216,11 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     uint32_t *qc = q_codes ? q_codes : reinterpret_cast<uint32_t *>(ws + L.off_qcodes);
     uint8_t *dst = dist ? dist : reinterpret_cast<uint8_t *>(ws + L.off_dist);
     const int64_t drow = dist ? dist_row_bytes : L.dist_row;
+    int32_t *idx = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(ws + L.off_idx);
+    uint32_t *flags = reinterpret_cast<uint32_t *>(ws + L.off_flags);
     uint32_t *hist = reinterpret_cast<uint32_t *>(ws + L.off_hist);
-    uint32_t *cnt_score = reinterpret_cast<uint32_t *>(ws + L.off_cnt_score);
+    uint32_t *cum = reinterpret_cast<uint32_t *>(ws + L.off_cum);
     uint32_t *cnt_attn = reinterpret_cast<uint32_t *>(ws + L.off_cnt_attn);
-    PlanHead *plan_head = reinterpret_cast<PlanHead *>(ws + L.off_plan_head);
-    PlanChunk *plan_chunk = reinterpret_cast<PlanChunk *>(ws + L.off_plan_chunk);
     const Events ev{events, s};
     cudaError_t e;
 
@@ -215,10 +236,9 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     p.V = V;
     p.seq_len = seq_len;
     p.q_out = qc;
-    p.flags = reinterpret_cast<uint32_t *>(ws + L.off_flags);
+    p.flags = flags;
     p.hist_total = hist;
     p.cnt_attn = cnt_attn;
-    p.cnt_score = cnt_score;
     p.ws_header = reinterpret_cast<uint32_t *>(ws);
     p.n_cap = n_cap;
     p.max_seq_len = max_seq_len;
@@ -226,7 +246,6 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     p.H_q = H_q;
     p.H_kv = H_kv;
     p.G = G;
-    p.zgroups = L.zgroups;
     p.kv_bf16 = kv_dtype == HATA_DT_BF16;
     if ((e = launch_prep(p, B * G + (k_new ? B : 0), s)) != cudaSuccess)
         return cuda_fail(e, "prep launch");
@@ -238,12 +257,9 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     sa.seq_len = seq_len;
     sa.dist = dst;
     sa.dist_row = drow;
-    sa.cum = reinterpret_cast<uint32_t *>(ws + L.off_cum);
+    sa.cum = cum;
     sa.hist_total = hist;
-    sa.plan_head = plan_head;
-    sa.plan_chunk = plan_chunk;
-    sa.cnt_score = cnt_score;
-    sa.sel_idx = sel_idx;
+    sa.flags = flags;
     sa.n_cap = n_cap;
     sa.max_seq_len = max_seq_len;
     sa.n_chunks = L.n_chunks;
@@ -252,35 +268,47 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     sa.H_kv = H_kv;
     sa.G = G;
     sa.zgroups = L.zgroups;
-    sa.topk = topk;
     if ((e = launch_score(sa, s)) != cudaSuccess) return cuda_fail(e, "score launch");
     if ((e = ev.record(2)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    SelectArgs se{};
+    se.seq_len = seq_len;
+    se.dist = dst;
+    se.dist_row = drow;
+    se.cum = cum;
+    se.hist_total = hist;
+    se.idx = idx;
+    se.n_cap = n_cap;
+    se.max_seq_len = max_seq_len;
+    se.n_chunks = L.n_chunks;
+    se.B = B;
+    se.H_q = H_q;
+    se.topk = topk;
+    if ((e = launch_select(se, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+    if ((e = ev.record(3)) != cudaSuccess) return cuda_fail(e, "event record");
 
     AttendArgs aa{};
     aa.q = q;
     aa.K = K;
     aa.V = V;
     aa.seq_len = seq_len;
-    aa.dist = dst;
-    aa.dist_row = drow;
-    aa.plan_head = plan_head;
-    aa.plan_chunk = plan_chunk;
+    aa.idx = idx;
     aa.part = reinterpret_cast<float *>(ws + L.off_part);
     aa.cnt_attn = cnt_attn;
+    aa.flags = flags;
     aa.out = out;
-    aa.sel_idx = sel_idx;
     aa.n_cap = n_cap;
     aa.max_seq_len = max_seq_len;
-    aa.n_chunks = L.n_chunks;
     aa.B = B;
     aa.H_q = H_q;
     aa.H_kv = H_kv;
     aa.G = G;
     aa.topk = topk;
+    aa.n_split = L.n_split;
     aa.scale_log2 = scale * 1.4426950408889634f;
     if ((e = launch_attend(aa, kv_dtype == HATA_DT_BF16, s)) != cudaSuccess)
         return cuda_fail(e, "attend launch");
-    if ((e = ev.record(3)) != cudaSuccess) return cuda_fail(e, "event record");
+    if ((e = ev.record(4)) != cudaSuccess) return cuda_fail(e, "event record");
     return ok();
 }
 

@@ -27,15 +27,28 @@ constexpr uint32_t kWsMagic = 0x48415441u;  // "HATA"
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+constexpr int kAttnMaxWorkers = 4096;   // upper bound of the attention stream-K workers
+constexpr int kSelSegChunks = 8;        // scoring chunks walked by one selection CTA
+
+// Most attention workers that can share one head: each of the P <= T
+// workers owns at least floor(T / P) >= r_min rows of the flat row space.
+inline int attn_max_contributors(int64_t BH, int topk)
+{
+    const int64_t T = BH * topk;
+    const int64_t r_min = T >= kAttnMaxWorkers ? T / kAttnMaxWorkers : 1;
+    const int64_t c = (topk + r_min - 1) / r_min + 1;
+    return int(c < kAttnMaxWorkers ? c : kAttnMaxWorkers);
+}
+
 // Decode workspace.  The first 256 B hold a header {magic, B}; one flag word
 // per batch row follows.  Everything else is rebuilt by every decode step.
 struct DecodeLayout {
-    int64_t n_chunks = 0;   // chunks of max_seq_len
+    int64_t n_chunks = 0;   // scoring chunks of max_seq_len
     int64_t dist_row = 0;   // bytes per (b, h_q) distance row
     int zgroups = 0;        // ceil(G / kScoreHeads)
+    int n_split = 0;        // attention partial slots per head
     size_t off_flags = 0, off_qcodes = 0, off_dist = 0, off_cum = 0, off_hist = 0,
-           off_plan_head = 0, off_plan_chunk = 0, off_part = 0, off_cnt_score = 0,
-           off_cnt_attn = 0, total = 0;
+           off_idx = 0, off_part = 0, off_cnt_attn = 0, total = 0;
 };
 
 inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
@@ -50,33 +63,21 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
     L->n_chunks = ceil_div(max_seq_len, kChunk);
     L->dist_row = L->n_chunks * kChunk;
     L->zgroups = int(ceil_div(G, kScoreHeads));
+    // the scoring kernel numbers its work items with 32-bit integers
+    if (int64_t(B) * H_kv * L->zgroups * L->n_chunks >= (int64_t(1) << 31)) return false;
+    L->n_split = attn_max_contributors(BH, topk);
     size_t o = 256;
     L->off_flags = o;      o = align_up(o + 4 * size_t(B), 256);
     L->off_qcodes = o;     o = align_up(o + 16 * size_t(BH), 256);
     L->off_dist = o;       o = align_up(o + size_t(BH) * L->dist_row, 256);
     L->off_cum = o;        o = align_up(o + 4 * size_t(BH) * L->n_chunks * kCumStride, 256);
     L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * kHistStride, 256);
-    L->off_plan_head = o;  o = align_up(o + 16 * size_t(BH), 256);
-    L->off_plan_chunk = o; o = align_up(o + 8 * size_t(BH) * L->n_chunks, 256);
-    L->off_part = o;       o = align_up(o + 4 * size_t(BH) * L->n_chunks * kPartStride, 256);
-    L->off_cnt_score = o;  o = align_up(o + 4 * size_t(B) * H_kv * L->zgroups, 256);
+    L->off_idx = o;        o = align_up(o + 4 * size_t(BH) * topk, 256);
+    L->off_part = o;       o = align_up(o + 4 * size_t(BH) * L->n_split * kPartStride, 256);
     L->off_cnt_attn = o;   o = align_up(o + 4 * size_t(BH), 256);
     L->total = o;
     return true;
 }
-
-// Per-head plan written by the last scoring CTA of a (b, kv-head) group.
-struct PlanHead {
-    int32_t T;       // boundary distance (-1: nothing selected)
-    int32_t k_eff;   // min(topk, seq_len)
-    int32_t n_less;  // keys with distance < T
-    int32_t ties;    // keys taken from the boundary bucket
-};
-
-struct PlanChunk {
-    int32_t off;     // first output slot of this chunk's selected keys
-    int32_t take;    // boundary-bucket keys this chunk contributes
-};
 
 // ------------------------------------------------------------------ args --
 struct PrepArgs {
@@ -93,10 +94,9 @@ struct PrepArgs {
     uint32_t *err_word;      // single OR-ed word (append API) or null
     uint32_t *hist_total;    // zeroed for every query row (decode) or null
     uint32_t *cnt_attn;      // zeroed for every query row (decode) or null
-    uint32_t *cnt_score;     // zeroed [B][H_kv][zgroups] (decode) or null
     uint32_t *ws_header;     // {magic, B} written (decode) or null
     int64_t n_cap, max_seq_len;
-    int B, H_q, H_kv, G, zgroups;
+    int B, H_q, H_kv, G;
     int kv_bf16;
 };
 
@@ -108,28 +108,34 @@ struct ScoreArgs {
     int64_t dist_row;
     uint32_t *cum;           // [B][H_q][n_chunks][kCumStride]
     uint32_t *hist_total;    // [B][H_q][kHistStride]
-    PlanHead *plan_head;     // [B][H_q]
-    PlanChunk *plan_chunk;   // [B][H_q][n_chunks]
-    uint32_t *cnt_score;     // [B][H_kv][zgroups]
-    int32_t *sel_idx;        // optional [B][H_q][topk] (only -1 padding written here)
+    uint32_t *flags;         // per-b flag words
     int64_t n_cap, max_seq_len, n_chunks;
-    int B, H_q, H_kv, G, zgroups, topk;
+    int B, H_q, H_kv, G, zgroups;
+};
+
+struct SelectArgs {
+    const int32_t *seq_len;
+    const uint8_t *dist;
+    int64_t dist_row;
+    const uint32_t *cum;
+    const uint32_t *hist_total;
+    int32_t *idx;            // [B][H_q][topk] ascending, -1 padded
+    int64_t n_cap, max_seq_len, n_chunks;
+    int B, H_q, topk;
 };
 
 struct AttendArgs {
     const float *q;
     const void *K, *V;
     const int32_t *seq_len;
-    const uint8_t *dist;
-    int64_t dist_row;
-    const PlanHead *plan_head;
-    const PlanChunk *plan_chunk;
-    float *part;             // [B][H_q][n_chunks][kPartStride]
+    const int32_t *idx;      // [B][H_q][topk]
+    float *part;             // [B][H_q][n_split][kPartStride]
     uint32_t *cnt_attn;      // [B][H_q]
+    uint32_t *flags;
     float *out;
-    int32_t *sel_idx;
-    int64_t n_cap, max_seq_len, n_chunks;
-    int B, H_q, H_kv, G, topk;
+    int64_t n_cap, max_seq_len;
+    int B, H_q, H_kv, G, topk, n_split;
+    int64_t n_workers;       // stream-K workers (set by the launcher)
     float scale_log2;        // scale * log2(e)
 };
 
@@ -164,12 +170,16 @@ inline bool dense_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int64_t 
     return true;
 }
 
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+cudaError_t ensure_smem_attr(const void *func, size_t bytes);
+
 // Launchers (each returns the cudaGetLastError() of its launch).
 cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const float *W,
                                 uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
                                 cudaStream_t s);
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s);
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
 cudaError_t launch_attend(const AttendArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_dense(const DenseArgs &a, bool bf16, cudaStream_t s);
 

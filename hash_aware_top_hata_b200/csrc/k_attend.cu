@@ -1,34 +1,37 @@
-// k_attend.cu -- top-k selection fused with gather + exact softmax attention.
+// k_attend.cu -- gather of the selected K/V rows + exact softmax attention.
 //
-// HATA review page (arXiv 2506.02572): "What carries the argument" (the top-k
-// indices select K/V for attention; the page's implementation fuses the
-// gather into FlashAttention) and major comment 1 (Algorithm 3: the top-k
-// over Hamming scores; boundary ties here go to the lower token index).
+// HATA review page (arXiv 2506.02572), "What carries the argument": the
+// top-k indices select K/V for attention, which the page runs as a fused
+// gather + FlashAttention over the selected keys.
 //
-// Grid: (chunk of 4096 tokens, b * H_q + h_q).  Each CTA
-//   1. reads its chunk's u8 distances (L2-resident from the scoring kernel)
-//      and the plan (T, take_c, off_c), and compacts, in token order, the keys
-//      with dist < T plus its share of dist == T keys into a shared-memory
-//      index list (two block scans; no sort);
-//   2. writes those indices to sel_idx (optional) at off_c -- so the global
-//      list comes out in ascending token order;
-//   3. gathers the selected K and V rows straight from the cache (each 16-lane
-//      half-warp owns one 256-byte bf16 row: one 128-bit load per lane, eight
-//      rows per half-warp in flight) and runs an online softmax in fp32,
-//      base-2 exponent with the scale folded into q;
-//   4. merges its eight half-warp states into one partial (m, l, acc[128]);
-//      the last CTA of the head (fence + arrival counter, no waiting) merges
-//      all chunk partials into out = acc / l.
-#include "block_scan.cuh"
+// Persistent, stream-K style.  The selected rows of all heads form one flat
+// space of B*H_q*topk rows (head bh owns [bh*topk, bh*topk + k_eff)); CTA k of
+// P owns the contiguous range [k*T/P, (k+1)*T/P), so every CTA moves the
+// same number of bytes whatever the distance distribution, and a head is
+// shared by at most a few CTAs.  Each CTA walks its range in stages of up to
+// 32 rows through a 4-deep ring in shared memory: while it computes stage s
+// the 16-byte cp.async copies of stages s+1..s+3 are in flight (for bf16,
+// 16 lanes per 256-byte row; on B200 this random-row gather runs at the
+// streaming HBM bandwidth, where one bulk-copy request per row reaches only
+// half of it).  Every 16-lane half-warp takes rows, computes q.k in fp32
+// with the softmax scale and log2(e) folded into q, and keeps an online
+// softmax state (m, l, acc[8 per lane]).  When a CTA leaves a head, its
+// eight half-warp states merge into one partial (m, l, acc[128]); the last
+// of the head's contributors to finish (fence + arrival counter, no
+// waiting) merges the partials into out = acc / l.
+#include <cuda_bf16.h>
+
 #include "hata_internal.cuh"
+#include "tma.cuh"
 
 namespace hata {
 namespace {
 
 constexpr int kWarps = kAttnThreads / 32;
-constexpr int kRowsPerHalf = 8;        // rows gathered per half-warp per round
 constexpr int kHalves = kWarps * 2;
-constexpr int kBytesPerThread = kChunk / kAttnThreads;  // 32 distances
+constexpr int kStageRows = 32;
+constexpr int kRing = 4;
+constexpr int kRowsPerHalf = kStageRows / kHalves;  // 4
 
 __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
 {
@@ -37,156 +40,217 @@ __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_
     return l < n_cap ? l : n_cap;
 }
 
-// 8 consecutive elements of a row (starting at element e0) as fp32.
 template <bool BF16>
-struct RowFrag;
+struct Rows {
+    static constexpr int kRowBytes = kD * (BF16 ? 2 : 4);
+    static constexpr int kPieces = kRowBytes / 16;                 // 16-byte pieces per row
+    static constexpr int kSlotBytes = 2 * kStageRows * kRowBytes;  // K and V
+};
 
-template <>
-struct RowFrag<true> {
-    uint4 v;
-    __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
-    __device__ __forceinline__ void load(const void *base, int64_t elem)
-    {
-        v = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(base) + elem));
-    }
-    __device__ __forceinline__ void to_f32(float (&f)[8]) const
-    {
+// 8 consecutive row elements (from shared memory) as fp32.
+template <bool BF16>
+__device__ __forceinline__ void frag8(const uint8_t *row, int l16, float (&f)[8])
+{
+    if (BF16) {
+        const uint4 v = reinterpret_cast<const uint4 *>(row)[l16];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             f[2 * i] = __uint_as_float(w[i] << 16);
             f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
+    } else {
+        const float4 x = reinterpret_cast<const float4 *>(row)[2 * l16];
+        const float4 y = reinterpret_cast<const float4 *>(row)[2 * l16 + 1];
+        f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+        f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
     }
-};
+}
 
-template <>
-struct RowFrag<false> {
-    float4 a, b;
-    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
-    __device__ __forceinline__ void load(const void *base, int64_t elem)
-    {
-        const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(base) + elem);
-        a = __ldg(p);
-        b = __ldg(p + 1);
-    }
-    __device__ __forceinline__ void to_f32(float (&f)[8]) const
-    {
-        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-    }
-};
-
-template <bool BF16>
-__global__ void __launch_bounds__(kAttnThreads) attend_kernel(AttendArgs a)
+// Flat row x -> index of the CTA whose range [k*T/P, (k+1)*T/P) holds it.
+__device__ __forceinline__ int64_t owner(int64_t x, int64_t T, int64_t P)
 {
-    const int c = blockIdx.x;
-    const size_t bh = blockIdx.y;
-    const int b = int(bh / a.H_q), hq = int(bh % a.H_q), h = hq / a.G;
-    const int64_t len = clamp_len(a.seq_len[b], a.max_seq_len, a.n_cap);
-    const int64_t nch = len > 0 ? ceil_div(len, kChunk) : 1;
-    if (c >= nch) return;
+    return ((x + 1) * P + T - 1) / T - 1;
+}
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    __shared__ int32_t idx_s[kChunk];
-    __shared__ int scan_s[kWarps + 1];
+struct Stage {
+    int bh;        // head (b * H_q + h_q)
+    int b, h;      // batch row and KV head of that head
+    int p0;        // first position in the head's index list
+    int n;         // rows of this stage (0: the placeholder row of an empty head)
+    bool last;     // last stage of this CTA in this head
+};
+
+// Walks one CTA's range in stages with incremental 32-bit cursors (no
+// division in the loop).  A head with k_eff == 0 still gets one placeholder
+// stage (n = 0) from the CTA that owns its first row, so that someone
+// writes its (zero) output.
+template <int kRows>
+struct Walker {
+    const AttendArgs *a;
+    int64_t remaining;   // rows of the CTA range not yet walked
+    int bh, b, hq, pos;  // cursor: head, its batch row / query head, position
+    int keff;            // min(topk, len(b))
+    int64_t len;
+
+    __device__ __forceinline__ void load_len()
+    {
+        len = clamp_len(__ldg(a->seq_len + b), a->max_seq_len, a->n_cap);
+        keff = int(int64_t(a->topk) < len ? int64_t(a->topk) : len);
+    }
+    __device__ __forceinline__ void init(const AttendArgs *args, int64_t beg, int64_t end)
+    {
+        a = args;
+        remaining = end - beg;
+        const int64_t h = beg / a->topk;  // once per CTA
+        bh = int(h);
+        pos = int(beg - h * a->topk);
+        b = bh / a->H_q;
+        hq = bh - b * a->H_q;
+        load_len();
+    }
+    __device__ __forceinline__ bool next(Stage &st)
+    {
+        while (remaining > 0) {
+            const int e = keff > 0 ? keff : 1;
+            if (pos >= e) {  // the rest of this head is empty: skip to the next head
+                remaining -= a->topk - pos;
+                pos = 0;
+                ++bh;
+                if (++hq == a->H_q) {
+                    hq = 0;
+                    ++b;
+                    if (remaining > 0) load_len();
+                }
+                continue;
+            }
+            const int seg = int(int64_t(e - pos) < remaining ? int64_t(e - pos) : remaining);
+            const int n = seg < kRows ? seg : kRows;
+            st.bh = bh;
+            st.b = b;
+            st.h = hq / a->G;
+            st.p0 = pos;
+            st.n = keff > 0 ? n : 0;
+            st.last = n == seg;
+            pos += n;
+            remaining -= n;
+            return true;
+        }
+        return false;
+    }
+};
+
+// fp32 K/V: CUDA-core path (16 lanes per row, shuffle-reduced dot products).
+template <bool BF16>
+__global__ void __launch_bounds__(kAttnThreads) attend_simt_kernel(AttendArgs a)
+{
+    using RW = Rows<BF16>;
+    constexpr int RB = RW::kRowBytes;
+    extern __shared__ __align__(128) uint8_t smem[];  // [kRing][K rows | V rows]
+    __shared__ int32_t rows_s[kRing][kStageRows];
     __shared__ float red_m[kHalves], red_l[kHalves];
     __shared__ __align__(16) float red_acc[kHalves][kD];
     __shared__ int s_last;
 
-    const PlanHead ph = a.plan_head[bh];
-    const PlanChunk pc = a.plan_chunk[bh * a.n_chunks + c];
-
-    // ---- 1. ordered compaction of this chunk's selected keys ----
-    const uint4 *dp = reinterpret_cast<const uint4 *>(a.dist + bh * a.dist_row +
-                                                      int64_t(c) * kChunk) + tid * 2;
-    const uint4 d0 = __ldg(dp), d1 = __ldg(dp + 1);
-    const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-    const uint32_t T4 = ph.T >= 0 ? uint32_t(ph.T) * 0x01010101u : 0u;
-    uint32_t lt[8], eq[8];
-    int n_lt = 0, n_eq = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        lt[k] = ph.T >= 0 ? __vcmpltu4(dw[k], T4) : 0u;
-        eq[k] = ph.T >= 0 ? __vcmpeq4(dw[k], T4) : 0u;
-        n_lt += __popc(lt[k]) >> 3;
-        n_eq += __popc(eq[k]) >> 3;
-    }
-    int tot;
-    const int eq_before = block_exclusive_scan<kAttnThreads>(n_eq, scan_s, &tot);
-    const int my_take = max(0, min(pc.take - eq_before, n_eq));
-    int total;
-    int wpos = block_exclusive_scan<kAttnThreads>(n_lt + my_take, scan_s, &total);
-    {
-        int eq_seen = 0;
-        const int32_t tok0 = int32_t(int64_t(c) * kChunk) + tid * kBytesPerThread;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const bool is_lt = (lt[k] >> (8 * e)) & 1u;
-                const bool is_eq = (eq[k] >> (8 * e)) & 1u;
-                const bool take = is_lt || (is_eq && eq_seen < my_take);
-                eq_seen += is_eq;
-                if (take) idx_s[wpos++] = tok0 + k * 4 + e;
-            }
-        }
-    }
-    __syncthreads();
-    if (a.sel_idx) {
-        int32_t *dst = a.sel_idx + bh * a.topk + pc.off;
-        const int lim = min(total, a.topk - pc.off);
-        for (int i = tid; i < lim; i += kAttnThreads) dst[i] = idx_s[i];
-    }
-
-    // ---- 3. gather + online softmax ----
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int half = lane >> 4, l16 = lane & 15, hw = warp * 2 + half;
-    float qv[8];
-    {
-        const float4 *qp = reinterpret_cast<const float4 *>(a.q + bh * kD + l16 * 8);
-        const float4 x = __ldg(qp), y = __ldg(qp + 1);
-        qv[0] = x.x; qv[1] = x.y; qv[2] = x.z; qv[3] = x.w;
-        qv[4] = y.x; qv[5] = y.y; qv[6] = y.z; qv[7] = y.w;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) qv[e] *= a.scale_log2;
-    }
-    const int64_t slab = (int64_t(b) * a.H_kv + h) * a.n_cap;  // row of token 0
-    float m = -INFINITY, l = 0.0f, acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    const int64_t T = int64_t(a.B) * a.H_q * a.topk, P = gridDim.x;
+    const int64_t beg = blockIdx.x * T / P, end = (blockIdx.x + 1) * T / P;
+    const uint8_t *Kg = static_cast<const uint8_t *>(a.K);
+    const uint8_t *Vg = static_cast<const uint8_t *>(a.V);
 
-    for (int base = 0; base < total; base += kHalves * kRowsPerHalf) {
-        RowFrag<BF16> kf[kRowsPerHalf], vf[kRowsPerHalf];
-        bool valid[kRowsPerHalf];
+    Walker<kStageRows> prod, cons;
+    prod.init(&a, beg, end);
+    cons.init(&a, beg, end);
+
+    // ---- producer: gather the rows of stage `st` into ring slot `slot` ----
+    // Each thread copies the same piece column p of rows i0, i0 + kRowStep, ...
+    constexpr int kRowStep = kAttnThreads / RW::kPieces;          // 8 (bf16) / 4 (fp32)
+    constexpr int kRowsPerThread = kStageRows / kRowStep;          // 4 / 8
+    auto issue = [&](const Stage &st, int slot) {
+        uint8_t *Ks = smem + size_t(slot) * RW::kSlotBytes;
+        uint8_t *Vs = Ks + kStageRows * RB;
+        const int64_t len = prod.len;  // the producer's cursor sits in this stage's head
+        const int64_t slab = (int64_t(st.b) * a.H_kv + st.h) * a.n_cap;
+        const int32_t *idx = a.idx + int64_t(st.bh) * a.topk + st.p0;
+        const int p = tid % RW::kPieces, i0 = tid / RW::kPieces;
+        int32_t rows[kRowsPerThread];
 #pragma unroll
-        for (int u = 0; u < kRowsPerHalf; ++u) {
-            const int ri = base + hw * kRowsPerHalf + u;
-            const int32_t row = ri < total ? idx_s[ri] : -1;
-            // distances past seq_len are 255 and never selected; the range
-            // check keeps even a corrupted distance row inside the cache
-            valid[u] = row >= 0 && row < len;
-            if (valid[u]) {
-                const int64_t e0 = (slab + row) * kD + l16 * 8;
-                kf[u].load(a.K, e0);
-                vf[u].load(a.V, e0);
-            } else {
-                kf[u].zero();  // weight 0 must meet a finite value
-                vf[u].zero();
-            }
+        for (int u = 0; u < kRowsPerThread; ++u) {  // all index loads first
+            const int i = i0 + u * kRowStep;
+            rows[u] = i < st.n ? __ldg(idx + i) : -1;
         }
-        float s[kRowsPerHalf];
+#pragma unroll
+        for (int u = 0; u < kRowsPerThread; ++u) {
+            const int i = i0 + u * kRowStep;
+            // the selection never yields an index outside [0, len); the check
+            // keeps a corrupted list from steering a copy outside the cache
+            const bool ok = rows[u] >= 0 && rows[u] < len;
+            if (ok) {
+                const int64_t off = (slab + rows[u]) * RB + p * 16;
+                cp_async16(Ks + i * RB + p * 16, Kg + off);
+                cp_async16(Vs + i * RB + p * 16, Vg + off);
+            }
+            if (p == 0) rows_s[slot][i] = ok ? rows[u] : -1;
+        }
+    };
+
+    Stage ps;
+    int n_issued = 0;
+    for (; n_issued < kRing - 1; ++n_issued) {
+        if (prod.next(ps)) issue(ps, n_issued);
+        cp_async_commit();
+    }
+
+    // q of the current head, scaled; online-softmax state
+    float qv[8], m = -INFINITY, l = 0.0f, acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qv[e] = acc[e] = 0.0f;
+    int64_t cur_bh = -1;
+    Stage cs;
+    for (int s = 0; cons.next(cs); ++s) {
+        // stage s has landed (the kRing-2 younger groups may still be in flight)
+        cp_async_wait<kRing - 2>();
+        __syncthreads();
+        if (prod.next(ps)) issue(ps, n_issued % kRing);
+        ++n_issued;
+        cp_async_commit();  // (possibly empty) group, keeps the accounting uniform
+
+        if (cs.bh != cur_bh) {
+            cur_bh = cs.bh;
+            const float4 *qp =
+                reinterpret_cast<const float4 *>(a.q + int64_t(cs.bh) * kD + l16 * 8);
+            const float4 x = __ldg(qp), y = __ldg(qp + 1);
+            qv[0] = x.x; qv[1] = x.y; qv[2] = x.z; qv[3] = x.w;
+            qv[4] = y.x; qv[5] = y.y; qv[6] = y.z; qv[7] = y.w;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qv[e] *= a.scale_log2;
+            m = -INFINITY;
+            l = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        }
+
+        const int slot = s % kRing;
+        const uint8_t *Ks = smem + size_t(slot) * RW::kSlotBytes;
+        const uint8_t *Vs = Ks + kStageRows * RB;
+        float sc[kRowsPerHalf];
         float mx = m;
 #pragma unroll
         for (int u = 0; u < kRowsPerHalf; ++u) {
-            float kx[8];
-            kf[u].to_f32(kx);
+            const int i = hw + u * kHalves;  // warp-uniform trip count: shuffles see all lanes
+            const bool valid = i < cs.n && rows_s[slot][i] >= 0;
             float p = 0.0f;
+            if (valid) {
+                float kx[8];
+                frag8<BF16>(Ks + i * RB, l16, kx);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p = fmaf(qv[e], kx[e], p);
+                for (int e = 0; e < 8; ++e) p = fmaf(qv[e], kx[e], p);
+            }
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-            s[u] = valid[u] ? p : -INFINITY;
-            mx = fmaxf(mx, s[u]);
+            sc[u] = valid ? p : -INFINITY;
+            mx = fmaxf(mx, sc[u]);
         }
         const float mref = mx == -INFINITY ? 0.0f : mx;
         const float alpha = exp2f(m - mref);
@@ -195,73 +259,458 @@ __global__ void __launch_bounds__(kAttnThreads) attend_kernel(AttendArgs a)
         for (int e = 0; e < 8; ++e) acc[e] *= alpha;
 #pragma unroll
         for (int u = 0; u < kRowsPerHalf; ++u) {
-            const float p = exp2f(s[u] - mref);
-            l += p;
-            float vx[8];
-            vf[u].to_f32(vx);
+            if (sc[u] != -INFINITY) {
+                const float p = exp2f(sc[u] - mref);
+                l += p;
+                float vx[8];
+                frag8<BF16>(Vs + (hw + u * kHalves) * RB, l16, vx);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(p, vx[e], acc[e]);
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(p, vx[e], acc[e]);
+            }
         }
         m = mx;
-    }
 
-    // ---- 4. merge half-warps, then chunks ----
-    if (l16 == 0) {
-        red_m[hw] = m;
-        red_l[hw] = l;
-    }
+        if (!cs.last) continue;
+        // ---- this CTA is done with head cs.bh: publish a partial ----
+        if (l16 == 0) {
+            red_m[hw] = m;
+            red_l[hw] = l;
+        }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red_acc[hw][l16 * 8 + e] = acc[e];
-    __syncthreads();
+        for (int e = 0; e < 8; ++e) red_acc[hw][l16 * 8 + e] = acc[e];
+        __syncthreads();
+        const int64_t h0 = int64_t(cs.bh) * a.topk;
+        const int ke = cons.keff;
+        const int64_t k_first = owner(h0, T, P);
+        const int64_t k_last = owner(h0 + (ke > 0 ? ke : 1) - 1, T, P);
+        const int slot_out = int(blockIdx.x - k_first);
+        const int n_contrib = int(k_last - k_first + 1);
+        {
+            float M = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kHalves; ++i) M = fmaxf(M, red_m[i]);
+            const float Mref = M == -INFINITY ? 0.0f : M;
+            float L = 0.0f, A = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kHalves; ++i) {
+                const float w = exp2f(red_m[i] - Mref);
+                L = fmaf(red_l[i], w, L);
+                A = fmaf(red_acc[i][tid], w, A);
+            }
+            float *pp = a.part + (int64_t(cs.bh) * a.n_split + slot_out) * kPartStride;
+            if (tid == 0) {
+                pp[0] = M;
+                pp[1] = L;
+            }
+            pp[4 + tid] = A;
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_last = atomicAdd(a.cnt_attn + cs.bh, 1u) == uint32_t(n_contrib - 1);
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            float M = -INFINITY, L = 0.0f, A = 0.0f;
+            const float *pp = a.part + int64_t(cs.bh) * a.n_split * kPartStride;
+            for (int c = 0; c < n_contrib; ++c, pp += kPartStride) {
+                const float mc = __ldcg(pp), lc = __ldcg(pp + 1), ac = __ldcg(pp + 4 + tid);
+                if (mc == -INFINITY) continue;
+                const float Mn = fmaxf(M, mc);
+                const float so = exp2f(M - Mn), sn = exp2f(mc - Mn);
+                L = L * so + lc * sn;
+                A = A * so + ac * sn;
+                M = Mn;
+            }
+            a.out[int64_t(cs.bh) * kD + tid] = L > 0.0f ? A / L : 0.0f;
+        }
+    }
+    cp_async_wait<0>();
+}
+
+// ------------------------------------------------------------------------
+// bf16 K/V: tensor-core path.
+//
+// Every warp is an independent stream-K worker: the flat row space is cut
+// into n_workers contiguous ranges (eight warps per CTA, one CTA per SM), so
+// a warp walks only its own rows and needs no block barrier.  Random
+// 256-byte row gathers on B200 see a loaded DRAM latency of several
+// microseconds; the copies are issued by many warps (one warp alone cannot
+// issue cp.async fast enough), each keeping a private ring of three 16-key
+// stages (K and V, 8 KB a stage) in flight two stages ahead of its
+// arithmetic, with 16-byte cp.async copies.  The CTA's slice of the flat
+// index list is loaded into shared memory up front, so no copy waits on an
+// index load.
+//
+// A warp computes S = q K^T and O += P V as mma.sync m16n8k16 bf16 tiles
+// with fp32 accumulation, fed by ldmatrix from an XOR-swizzled layout
+// (16-byte piece p of key row r sits at piece p ^ (r & 7), so the eight rows
+// one ldmatrix reads hit eight different bank groups).  The A operands are
+// the query (resp. the softmax weights) split into two bf16 rows,
+// hi = bf16(x) and lo = bf16(x - hi): rows 0 and 1 of the 16-row tile, whose
+// sum carries ~16 mantissa bits, so the tensor cores reproduce the fp32
+// result (the other 14 rows are zero).  The softmax rescale is lazy: the
+// reference maximum moves only when a score exceeds it by more than 2^8
+// (exact: weights stay <= 2^8), which skips rescaling the 64 accumulator
+// registers almost always.  When a warp leaves a head it publishes a partial
+// (m, l, acc[128]); the head's last contributor merges them.
+namespace tc {
+
+constexpr int kSub = 16;                           // keys per stage
+constexpr int kRingW = 3;                          // stages per warp ring
+constexpr int kTcWarps = 8;
+constexpr int kThreads = 32 * kTcWarps;
+constexpr int kRowB = kD * 2;                      // bf16 row bytes
+constexpr int kStageBytes = 2 * kSub * kRowB;      // K + V
+constexpr int kIdxCap = 4096;                      // indices of the CTA slice kept in smem
+constexpr float kLazy = 8.0f;                      // rescale threshold, log2 units
+constexpr size_t kRingBytes = size_t(kTcWarps) * kRingW * kStageBytes;
+constexpr size_t kSmem = kRingBytes + sizeof(int32_t) * kIdxCap;
+
+__device__ __forceinline__ uint32_t swz(int row, int piece)
+{
+    return uint32_t(row * kRowB + ((piece ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// d += A(16x16, rows 8..15 zero) * B(16x8); a0/a2: row g, k and k+8.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// x as the bf16 row `part` of a hi/lo pair: part 0 -> bf16(x), 1 -> bf16(x - bf16(x)).
+__device__ __forceinline__ float split(float x, int part)
+{
+    const float hi = __bfloat162float(__float2bfloat16_rn(x));
+    return part == 0 ? hi : x - hi;
+}
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes));
+}
+
+// 2^x on the special-function unit (relative error ~2^-22; -inf -> +0).
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Per-lane ldmatrix offsets inside a stage (constant for a warp's life):
+// koff[kq]: key rows (lane & 7), 16-byte pieces kq*4 + (lane >> 3), for S;
+// voff[j2]: key rows (mi & 1)*8 + (lane & 7), pieces 2*j2 + (mi >> 1), for P V.
+struct LaneOffsets {
+    uint32_t koff[4], voff[8];
+    __device__ __forceinline__ explicit LaneOffsets(int lane)
     {
-        float M = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < kHalves; ++i) M = fmaxf(M, red_m[i]);
-        const float Mref = M == -INFINITY ? 0.0f : M;
-        float L = 0.0f, A = 0.0f;
+        for (int kq = 0; kq < 4; ++kq) koff[kq] = swz(lane & 7, kq * 4 + (lane >> 3));
+        const int mi = lane >> 3;
 #pragma unroll
-        for (int i = 0; i < kHalves; ++i) {
-            const float w = exp2f(red_m[i] - Mref);
-            L = fmaf(red_l[i], w, L);
-            A = fmaf(red_acc[i][tid], w, A);
+        for (int j2 = 0; j2 < 8; ++j2) voff[j2] = swz((mi & 1) * 8 + (lane & 7), 2 * j2 + (mi >> 1));
+    }
+};
+
+// One 16-key stage of one warp: S = q K^T, online softmax, O += P V.
+__device__ __forceinline__ void attend_stage(int n, uint32_t Ks, const int32_t *rows,
+                                             const uint32_t (&qa)[8][2], const LaneOffsets &lo,
+                                             float (&O)[16][4], float &m_ref, float &l_part,
+                                             int lane)
+{
+    const uint32_t Vs = Ks + kSub * kRowB;
+    const int q4 = lane & 3, part = (lane >> 2) & 1;
+    // ---- S = q K^T: two n-tiles of 8 keys; even / odd k-tiles accumulate
+    //      separately so each dependent mma chain is four deep ----
+    float S[2][2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) S[nt][h][0] = S[nt][h][1] = S[nt][h][2] = S[nt][h][3] = 0.0f;
+#pragma unroll
+    for (int kq = 0; kq < 4; ++kq) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t b0, b1, b2, b3;
+            // rows nt*8 + (lane & 7): the +8 row offset leaves the swizzle unchanged
+            ldsm_x4(Ks + nt * 8 * kRowB + lo.koff[kq], b0, b1, b2, b3);
+            mma16816(S[nt][0], qa[2 * kq][0], qa[2 * kq][1], b0, b1);
+            mma16816(S[nt][1], qa[2 * kq + 1][0], qa[2 * kq + 1][1], b2, b3);
         }
-        float *pp = a.part + (bh * a.n_chunks + c) * kPartStride;
-        if (tid == 0) {
-            pp[0] = M;
-            pp[1] = L;
+    }
+    // ---- scores of keys (nt*8 + 2*q4 + e): even + odd k-tiles, hi row + lo row ----
+    float sc[4] = {S[0][0][0] + S[0][1][0], S[0][0][1] + S[0][1][1], S[1][0][0] + S[1][1][0],
+                   S[1][0][1] + S[1][1][1]};
+    bool valid[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        sc[e] += __shfl_xor_sync(0xffffffffu, sc[e], 4);
+        const int key = (e >> 1) * 8 + 2 * q4 + (e & 1);
+        valid[e] = lane < 8 && key < n && rows[key] >= 0;
+        if (!valid[e]) sc[e] = -INFINITY;
+    }
+    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = __shfl_sync(0xffffffffu, mx, 0);  // warp-uniform
+    if (mx == -INFINITY) return;
+    if (mx > m_ref + kLazy) {
+        const float alpha = fast_exp2(m_ref - mx);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            O[j][0] *= alpha; O[j][1] *= alpha; O[j][2] *= alpha; O[j][3] *= alpha;
         }
-        pp[4 + tid] = A;
+        l_part *= alpha;
+        m_ref = mx;
+    }
+    float pv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float pe = valid[e] ? fast_exp2(sc[e] - m_ref) : 0.0f;
+        l_part += pe;
+        pv[e] = split(pe, part);
+    }
+    const uint32_t a0 = lane < 8 ? pack2(pv[0], pv[1]) : 0u;
+    const uint32_t a2 = lane < 8 ? pack2(pv[2], pv[3]) : 0u;
+    // ---- O += P V: 16 n-tiles of 8 dims, one k-tile of 16 keys ----
+#pragma unroll
+    for (int j2 = 0; j2 < 8; ++j2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(Vs + lo.voff[j2], b0, b1, b2, b3);
+        mma16816(O[2 * j2], a0, a2, b0, b1);
+        mma16816(O[2 * j2 + 1], a0, a2, b2, b3);
+    }
+}
+
+// A warp is done with head cs.bh: publish its partial (m, l, acc[128]); the
+// last of the head's contributors (fence + arrival counter, no waiting)
+// merges all partials into out = acc / l.
+__device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, int keff,
+                                        int64_t wid, int64_t NW, int64_t T,
+                                        const float (&O)[16][4], float m_ref, float l_part,
+                                        int lane)
+{
+    const int q4 = lane & 3;
+    const int64_t h0 = int64_t(cs.bh) * a.topk;
+    const int64_t k_first = owner(h0, T, NW);
+    const int64_t k_last = owner(h0 + (keff > 0 ? keff : 1) - 1, T, NW);
+    const int n_contrib = int(k_last - k_first + 1);
+    float *pp = a.part + (int64_t(cs.bh) * a.n_split + (wid - k_first)) * kPartStride;
+    float lw = lane < 4 ? l_part : 0.0f;  // lanes 4-7 repeat lanes 0-3's weights
+    lw += __shfl_xor_sync(0xffffffffu, lw, 1);
+    lw += __shfl_xor_sync(0xffffffffu, lw, 2);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float o = O[j][e] + __shfl_xor_sync(0xffffffffu, O[j][e], 4);  // hi + lo rows
+            if (lane < 4) pp[4 + 8 * j + 2 * q4 + e] = o;
+        }
+    }
+    if (lane == 0) {
+        pp[0] = m_ref;
+        pp[1] = lw;
     }
     __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(a.cnt_attn + bh, 1u) == uint32_t(nch - 1);
-    __syncthreads();
-    if (!s_last) return;
+    __syncwarp();
+    unsigned last = 0;
+    if (lane == 0) last = atomicAdd(a.cnt_attn + cs.bh, 1u) == uint32_t(n_contrib - 1);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
     __threadfence();
-
-    float M = -INFINITY, L = 0.0f, A = 0.0f;
-    const float *pp = a.part + bh * a.n_chunks * kPartStride;
-    for (int64_t cc = 0; cc < nch; ++cc, pp += kPartStride) {
-        const float mc = __ldcg(pp), lc = __ldcg(pp + 1), ac = __ldcg(pp + 4 + tid);
+    float M = -INFINITY, L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const float *pc = a.part + int64_t(cs.bh) * a.n_split * kPartStride;
+    for (int c = 0; c < n_contrib; ++c, pc += kPartStride) {
+        const float mc = __ldcg(pc), lc = __ldcg(pc + 1);
         if (mc == -INFINITY) continue;
         const float Mn = fmaxf(M, mc);
-        const float so = exp2f(M - Mn), sn = exp2f(mc - Mn);
+        const float so = fast_exp2(M - Mn), sn = fast_exp2(mc - Mn);
         L = L * so + lc * sn;
-        A = A * so + ac * sn;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) A[i] = A[i] * so + __ldcg(pc + 4 + lane + 32 * i) * sn;
         M = Mn;
     }
-    a.out[bh * kD + tid] = L > 0.0f ? A / L : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        a.out[int64_t(cs.bh) * kD + lane + 32 * i] = L > 0.0f ? A[i] / L : 0.0f;
+}
+
+}  // namespace tc
+
+__global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a)
+{
+    using namespace tc;
+    extern __shared__ __align__(128) uint8_t smem[];  // [warp][kRingW][K | V], then indices
+    __shared__ int32_t rows_s[kTcWarps][kRingW][kSub];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t T = int64_t(a.B) * a.H_q * a.topk;
+    const int64_t NW = a.n_workers;  // warps that own rows (<= T, so none is empty)
+    const int64_t wid = int64_t(blockIdx.x) * kTcWarps + warp;
+    const int64_t cta_beg = int64_t(blockIdx.x) * kTcWarps * T / NW;
+    int64_t cta_end = (int64_t(blockIdx.x) + 1) * kTcWarps;
+    cta_end = (cta_end < NW ? cta_end : NW) * T / NW;
+    const uint8_t *Kg = static_cast<const uint8_t *>(a.K);
+    const uint8_t *Vg = static_cast<const uint8_t *>(a.V);
+    const uint32_t wring = smem_addr(smem) + uint32_t(warp * kRingW * kStageBytes);
+    int32_t *idx_s = reinterpret_cast<int32_t *>(smem + kRingBytes);
+
+    // the CTA's slice of the index list (the first kIdxCap of it), coalesced
+    if (cta_beg < cta_end) {
+        const int64_t n_s = cta_end - cta_beg < kIdxCap ? cta_end - cta_beg : kIdxCap;
+        for (int64_t i = tid; i < n_s; i += kThreads) idx_s[i] = __ldg(a.idx + cta_beg + i);
+    }
+    __syncthreads();
+    if (wid >= NW) return;
+    const int64_t beg = wid * T / NW, end = (wid + 1) * T / NW;
+    auto index_of = [&](int64_t x) {  // flat row -> key index
+        return x - cta_beg < kIdxCap ? idx_s[x - cta_beg] : __ldg(a.idx + x);
+    };
+
+    Walker<kSub> prod, cons;
+    prod.init(&a, beg, end);
+    cons.init(&a, beg, end);
+    int64_t prod_x = beg;  // flat row of the producer walker's position
+    int n_issued = 0;
+    const int p = lane & 15, rb = lane >> 4;  // lane = piece p of rows rb, rb+2, ...
+    uint32_t doff[kSub / 2];                   // this lane's swizzled destinations
+#pragma unroll
+    for (int u = 0; u < kSub / 2; ++u) doff[u] = swz(rb + 2 * u, p);
+
+    // gather this warp's next stage into its ring (always commits one group)
+    auto issue_next = [&]() {
+        Stage st;
+        const int64_t before = prod.remaining;
+        if (prod.next(st)) {
+            const int64_t used = before - prod.remaining;  // skipped + this stage's rows
+            const int64_t x0 = prod_x + used - st.n;
+            prod_x += used;
+            const int slot = n_issued++ % kRingW;
+            const uint32_t Ks = wring + uint32_t(slot * kStageBytes), Vs = Ks + kSub * kRowB;
+            const int64_t slab = (int64_t(st.b) * a.H_kv + st.h) * a.n_cap;
+#pragma unroll
+            for (int u = 0; u < kSub / 2; ++u) {
+                const int r = rb + 2 * u;
+                const int32_t row = r < st.n ? index_of(x0 + r) : -1;
+                // the selection never yields an index outside [0, len); the
+                // check keeps a corrupted list from steering a copy outside
+                // the cache.  Rows without a key are zero-filled.
+                const bool ok = row >= 0 && row < prod.len;
+                const int64_t off = ok ? (slab + row) * kRowB + p * 16 : 0;
+                cp_async16_zfill(Ks + doff[u], Kg + off, ok ? 16u : 0u);
+                cp_async16_zfill(Vs + doff[u], Vg + off, ok ? 16u : 0u);
+                if (p == 0) rows_s[warp][slot][r] = ok ? row : -1;
+            }
+        }
+        cp_async_commit();
+    };
+    for (int i = 0; i < kRingW - 1; ++i) issue_next();
+
+    const int g4 = lane >> 2, q4 = lane & 3;   // mma fragment coordinates
+    const int part = g4 & 1;                    // lanes 0-3: hi row, 4-7: lo row
+    const LaneOffsets lo(lane);
+    uint32_t qa[8][2];
+    float O[16][4];
+    float m_ref = -INFINITY, l_part = 0.0f;
+    int cur_bh = -1;
+    Stage cs;
+    for (int s = 0; cons.next(cs); ++s) {
+        if (cs.bh != cur_bh) {  // a new head: its query as hi/lo bf16 rows, fresh state
+            cur_bh = cs.bh;
+            const float *q = a.q + int64_t(cs.bh) * kD;
+#pragma unroll
+            for (int kt = 0; kt < 8; ++kt) {
+                const int d0 = 16 * kt + 2 * q4;
+                if (lane < 8) {
+                    const float2 x = __ldg(reinterpret_cast<const float2 *>(q + d0));
+                    const float2 y = __ldg(reinterpret_cast<const float2 *>(q + d0 + 8));
+                    qa[kt][0] = pack2(split(x.x * a.scale_log2, part), split(x.y * a.scale_log2, part));
+                    qa[kt][1] = pack2(split(y.x * a.scale_log2, part), split(y.y * a.scale_log2, part));
+                } else {
+                    qa[kt][0] = qa[kt][1] = 0u;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
+            m_ref = -INFINITY;
+            l_part = 0.0f;
+        }
+
+        cp_async_wait<kRingW - 2>();
+        __syncwarp();
+        const int slot = s % kRingW;
+        issue_next();
+        attend_stage(cs.n, wring + uint32_t(slot * kStageBytes), rows_s[warp][slot], qa, lo, O,
+                     m_ref, l_part, lane);
+
+        if (cs.last) publish(a, cs, cons.keff, wid, NW, T, O, m_ref, l_part, lane);
+    }
+    cp_async_wait<0>();
+}
+
+template <typename Kernel>
+cudaError_t occupancy_grid(Kernel kernel, int threads, size_t smem, int64_t *grid)
+{
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kernel), smem)) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+    *grid = int64_t(per_sm > 0 ? per_sm : 1) * sms;
+    return e;
 }
 
 }  // namespace
 
-cudaError_t launch_attend(const AttendArgs &a, bool bf16, cudaStream_t s)
+cudaError_t launch_attend(const AttendArgs &args, bool bf16, cudaStream_t s)
 {
-    const dim3 grid(unsigned(a.n_chunks), unsigned(a.B * a.H_q));
-    if (bf16)
-        attend_kernel<true><<<grid, kAttnThreads, 0, s>>>(a);
-    else
-        attend_kernel<false><<<grid, kAttnThreads, 0, s>>>(a);
+    AttendArgs a = args;
+    const int64_t T = int64_t(a.B) * a.H_q * a.topk;
+    int64_t P = 0;
+    if (bf16) {
+        if (cudaError_t e = occupancy_grid(attend_tc_kernel, tc::kThreads, tc::kSmem, &P)) return e;
+        int64_t NW = P * tc::kTcWarps;
+        if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
+        if (NW > T) NW = T;
+        a.n_workers = NW;
+        attend_tc_kernel<<<unsigned(ceil_div(NW, tc::kTcWarps)), tc::kThreads, tc::kSmem, s>>>(a);
+        return cudaGetLastError();
+    }
+    constexpr size_t kSmemF32 = size_t(kRing) * Rows<false>::kSlotBytes;
+    if (cudaError_t e = occupancy_grid(attend_simt_kernel<false>, kAttnThreads, kSmemF32, &P))
+        return e;
+    if (P > kAttnMaxWorkers) P = kAttnMaxWorkers;
+    if (P > T) P = T;
+    a.n_workers = P;
+    attend_simt_kernel<false><<<unsigned(P), kAttnThreads, kSmemF32, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@
 // optionally its K/V rows) and clears the per-step counters the scoring
 // kernel accumulates into.
 #include "hata_internal.cuh"
+#include "tma.cuh"
 
 namespace hata {
 namespace {
@@ -50,19 +51,6 @@ __device__ __forceinline__ void load_w_column(const float *__restrict__ Wh, int 
 {
 #pragma unroll
     for (int i = 0; i < kD; ++i) w[i] = __ldg(Wh + i * kRbit + j);
-}
-
-// One head's W_H [kD][kRbit] into shared memory (all loads in flight at once).
-__device__ __forceinline__ void stage_w(const float *__restrict__ Wh, float *__restrict__ ws)
-{
-    constexpr int kVec = kD * kRbit / 4;
-    const float4 *src = reinterpret_cast<const float4 *>(Wh);
-    float4 *dst = reinterpret_cast<float4 *>(ws);
-    float4 v[kVec / kD];
-#pragma unroll
-    for (int m = 0; m < kVec / kD; ++m) v[m] = __ldg(src + m * kD + threadIdx.x);
-#pragma unroll
-    for (int m = 0; m < kVec / kD; ++m) dst[m * kD + threadIdx.x] = v[m];
 }
 
 // xs: [kD][R] floats (row r of the group in column r); ws: W_H in shared
@@ -164,23 +152,24 @@ __global__ void __launch_bounds__(kD) prep_kernel(PrepArgs a)
     const int rows = nq + nk;
     const int r0 = blockIdx.x * R;
 
-    if (blockIdx.x == 0) {
-        if (a.cnt_score)
-            for (int i = j; i < a.B * a.zgroups; i += kD) {
-                const int b = i / a.zgroups, z = i % a.zgroups;
-                a.cnt_score[(size_t(b) * a.H_kv + h) * a.zgroups + z] = 0u;
-            }
-        if (a.ws_header && h == 0 && j == 0) {
-            a.ws_header[0] = kWsMagic;
-            a.ws_header[1] = uint32_t(a.B);
-        }
+    if (a.ws_header && blockIdx.x == 0 && h == 0 && j == 0) {
+        a.ws_header[0] = kWsMagic;
+        a.ws_header[1] = uint32_t(a.B);
     }
     if (r0 >= rows) return;
 
-    extern __shared__ __align__(16) float smem[];
-    float *ws = smem;                 // [kD][kRbit]
-    float *xs = smem + kD * kRbit;    // [kD][R]
-    stage_w(a.W + size_t(h) * kD * kRbit, ws);
+    extern __shared__ __align__(128) float smem[];
+    float *ws = smem;                 // [kD][kRbit]: this head's W_H
+    float *xs = smem + kD * kRbit;    // [kD][R]: the rows, one per column
+    __shared__ uint64_t bar;
+    if (j == 0) {
+        // the whole 64 KB W_H in one bulk copy, overlapping the row staging
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        constexpr uint32_t kWBytes = sizeof(float) * kD * kRbit;
+        mbar_arrive_expect_tx(&bar, kWBytes);
+        bulk_g2s(ws, a.W + size_t(h) * kD * kRbit, kWBytes, &bar);
+    }
 
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -206,7 +195,16 @@ __global__ void __launch_bounds__(kD) prep_kernel(PrepArgs a)
         }
         xs[j * R + r] = x;
     }
-    __syncthreads();
+    const bool landed = mbar_wait(&bar, 0);
+    if (__syncthreads_or(!landed)) {
+        if (j == 0) {
+            if (a.flags)
+                for (int b = 0; b < a.B; ++b) atomicOr(a.flags + b, HATA_FLAG_TIMEOUT);
+            if (a.err_word) atomicOr(a.err_word, HATA_FLAG_TIMEOUT);
+            (void)mbar_wait(&bar, 0);
+        }
+        return;
+    }
     uint32_t words[R];
     hash_group_smem<R>(xs, ws, words);
 
@@ -254,15 +252,9 @@ cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const f
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s)
 {
     constexpr size_t kSmem = sizeof(float) * (kD * kRbit + kD * kPrepRows);
-    static const cudaError_t attr_err = [] {
-        cudaError_t e = cudaFuncSetAttribute(prep_kernel<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(prep_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
-        return e;
-    }();
-    if (attr_err != cudaSuccess) return attr_err;
+    const void *fn = a.kv_bf16 ? reinterpret_cast<const void *>(prep_kernel<true>)
+                               : reinterpret_cast<const void *>(prep_kernel<false>);
+    if (cudaError_t e = ensure_smem_attr(fn, kSmem)) return e;
     const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRows)), unsigned(a.H_kv));
     if (a.kv_bf16)
         prep_kernel<true><<<grid, kD, kSmem, s>>>(a);

@@ -68,6 +68,7 @@ typedef enum hata_dtype {
 /* Device-side check flags (OR-ed into the error word). */
 #define HATA_FLAG_SEQ_LEN_RANGE 1u  /* seq_len[b] < 0, > max_seq_len or > n_cap: clamped */
 #define HATA_FLAG_POS_RANGE     2u  /* an append position outside [0, n_cap): skipped  */
+#define HATA_FLAG_TIMEOUT       4u  /* a bounded wait on an asynchronous copy gave up  */
 
 /* ABI revision; bumps whenever a signature below changes. */
 int hata_abi_version(void);
@@ -127,7 +128,7 @@ int64_t hata_dist_row_bytes(int64_t max_seq_len);
  *      accumulation, exact softmax over S only).  seq_len[b] == 0 gives 0.
  * Arguments:
  *   q         [B][H_q][d] fp32
- *   W_H       [H_kv][d][r] fp32
+ *   W_H       [H_kv][d][r] fp32, 16-byte aligned
  *   codes     [B][H_kv][n_cap][r/32]; written only by the optional append
  *   K, V      [B][H_kv][n_cap][d] kv_dtype; written only when v_new is given
  *   seq_len   [B] int32, device: keys 0 .. seq_len[b]-1 take part
@@ -144,8 +145,9 @@ int64_t hata_dist_row_bytes(int64_t max_seq_len);
  *             Hamming distances (0..128); positions seq_len[b] ..
  *             hata_dist_row_bytes(max_seq_len)-1 hold 255;
  *             dist_row_bytes >= hata_dist_row_bytes(max_seq_len), multiple of 16
- *   events    optional array of 4 cudaEvent_t recorded on `stream` before the
- *             first kernel and after each of the three kernels (profiling)
+ *   events    optional array of 5 cudaEvent_t recorded on `stream` before the
+ *             first kernel and after each of the four kernels (prep, score,
+ *             select, attend) -- a profiling hook
  */
 hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
                                void *V, hata_dtype_t kv_dtype, int64_t n_cap,
