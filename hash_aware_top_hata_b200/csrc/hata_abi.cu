@@ -71,6 +71,8 @@ struct Events {
 
 namespace hata {
 
+hata_status_t report_error(hata_status_t st, const char *msg) { return fail(st, "%s", msg); }
+
 cudaError_t ensure_smem_attr(const void *func, size_t bytes)
 {
     static std::mutex mu;

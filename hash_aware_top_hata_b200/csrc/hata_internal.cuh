@@ -170,6 +170,9 @@ inline bool dense_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int64_t 
     return true;
 }
 
+// Records msg as hata_last_error() of this thread and returns st.
+hata_status_t report_error(hata_status_t st, const char *msg);
+
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
 cudaError_t ensure_smem_attr(const void *func, size_t bytes);
 

@@ -27,6 +27,8 @@ HATA_DT_BF16 = 0
 HATA_DT_F32 = 1
 HATA_FLAG_SEQ_LEN_RANGE = 1
 HATA_FLAG_POS_RANGE = 2
+HATA_FLAG_TIMEOUT = 4
+HATA_NOALLOC_WORKSPACE_BYTES = 64 << 20
 D = 128
 RBIT = 128
 
@@ -50,6 +52,8 @@ _SIGS = {
     "hata_dist_row_bytes": ([I64], I64),
     "hata_decode_step": ([P, P, P, P, P, I, I64, P, I64, P, P, I, I, I, I, I, I, F, P, U64, P,
                           P, P, P, I64, P, P], I),
+    "hata_decode_step_noalloc": ([P, P, P, P, P, I, I64, P, I64, P, P, I, I, I, I, I, I, F, P,
+                                  P, P, P, I64, P, P], I),
     "hata_workspace_check": ([P, U64, P, P], I),
     "hata_dense_workspace_size": ([I, I, I, I64], U64),
     "hata_dense_decode": ([P, P, P, I, I64, P, I64, I, I, I, I, F, P, U64, P, P], I),
@@ -210,6 +214,49 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
         max_seq_len, _ptr(k_new), _ptr(v_new), B, H_q, H_kv, d, W_H.shape[2], topk,
         float(scale), _ptr(workspace), workspace.numel(), _ptr(out), _ptr(sel_idx),
         _ptr(q_codes), _ptr(dist), drow, ev, _stream(stream)), "hata_decode_step")
+
+
+def hata_decode_step_noalloc(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor,
+                             K: torch.Tensor, V: torch.Tensor, seq_len: torch.Tensor,
+                             max_seq_len: int, topk: int, scale: float, out: torch.Tensor,
+                             k_new: torch.Tensor | None = None, v_new: torch.Tensor | None = None,
+                             sel_idx: torch.Tensor | None = None,
+                             q_codes: torch.Tensor | None = None,
+                             dist: torch.Tensor | None = None, events=None, stream=None) -> None:
+    """hata_decode_step with the library's fixed device scratch instead of a
+    caller workspace, for callers that cannot allocate device memory (see
+    include/hata.h).  Calls on one device share that scratch: keep them
+    ordered on one stream."""
+    _need(q, "q", torch.float32, 3)
+    _need(W_H, "W_H", torch.float32, 3)
+    _need(codes, "codes", torch.int32, 4)
+    _need(K, "K", ndim=4)
+    _need(V, "V", ndim=4)
+    _need(seq_len, "seq_len", torch.int32, 1)
+    _need(out, "out", torch.float32, 3)
+    for t, name in ((k_new, "k_new"), (v_new, "v_new")):
+        if t is not None:
+            _need(t, name, K.dtype, 3)
+    if sel_idx is not None:
+        _need(sel_idx, "sel_idx", torch.int32, 3)
+    if q_codes is not None:
+        _need(q_codes, "q_codes", torch.int32, 3)
+    drow = 0
+    if dist is not None:
+        _need(dist, "dist", torch.uint8, 3)
+        drow = dist.shape[2]
+    B, H_q, d = q.shape
+    H_kv, n_cap = K.shape[1], K.shape[2]
+    ev = None
+    if events is not None:
+        if len(events) != 5:
+            raise ValueError("events: give 5 torch.cuda.Event (recorded around the 4 kernels)")
+        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+    _check(lib().hata_decode_step_noalloc(
+        _ptr(q), _ptr(W_H), _ptr(codes), _ptr(K), _ptr(V), _kv_code(K), n_cap, _ptr(seq_len),
+        max_seq_len, _ptr(k_new), _ptr(v_new), B, H_q, H_kv, d, W_H.shape[2], topk,
+        float(scale), _ptr(out), _ptr(sel_idx), _ptr(q_codes), _ptr(dist), drow, ev,
+        _stream(stream)), "hata_decode_step_noalloc")
 
 
 def hata_workspace_check(workspace: torch.Tensor, stream=None) -> int:

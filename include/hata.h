@@ -158,6 +158,40 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
                                int64_t dist_row_bytes, void *const *events, void *stream);
 
 /* ------------------------------------------------------------------------
+ * hata_decode_step_noalloc -- hata_decode_step for callers that cannot
+ * allocate device memory (no counterpart in the HATA paper: this is a
+ * deployment convenience).  Some callers may not call cudaMalloc -- a plugin
+ * inside a serving engine that hands all device memory to its own pool, or
+ * code on a latency-critical path where cudaMalloc's implicit device
+ * synchronisation is not allowed.  They still pass every input and output;
+ * the decode scratch comes from a fixed array of
+ * HATA_NOALLOC_WORKSPACE_BYTES in the library's device image, which every
+ * GPU that loads the library holds until the process exits.
+ *   - Arguments and results are those of hata_decode_step without
+ *     workspace / workspace_bytes.
+ *   - Sizes whose scratch (hata_decode_workspace_size) exceeds the fixed
+ *     buffer are rejected with HATA_ERR_INVALID_ARG before anything runs.
+ *   - The first call on each device looks the buffer's device address up
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Nothing in the buffer needs to start at zero: every step rebuilds the
+ *     counters and histograms it uses.  All calls on a device share the one
+ *     buffer, so calls that may overlap on the GPU (different streams
+ *     without ordering between them) race: order them on one stream.
+ *   - hata_workspace_check cannot see this buffer; device-side flags of
+ *     this entry point are not reported.
+ * The call allocates nothing (no cudaMalloc / cudaFree / allocating
+ * library routine). */
+#define HATA_NOALLOC_WORKSPACE_BYTES (64u << 20)
+hata_status_t hata_decode_step_noalloc(const float *q, const float *W_H, uint32_t *codes,
+                                       void *K, void *V, hata_dtype_t kv_dtype, int64_t n_cap,
+                                       const int32_t *seq_len, int64_t max_seq_len,
+                                       const void *k_new, const void *v_new, int B, int H_q,
+                                       int H_kv, int d, int r, int topk, float scale, float *out,
+                                       int32_t *sel_idx, uint32_t *q_codes, uint8_t *dist,
+                                       int64_t dist_row_bytes, void *const *events, void *stream);
+
+/* ------------------------------------------------------------------------
  * hata_workspace_check -- synchronises `stream`, reads and clears the
  * device-side check flags of a decode workspace.  Returns HATA_OK if none
  * fired, HATA_ERR_DEVICE_CHECK otherwise (flags, if non-NULL, receives them). */
