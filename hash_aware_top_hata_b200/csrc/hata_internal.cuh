@@ -28,7 +28,7 @@ __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kAttnMaxWorkers = 4096;   // upper bound of the attention stream-K workers
-constexpr int kSelSegChunks = 8;        // scoring chunks walked by one selection CTA
+constexpr int kSelSegChunks = 2;        // scoring chunks walked by one selection CTA
 
 // Most attention workers that can share one head: each of the P <= T
 // workers owns at least floor(T / P) >= r_min rows of the flat row space.

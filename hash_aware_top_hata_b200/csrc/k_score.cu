@@ -143,6 +143,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(ScoreArgs a)
         const int v = sub_valid(r, s);
 
         const bool landed = mbar_wait(&S.full[j % kRing], uint32_t((j / kRing) & 1));
+        // the distance tile of sub-block j was last stored by bulk group j-2:
+        // let it finish reading (it was issued a whole sub-block ago) before
+        // the barrier that releases the tile writes
+        if (tid == 0) bulk_wait_read<1>();
         if (__syncthreads_or(!landed)) {
             // a copy never completed: flag it and stop (the wait was bounded)
             if (tid == 0) atomicOr(a.flags + r.b, HATA_FLAG_TIMEOUT);
@@ -165,7 +169,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(ScoreArgs a)
             }
         }
         fence_async_shared();          // tile writes -> visible to the bulk store
-        if (tid == 0) bulk_wait_read<0>();  // the other tile's store has read it
         __syncthreads();
         if (tid == 0) {
             const int64_t off = int64_t(r.c) * kChunk + int64_t(s) * kSub;

@@ -26,10 +26,11 @@
 namespace hata {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
-constexpr int kPerThread = kChunk / kThreads;  // 16 distances
-static_assert(kPerThread == 16, "one 16-byte load per thread per chunk");
+constexpr int kPerThread = kChunk / kThreads;  // 32 distances: two 16-byte loads
+static_assert(kPerThread == 32, "two 16-byte loads per thread per chunk");
+static_assert(kSelSegChunks == 2, "the distances of a segment are loaded up front");
 
 __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
 {
@@ -75,9 +76,16 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a)
         for (int i = k_eff + tid; i < a.topk; i += kThreads) idx[i] = -1;
     if (k_eff <= 0) return;
 
-    // first chunk's distances: in flight while T and the offsets are found
+    // the segment's distances: in flight while T and the offsets are found
     const uint8_t *drow = a.dist + bh * a.dist_row;
-    uint4 dv = __ldg(reinterpret_cast<const uint4 *>(drow + c0 * kChunk) + tid);
+    uint4 dv[kSelSegChunks][2];
+#pragma unroll
+    for (int k = 0; k < kSelSegChunks; ++k) {
+        const uint4 *dp = reinterpret_cast<const uint4 *>(drow + (c0 + k) * kChunk) + 2 * tid;
+        const bool in = c0 + k < c1;
+        dv[k][0] = in ? __ldg(dp) : make_uint4(0, 0, 0, 0);
+        dv[k][1] = in ? __ldg(dp + 1) : make_uint4(0, 0, 0, 0);
+    }
 
     // ---- T from the head's total histogram ----
     if (warp == 0) {
@@ -134,19 +142,21 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a)
 
     // ---- ordered compaction, chunk by chunk ----
     const uint32_t T4 = uint32_t(T) * 0x01010101u;
-    for (int64_t c = c0; c < c1; ++c) {
-        const uint4 cur = dv;
-        if (c + 1 < c1) dv = __ldg(reinterpret_cast<const uint4 *>(drow + (c + 1) * kChunk) + tid);
-        const uint32_t dw[4] = {cur.x, cur.y, cur.z, cur.w};
-        // byte masks (0xff / 0x00) -> one bit per distance: byte e of word k
-        // becomes bit 4k + e (the multiply gathers bits 7, 15, 23, 31 into 28..31)
+#pragma unroll
+    for (int k = 0; k < kSelSegChunks; ++k) {
+        const int64_t c = c0 + k;
+        if (c >= c1) break;
+        const uint32_t dw[8] = {dv[k][0].x, dv[k][0].y, dv[k][0].z, dv[k][0].w,
+                                dv[k][1].x, dv[k][1].y, dv[k][1].z, dv[k][1].w};
+        // byte masks (0xff / 0x00) -> one bit per distance: byte e of word w
+        // becomes bit 4w + e (the multiply gathers bits 7, 15, 23, 31 into 28..31)
         uint32_t lt_bits = 0, eq_bits = 0;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t lt = __vcmpltu4(dw[k], T4) & 0x80808080u;
-            const uint32_t eq = __vcmpeq4(dw[k], T4) & 0x80808080u;
-            lt_bits |= ((lt * 0x00204081u) >> 28) << (4 * k);
-            eq_bits |= ((eq * 0x00204081u) >> 28) << (4 * k);
+        for (int w = 0; w < 8; ++w) {
+            const uint32_t lt = __vcmpltu4(dw[w], T4) & 0x80808080u;
+            const uint32_t eq = __vcmpeq4(dw[w], T4) & 0x80808080u;
+            lt_bits |= ((lt * 0x00204081u) >> 28) << (4 * w);
+            eq_bits |= ((eq * 0x00204081u) >> 28) << (4 * w);
         }
         const int n_lt = __popc(lt_bits), n_eq = __popc(eq_bits);
         // one scan of the packed pair (each count <= 4096 per chunk)
