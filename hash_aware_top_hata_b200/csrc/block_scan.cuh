@@ -39,3 +39,45 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *scratch, int *to
 }
 
 }  // namespace hata
+
+namespace hata {
+
+// Exclusive prefix sums of two counters (a, b) over the block at once, in
+// threadIdx.x order; *ta / *tb get the block sums.  scratch: >= NT/32 + 1
+// int2 of shared memory.  Every thread must call it; two block barriers,
+// plus one at the end so that scratch may be reused right after.
+template <int NT>
+__device__ __forceinline__ int2 block_exclusive_scan2(int a, int b, int2 *scratch, int *ta, int *tb)
+{
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int na = __shfl_up_sync(0xffffffffu, ia, o);
+        const int nb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) { ia += na; ib += nb; }
+    }
+    if (lane == 31) scratch[warp] = make_int2(ia, ib);
+    __syncthreads();
+    if (warp == 0) {
+        const int2 w = lane < NW ? scratch[lane] : make_int2(0, 0);
+        int wa = w.x, wb = w.y;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int na = __shfl_up_sync(0xffffffffu, wa, o);
+            const int nb = __shfl_up_sync(0xffffffffu, wb, o);
+            if (lane >= o) { wa += na; wb += nb; }
+        }
+        if (lane < NW) scratch[lane] = make_int2(wa - w.x, wb - w.y);
+        if (lane == NW - 1) scratch[NW] = make_int2(wa, wb);
+    }
+    __syncthreads();
+    const int2 base = scratch[warp];
+    *ta = scratch[NW].x;
+    *tb = scratch[NW].y;
+    __syncthreads();
+    return make_int2(base.x + ia - a, base.y + ib - b);
+}
+
+}  // namespace hata

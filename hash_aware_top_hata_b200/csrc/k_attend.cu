@@ -411,11 +411,6 @@ __device__ __forceinline__ float split(float x, int part)
     return part == 0 ? hi : x - hi;
 }
 
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes));
-}
-
 // 2^x on the special-function unit (relative error ~2^-22; -inf -> +0).
 __device__ __forceinline__ float fast_exp2(float x)
 {

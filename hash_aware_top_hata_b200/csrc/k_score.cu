@@ -5,28 +5,31 @@
 // the Hamming score; major comment 1 (Algorithm 3): the top-k runs over
 // these 129 possible scores.
 //
-// Persistent kernel.  Work items are (b, h_kv, group of <= 8 query heads,
-// chunk of 4096 tokens); CTA k takes items k, k + gridDim.x, ...  Each item's
-// 64 KB of 16-byte codes streams through a 3-deep ring of 16 KB shared-memory
-// buffers filled by the bulk-copy engine (cp.async.bulk issued by one
-// thread, mbarrier completion), so the code stream is read from HBM exactly
-// once per KV head and its latency hides behind the arithmetic of the
-// previous sub-block.  Every code is scored against all query heads of its
-// group:
+// Work items are (b, h_kv, group of <= 8 query heads, chunk of 4096 tokens);
+// CTA k takes items k, k + gridDim.x, ...  Inside an item every warp streams
+// its own 512 tokens as four 128-token units, with no block-wide barrier:
+// lane l owns tokens l, l+32, l+64, l+96 of a unit (four coalesced 16-byte
+// loads per warp instruction).  The loads are asynchronous copies
+// (cp.async) into a per-warp ring of kRing units in shared memory, issued
+// kRing-1 units ahead; every lane reads back only the bytes it copied, so a
+// lane's own wait_group is the only synchronisation, and the codes in
+// flight cost no registers.  The code stream is read from HBM exactly once
+// per KV head.  Each code is scored against every query head of the group:
 //
 //   x_w = code_w XOR q_w (w = 0..3)
 //   (s, c)    = full-add(x0, x1, x2)    -- bitwise carry-save adder
 //   (ones, c2) = half-add(s, x3)
 //   dist = popc(ones) + 2 popc(c XOR c2) + 4 popc(c AND c2)
 //
-// i.e. three population counts instead of four: POPC issues at a quarter of
-// the integer rate on sm_100a, and it is what bounds this kernel.
+// i.e. three population counts instead of four: POPC issues at an eighth of
+// the integer-logic rate on sm_100a, and it is what bounds the arithmetic.
 //
-// Per query head the kernel writes the u8 distance row (through a
-// shared-memory tile and a bulk store; the row stays L2-resident for the
-// selection kernel) and a 129-bin histogram per chunk (per-warp shared
-// counters), published as a cumulative histogram per chunk plus atomic adds
-// into the head's total histogram.
+// Per query head the kernel stores the u8 distance row (32 lanes write 32
+// consecutive bytes per store; the row stays L2-resident for the selection
+// kernel) and counts a 129-bin histogram per chunk in shared memory.  The
+// block's single barrier per item closes the chunk: warp g publishes head
+// g's histogram as a cumulative histogram (for the selection's offsets) and
+// adds its non-zero bins into the head's total histogram.
 #include "block_scan.cuh"
 #include "hata_internal.cuh"
 #include "tma.cuh"
@@ -34,11 +37,12 @@
 namespace hata {
 namespace {
 
-constexpr int kWarps = kScoreThreads / 32;
-constexpr int kSub = 1024;                    // tokens per staged sub-block (16 KB)
-constexpr int kSubsPerChunk = kChunk / kSub;  // 4
-constexpr int kRing = 3;
-constexpr int kTokPerThread = kSub / kScoreThreads;  // 4
+constexpr int kWarps = kScoreThreads / 32;              // 8
+constexpr int kUnit = 128;                              // tokens per warp step
+constexpr int kUnitsPerWarp = kChunk / (kWarps * kUnit);  // 4
+constexpr int kRing = 4;                                // units per warp ring
+static_assert(kUnitsPerWarp * kWarps * kUnit == kChunk, "warps tile a chunk");
+static_assert(kScoreHeads <= kWarps, "one publishing warp per head");
 
 __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
 {
@@ -57,169 +61,174 @@ __device__ __forceinline__ int hamming128(const uint4 &k, const uint4 &q)
 }
 
 struct Item {
-    int b, h, z, c;
+    int b, h, c, ng;
     int64_t len;
+    size_t bh0;  // b * H_q + first query head of the group
 };
-static_assert(kChunk % kSub == 0, "sub-blocks tile a chunk");
 
 struct ScoreSmem {
-    uint4 codes[kRing][kSub];               // 48 KB ring of staged codes
-    uint8_t dist[2][kScoreHeads][kSub];     // 16 KB double-buffered distance tiles
-    uint32_t hist[kWarps][kScoreHeads][kBins];
-    uint32_t chist[kScoreHeads][kBins];
-    uint64_t full[kRing];
+    uint4 ring[kWarps][kRing][kUnit];            // 64 KB of staged codes
+    uint4 qs[2][kScoreHeads];                    // query codes, by item parity
+    uint32_t hist[2][kScoreHeads][kHistStride];  // chunk histograms, by item parity
 };
 
+// Histogram increment: one shared-memory reduction, no return value.
+__device__ __forceinline__ void red_shared_add1(uint32_t addr)
+{
+    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
+}
+
 template <int GB>
-__global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(ScoreArgs a)
+__global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ScoreSmem &S = *reinterpret_cast<ScoreSmem *>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // item -> (b, h_kv, head group, chunk): 32-bit arithmetic, once per item
-    auto item_of = [&](int it) {
+    // item -> (b, h_kv, head group, chunk): 32-bit arithmetic
+    auto item_of = [&](int k) {
+        const int it = int(blockIdx.x) + k * int(gridDim.x);
         Item r;
         r.c = it % int(a.n_chunks);
         int g = it / int(a.n_chunks);
-        r.z = g % a.zgroups;
+        const int z = g % a.zgroups;
         g /= a.zgroups;
         r.h = g % a.H_kv;
         r.b = g / a.H_kv;
         r.len = clamp_len(__ldg(a.seq_len + r.b), a.max_seq_len, a.n_cap);
+        const int g0 = z * kScoreHeads;
+        r.ng = min(GB, a.G - g0);
+        r.bh0 = size_t(r.b) * a.H_q + size_t(r.h) * a.G + g0;
         return r;
     };
-    // tokens of sub-block s of item r that hold real codes
-    auto sub_valid = [&](const Item &r, int s) -> int {
-        const int64_t v = r.len - (int64_t(r.c) * kChunk + int64_t(s) * kSub);
-        return v <= 0 ? 0 : (v >= kSub ? kSub : int(v));
-    };
-    // sub-block j of this CTA's sequence into ring slot j % kRing (thread 0)
-    auto issue = [&](int j) {
-        const Item r = item_of(int(blockIdx.x) + (j / kSubsPerChunk) * int(gridDim.x));
-        const int s = j % kSubsPerChunk;
-        const int v = sub_valid(r, s);
-        uint64_t *bar = &S.full[j % kRing];
-        mbar_arrive_expect_tx(bar, uint32_t(v) * 16u);
-        if (v > 0) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.codes) +
-                               ((int64_t(r.b) * a.H_kv + r.h) * a.n_cap +
-                                int64_t(r.c) * kChunk + int64_t(s) * kSub);
-            bulk_g2s(S.codes[j % kRing], src, uint32_t(v) * 16u, bar);
+    // the query codes of item k into qs[k & 1] (threads 0 .. 4*GB-1)
+    auto stage_q = [&](int k) {
+        if (tid < 4 * GB) {
+            const Item r = item_of(k);
+            const int g = tid >> 2, w = tid & 3;
+            reinterpret_cast<uint32_t *>(&S.qs[k & 1][0])[tid] =
+                g < r.ng ? __ldg(a.qcodes + (r.bh0 + g) * kWords + w) : 0u;
         }
     };
-
-    if (tid == 0) {
-        for (int i = 0; i < kRing; ++i) mbar_init(&S.full[i], 1);
-        fence_mbar_init();
-    }
-    for (int i = tid; i < kWarps * kScoreHeads * kBins; i += kScoreThreads)
-        (&S.hist[0][0][0])[i] = 0u;
-    __syncthreads();
 
     const int n_items = int(int64_t(a.B) * a.H_kv * a.zgroups * a.n_chunks);
     const int my_items =
         int(blockIdx.x) < n_items ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
-    const int n_subs = my_items * kSubsPerChunk;
-    if (tid == 0)
-        for (int j = 0; j < kRing && j < n_subs; ++j) issue(j);
+    if (my_items == 0) return;
+    for (int i = tid; i < 2 * kScoreHeads * kHistStride; i += kScoreThreads)
+        (&S.hist[0][0][0])[i] = 0u;
+    stage_q(0);
+    if (my_items > 1) stage_q(1);
+    __syncthreads();
 
-    Item r{};
-    int ng = 0;
-    size_t bh0 = 0;
-    uint4 qc[GB];
-    for (int j = 0; j < n_subs; ++j) {
-        const int s = j % kSubsPerChunk;
-        if (s == 0) {  // a new item: decode it and fetch its query codes once
-            r = item_of(int(blockIdx.x) + (j / kSubsPerChunk) * int(gridDim.x));
-            const int g0 = r.z * kScoreHeads;
-            ng = min(GB, a.G - g0);
-            bh0 = size_t(r.b) * a.H_q + size_t(r.h) * a.G + g0;
+    const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes);
+    const int n_units = my_items * kUnitsPerWarp;
+    // copy this warp's unit j (of its item sequence) into ring slot j % kRing;
+    // tokens past len are zero-filled without reading memory.  Always
+    // commits one group (empty past the end) so the group count stays exact.
+    Item ld = item_of(0);
+    auto issue = [&](int j) {
+        asm volatile("" ::: "memory");  // earlier reads of the ring stay before the copies
+        if (j < n_units) {
+            const int u = j % kUnitsPerWarp;
+            if (u == 0 && j > 0) ld = item_of(j / kUnitsPerWarp);
+            const int64_t t0 = int64_t(ld.c) * kChunk + (warp * kUnitsPerWarp + u) * kUnit + lane;
+            const uint4 *src = codes + (int64_t(ld.b) * a.H_kv + ld.h) * a.n_cap + t0;
+            const uint32_t dst = smem_addr(&S.ring[warp][j % kRing][lane]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const bool ok = t0 + 32 * i < ld.len;
+                cp_async16_zfill(dst + 512u * i, ok ? src + 32 * i : codes, ok ? 16u : 0u);
+            }
+        }
+        cp_async_commit();
+    };
+    for (int j = 0; j < kRing - 1; ++j) issue(j);
+
+    Item cp = item_of(0);  // item of the unit being scored
+    for (int j = 0; j < n_units; ++j) {
+        const int k = j / kUnitsPerWarp, u = j % kUnitsPerWarp;
+        issue(j + kRing - 1);
+        cp_async_wait<kRing - 1>();  // this lane's copies of unit j have landed
+        uint4 cur[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cur[i] = S.ring[warp][j % kRing][lane + 32 * i];
+        if (u == 0 && j > 0) cp = item_of(k);
+        const int p = k & 1;
+        const int64_t t0 = int64_t(cp.c) * kChunk + (warp * kUnitsPerWarp + u) * kUnit;
+        const int64_t nv64 = cp.len - t0;
+        const int nv = nv64 <= 0 ? 0 : (nv64 >= kUnit ? kUnit : int(nv64));
+        uint8_t *row0 = a.dist + cp.bh0 * a.dist_row + t0;
+        if (nv == 0) {
+            // past seq_len: pad bytes only (4 per lane, 128 per head)
 #pragma unroll
             for (int g = 0; g < GB; ++g)
-                qc[g] = g < ng ? reinterpret_cast<const uint4 *>(a.qcodes)[bh0 + g]
-                               : make_uint4(0, 0, 0, 0);
-        }
-        const int v = sub_valid(r, s);
-
-        const bool landed = mbar_wait(&S.full[j % kRing], uint32_t((j / kRing) & 1));
-        // the distance tile of sub-block j was last stored by bulk group j-2:
-        // let it finish reading (it was issued a whole sub-block ago) before
-        // the barrier that releases the tile writes
-        if (tid == 0) bulk_wait_read<1>();
-        if (__syncthreads_or(!landed)) {
-            // a copy never completed: flag it and stop (the wait was bounded)
-            if (tid == 0) atomicOr(a.flags + r.b, HATA_FLAG_TIMEOUT);
-            break;
-        }
-        const uint4 *buf = S.codes[j % kRing];
-        uint8_t(*tile)[kSub] = S.dist[j & 1];
-#pragma unroll
-        for (int u = 0; u < kTokPerThread; ++u) {
-            const int t = u * kScoreThreads + tid;
-            const bool valid = t < v;
-            const uint4 cv = valid ? buf[t] : make_uint4(0, 0, 0, 0);
+                if (g < cp.ng)
+                    reinterpret_cast<uint32_t *>(row0 + g * a.dist_row)[lane] = 0xffffffffu;
+        } else {
 #pragma unroll
             for (int g = 0; g < GB; ++g) {
-                if (g < ng) {
-                    const int d = hamming128(cv, qc[g]);
-                    tile[g][t] = valid ? uint8_t(d) : kDistPad;
-                    if (valid) atomicAdd(&S.hist[warp][g][d], 1u);
-                }
-            }
-        }
-        fence_async_shared();          // tile writes -> visible to the bulk store
-        __syncthreads();
-        if (tid == 0) {
-            const int64_t off = int64_t(r.c) * kChunk + int64_t(s) * kSub;
-            for (int g = 0; g < ng; ++g)
-                bulk_s2g(a.dist + (bh0 + g) * a.dist_row + off, tile[g], kSub);
-            bulk_commit();
-            if (j + kRing < n_subs) issue(j + kRing);
-        }
-
-        const int64_t nch = r.len > 0 ? ceil_div(r.len, kChunk) : 1;
-        if (s == kSubsPerChunk - 1 && r.c < nch) {
-            // ---- chunk done: publish its histogram ----
-            for (int i = tid; i < ng * kBins; i += kScoreThreads) {
-                const int g = i / kBins, t = i % kBins;
-                uint32_t sum = 0;
+                if (g < cp.ng) {
+                    const uint4 q = S.qs[p][g];
+                    uint8_t *row = row0 + g * a.dist_row + lane;
+                    const uint32_t H = smem_addr(S.hist[p][g]);
+                    if (nv == kUnit) {
 #pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    sum += S.hist[w][g][t];
-                    S.hist[w][g][t] = 0u;
+                        for (int i = 0; i < 4; ++i) {
+                            const int d = hamming128(cur[i], q);
+                            __stcg(row + 32 * i, uint8_t(d));
+                            red_shared_add1(H + 4u * uint32_t(d));
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int d = hamming128(cur[i], q);
+                            const bool valid = lane + 32 * i < nv;
+                            __stcg(row + 32 * i, valid ? uint8_t(d) : kDistPad);
+                            if (valid) red_shared_add1(H + 4u * uint32_t(d));
+                        }
+                    }
                 }
-                S.chist[g][t] = sum;
             }
+        }
+        if (u == kUnitsPerWarp - 1) {
+            // ---- chunk done (all warps): publish its histogram ----
             __syncthreads();
-            if (warp < ng) {
+            const int64_t nch = cp.len > 0 ? ceil_div(cp.len, kChunk) : 1;
+            if (warp < cp.ng) {
                 const int g = warp;
-                const size_t bh = bh0 + g;
+                uint32_t *H = S.hist[p][g];
                 uint32_t vv[5];
                 uint32_t run = 0;
 #pragma unroll
                 for (int e = 0; e < 5; ++e) {
                     const int t = lane * 5 + e;
-                    vv[e] = t < kBins ? S.chist[g][t] : 0u;
+                    vv[e] = t < kBins ? H[t] : 0u;
                     run += vv[e];
                 }
-                uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
-                uint32_t *cp = a.cum + (bh * a.n_chunks + r.c) * kCumStride;
+                if (cp.c < nch) {
+                    const size_t bh = cp.bh0 + g;
+                    uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
+                    uint32_t *cum = a.cum + (bh * a.n_chunks + cp.c) * kCumStride;
 #pragma unroll
-                for (int e = 0; e < 5; ++e) {
-                    const int t = lane * 5 + e;
-                    acc += vv[e];
-                    if (t < kBins) {
-                        cp[t] = acc;
-                        if (vv[e]) atomicAdd(a.hist_total + bh * kHistStride + t, vv[e]);
+                    for (int e = 0; e < 5; ++e) {
+                        const int t = lane * 5 + e;
+                        acc += vv[e];
+                        if (t < kBins) {
+                            cum[t] = acc;
+                            if (vv[e]) atomicAdd(a.hist_total + bh * kHistStride + t, vv[e]);
+                        }
                     }
                 }
+#pragma unroll
+                for (int e = 0; e < 5; ++e)
+                    if (lane * 5 + e < kBins) H[lane * 5 + e] = 0u;
             }
-            // chist is next rewritten only after four more sub-blocks, each
-            // closed by a __syncthreads
+            // qs[p] is free (item k is scored): stage item k + 2's query codes
+            if (k + 2 < my_items) stage_q(k + 2);
         }
     }
-    if (tid == 0) bulk_wait_all();
+    cp_async_wait<0>();
 }
 
 template <int GB>
