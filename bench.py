@@ -225,6 +225,11 @@ def config_dict(cfg, l2: str) -> dict:
 
 # ---------------------------------------------------------------- GPU arm --
 
+def _num(x, nd):
+    """x rounded, or None (JSON null) when it was not measured."""
+    return None if x != x else round(x, nd)
+
+
 def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, world):
     """e2e (host buffers in, host result out, through the same C ABI) and the
     dense decode attention at the same shape."""
@@ -232,7 +237,7 @@ def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, w
     B, Hq, Hkv, N = cfg.B, cfg.H_q, cfg.H_kv, cfg.N
     scale = 1.0 / math.sqrt(128)
     kv_elt = 2 if cfg.kv_dtype == "bf16" else 4
-    t0 = W_steps + K_steps
+    t0 = W_steps + 2 * K_steps  # steps after the timed and the breakdown passes
     q_h = w.q[t0:t0 + K_steps].cpu().pin_memory()
     kn_h = w.k_new[t0:t0 + K_steps].cpu().pin_memory()
     vn_h = w.v_new[t0:t0 + K_steps].cpu().pin_memory()
@@ -278,7 +283,7 @@ def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, w
 def run_hata(args, world, rank, local):
     cfg = bench_config(args)
     K_steps, W_steps = args.steps, args.warmup
-    total_steps = W_steps + 2 * K_steps
+    total_steps = W_steps + 3 * K_steps
     seed = wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config) + 1000 * rank
     dev = torch.device("cuda", torch.cuda.current_device())
     w = wl.make_workload(cfg, seed, device=dev, steps=total_steps)
@@ -306,27 +311,39 @@ def run_hata(args, world, rank, local):
     torch.cuda.synchronize()
     H.hata_workspace_check(ws)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K_steps)]
-    for e4 in evs:  # torch creates the CUDA event on first record; the library needs handles
-        for e in e4:
-            e.record(stream)
-    torch.cuda.synchronize()
+    # timed region: the step alone (no events between its kernels, so each
+    # kernel's launch overlaps its predecessor), bracketed by two events
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
         wall0 = time.perf_counter()
         for i in range(K_steps):
             flush()
-            step(W_steps + i, evs[i])
+            evs[i][0].record(stream)
+            step(W_steps + i)
+            evs[i][1].record(stream)
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
         barrier(world)
     H.hata_workspace_check(ws)
-    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
-    prep_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    score_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    select_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    attend_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+
+    # per-kernel breakdown (untimed pass): events between the four kernels
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K_steps)]
+    for e5 in kevs:  # torch creates the CUDA event on first record; the library needs handles
+        for e in e5:
+            e.record(stream)
+    torch.cuda.synchronize()
+    for i in range(K_steps):
+        flush()
+        step(W_steps + K_steps + i, kevs[i])
+    torch.cuda.synchronize()
+    prep_ms = [e[0].elapsed_time(e[1]) for e in kevs]
+    score_ms = [e[1].elapsed_time(e[2]) for e in kevs]
+    select_ms = [e[2].elapsed_time(e[3]) for e in kevs]
+    attend_ms = [e[3].elapsed_time(e[4]) for e in kevs]
+    split_ms = [e[0].elapsed_time(e[4]) for e in kevs]
     ms = statistics.mean(step_ms)
     ms_max = max_over_ranks(world, ms)
 
@@ -360,10 +377,11 @@ def run_hata(args, world, rank, local):
                        "score": round(score_s * 1e6, 2),
                        "select": round(statistics.mean(select_ms) * 1e3, 2),
                        "attend": round(attend_s * 1e6, 2),
+                       "sum_with_events": round(statistics.mean(split_ms) * 1e3, 2),
                        "score_gbs": round(code_bytes / score_s / 1e9, 1)},
-        "dense_us": round(dense_ms * 1e3, 1),
-        "speedup_vs_dense": round(dense_ms / ms, 2),
-        "e2e": {"value": round(e2e_ms * 1e3, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "dense_us": _num(dense_ms * 1e3, 1),
+        "speedup_vs_dense": _num(dense_ms / ms, 2),
+        "e2e": {"value": _num(e2e_ms * 1e3, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 4 * K_steps,
         "clocks": clk.summary(),

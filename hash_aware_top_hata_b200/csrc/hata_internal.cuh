@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/hata.h"
 
 namespace hata {
@@ -168,6 +170,37 @@ inline bool dense_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int64_t 
     *off_cnt = o;   o = align_up(o + 4 * size_t(B) * H_kv * ceil_div(G, kDenseHeads), 256);
     *total = o;
     return true;
+}
+
+// ------------------------------------------- programmatic dependent launch --
+// The kernels after the first of a decode step are launched with programmatic
+// stream serialization: a dependent grid may be scheduled while its
+// predecessor still runs, so its launch latency hides behind that kernel.
+// Every such kernel lets its own dependent go (pdl_trigger) and then waits
+// for its predecessor to complete, with all its memory writes visible
+// (pdl_wait), before it reads anything the predecessor produced.  Both are
+// no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args &&...args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Records msg as hata_last_error() of this thread and returns st.

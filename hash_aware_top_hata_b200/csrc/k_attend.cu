@@ -148,6 +148,8 @@ __global__ void __launch_bounds__(kAttnThreads) attend_simt_kernel(AttendArgs a)
     constexpr int RB = RW::kRowBytes;
     extern __shared__ __align__(128) uint8_t smem[];  // [kRing][K rows | V rows]
     __shared__ int32_t rows_s[kRing][kStageRows];
+    pdl_trigger();
+    pdl_wait();  // the selected index lists
     __shared__ float red_m[kHalves], red_l[kHalves];
     __shared__ __align__(16) float red_acc[kHalves][kD];
     __shared__ int s_last;
@@ -564,6 +566,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     using namespace tc;
     extern __shared__ __align__(128) uint8_t smem[];  // [warp][kRingW][K | V], then indices
     __shared__ int32_t rows_s[kTcWarps][kRingW][kSub];
+    pdl_trigger();
+    pdl_wait();  // the selected index lists
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = int64_t(a.B) * a.H_q * a.topk;
@@ -696,8 +700,8 @@ cudaError_t launch_attend(const AttendArgs &args, bool bf16, cudaStream_t s)
         if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
         if (NW > T) NW = T;
         a.n_workers = NW;
-        attend_tc_kernel<<<unsigned(ceil_div(NW, tc::kTcWarps)), tc::kThreads, tc::kSmem, s>>>(a);
-        return cudaGetLastError();
+        return launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
+                          dim3(tc::kThreads), tc::kSmem, s, a);
     }
     constexpr size_t kSmemF32 = size_t(kRing) * Rows<false>::kSlotBytes;
     if (cudaError_t e = occupancy_grid(attend_simt_kernel<false>, kAttnThreads, kSmemF32, &P))
@@ -705,8 +709,8 @@ cudaError_t launch_attend(const AttendArgs &args, bool bf16, cudaStream_t s)
     if (P > kAttnMaxWorkers) P = kAttnMaxWorkers;
     if (P > T) P = T;
     a.n_workers = P;
-    attend_simt_kernel<false><<<unsigned(P), kAttnThreads, kSmemF32, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(attend_simt_kernel<false>, dim3(unsigned(P)), dim3(kAttnThreads), kSmemF32,
+                      s, a);
 }
 
 }  // namespace hata

@@ -20,7 +20,6 @@
 // optionally its K/V rows) and clears the per-step counters the scoring
 // kernel accumulates into.
 #include "hata_internal.cuh"
-#include "tma.cuh"
 
 namespace hata {
 namespace {
@@ -53,35 +52,9 @@ __device__ __forceinline__ void load_w_column(const float *__restrict__ Wh, int 
     for (int i = 0; i < kD; ++i) w[i] = __ldg(Wh + i * kRbit + j);
 }
 
-// xs: [kD][R] floats (row r of the group in column r); ws: W_H in shared
-// memory.  Returns, for every row, the ballot of this warp's 32 bits = code
-// word (threadIdx.x / 32).
-template <int R>
-__device__ __forceinline__ void hash_group_smem(const float *__restrict__ xs,
-                                                const float *__restrict__ ws,
-                                                uint32_t (&words)[R])
-{
-    const int j = threadIdx.x;
-    float acc[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0.0f;
-#pragma unroll 8
-    for (int i = 0; i < kD; ++i) {
-        const float w = ws[i * kRbit + j];
-#pragma unroll
-        for (int r4 = 0; r4 < R / 4; ++r4) {
-            const float4 x = reinterpret_cast<const float4 *>(xs + i * R)[r4];
-            acc[4 * r4 + 0] = __fmaf_rn(x.x, w, acc[4 * r4 + 0]);
-            acc[4 * r4 + 1] = __fmaf_rn(x.y, w, acc[4 * r4 + 1]);
-            acc[4 * r4 + 2] = __fmaf_rn(x.z, w, acc[4 * r4 + 2]);
-            acc[4 * r4 + 3] = __fmaf_rn(x.w, w, acc[4 * r4 + 3]);
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) words[r] = __ballot_sync(0xffffffffu, acc[r] > 0.0f);
-}
-
-// Same with column j of W_H held in registers (prefill: many row groups per CTA).
+// xs: [kD][R] floats (row r of the group in column r); w: column j of W_H
+// (j = threadIdx.x) in registers.  Returns, for every row, the ballot of this
+// warp's 32 bits = code word (threadIdx.x / 32).
 template <int R>
 __device__ __forceinline__ void hash_group(const float *__restrict__ xs, const float (&w)[kD],
                                            uint32_t (&words)[R])
@@ -158,18 +131,11 @@ __global__ void __launch_bounds__(kD) prep_kernel(PrepArgs a)
     }
     if (r0 >= rows) return;
 
-    extern __shared__ __align__(128) float smem[];
-    float *ws = smem;                 // [kD][kRbit]: this head's W_H
-    float *xs = smem + kD * kRbit;    // [kD][R]: the rows, one per column
-    __shared__ uint64_t bar;
-    if (j == 0) {
-        // the whole 64 KB W_H in one bulk copy, overlapping the row staging
-        mbar_init(&bar, 1);
-        fence_mbar_init();
-        constexpr uint32_t kWBytes = sizeof(float) * kD * kRbit;
-        mbar_arrive_expect_tx(&bar, kWBytes);
-        bulk_g2s(ws, a.W + size_t(h) * kD * kRbit, kWBytes, &bar);
-    }
+    // column j of this head's W_H: 128 coalesced loads in flight while the
+    // rows are staged
+    float w[kD];
+    load_w_column(a.W + size_t(h) * kD * kRbit, j, w);
+    __shared__ __align__(16) float xs[kD * R];  // [kD][R]: the rows, one per column
 
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -195,18 +161,9 @@ __global__ void __launch_bounds__(kD) prep_kernel(PrepArgs a)
         }
         xs[j * R + r] = x;
     }
-    const bool landed = mbar_wait(&bar, 0);
-    if (__syncthreads_or(!landed)) {
-        if (j == 0) {
-            if (a.flags)
-                for (int b = 0; b < a.B; ++b) atomicOr(a.flags + b, HATA_FLAG_TIMEOUT);
-            if (a.err_word) atomicOr(a.err_word, HATA_FLAG_TIMEOUT);
-            (void)mbar_wait(&bar, 0);
-        }
-        return;
-    }
+    __syncthreads();
     uint32_t words[R];
-    hash_group_smem<R>(xs, ws, words);
+    hash_group<R>(xs, w, words);
 
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -251,15 +208,11 @@ cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const f
 
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s)
 {
-    constexpr size_t kSmem = sizeof(float) * (kD * kRbit + kD * kPrepRows);
-    const void *fn = a.kv_bf16 ? reinterpret_cast<const void *>(prep_kernel<true>)
-                               : reinterpret_cast<const void *>(prep_kernel<false>);
-    if (cudaError_t e = ensure_smem_attr(fn, kSmem)) return e;
     const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRows)), unsigned(a.H_kv));
     if (a.kv_bf16)
-        prep_kernel<true><<<grid, kD, kSmem, s>>>(a);
+        prep_kernel<true><<<grid, kD, 0, s>>>(a);
     else
-        prep_kernel<false><<<grid, kD, kSmem, s>>>(a);
+        prep_kernel<false><<<grid, kD, 0, s>>>(a);
     return cudaGetLastError();
 }
 

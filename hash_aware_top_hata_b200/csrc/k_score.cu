@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a)
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ScoreSmem &S = *reinterpret_cast<ScoreSmem *>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_trigger();
+    pdl_wait();  // query codes, the appended key code and cleared counters
 
     // item -> (b, h_kv, head group, chunk): 32-bit arithmetic
     auto item_of = [&](int k) {
@@ -245,8 +247,8 @@ cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     const int64_t cap = int64_t(per_sm > 0 ? per_sm : 1) * sms;
     const int64_t items = int64_t(a.B) * a.H_kv * a.zgroups * a.n_chunks;
-    score_kernel<GB><<<unsigned(items < cap ? items : cap), kScoreThreads, sizeof(ScoreSmem), s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(score_kernel<GB>, dim3(unsigned(items < cap ? items : cap)),
+                      dim3(kScoreThreads), sizeof(ScoreSmem), s, a);
 }
 
 }  // namespace

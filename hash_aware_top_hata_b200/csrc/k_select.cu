@@ -94,6 +94,8 @@ __device__ __forceinline__ uint32_t to_token_order(uint32_t m)
 
 __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a, int parts)
 {
+    pdl_trigger();
+    pdl_wait();  // distances and histograms of the scoring kernel
     const int part = blockIdx.x;
     const size_t bh = blockIdx.y;
     const int b = int(bh / a.H_q);
@@ -271,8 +273,7 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t s)
     int64_t parts = slots / heads;
     parts = parts < 1 ? 1 : (parts > tiles ? tiles : parts);
     const dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(heads));
-    select_kernel<<<grid, kThreads, 0, s>>>(a, int(parts));
-    return cudaGetLastError();
+    return launch_pdl(select_kernel, grid, dim3(kThreads), 0, s, a, int(parts));
 }
 
 }  // namespace hata
