@@ -221,7 +221,6 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     int32_t *idx = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(ws + L.off_idx);
     uint32_t *flags = reinterpret_cast<uint32_t *>(ws + L.off_flags);
     uint32_t *hist = reinterpret_cast<uint32_t *>(ws + L.off_hist);
-    uint32_t *cum = reinterpret_cast<uint32_t *>(ws + L.off_cum);
     uint32_t *cnt_attn = reinterpret_cast<uint32_t *>(ws + L.off_cnt_attn);
     const Events ev{events, s};
     cudaError_t e;
@@ -239,7 +238,8 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     p.seq_len = seq_len;
     p.q_out = qc;
     p.flags = flags;
-    p.hist_total = hist;
+    p.hist = hist;
+    p.hist_row_words = L.n_tiles * kHistStride;
     p.cnt_attn = cnt_attn;
     p.ws_header = reinterpret_cast<uint32_t *>(ws);
     p.n_cap = n_cap;
@@ -259,12 +259,10 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     sa.seq_len = seq_len;
     sa.dist = dst;
     sa.dist_row = drow;
-    sa.cum = cum;
-    sa.hist_total = hist;
-    sa.flags = flags;
+    sa.hist = hist;
     sa.n_cap = n_cap;
     sa.max_seq_len = max_seq_len;
-    sa.n_chunks = L.n_chunks;
+    sa.n_tiles = L.n_tiles;
     sa.B = B;
     sa.H_q = H_q;
     sa.H_kv = H_kv;
@@ -277,12 +275,11 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     se.seq_len = seq_len;
     se.dist = dst;
     se.dist_row = drow;
-    se.cum = cum;
-    se.hist_total = hist;
+    se.hist = hist;
     se.idx = idx;
     se.n_cap = n_cap;
     se.max_seq_len = max_seq_len;
-    se.n_chunks = L.n_chunks;
+    se.n_tiles = L.n_tiles;
     se.B = B;
     se.H_q = H_q;
     se.topk = topk;

@@ -19,8 +19,8 @@ constexpr int kChunk = 4096;            // tokens per scoring / selection chunk
 constexpr int kScoreThreads = 256;
 constexpr int kScoreHeads = 8;          // query heads scored per code load (one CTA)
 constexpr int kAttnThreads = 128;
-constexpr int kCumStride = 132;         // u32 per (head, chunk) cumulative histogram
-constexpr int kHistStride = 132;        // u32 per head total histogram
+constexpr int kHistStride = 132;        // u32 per (head, tile) histogram row (129 bins)
+constexpr int kTile = 32768;            // tokens per histogram tile / selection tile
 constexpr int kPartStride = 132;        // f32 per (head, chunk) partial: m, l, -, -, acc[128]
 constexpr int kPrepRows = 4;            // rows hashed together by one prep CTA
 constexpr uint8_t kDistPad = 255;       // distance stored past seq_len
@@ -30,7 +30,6 @@ __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kAttnMaxWorkers = 4096;   // upper bound of the attention stream-K workers
-constexpr int kSelSegChunks = 2;        // scoring chunks walked by one selection CTA
 
 // Most attention workers that can share one head: each of the P <= T
 // workers owns at least floor(T / P) >= r_min rows of the flat row space.
@@ -45,12 +44,13 @@ inline int attn_max_contributors(int64_t BH, int topk)
 // Decode workspace.  The first 256 B hold a header {magic, B}; one flag word
 // per batch row follows.  Everything else is rebuilt by every decode step.
 struct DecodeLayout {
-    int64_t n_chunks = 0;   // scoring chunks of max_seq_len
+    int64_t n_chunks = 0;   // 4096-token chunks of max_seq_len
     int64_t dist_row = 0;   // bytes per (b, h_q) distance row
+    int64_t n_tiles = 0;    // 32K-token histogram tiles of a distance row
     int zgroups = 0;        // ceil(G / kScoreHeads)
     int n_split = 0;        // attention partial slots per head
-    size_t off_flags = 0, off_qcodes = 0, off_dist = 0, off_cum = 0, off_hist = 0,
-           off_idx = 0, off_part = 0, off_cnt_attn = 0, total = 0;
+    size_t off_flags = 0, off_qcodes = 0, off_dist = 0, off_hist = 0, off_idx = 0,
+           off_part = 0, off_cnt_attn = 0, total = 0;
 };
 
 inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
@@ -64,16 +64,16 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
     const int G = H_q / H_kv;
     L->n_chunks = ceil_div(max_seq_len, kChunk);
     L->dist_row = L->n_chunks * kChunk;
+    L->n_tiles = ceil_div(L->dist_row, kTile);
     L->zgroups = int(ceil_div(G, kScoreHeads));
-    // the scoring kernel numbers its work items with 32-bit integers
-    if (int64_t(B) * H_kv * L->zgroups * L->n_chunks >= (int64_t(1) << 31)) return false;
+    // the scoring kernel numbers its 128-token units with 32-bit integers
+    if (int64_t(B) * H_kv * L->zgroups * (L->dist_row / 128) >= (int64_t(1) << 31)) return false;
     L->n_split = attn_max_contributors(BH, topk);
     size_t o = 256;
     L->off_flags = o;      o = align_up(o + 4 * size_t(B), 256);
     L->off_qcodes = o;     o = align_up(o + 16 * size_t(BH), 256);
     L->off_dist = o;       o = align_up(o + size_t(BH) * L->dist_row, 256);
-    L->off_cum = o;        o = align_up(o + 4 * size_t(BH) * L->n_chunks * kCumStride, 256);
-    L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * kHistStride, 256);
+    L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * L->n_tiles * kHistStride, 256);
     L->off_idx = o;        o = align_up(o + 4 * size_t(BH) * topk, 256);
     L->off_part = o;       o = align_up(o + 4 * size_t(BH) * L->n_split * kPartStride, 256);
     L->off_cnt_attn = o;   o = align_up(o + 4 * size_t(BH), 256);
@@ -94,7 +94,8 @@ struct PrepArgs {
     uint32_t *q_out;         // [B][H_q][4]
     uint32_t *flags;         // per-b flag words (decode) or null
     uint32_t *err_word;      // single OR-ed word (append API) or null
-    uint32_t *hist_total;    // zeroed for every query row (decode) or null
+    uint32_t *hist;          // [B][H_q][hist_row_words] zeroed (decode) or null
+    int64_t hist_row_words;  // n_tiles * kHistStride
     uint32_t *cnt_attn;      // zeroed for every query row (decode) or null
     uint32_t *ws_header;     // {magic, B} written (decode) or null
     int64_t n_cap, max_seq_len;
@@ -108,10 +109,8 @@ struct ScoreArgs {
     const int32_t *seq_len;
     uint8_t *dist;           // [B][H_q][dist_row]
     int64_t dist_row;
-    uint32_t *cum;           // [B][H_q][n_chunks][kCumStride]
-    uint32_t *hist_total;    // [B][H_q][kHistStride]
-    uint32_t *flags;         // per-b flag words
-    int64_t n_cap, max_seq_len, n_chunks;
+    uint32_t *hist;          // [B][H_q][n_tiles][kHistStride], zeroed by prep
+    int64_t n_cap, max_seq_len, n_tiles;
     int B, H_q, H_kv, G, zgroups;
 };
 
@@ -119,10 +118,9 @@ struct SelectArgs {
     const int32_t *seq_len;
     const uint8_t *dist;
     int64_t dist_row;
-    const uint32_t *cum;
-    const uint32_t *hist_total;
+    const uint32_t *hist;    // [B][H_q][n_tiles][kHistStride]
     int32_t *idx;            // [B][H_q][topk] ascending, -1 padded
-    int64_t n_cap, max_seq_len, n_chunks;
+    int64_t n_cap, max_seq_len, n_tiles;
     int B, H_q, topk;
 };
 

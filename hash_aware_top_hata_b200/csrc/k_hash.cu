@@ -20,6 +20,7 @@
 // optionally its K/V rows) and clears the per-step counters the scoring
 // kernel accumulates into.
 #include "hata_internal.cuh"
+#include "tma.cuh"
 
 namespace hata {
 namespace {
@@ -115,79 +116,111 @@ __global__ void __launch_bounds__(kD) hash_prefill_kernel(const void *__restrict
 
 // --------------------------------------------------------- decode prep --
 // Rows of KV head h: B*G query rows (b-major), then B appended-key rows.
+// A CTA takes kPrepRows rows of one head with 128 threads per row (thread j
+// of a row owns bit j).  The head's W_H is staged once in shared memory
+// (asynchronous 16-byte copies by all threads) next to the rows, so every
+// step of a chain reads its two operands from shared memory at addresses
+// known in advance: the loads run ahead of the dependent FMAs instead of
+// exposing their latency at each of the 128 steps.
+constexpr int kPrepThreads = kD * kPrepRows;
+
 template <bool BF16>
-__global__ void __launch_bounds__(kD) prep_kernel(PrepArgs a)
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
 {
-    constexpr int R = kPrepRows;
-    const int h = blockIdx.y, j = threadIdx.x;
+    const int h = blockIdx.y;
+    const int r = threadIdx.x / kD, j = threadIdx.x % kD;
     const int nq = a.q ? a.B * a.G : 0;
     const int nk = a.k_new ? a.B : 0;
     const int rows = nq + nk;
-    const int r0 = blockIdx.x * R;
+    const int r0 = blockIdx.x * kPrepRows;
+    const int row = r0 + r;
 
-    if (a.ws_header && blockIdx.x == 0 && h == 0 && j == 0) {
+    if (a.ws_header && blockIdx.x == 0 && h == 0 && threadIdx.x == 0) {
         a.ws_header[0] = kWsMagic;
         a.ws_header[1] = uint32_t(a.B);
     }
     if (r0 >= rows) return;
 
-    // column j of this head's W_H: 128 coalesced loads in flight while the
-    // rows are staged
-    float w[kD];
-    load_w_column(a.W + size_t(h) * kD * kRbit, j, w);
-    __shared__ __align__(16) float xs[kD * R];  // [kD][R]: the rows, one per column
-
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const int row = r0 + r;
-        float x = 0.0f;
-        if (row < nq) {
-            const int b = row / a.G, g = row % a.G, hq = h * a.G + g;
-            const size_t bh = size_t(b) * a.H_q + hq;
-            x = a.q[bh * kD + j];
-            if (a.hist_total)
-                for (int t = j; t < kHistStride; t += kD) a.hist_total[bh * kHistStride + t] = 0u;
-            if (a.cnt_attn && j == 0) a.cnt_attn[bh] = 0u;
-            if (a.flags && h == 0 && g == 0 && j == 0) {
-                const int64_t sl = a.seq_len[b];
-                uint32_t f = 0;
-                if (sl < 0 || sl > a.max_seq_len || sl > a.n_cap) f |= HATA_FLAG_SEQ_LEN_RANGE;
-                if (a.k_new && (sl - 1 < 0 || sl - 1 >= a.n_cap)) f |= HATA_FLAG_POS_RANGE;
-                a.flags[b] = f;
-            }
-        } else if (row < rows) {
-            const int b = row - nq;
-            x = load_x<BF16>(a.k_new, (int64_t(b) * a.H_kv + h) * kD + j);
-        }
-        xs[j * R + r] = x;
+    extern __shared__ __align__(16) float smem[];
+    float *ws = smem;                  // [kD][kRbit]: this head's W_H
+    float *xs = smem + kD * kRbit;     // [kPrepRows][kD]: the rows
+    {
+        const float *Wh = a.W + size_t(h) * kD * kRbit;
+        const uint32_t base = smem_addr(ws);
+        for (int c = threadIdx.x; c < kD * kRbit / 4; c += kPrepThreads)
+            cp_async16_zfill(base + 16u * c, Wh + 4 * c, 16u);
+        cp_async_commit();
     }
-    __syncthreads();
-    uint32_t words[R];
-    hash_group<R>(xs, w, words);
 
+    float x = 0.0f;
+    if (row < nq) {
+        const int b = row / a.G, g = row % a.G, hq = h * a.G + g;
+        const size_t bh = size_t(b) * a.H_q + hq;
+        x = a.q[bh * kD + j];
+        if (a.hist)
+            for (int64_t t = j; t < a.hist_row_words; t += kD) a.hist[bh * a.hist_row_words + t] = 0u;
+        if (a.cnt_attn && j == 0) a.cnt_attn[bh] = 0u;
+        if (a.flags && h == 0 && g == 0 && j == 0) {
+            const int64_t sl = a.seq_len[b];
+            uint32_t f = 0;
+            if (sl < 0 || sl > a.max_seq_len || sl > a.n_cap) f |= HATA_FLAG_SEQ_LEN_RANGE;
+            if (a.k_new && (sl - 1 < 0 || sl - 1 >= a.n_cap)) f |= HATA_FLAG_POS_RANGE;
+            a.flags[b] = f;
+        }
+    } else if (row < rows) {
+        const int b = row - nq;
+        x = load_x<BF16>(a.k_new, (int64_t(b) * a.H_kv + h) * kD + j);
+    }
+    xs[r * kD + j] = x;
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // the fixed-order chain acc = fmaf(x_i, W[i][j], acc), i = 0..127
+    // (operands of block i0 + 16 are loaded before block i0 is multiplied in)
+    constexpr int kBlk = 16;
+    const float4 *xr = reinterpret_cast<const float4 *>(xs + r * kD);
+    float xa[kBlk], wa[kBlk], xb[kBlk], wb[kBlk];
+    auto fetch = [&](int i0, float (&xv)[kBlk], float (&wv)[kBlk]) {
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const int row = r0 + r;
-        if (row < nq) {
-            if ((j & 31) == 0) {
-                const int b = row / a.G, g = row % a.G;
-                const size_t bh = size_t(b) * a.H_q + h * a.G + g;
-                a.q_out[bh * kWords + (j >> 5)] = words[r];
+        for (int k = 0; k < kBlk / 4; ++k) {
+            const float4 v = xr[i0 / 4 + k];
+            xv[4 * k] = v.x, xv[4 * k + 1] = v.y, xv[4 * k + 2] = v.z, xv[4 * k + 3] = v.w;
+        }
+#pragma unroll
+        for (int k = 0; k < kBlk; ++k) wv[k] = ws[(i0 + k) * kRbit + j];
+    };
+    float acc = 0.0f;
+    fetch(0, xa, wa);
+#pragma unroll
+    for (int i0 = 0; i0 < kD; i0 += 2 * kBlk) {
+        fetch(i0 + kBlk, xb, wb);
+#pragma unroll
+        for (int k = 0; k < kBlk; ++k) acc = __fmaf_rn(xa[k], wa[k], acc);
+        if (i0 + 2 * kBlk < kD) fetch(i0 + 2 * kBlk, xa, wa);
+#pragma unroll
+        for (int k = 0; k < kBlk; ++k) acc = __fmaf_rn(xb[k], wb[k], acc);
+    }
+    const uint32_t word = __ballot_sync(0xffffffffu, acc > 0.0f);
+
+    if (row < nq) {
+        if ((j & 31) == 0) {
+            const int b = row / a.G, g = row % a.G;
+            const size_t bh = size_t(b) * a.H_q + h * a.G + g;
+            a.q_out[bh * kWords + (j >> 5)] = word;
+        }
+    } else if (row < rows) {
+        const int b = row - nq;
+        const int64_t pos = a.pos ? int64_t(a.pos[b]) : int64_t(a.seq_len[b]) - 1;
+        if (pos >= 0 && pos < a.n_cap) {
+            const int64_t crow = (int64_t(b) * a.H_kv + h) * a.n_cap + pos;
+            if ((j & 31) == 0) a.codes[crow * kWords + (j >> 5)] = word;
+            if (a.v_new) {
+                const int64_t src = (int64_t(b) * a.H_kv + h) * kD + j;
+                store_x<BF16>(a.K, crow * kD + j, a.k_new, src);
+                store_x<BF16>(a.V, crow * kD + j, a.v_new, src);
             }
-        } else if (row < rows) {
-            const int b = row - nq;
-            const int64_t pos = a.pos ? int64_t(a.pos[b]) : int64_t(a.seq_len[b]) - 1;
-            if (pos >= 0 && pos < a.n_cap) {
-                const int64_t crow = (int64_t(b) * a.H_kv + h) * a.n_cap + pos;
-                if ((j & 31) == 0) a.codes[crow * kWords + (j >> 5)] = words[r];
-                if (a.v_new) {
-                    const int64_t src = (int64_t(b) * a.H_kv + h) * kD + j;
-                    store_x<BF16>(a.K, crow * kD + j, a.k_new, src);
-                    store_x<BF16>(a.V, crow * kD + j, a.v_new, src);
-                }
-            } else if (a.err_word && j == 0) {
-                atomicOr(a.err_word, HATA_FLAG_POS_RANGE);
-            }
+        } else if (a.err_word && j == 0) {
+            atomicOr(a.err_word, HATA_FLAG_POS_RANGE);
         }
     }
 }
@@ -208,11 +241,15 @@ cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const f
 
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s)
 {
+    constexpr size_t kSmem = sizeof(float) * (kD * kRbit + kD * kPrepRows);
+    const void *fn = a.kv_bf16 ? reinterpret_cast<const void *>(prep_kernel<true>)
+                               : reinterpret_cast<const void *>(prep_kernel<false>);
+    if (cudaError_t e = ensure_smem_attr(fn, kSmem)) return e;
     const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRows)), unsigned(a.H_kv));
     if (a.kv_bf16)
-        prep_kernel<true><<<grid, kD, 0, s>>>(a);
+        prep_kernel<true><<<grid, kPrepThreads, kSmem, s>>>(a);
     else
-        prep_kernel<false><<<grid, kD, 0, s>>>(a);
+        prep_kernel<false><<<grid, kPrepThreads, kSmem, s>>>(a);
     return cudaGetLastError();
 }
 

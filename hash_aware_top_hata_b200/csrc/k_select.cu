@@ -10,18 +10,16 @@
 //   S     = {n : dist[n] < T}  +  the r = k_eff - #(dist < T) lowest-index
 //           keys with dist[n] == T.
 //
-// Grid: (part, b * H_q + h_q), 256 threads.  A tile is 256 x 128 = 32K
-// tokens, each thread owning 128 consecutive distances (eight 16-byte
-// loads); the launcher splits each head's tiles into as many parts as fill
-// one wave of CTAs, and a CTA walks its part's tiles in order, carrying the
-// counts.  The CTA issues its first tile's loads, finds T from the head's
-// total histogram and -- for parts after the first -- the keys below T and
-// the boundary keys before the part from the scoring kernel's cumulative
-// chunk histograms.  Each thread turns its 128 distances into "< T" and
-// "== T" bit masks with byte-wise integer compares, ONE block scan of the
-// two counts gives every thread its output position, and the ties a thread
-// may take follow from the ties before it: taken_before = min(ties_before,
-// room).  Indices are written straight to the head's list, ascending.
+// Grid: (32K-token tile, b * H_q + h_q), 256 threads, each thread owning 128
+// consecutive distances (eight 16-byte loads, issued first).  Warp 0 sums
+// the head's tile histograms (written by the scoring kernel) while they are
+// in flight: the total gives T and r, the tiles before this one the keys
+// below T and at T already placed.
+// Each thread turns its 128 distances into "< T" and "== T" bit masks with
+// byte-wise integer compares, ONE block scan of the two counts gives every
+// thread its output position, and the ties a thread may take follow from
+// the ties before it: taken_before = min(ties_before, room).  Indices are
+// written straight to the head's list, ascending.
 #include "block_scan.cuh"
 #include "hata_internal.cuh"
 
@@ -33,9 +31,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kPer = 128;                               // distances per thread
 constexpr int kPieces = kPer / 16;                      // 16-byte loads per thread
 constexpr int kGroups = kPer / 32;                      // 32-distance mask words
-constexpr int64_t kTile = int64_t(kThreads) * kPer;     // 32K tokens
-static_assert(kTile % kChunk == 0, "a tile is whole scoring chunks");
-constexpr int kTileChunks = int(kTile / kChunk);
+static_assert(kThreads * kPer == kTile, "a CTA covers one histogram tile per pass");
 
 __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
 {
@@ -63,21 +59,6 @@ __device__ __forceinline__ uint32_t byte_eq_mask(uint32_t w, uint32_t T4)
     return ~(t | x) & 0x80808080u;
 }
 
-// Block-wide sum of a 64-bit value (all threads get the total).
-__device__ __forceinline__ int64_t block_sum64(int64_t v, int64_t *scratch)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    int64_t t = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) t += scratch[w];
-    __syncthreads();
-    return t;
-}
-
 // Mask word of 32 distances, bit 8e + w <-> distance 4w + e; the same bits
 // in token order (bit 4w + e).  Only words that select something need it.
 __device__ __forceinline__ uint32_t to_token_order(uint32_t m)
@@ -92,167 +73,188 @@ __device__ __forceinline__ uint32_t to_token_order(uint32_t m)
     return t;
 }
 
-__global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a, int parts)
+// T = the smallest distance t with #(dist <= t) >= k_eff, #(dist < T), and
+// the keys below T and at T in the tiles before `tile`, from head bh's tile
+// histograms.  One warp; lane l owns bins 5l .. 5l+4; out: {T, #(< T),
+// below-T before the tile, at-T before the tile}.
+__device__ __forceinline__ void head_threshold(const SelectArgs &a, size_t bh, int k_eff, int tile,
+                                               int lane, int *out)
+{
+    constexpr int kRegTiles = 8;  // rows held in registers: one round trip to L2
+    const uint32_t *hrow = a.hist + bh * size_t(a.n_tiles) * kHistStride;
+    const int n_tiles = int(a.n_tiles);
+    auto row_bins = [&](int t, uint32_t (&v)[5]) {
+#pragma unroll
+        for (int e = 0; e < 5; ++e)
+            v[e] = lane * 5 + e < kBins ? __ldg(hrow + t * kHistStride + lane * 5 + e) : 0u;
+    };
+    uint32_t rv[kRegTiles][5];
+#pragma unroll
+    for (int t = 0; t < kRegTiles; ++t) {
+        if (t < n_tiles) {
+            row_bins(t, rv[t]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 5; ++e) rv[t][e] = 0u;
+        }
+    }
+    uint32_t tot[5] = {0u, 0u, 0u, 0u, 0u}, pre[5] = {0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int t = 0; t < kRegTiles; ++t)
+#pragma unroll
+        for (int e = 0; e < 5; ++e) {
+            tot[e] += rv[t][e];
+            pre[e] += t < tile ? rv[t][e] : 0u;
+        }
+    for (int t = kRegTiles; t < n_tiles; ++t) {  // long contexts only
+        uint32_t v[5];
+        row_bins(t, v);
+#pragma unroll
+        for (int e = 0; e < 5; ++e) {
+            tot[e] += v[e];
+            pre[e] += t < tile ? v[e] : 0u;
+        }
+    }
+    const uint32_t run = tot[0] + tot[1] + tot[2] + tot[3] + tot[4];
+    uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
+    int Tl = -1;
+    uint32_t less_l = 0;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+        if (Tl < 0 && lane * 5 + e < kBins && acc + tot[e] >= uint32_t(k_eff)) {
+            Tl = lane * 5 + e;
+            less_l = acc;
+        }
+        acc += tot[e];
+    }
+    // cumulative counts are monotone: the lowest lane that found a bin holds T
+    const unsigned found = __ballot_sync(0xffffffffu, Tl >= 0);
+    const int src = found ? __ffs(int(found)) - 1 : 0;
+    const int T = found ? __shfl_sync(0xffffffffu, Tl, src) : 128;  // unreachable fallback
+    const int n_less = found ? __shfl_sync(0xffffffffu, int(less_l), src) : 0;
+    int l = 0, q = 0;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+        const int bin = lane * 5 + e;
+        l += bin < T ? int(pre[e]) : 0;
+        q += bin == T ? int(pre[e]) : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+        q += __shfl_xor_sync(0xffffffffu, q, o);
+    }
+    if (lane == 0) {
+        out[0] = T;
+        out[1] = n_less;
+        out[2] = l;
+        out[3] = q;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
 {
     pdl_trigger();
-    pdl_wait();  // distances and histograms of the scoring kernel
-    const int part = blockIdx.x;
+    pdl_wait();  // distances and tile histograms of the scoring kernel
+    const int tile = blockIdx.x;
     const size_t bh = blockIdx.y;
-    const int b = int(bh / a.H_q);
-    const int64_t len = clamp_len(a.seq_len[b], a.max_seq_len, a.n_cap);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int k_eff = int(int64_t(a.topk) < len ? int64_t(a.topk) : len);
+    const int b = int(bh) / a.H_q;
+    const int len = int(clamp_len(a.seq_len[b], a.max_seq_len, a.n_cap));
+    const int tid = threadIdx.x;
+    const int k_eff = a.topk < len ? a.topk : len;
     int32_t *idx = a.idx + bh * a.topk;
-    const int64_t n_tiles = ceil_div(len, kTile);
-    const int64_t t_beg = int64_t(part) * n_tiles / parts;
-    const int64_t t_end = int64_t(part + 1) * n_tiles / parts;
 
     __shared__ int2 scan_s[kWarps + 1];
-    __shared__ int64_t red_s[kWarps];
-    __shared__ int s_T, s_nless;
+    __shared__ int s_thr[4];
 
-    if (part == 0)
+    if (tile == 0)
         for (int i = k_eff + tid; i < a.topk; i += kThreads) idx[i] = -1;
-    if (k_eff <= 0 || t_beg >= t_end) return;
+    if (k_eff <= 0 || tile * kTile >= len) return;
 
+    // this thread's 128 distances (bytes past the row read as padding)
     const uint8_t *drow = a.dist + bh * a.dist_row;
-    // this thread's 128 distances of tile t (bytes past the row read as padding)
+    const int my0 = tile * kTile + tid * kPer;
     uint4 dv[kPieces];
-    auto load_tile = [&](int64_t t) {
-        const int64_t my0 = t * kTile + int64_t(tid) * kPer;
 #pragma unroll
-        for (int v = 0; v < kPieces; ++v) {
-            const int64_t o = my0 + 16 * v;
-            dv[v] = o < a.dist_row ? __ldg(reinterpret_cast<const uint4 *>(drow + o))
-                                   : make_uint4(~0u, ~0u, ~0u, ~0u);
-        }
-    };
-    load_tile(t_beg);  // in flight while T and the offsets are found
+    for (int v = 0; v < kPieces; ++v)
+        dv[v] = my0 + 16 * v < a.dist_row
+                    ? __ldg(reinterpret_cast<const uint4 *>(drow + my0 + 16 * v))
+                    : make_uint4(~0u, ~0u, ~0u, ~0u);
 
-    // ---- T from the head's total histogram ----
-    if (warp == 0) {
-        const uint32_t *ht = a.hist_total + bh * kHistStride;
-        uint32_t v[5];
-        uint32_t run = 0;
-#pragma unroll
-        for (int e = 0; e < 5; ++e) {
-            const int t = lane * 5 + e;
-            v[e] = t < kBins ? __ldg(ht + t) : 0u;
-            run += v[e];
-        }
-        uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
-        int T = -1;
-        uint32_t less = 0;
-#pragma unroll
-        for (int e = 0; e < 5; ++e) {
-            if (T < 0 && lane * 5 + e < kBins && acc + v[e] >= uint32_t(k_eff)) {
-                T = lane * 5 + e;
-                less = acc;
-            }
-            acc += v[e];
-        }
-        // cumulative counts are monotone: the lowest lane that found a bin holds T
-        const unsigned found = __ballot_sync(0xffffffffu, T >= 0);
-        const int src = found ? __ffs(int(found)) - 1 : 0;
-        const int Tf = __shfl_sync(0xffffffffu, T, src);
-        const int nl = __shfl_sync(0xffffffffu, int(less), src);
-        if (lane == 0) {
-            s_T = found ? Tf : 128;  // unreachable fallback: every key qualifies
-            s_nless = found ? nl : 0;
-        }
-    }
+    // ---- warp 0: T, #(dist < T) and the keys below T / at T in the tiles
+    // before this one, from the head's tile histograms (one round trip to L2
+    // for up to kRegTiles tiles, overlapping the distance loads) ----
+    if (tid < 32) head_threshold(a, bh, k_eff, tile, tid, s_thr);
     __syncthreads();
-    const int T = s_T;
-    const int r_ties = k_eff - s_nless;  // boundary keys taken over the whole head
+    const int T = s_thr[0], n_less = s_thr[1], lp = s_thr[2], tp = s_thr[3];
+    const int r_ties = k_eff - n_less;  // boundary keys taken over the whole head
+    const int less_before = lp, ties_before = tp;
+    if (less_before + (ties_before < r_ties ? ties_before : r_ties) >= k_eff)
+        return;  // every key of the head is placed before this tile (CTA-uniform)
 
-    // ---- keys (< T) and boundary keys (== T) before this part ----
-    int64_t less_before = 0, ties_before = 0;
-    if (t_beg > 0) {
-        const int64_t c0 = t_beg * kTileChunks;
-        int64_t lsum = 0, tsum = 0;
-        for (int64_t cc = tid; cc < c0; cc += kThreads) {
-            const uint32_t *cp = a.cum + (bh * a.n_chunks + cc) * kCumStride;
-            const uint32_t le = T > 0 ? __ldg(cp + T - 1) : 0u;
-            lsum += le;
-            tsum += __ldg(cp + T) - le;
+    // ---- masks: group m = pieces 2m, 2m+1 = distances 32m .. 32m+31 ----
+    const uint32_t T4 = uint32_t(T) * 0x01010101u;
+    uint32_t lt_bits[kGroups], eq_bits[kGroups];
+    int n_lt = 0, n_eq = 0;
+#pragma unroll
+    for (int m = 0; m < kGroups; ++m) {
+        const uint32_t dw[8] = {dv[2 * m].x,     dv[2 * m].y,     dv[2 * m].z,     dv[2 * m].w,
+                                dv[2 * m + 1].x, dv[2 * m + 1].y, dv[2 * m + 1].z, dv[2 * m + 1].w};
+        uint32_t lb = 0, eb = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            // flag of byte e at bit 8e + 7 -> bit 8e + w
+            lb |= byte_lt_mask(dw[w], T4) >> (7 - w);
+            eb |= byte_eq_mask(dw[w], T4) >> (7 - w);
         }
-        less_before = block_sum64(lsum, red_s);
-        ties_before = block_sum64(tsum, red_s);
+        lt_bits[m] = lb;
+        eq_bits[m] = eb;
+        n_lt += __popc(lb);
+        n_eq += __popc(eb);
     }
 
-    const uint32_t T4 = uint32_t(T) * 0x01010101u;
-    for (int64_t t = t_beg; t < t_end; ++t) {
-        if (less_before + (ties_before < r_ties ? ties_before : r_ties) >= k_eff) break;
-        if (t > t_beg) load_tile(t);
-        // ---- masks: group m = pieces 2m, 2m+1 = distances 32m .. 32m+31 ----
-        uint32_t lt_bits[kGroups], eq_bits[kGroups];
-        int n_lt = 0, n_eq = 0;
-#pragma unroll
-        for (int m = 0; m < kGroups; ++m) {
-            const uint32_t dw[8] = {dv[2 * m].x,     dv[2 * m].y,     dv[2 * m].z,
-                                    dv[2 * m].w,     dv[2 * m + 1].x, dv[2 * m + 1].y,
-                                    dv[2 * m + 1].z, dv[2 * m + 1].w};
-            uint32_t lb = 0, eb = 0;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                // flag of byte e at bit 8e + 7 -> bit 8e + w
-                lb |= byte_lt_mask(dw[w], T4) >> (7 - w);
-                eb |= byte_eq_mask(dw[w], T4) >> (7 - w);
-            }
-            lt_bits[m] = lb;
-            eq_bits[m] = eb;
-            n_lt += __popc(lb);
-            n_eq += __popc(eb);
-        }
+    int tile_lt, tile_eq;
+    const int2 before = block_exclusive_scan2<kThreads>(n_lt, n_eq, scan_s, &tile_lt, &tile_eq);
+    const int room = r_ties - ties_before > 0 ? r_ties - ties_before : 0;  // ties left
+    const int take_tile = room < tile_eq ? room : tile_eq;
+    const int taken_before = before.y < take_tile ? before.y : take_tile;
+    int my_take = take_tile - before.y;
+    my_take = my_take < 0 ? 0 : (my_take > n_eq ? n_eq : my_take);
 
-        int tile_lt, tile_eq;
-        const int2 before =
-            block_exclusive_scan2<kThreads>(n_lt, n_eq, scan_s, &tile_lt, &tile_eq);
-        const int64_t room = r_ties - ties_before > 0 ? r_ties - ties_before : 0;  // ties left
-        const int take_tile = int(room < tile_eq ? room : tile_eq);
-        const int taken_before = before.y < take_tile ? before.y : take_tile;
-        int my_take = take_tile - before.y;
-        my_take = my_take < 0 ? 0 : (my_take > n_eq ? n_eq : my_take);
-
-        int64_t pos = less_before + (ties_before < r_ties ? ties_before : r_ties) + before.x +
-                      taken_before;
-        const int32_t tok0 = int32_t(t * kTile + int64_t(tid) * kPer);
+    int pos = less_before + (ties_before < r_ties ? ties_before : r_ties) + before.x + taken_before;
 #pragma unroll
-        for (int m = 0; m < kGroups; ++m) {
-            uint32_t sel = lt_bits[m];
-            if (my_take > 0 && eq_bits[m]) {
-                const int ne = __popc(eq_bits[m]);
-                if (my_take >= ne) {  // every tie of this word
-                    sel |= eq_bits[m];
-                    my_take -= ne;
-                } else {              // the lowest-index my_take ties
-                    uint32_t eqt = to_token_order(eq_bits[m]);
-                    uint32_t selt = to_token_order(sel);
-                    for (; my_take > 0; --my_take) {
-                        selt |= eqt & (0u - eqt);
-                        eqt &= eqt - 1u;
-                    }
-                    while (selt) {
-                        const int e = __ffs(int(selt)) - 1;
-                        selt &= selt - 1u;
-                        if (pos < a.topk) idx[pos] = tok0 + 32 * m + e;
-                        ++pos;
-                    }
-                    continue;
+    for (int m = 0; m < kGroups; ++m) {
+        uint32_t sel = lt_bits[m];
+        if (my_take > 0 && eq_bits[m]) {
+            const int ne = __popc(eq_bits[m]);
+            if (my_take >= ne) {  // every tie of this word
+                sel |= eq_bits[m];
+                my_take -= ne;
+            } else {              // the lowest-index my_take ties
+                uint32_t eqt = to_token_order(eq_bits[m]), kept = 0u;
+                for (; my_take > 0; --my_take) {
+                    kept |= eqt & (0u - eqt);
+                    eqt &= eqt - 1u;
                 }
-            }
-            if (sel) {
-                uint32_t selt = to_token_order(sel);
+                uint32_t selt = to_token_order(sel) | kept;
                 while (selt) {
                     const int e = __ffs(int(selt)) - 1;
                     selt &= selt - 1u;
-                    if (pos < a.topk) idx[pos] = tok0 + 32 * m + e;
+                    if (pos < a.topk) idx[pos] = my0 + 32 * m + e;
                     ++pos;
                 }
+                continue;
             }
         }
-        less_before += tile_lt;
-        ties_before += tile_eq;
+        if (sel) {
+            uint32_t selt = to_token_order(sel);
+            while (selt) {
+                const int e = __ffs(int(selt)) - 1;
+                selt &= selt - 1u;
+                if (pos < a.topk) idx[pos] = my0 + 32 * m + e;
+                ++pos;
+            }
+        }
     }
 }
 
@@ -260,20 +262,10 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a, int p
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s)
 {
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel, kThreads, 0);
-    if (e != cudaSuccess) return e;
-    // as many parts per head as fill one wave (at least one, at most a tile each)
-    const int64_t heads = int64_t(a.B) * a.H_q;
-    const int64_t slots = int64_t(per_sm > 0 ? per_sm : 1) * sms;
-    const int64_t tiles = ceil_div(a.max_seq_len, kTile);
-    int64_t parts = slots / heads;
-    parts = parts < 1 ? 1 : (parts > tiles ? tiles : parts);
-    const dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(heads));
-    return launch_pdl(select_kernel, grid, dim3(kThreads), 0, s, a, int(parts));
+    // one CTA per (32K-token tile, head)
+    const dim3 grid(static_cast<unsigned>(ceil_div(a.max_seq_len, kTile)),
+                    static_cast<unsigned>(int64_t(a.B) * a.H_q));
+    return launch_pdl(select_kernel, grid, dim3(kThreads), 0, s, a);
 }
 
 }  // namespace hata
