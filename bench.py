@@ -119,7 +119,7 @@ def dist_setup(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        backend = "nccl" if args.impl == "hata" else "gloo"
+        backend = "nccl" if args.impl == "hata" and torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
@@ -138,41 +138,59 @@ def max_over_ranks(world, x: float) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 # ------------------------------------------------------------ oracle (CPU) --
 
+class OracleSample:
+    """A bounded sample of the workload for the CPU oracle: `n_heads` query
+    heads at context n_len, their slabs' key codes hashed once up front (the
+    decode step itself only hashes the query)."""
+
+    def __init__(self, cfg, w, n_heads: int, n_len: int):
+        import oracle
+        self.cfg, self.n_len = cfg, n_len
+        G = cfg.G
+        self.heads = [(b, hq) for b in range(cfg.B) for hq in range(cfg.H_q)][
+            :: max(1, cfg.B * cfg.H_q // n_heads)][:n_heads]
+        self.Wn = w.W_H.cpu().numpy()
+        self.slabs, self.codes = {}, {}
+        for b, hq in self.heads:
+            h = hq // G
+            if (b, h) not in self.slabs:
+                K = wl.to_numpy_kv(w.K[b, h, :n_len])
+                V = wl.to_numpy_kv(w.V[b, h, :n_len])
+                self.slabs[(b, h)] = (K, V)
+                self.codes[(b, h)] = oracle.hash_keys(K[None, None], self.Wn[h][None])[0, 0]
+        self.qs = {(b, hq): w.q[0, b, hq].cpu().numpy() for b, hq in self.heads}
+
+    def seconds_per_head(self) -> float:
+        """Time the oracle's decode step over the sample; seconds per head."""
+        import oracle
+        t0 = time.perf_counter()
+        for b, hq in self.heads:
+            h = hq // self.cfg.G
+            K, V = self.slabs[(b, h)]
+            oracle.decode_head(self.qs[(b, hq)], self.Wn[h], self.codes[(b, h)], K, V,
+                               self.n_len, self.cfg.topk, 1.0 / math.sqrt(128))
+        return (time.perf_counter() - t0) / len(self.heads)
+
+    def describe(self) -> str:
+        c = self.cfg
+        return (f"oracle decode (hash q, Hamming over {self.n_len} codes, sorted top-{c.topk}, "
+                f"fp64 attention) on {len(self.heads)} of {c.B * c.H_q} query heads, scaled to "
+                f"a full step; key codes hashed before timing")
+
+
 def oracle_sample(cfg, w, n_heads: int, n_len: int):
     """Time the CPU oracle on `n_heads` query heads of the workload at
     context n_len; returns (seconds per head, description)."""
-    import numpy as np
-    import oracle
-    G = cfg.G
-    heads = [(b, hq) for b in range(cfg.B) for hq in range(cfg.H_q)][:: max(1, cfg.B * cfg.H_q
-                                                                          // n_heads)][:n_heads]
-    Wn = w.W_H.cpu().numpy()
-    slabs, codes = {}, {}
-    for b, hq in heads:
-        h = hq // G
-        if (b, h) not in slabs:
-            K = wl.to_numpy_kv(w.K[b, h, :n_len])
-            V = wl.to_numpy_kv(w.V[b, h, :n_len])
-            slabs[(b, h)] = (K, V)
-            codes[(b, h)] = oracle.hash_keys(K[None, None], Wn[h][None])[0, 0]
-    qs = {(b, hq): w.q[0, b, hq].cpu().numpy() for b, hq in heads}
-    t0 = time.perf_counter()
-    for b, hq in heads:
-        h = hq // G
-        K, V = slabs[(b, h)]
-        oracle.decode_head(qs[(b, hq)], Wn[h], codes[(b, h)], K, V, n_len, cfg.topk,
-                           1.0 / math.sqrt(128))
-    el = time.perf_counter() - t0
-    desc = (f"oracle decode (hash q, Hamming over {n_len} codes, sorted top-{cfg.topk}, fp64 "
-            f"attention) on {len(heads)} of {cfg.B * cfg.H_q} query heads, scaled to a full step")
-    return el / len(heads), desc
+    s = OracleSample(cfg, w, n_heads, n_len)
+    return s.seconds_per_head(), s.describe()
 
 
 def bench_config(args):
@@ -192,16 +210,13 @@ def run_reference(args, world, rank):
     cfg = bench_config(args)
     w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config), device="cpu"
                          if not torch.cuda.is_available() else "cuda", steps=1)
-    per_head, desc = oracle_sample(cfg, w, n_heads=2, n_len=cfg.N)
+    sample = OracleSample(cfg, w, n_heads=2, n_len=cfg.N)
     heads_total = cfg.B * cfg.H_q
-    # each "step" re-times a bounded sample (two heads) and scales to the full step
-    import oracle  # noqa: F401
+    # each step times the same bounded sample (two heads) and scales it to a full step
     for _ in range(args.warmup):
-        oracle_sample(cfg, w, n_heads=1, n_len=cfg.N)
-    times = []
-    for _ in range(args.steps):
-        ph, _ = oracle_sample(cfg, w, n_heads=2, n_len=cfg.N)
-        times.append(ph * heads_total)
+        sample.seconds_per_head()
+    times = [sample.seconds_per_head() * heads_total for _ in range(args.steps)]
+    desc = sample.describe()
     us = statistics.mean(times) * 1e6
     line = {
         "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": UNIT,
