@@ -232,6 +232,24 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def profiled_traffic(cfg, kernel: str, src: str):
+    """DRAM bytes per launch of `kernel` from its committed ncu summary under
+    profiles/, or None when there is none for this workload or the kernel's
+    source has changed since the capture (hash recorded in the summary)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{cfg.name}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"sha256\[:16\] = `([0-9a-f]+)`", text)
+    m_traffic = re.search(r"traffic_mb: ([0-9.]+)", text)
+    if not (m_hash and m_traffic):
+        return None
+    now = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
+    return round(float(m_traffic.group(1)) * 1e6) if now == m_hash.group(1) else None
+
+
 def config_dict(cfg, l2: str) -> dict:
     return {"workload": cfg.name, "B": cfg.B, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
             "context": cfg.N, "topk": cfg.topk, "head_dim": 128, "rbit": 128,
@@ -383,7 +401,9 @@ def run_hata(args, world, rank, local):
         "config": config_dict(cfg, "flushed before every timed step (512 MiB read)"),
         "roofline": {"bound": "hbm", "kernel": "attend (gather + softmax)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(cfg, "attend_tc_kernel",
+                                                 "hash_aware_top_hata_b200/csrc/k_attend.cu"),
                      "peak_kind": peak_kind, "algorithmic_bytes_per_launch": attend_bytes},
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
                           "frac_of_measured": round(step_bytes / (ms / 1e3) / 1e9 / peak, 4),
