@@ -174,17 +174,17 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     // this thread's 128 distances (bytes past the row read as padding)
     const uint8_t *drow = a.dist + bh * a.dist_row;
     const int my0 = tile * kTile + tid * kPer;
+    // ---- warp 0 first finds T, #(dist < T) and the keys below T / at T in
+    // the tiles before this one from the head's tile histograms (one round
+    // trip to L2 for up to kRegTiles tiles), ahead of its own distance loads;
+    // the other warps' distance loads are in flight meanwhile ----
+    if (tid < 32) head_threshold(a, bh, k_eff, tile, tid, s_thr);
     uint4 dv[kPieces];
 #pragma unroll
     for (int v = 0; v < kPieces; ++v)
         dv[v] = my0 + 16 * v < a.dist_row
                     ? __ldg(reinterpret_cast<const uint4 *>(drow + my0 + 16 * v))
                     : make_uint4(~0u, ~0u, ~0u, ~0u);
-
-    // ---- warp 0: T, #(dist < T) and the keys below T / at T in the tiles
-    // before this one, from the head's tile histograms (one round trip to L2
-    // for up to kRegTiles tiles, overlapping the distance loads) ----
-    if (tid < 32) head_threshold(a, bh, k_eff, tile, tid, s_thr);
     __syncthreads();
     const int T = s_thr[0], n_less = s_thr[1], lp = s_thr[2], tp = s_thr[3];
     const int r_ties = k_eff - n_less;  // boundary keys taken over the whole head
