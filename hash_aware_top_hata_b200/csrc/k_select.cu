@@ -22,6 +22,7 @@
 // written straight to the head's list, ascending.
 #include "block_scan.cuh"
 #include "hata_internal.cuh"
+#include "tma.cuh"
 
 namespace hata {
 namespace {
@@ -166,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
 
     __shared__ int2 scan_s[kWarps + 1];
     __shared__ int s_thr[4];
+    __shared__ __align__(16) uint8_t dist_s[kThreads * kPer];  // the tile's distances
 
     if (tile == 0)
         for (int i = k_eff + tid; i < a.topk; i += kThreads) idx[i] = -1;
@@ -179,11 +181,29 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     // trip to L2 for up to kRegTiles tiles), ahead of its own distance loads;
     // the other warps' distance loads are in flight meanwhile ----
     if (tid < 32) head_threshold(a, bh, k_eff, tile, tid, s_thr);
+    // the warp's 4 KB arrive by coalesced 16-byte copies (lane l: bytes
+    // 16l .. 16l+15 of each 512-byte block) into a swizzled shared tile,
+    // piece v of thread t at t*128 + 16*(v ^ (t & 7)), so that each thread
+    // then reads its own 128 bytes without bank conflicts
+    const uint32_t sbase = smem_addr(dist_s);
+    const int wbase = (tid >> 5) * 32 * kPer;  // this warp's first byte in the tile
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) {
+        const int byte = wbase + k * 512 + (tid & 31) * 16;
+        const int t = byte >> 7, v = (byte >> 4) & 7;
+        const int64_t g = int64_t(tile) * kTile + byte;
+        const bool in = g < a.dist_row;  // past the row: no read (padding below)
+        cp_async16_zfill(sbase + uint32_t(t * kPer + 16 * (v ^ (t & 7))), in ? drow + g : drow,
+                         in ? 16u : 0u);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
     uint4 dv[kPieces];
 #pragma unroll
     for (int v = 0; v < kPieces; ++v)
         dv[v] = my0 + 16 * v < a.dist_row
-                    ? __ldg(reinterpret_cast<const uint4 *>(drow + my0 + 16 * v))
+                    ? *reinterpret_cast<const uint4 *>(dist_s + tid * kPer + 16 * (v ^ (tid & 7)))
                     : make_uint4(~0u, ~0u, ~0u, ~0u);
     __syncthreads();
     const int T = s_thr[0], n_less = s_thr[1], lp = s_thr[2], tp = s_thr[3];
