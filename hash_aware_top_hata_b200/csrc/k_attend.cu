@@ -507,8 +507,8 @@ __device__ __forceinline__ void attend_stage(int n, uint32_t Ks, const int32_t *
 }
 
 // A warp is done with head cs.bh: publish its partial (m, l, acc[128]); the
-// last of the head's contributors (fence + arrival counter, no waiting)
-// merges all partials into out = acc / l.
+// last of the head's contributors (acquire-release arrival counter, no
+// waiting) merges all partials into out = acc / l.
 __device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, int keff,
                                         int64_t wid, int64_t NW, int64_t T,
                                         const float (&O)[16][4], float m_ref, float l_part,
@@ -535,24 +535,34 @@ __device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, in
         pp[0] = m_ref;
         pp[1] = lw;
     }
-    __threadfence();
-    __syncwarp();
+    __syncwarp();  // the warp's partial writes happen before lane 0's release
     unsigned last = 0;
-    if (lane == 0) last = atomicAdd(a.cnt_attn + cs.bh, 1u) == uint32_t(n_contrib - 1);
+    if (lane == 0) {
+        uint32_t prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(prev)
+                     : "l"(a.cnt_attn + cs.bh)
+                     : "memory");
+        last = prev == uint32_t(n_contrib - 1);
+    }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
-    __threadfence();
-    float M = -INFINITY, L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    __threadfence();  // (last contributor only) every lane reads after the acquire
+    // merge: the global maximum first, then the rescaled sums, loads batched
     const float *pc = a.part + int64_t(cs.bh) * a.n_split * kPartStride;
-    for (int c = 0; c < n_contrib; ++c, pc += kPartStride) {
-        const float mc = __ldcg(pc), lc = __ldcg(pc + 1);
-        if (mc == -INFINITY) continue;
-        const float Mn = fmaxf(M, mc);
-        const float so = fast_exp2(M - Mn), sn = fast_exp2(mc - Mn);
-        L = L * so + lc * sn;
+    float M = -INFINITY;
+    for (int c = 0; c < n_contrib; ++c) M = fmaxf(M, __ldcg(pc + c * kPartStride));
+    float L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (M != -INFINITY) {
+#pragma unroll 4
+        for (int c = 0; c < n_contrib; ++c) {
+            const float *q = pc + c * kPartStride;
+            const float mc = __ldcg(q);
+            const float w = mc == -INFINITY ? 0.0f : fast_exp2(mc - M);
+            L += __ldcg(q + 1) * w;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) A[i] = A[i] * so + __ldcg(pc + 4 + lane + 32 * i) * sn;
-        M = Mn;
+            for (int i = 0; i < 4; ++i) A[i] += __ldcg(q + 4 + lane + 32 * i) * w;
+        }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
