@@ -313,10 +313,112 @@ def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, w
     return e2e_ms, h2d, d2h, dense_ms
 
 
+def more_legs(cfg, w, codes, ws, out, seq, flush, stream, t0, K_steps):
+    """Labelled side measurements of the same workload: warm-L2 step time,
+    needle recall, prefill key encoding against the FP32 peak, torch SDPA
+    dense decode, and K_steps consecutive decode steps replayed from one
+    CUDA Graph."""
+    B, Hq, Hkv, N, G = cfg.B, cfg.H_q, cfg.H_kv, cfg.N, cfg.G
+    scale = 1.0 / math.sqrt(128)
+    dev = out.device
+    res = {}
+
+    def ev_pair():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    # ---- warm L2: the same step with no flush in between ----
+    evs = [ev_pair() for _ in range(K_steps)]
+    for i in range(K_steps):
+        evs[i][0].record(stream)
+        H.hata_decode_step(w.q[t0 + i], w.W_H, codes, w.K, w.V, seq[t0 + i], w.n_cap, cfg.topk,
+                           scale, ws, out, k_new=w.k_new[t0 + i], v_new=w.v_new[t0 + i])
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    res["warm_l2_us"] = round(statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3, 2)
+
+    # ---- needle recall: needles kept in the selected set of each group's
+    # first query head (the head the needles point at) ----
+    if cfg.needles > 0:
+        sel = torch.empty((B, Hq, cfg.topk), dtype=torch.int32, device=dev)
+        H.hata_decode_step(w.q[0], w.W_H, codes, w.K, w.V, seq[t0 + K_steps], w.n_cap,
+                           cfg.topk, scale, ws, out, sel_idx=sel)
+        torch.cuda.synchronize()
+        sel_c = sel.cpu()
+        hits = total = 0
+        for b in range(B):
+            for h in range(Hkv):
+                nd = set(x for x in w.planted[b, h].tolist() if x >= 0)
+                got = set(sel_c[b, h * G].tolist())
+                hits += len(nd & got)
+                total += len(nd)
+        res["needle_recall"] = round(hits / max(total, 1), 4)
+
+    # ---- prefill key encoding (hata_hash_keys over the whole cache) ----
+    pe = [ev_pair() for _ in range(3)]
+    for i in range(4):
+        flush()
+        if i >= 1:
+            pe[i - 1][0].record(stream)
+        H.hata_hash_keys(w.K, w.W_H, codes, 0, N)
+        if i >= 1:
+            pe[i - 1][1].record(stream)
+    torch.cuda.synchronize()
+    t = statistics.median(a.elapsed_time(b) for a, b in pe) / 1e3
+    flops = 2.0 * B * Hkv * N * 128 * 128
+    fp32_peak = 148 * 128 * 2 * 1.965e9  # nominal: SMs x FP32 lanes x FMA x max clock
+    res["prefill_hash"] = {"us": round(t * 1e6, 1), "keys_per_s": round(B * Hkv * N / t, 0),
+                           "tflops": round(flops / t / 1e12, 2),
+                           "frac_of_fp32_nominal": round(flops / t / fp32_peak, 3)}
+
+    # ---- torch SDPA dense decode at the same shape (context) ----
+    try:
+        qs = w.q[0].to(w.K.dtype)[:, :, None, :]
+        Kd, Vd = w.K[:, :, :N], w.V[:, :, :N]
+        torch.nn.functional.scaled_dot_product_attention(qs, Kd, Vd, enable_gqa=True)
+        se = [ev_pair() for _ in range(5)]
+        for i in range(5):
+            flush()
+            se[i][0].record(stream)
+            torch.nn.functional.scaled_dot_product_attention(qs, Kd, Vd, enable_gqa=True)
+            se[i][1].record(stream)
+        torch.cuda.synchronize()
+        res["sdpa_dense_us"] = round(statistics.median(a.elapsed_time(b) for a, b in se) * 1e3, 1)
+    except Exception as e:  # an older torch without enable_gqa: not measured
+        res["sdpa_dense_us"] = None
+        res["sdpa_note"] = type(e).__name__
+
+    # ---- K_steps consecutive decode steps captured once and replayed ----
+    g = torch.cuda.CUDAGraph()
+    gs = torch.cuda.Stream()
+    gs.wait_stream(stream)
+    with torch.cuda.stream(gs):
+        with torch.cuda.graph(g, stream=gs):
+            for i in range(K_steps):
+                H.hata_decode_step(w.q[t0 + i], w.W_H, codes, w.K, w.V, seq[t0 + i], w.n_cap,
+                                   cfg.topk, scale, ws, out, k_new=w.k_new[t0 + i],
+                                   v_new=w.v_new[t0 + i])
+    stream.wait_stream(gs)
+    g.replay()  # warm
+    torch.cuda.synchronize()
+    gr = [ev_pair() for _ in range(3)]
+    for i in range(3):
+        flush()
+        gr[i][0].record(stream)
+        g.replay()
+        gr[i][1].record(stream)
+    torch.cuda.synchronize()
+    res["graph_us_per_step"] = round(
+        statistics.median(a.elapsed_time(b) for a, b in gr) * 1e3 / K_steps, 2)
+    res["graph_steps"] = K_steps
+    del g
+    return res
+
+
 def run_hata(args, world, rank, local):
     cfg = bench_config(args)
     K_steps, W_steps = args.steps, args.warmup
-    total_steps = W_steps + 3 * K_steps
+    G_steps = min(K_steps, 16)  # side legs: warm-L2 steps and the CUDA Graph
+    total_steps = W_steps + 3 * K_steps + G_steps + 1
     seed = wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config) + 1000 * rank
     dev = torch.device("cuda", torch.cuda.current_device())
     w = wl.make_workload(cfg, seed, device=dev, steps=total_steps)
@@ -381,9 +483,12 @@ def run_hata(args, world, rank, local):
     ms_max = max_over_ranks(world, ms)
 
     e2e_ms, h2d, d2h, dense_ms = float("nan"), 0, 0, float("nan")
+    side = None
     if not args.no_extras:
         e2e_ms, h2d, d2h, dense_ms = extras(args, cfg, w, codes, ws, out, seq, flush, stream,
                                             W_steps, K_steps, world)
+        side = more_legs(cfg, w, codes, ws, out, seq, flush, stream, W_steps + 3 * K_steps,
+                         G_steps)
     # ---- roofline ----
     peak, peak_kind = measured_peaks()
     kv_row = 128 * kv_elt
@@ -418,6 +523,7 @@ def run_hata(args, world, rank, local):
         "speedup_vs_dense": _num(dense_ms / ms, 2),
         "e2e": {"value": _num(e2e_ms * 1e3, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
+        "side": side,
         "gpu_launches": 4 * K_steps,
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
