@@ -82,8 +82,13 @@ cudaError_t ensure_smem_attr(const void *func, size_t bytes)
     const uint64_t bit = dev < 64 ? uint64_t(1) << dev : 0;
     std::lock_guard<std::mutex> lock(mu);
     if (bit && (done[func] & bit)) return cudaSuccess;
-    const cudaError_t e =
+    cudaError_t e =
         cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    // every kernel of the step prefers the largest shared-memory carveout, so
+    // the SMs keep one L1/shared split from kernel to kernel
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 int(cudaSharedmemCarveoutMaxShared));
     if (e == cudaSuccess) done[func] |= bit;
     return e;
 }

@@ -204,7 +204,8 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Records msg as hata_last_error() of this thread and returns st.
 hata_status_t report_error(hata_status_t st, const char *msg);
 
-// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+// Opt a kernel into `bytes` of dynamic shared memory (more than 48 KB needs
+// it) and the largest shared-memory carveout, once per device.
 cudaError_t ensure_smem_attr(const void *func, size_t bytes);
 
 // Launchers (each returns the cudaGetLastError() of its launch).

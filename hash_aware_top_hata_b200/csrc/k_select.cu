@@ -282,6 +282,8 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s)
 {
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(select_kernel), 0))
+        return e;
     // one CTA per (32K-token tile, head)
     const dim3 grid(static_cast<unsigned>(ceil_div(a.max_seq_len, kTile)),
                     static_cast<unsigned>(int64_t(a.B) * a.H_q));
