@@ -41,18 +41,11 @@ __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_
     return l < n_cap ? l : n_cap;
 }
 
-// Byte-wise compares of four distances (bytes of w: 0..128 or the pad 255)
-// against T (0..128, in every byte of T4), plain integer logic: bit 7 of
-// each byte of the result is the answer, the other bits are zero.
-//   d < T:  (d | 0x80) - T never borrows across bytes (T <= 128); its bit 7
-//           is set iff d >= T when d < 128, and d >= 128 is never below T.
-//   d == T: x = d ^ T is zero iff equal; (x & 0x7f) + 0x7f sets bit 7 iff
-//           the low seven bits of x are not all zero (no carry out).
-__device__ __forceinline__ uint32_t byte_lt_mask(uint32_t w, uint32_t T4)
-{
-    const uint32_t y = (w | 0x80808080u) - T4;
-    return ~(w | y) & 0x80808080u;
-}
+// Byte-wise zero test of four distances (bytes of w: 0..128 or the pad
+// 255) against T4 (one value in every byte), plain integer logic: bit 7 of
+// each byte of the result is set iff the byte equals T; the other bits are
+// zero.  x = d ^ T is zero iff equal; (x & 0x7f) + 0x7f sets bit 7 iff the
+// low seven bits of x are not all zero (no carry out).
 __device__ __forceinline__ uint32_t byte_eq_mask(uint32_t w, uint32_t T4)
 {
     const uint32_t x = w ^ T4;
@@ -213,24 +206,33 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
         return;  // every key of the head is placed before this tile (CTA-uniform)
 
     // ---- masks: group m = pieces 2m, 2m+1 = distances 32m .. 32m+31 ----
-    const uint32_t T4 = uint32_t(T) * 0x01010101u;
+    // "< T" and "<= T" from one (d | 0x80) per byte: (d | 0x80) - t never
+    // borrows for t <= 128, so only T = 128 (where "<= T" means "not the pad
+    // 255") needs the zero-byte test.  Ties = "<= T" and not "< T".  Flags
+    // move into the packed word with a multiply-high and an add (a right
+    // shift of the word so far; the bits never overlap).
+    const uint32_t T4 = uint32_t(T) * 0x01010101u, T4p = T4 + 0x01010101u;
     uint32_t lt_bits[kGroups], eq_bits[kGroups];
     int n_lt = 0, n_eq = 0;
 #pragma unroll
     for (int m = 0; m < kGroups; ++m) {
         const uint32_t dw[8] = {dv[2 * m].x,     dv[2 * m].y,     dv[2 * m].z,     dv[2 * m].w,
                                 dv[2 * m + 1].x, dv[2 * m + 1].y, dv[2 * m + 1].z, dv[2 * m + 1].w};
-        uint32_t lb = 0, eb = 0;
+        uint32_t lb = 0, le = 0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            // flag of byte e at bit 8e + 7 -> bit 8e + w
-            lb |= byte_lt_mask(dw[w], T4) >> (7 - w);
-            eb |= byte_eq_mask(dw[w], T4) >> (7 - w);
+            const uint32_t wh = dw[w] | 0x80808080u;
+            const uint32_t lt = ~(dw[w] | (wh - T4)) & 0x80808080u;
+            const uint32_t lq = T < 128 ? ~(dw[w] | (wh - T4p)) & 0x80808080u
+                                        : ~byte_eq_mask(dw[w], 0xffffffffu) & 0x80808080u;
+            // flag of byte e: bit 8e + 7 of word w -> bit 8e + w of the group
+            lb = __umulhi(lb, 0x80000000u) + lt;
+            le = __umulhi(le, 0x80000000u) + lq;
         }
         lt_bits[m] = lb;
-        eq_bits[m] = eb;
+        eq_bits[m] = le & ~lb;
         n_lt += __popc(lb);
-        n_eq += __popc(eb);
+        n_eq += __popc(eq_bits[m]);
     }
 
     int tile_lt, tile_eq;
