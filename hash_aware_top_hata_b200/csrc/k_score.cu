@@ -42,7 +42,7 @@ namespace {
 
 constexpr int kWarps = kScoreThreads / 32;  // 8
 constexpr int kUnit = 128;                  // tokens per warp step
-constexpr int kRing = 4;                    // units per warp ring
+constexpr int kRing = 2;                    // units per warp ring
 constexpr int kTileUnits = kTile / kUnit;   // 256
 constexpr int kMaxKeys = 3;                 // (slab, tile) histograms per CTA range
 
@@ -71,7 +71,7 @@ struct Slab {
 
 template <int GB>
 struct ScoreSmem {
-    uint4 ring[kWarps][kRing][kUnit];        // 64 KB of staged codes
+    uint4 ring[kWarps][kRing][kUnit];        // 32 KB of staged codes
     uint4 qs[kMaxKeys][GB];                  // query codes of each key's slab
     uint32_t hist[kMaxKeys][GB][kHistStride];
     uint8_t tile[kWarps][GB < 4 ? 4 : (GB + 3) / 4 * 4][kUnit];  // a unit's distances
@@ -112,7 +112,7 @@ __device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *q
 }
 
 template <int GB>
-__global__ void __launch_bounds__(kScoreThreads, 3) score_kernel(ScoreArgs a)
+__global__ void __launch_bounds__(kScoreThreads, 4) score_kernel(ScoreArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ScoreSmem<GB> &S = *reinterpret_cast<ScoreSmem<GB> *>(smem_raw);
