@@ -200,6 +200,8 @@ def bench_config(args):
     if args.context or args.batch:
         cfg = wl.scaled(cfg, N=args.context or cfg.N, B=args.batch or cfg.B,
                         topk=max(1, round(cfg.topk * (args.context or cfg.N) / cfg.N)))
+    if getattr(args, "topk", 0):
+        cfg = wl.scaled(cfg, N=cfg.N, topk=args.topk, name=f"{cfg.name}@k{args.topk}")
     return cfg
 
 
@@ -524,7 +526,7 @@ def run_hata(args, world, rank, local):
         "e2e": {"value": _num(e2e_ms * 1e3, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "side": side,
-        "gpu_launches": 4 * K_steps,
+        "gpu_launches": 5 * K_steps,  # prep, score, select, attend, combine
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
     }
@@ -547,6 +549,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--context", type=int, default=0, help="override the context length")
     ap.add_argument("--batch", type=int, default=0, help="override the batch size")
+    ap.add_argument("--topk", type=int, default=0, help="override the top-k budget")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e, dense and CPU legs (profiling runs)")
     args = ap.parse_args()

@@ -226,7 +226,6 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     int32_t *idx = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(ws + L.off_idx);
     uint32_t *flags = reinterpret_cast<uint32_t *>(ws + L.off_flags);
     uint32_t *hist = reinterpret_cast<uint32_t *>(ws + L.off_hist);
-    uint32_t *cnt_attn = reinterpret_cast<uint32_t *>(ws + L.off_cnt_attn);
     const Events ev{events, s};
     cudaError_t e;
 
@@ -245,7 +244,6 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     p.flags = flags;
     p.hist = hist;
     p.hist_row_words = L.n_tiles * kHistStride;
-    p.cnt_attn = cnt_attn;
     p.ws_header = reinterpret_cast<uint32_t *>(ws);
     p.n_cap = n_cap;
     p.max_seq_len = max_seq_len;
@@ -298,7 +296,6 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     aa.seq_len = seq_len;
     aa.idx = idx;
     aa.part = reinterpret_cast<float *>(ws + L.off_part);
-    aa.cnt_attn = cnt_attn;
     aa.flags = flags;
     aa.out = out;
     aa.n_cap = n_cap;

@@ -50,7 +50,7 @@ struct DecodeLayout {
     int zgroups = 0;        // ceil(G / kScoreHeads)
     int n_split = 0;        // attention partial slots per head
     size_t off_flags = 0, off_qcodes = 0, off_dist = 0, off_hist = 0, off_idx = 0,
-           off_part = 0, off_cnt_attn = 0, total = 0;
+           off_part = 0, total = 0;
 };
 
 inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
@@ -76,7 +76,6 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
     L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * L->n_tiles * kHistStride, 256);
     L->off_idx = o;        o = align_up(o + 4 * size_t(BH) * topk, 256);
     L->off_part = o;       o = align_up(o + 4 * size_t(BH) * L->n_split * kPartStride, 256);
-    L->off_cnt_attn = o;   o = align_up(o + 4 * size_t(BH), 256);
     L->total = o;
     return true;
 }
@@ -96,7 +95,6 @@ struct PrepArgs {
     uint32_t *err_word;      // single OR-ed word (append API) or null
     uint32_t *hist;          // [B][H_q][hist_row_words] zeroed (decode) or null
     int64_t hist_row_words;  // n_tiles * kHistStride
-    uint32_t *cnt_attn;      // zeroed for every query row (decode) or null
     uint32_t *ws_header;     // {magic, B} written (decode) or null
     int64_t n_cap, max_seq_len;
     int B, H_q, H_kv, G;
@@ -130,7 +128,6 @@ struct AttendArgs {
     const int32_t *seq_len;
     const int32_t *idx;      // [B][H_q][topk]
     float *part;             // [B][H_q][n_split][kPartStride]
-    uint32_t *cnt_attn;      // [B][H_q]
     uint32_t *flags;
     float *out;
     int64_t n_cap, max_seq_len;

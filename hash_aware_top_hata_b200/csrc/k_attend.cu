@@ -16,9 +16,10 @@
 // half of it).  Every 16-lane half-warp takes rows, computes q.k in fp32
 // with the softmax scale and log2(e) folded into q, and keeps an online
 // softmax state (m, l, acc[8 per lane]).  When a CTA leaves a head, its
-// eight half-warp states merge into one partial (m, l, acc[128]); the last
-// of the head's contributors to finish (fence + arrival counter, no
-// waiting) merges the partials into out = acc / l.
+// eight half-warp states merge into one partial (m, l, acc[128]) in the
+// head's slot for that CTA.  A separate combine launch (chained by
+// programmatic dependent launch) merges each head's slots into
+// out = acc / l, so no worker waits for another or merges behind the others.
 #include <cuda_bf16.h>
 
 #include "hata_internal.cuh"
@@ -152,7 +153,6 @@ __global__ void __launch_bounds__(kAttnThreads) attend_simt_kernel(AttendArgs a)
     pdl_wait();  // the selected index lists
     __shared__ float red_m[kHalves], red_l[kHalves];
     __shared__ __align__(16) float red_acc[kHalves][kD];
-    __shared__ int s_last;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int half = lane >> 4, l16 = lane & 15, hw = warp * 2 + half;
@@ -281,12 +281,7 @@ __global__ void __launch_bounds__(kAttnThreads) attend_simt_kernel(AttendArgs a)
 #pragma unroll
         for (int e = 0; e < 8; ++e) red_acc[hw][l16 * 8 + e] = acc[e];
         __syncthreads();
-        const int64_t h0 = int64_t(cs.bh) * a.topk;
-        const int ke = cons.keff;
-        const int64_t k_first = owner(h0, T, P);
-        const int64_t k_last = owner(h0 + (ke > 0 ? ke : 1) - 1, T, P);
-        const int slot_out = int(blockIdx.x - k_first);
-        const int n_contrib = int(k_last - k_first + 1);
+        const int slot_out = int(blockIdx.x - owner(int64_t(cs.bh) * a.topk, T, P));
         {
             float M = -INFINITY;
 #pragma unroll
@@ -306,25 +301,7 @@ __global__ void __launch_bounds__(kAttnThreads) attend_simt_kernel(AttendArgs a)
             }
             pp[4 + tid] = A;
         }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) s_last = atomicAdd(a.cnt_attn + cs.bh, 1u) == uint32_t(n_contrib - 1);
-        __syncthreads();
-        if (s_last) {
-            __threadfence();
-            float M = -INFINITY, L = 0.0f, A = 0.0f;
-            const float *pp = a.part + int64_t(cs.bh) * a.n_split * kPartStride;
-            for (int c = 0; c < n_contrib; ++c, pp += kPartStride) {
-                const float mc = __ldcg(pp), lc = __ldcg(pp + 1), ac = __ldcg(pp + 4 + tid);
-                if (mc == -INFINITY) continue;
-                const float Mn = fmaxf(M, mc);
-                const float so = exp2f(M - Mn), sn = exp2f(mc - Mn);
-                L = L * so + lc * sn;
-                A = A * so + ac * sn;
-                M = Mn;
-            }
-            a.out[int64_t(cs.bh) * kD + tid] = L > 0.0f ? A / L : 0.0f;
-        }
+        __syncthreads();  // red_* are rewritten by the next head
     }
     cp_async_wait<0>();
 }
@@ -343,18 +320,19 @@ __global__ void __launch_bounds__(kAttnThreads) attend_simt_kernel(AttendArgs a)
 // index list is loaded into shared memory up front, so no copy waits on an
 // index load.
 //
-// A warp computes S = q K^T and O += P V as mma.sync m16n8k16 bf16 tiles
-// with fp32 accumulation, fed by ldmatrix from an XOR-swizzled layout
-// (16-byte piece p of key row r sits at piece p ^ (r & 7), so the eight rows
-// one ldmatrix reads hit eight different bank groups).  The A operands are
-// the query (resp. the softmax weights) split into two bf16 rows,
-// hi = bf16(x) and lo = bf16(x - hi): rows 0 and 1 of the 16-row tile, whose
-// sum carries ~16 mantissa bits, so the tensor cores reproduce the fp32
-// result (the other 14 rows are zero).  The softmax rescale is lazy: the
-// reference maximum moves only when a score exceeds it by more than 2^8
-// (exact: weights stay <= 2^8), which skips rescaling the 64 accumulator
-// registers almost always.  When a warp leaves a head it publishes a partial
-// (m, l, acc[128]); the head's last contributor merges them.
+// A warp computes its 16-key stages as mma.sync m16n8k16 bf16 tiles with
+// fp32 accumulation and the keys along M: S^T = K Q^T, then O^T += V^T P^T,
+// 8 + 8 mma per stage, fed by ldmatrix (transposed for V) from an
+// XOR-swizzled layout (16-byte piece p of key row r sits at piece
+// p ^ (r & 7), so the eight rows one ldmatrix reads hit eight different bank
+// groups).  The B operands are the query (resp. the softmax weights) split
+// into two bf16 columns, hi = bf16(x) and lo = bf16(x - hi), whose sum
+// carries ~16 mantissa bits, so the tensor cores reproduce the fp32 result;
+// the two columns are summed inside a lane.  The softmax rescale is lazy:
+// the reference maximum moves only when a score exceeds it by more than 2^8
+// (exact: weights stay <= 2^8), which skips rescaling the 32 accumulator
+// registers almost always.  When a warp leaves a head it writes a partial
+// (m, l, acc[128]) for the combine kernel.
 namespace tc {
 
 constexpr int kSub = 16;                           // keys per stage
@@ -389,17 +367,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
                  : "r"(addr));
 }
 
-// d += A(16x16, rows 8..15 zero) * B(16x8); a0/a2: row g, k and k+8.
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
-                                         uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -421,67 +388,89 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// Per-lane ldmatrix offsets inside a stage (constant for a warp's life):
-// koff[kq]: key rows (lane & 7), 16-byte pieces kq*4 + (lane >> 3), for S;
-// voff[j2]: key rows (mi & 1)*8 + (lane & 7), pieces 2*j2 + (mi >> 1), for P V.
+// d += A(16x16) * B(16x8), all four A registers live.
+__device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Per-lane ldmatrix offsets inside a stage (constant for a warp's life).
+// Matrix mi = lane >> 3 of an x4 load, row lane & 7 of it:
+//   K (A = 16 keys x 16 dims of k-tile kt): key (mi & 1)*8 + (lane & 7),
+//     16-byte piece 2 kt + (mi >> 1);
+//   V (A = 16 dims of m-tile mt x 16 keys, transposed load): key
+//     (mi >> 1)*8 + (lane & 7), piece 2 mt + (mi & 1).
+// Piece 2t + b swizzles to (2t + b) ^ (r & 7) = ((b ^ (r & 7)) ^ 2t), so tile
+// t's offset is the tile-0 offset XOR (t << 5).
 struct LaneOffsets {
-    uint32_t koff[4], voff[8];
+    uint32_t k0, v0;
     __device__ __forceinline__ explicit LaneOffsets(int lane)
     {
-#pragma unroll
-        for (int kq = 0; kq < 4; ++kq) koff[kq] = swz(lane & 7, kq * 4 + (lane >> 3));
-        const int mi = lane >> 3;
-#pragma unroll
-        for (int j2 = 0; j2 < 8; ++j2) voff[j2] = swz((mi & 1) * 8 + (lane & 7), 2 * j2 + (mi >> 1));
+        const int mi = lane >> 3, r7 = lane & 7;
+        k0 = swz((mi & 1) * 8 + r7, mi >> 1);
+        v0 = swz((mi >> 1) * 8 + r7, mi & 1);
     }
+    __device__ __forceinline__ uint32_t k(int kt) const { return k0 ^ uint32_t(kt << 5); }
+    __device__ __forceinline__ uint32_t v(int mt) const { return v0 ^ uint32_t(mt << 5); }
 };
 
-// One 16-key stage of one warp: S = q K^T, online softmax, O += P V.
+// One 16-key stage of one warp.  Keys run along the M dimension of the
+// tiles: S^T = K Q^T with B = [q_hi q_lo 0 ...] (16 dims x 8 columns), then
+// O^T += V^T P^T with B = [p_hi p_lo 0 ...] (16 keys x 8 columns), so each
+// stage is 8 + 8 mma and the hi + lo columns are summed inside a lane.
+// Lane (g = lane / 4, t = lane % 4) of an m16n8 accumulator holds rows g and
+// g + 8, columns 2t and 2t + 1: only lanes with t == 0 see the two live
+// columns.  O[mt] in those lanes: dims 16 mt + g (O[mt][0] + O[mt][1]) and
+// 16 mt + g + 8 (O[mt][2] + O[mt][3]).
 __device__ __forceinline__ void attend_stage(int n, uint32_t Ks, const int32_t *rows,
-                                             const uint32_t (&qa)[8][2], const LaneOffsets &lo,
-                                             float (&O)[16][4], float &m_ref, float &l_part,
+                                             const uint32_t (&qb)[8][2], const LaneOffsets &lo,
+                                             float (&O)[8][4], float &m_ref, float &l_part,
                                              int lane)
 {
     const uint32_t Vs = Ks + kSub * kRowB;
-    const int q4 = lane & 3, part = (lane >> 2) & 1;
-    // ---- S = q K^T: two n-tiles of 8 keys; even / odd k-tiles accumulate
-    //      separately so each dependent mma chain is four deep ----
-    float S[2][2][4];
+    const int g = lane >> 2, t = lane & 3;
+    // keys of the stage that hold a row
+    const uint32_t vmask =
+        __ballot_sync(0xffffffffu, lane < kSub && lane < n && rows[lane < kSub ? lane : 0] >= 0);
+    // ---- S^T = K Q^T: even / odd k-tiles in separate accumulators ----
+    float S[2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int h = 0; h < 2; ++h) S[h][0] = S[h][1] = S[h][2] = S[h][3] = 0.0f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) S[nt][h][0] = S[nt][h][1] = S[nt][h][2] = S[nt][h][3] = 0.0f;
-#pragma unroll
-    for (int kq = 0; kq < 4; ++kq) {
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            uint32_t b0, b1, b2, b3;
-            // rows nt*8 + (lane & 7): the +8 row offset leaves the swizzle unchanged
-            ldsm_x4(Ks + nt * 8 * kRowB + lo.koff[kq], b0, b1, b2, b3);
-            mma16816(S[nt][0], qa[2 * kq][0], qa[2 * kq][1], b0, b1);
-            mma16816(S[nt][1], qa[2 * kq + 1][0], qa[2 * kq + 1][1], b2, b3);
-        }
+    for (int kt = 0; kt < 8; ++kt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(Ks + lo.k(kt), a0, a1, a2, a3);
+        mma16816_full(S[kt & 1], a0, a1, a2, a3, qb[kt][0], qb[kt][1]);
     }
-    // ---- scores of keys (nt*8 + 2*q4 + e): even + odd k-tiles, hi row + lo row ----
-    float sc[4] = {S[0][0][0] + S[0][1][0], S[0][0][1] + S[0][1][1], S[1][0][0] + S[1][1][0],
-                   S[1][0][1] + S[1][1][1]};
+    // lanes t == 0: key g (columns hi + lo) and key g + 8
+    const float s_g = (S[0][0] + S[1][0]) + (S[0][1] + S[1][1]);
+    const float s_g8 = (S[0][2] + S[1][2]) + (S[0][3] + S[1][3]);
+    // every lane takes keys 2t, 2t + 1, 2t + 8, 2t + 9 (the P^T fragment's rows)
+    float sc[4];
+    sc[0] = __shfl_sync(0xffffffffu, s_g, 8 * t);
+    sc[2] = __shfl_sync(0xffffffffu, s_g8, 8 * t);
+    sc[1] = __shfl_sync(0xffffffffu, s_g, 8 * t + 4);
+    sc[3] = __shfl_sync(0xffffffffu, s_g8, 8 * t + 4);
     bool valid[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        sc[e] += __shfl_xor_sync(0xffffffffu, sc[e], 4);
-        const int key = (e >> 1) * 8 + 2 * q4 + (e & 1);
-        valid[e] = lane < 8 && key < n && rows[key] >= 0;
+        const int key = 2 * t + (e & 1) + 8 * (e >> 1);
+        valid[e] = (vmask >> key) & 1u;
         if (!valid[e]) sc[e] = -INFINITY;
     }
     float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    mx = __shfl_sync(0xffffffffu, mx, 0);  // warp-uniform
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));  // the same in every lane
     if (mx == -INFINITY) return;
     if (mx > m_ref + kLazy) {
         const float alpha = fast_exp2(m_ref - mx);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
             O[j][0] *= alpha; O[j][1] *= alpha; O[j][2] *= alpha; O[j][3] *= alpha;
         }
         l_part *= alpha;
@@ -492,81 +481,42 @@ __device__ __forceinline__ void attend_stage(int n, uint32_t Ks, const int32_t *
     for (int e = 0; e < 4; ++e) {
         const float pe = valid[e] ? fast_exp2(sc[e] - m_ref) : 0.0f;
         l_part += pe;
-        pv[e] = split(pe, part);
+        pv[e] = split(pe, g & 1);
     }
-    const uint32_t a0 = lane < 8 ? pack2(pv[0], pv[1]) : 0u;
-    const uint32_t a2 = lane < 8 ? pack2(pv[2], pv[3]) : 0u;
-    // ---- O += P V: 16 n-tiles of 8 dims, one k-tile of 16 keys ----
+    const uint32_t b0 = g < 2 ? pack2(pv[0], pv[1]) : 0u;
+    const uint32_t b1 = g < 2 ? pack2(pv[2], pv[3]) : 0u;
+    // ---- O^T += V^T P^T: 8 m-tiles of 16 dims, one k-tile of 16 keys ----
 #pragma unroll
-    for (int j2 = 0; j2 < 8; ++j2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(Vs + lo.voff[j2], b0, b1, b2, b3);
-        mma16816(O[2 * j2], a0, a2, b0, b1);
-        mma16816(O[2 * j2 + 1], a0, a2, b2, b3);
+    for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(Vs + lo.v(mt), a0, a1, a2, a3);
+        mma16816_full(O[mt], a0, a1, a2, a3, b0, b1);
     }
 }
 
-// A warp is done with head cs.bh: publish its partial (m, l, acc[128]); the
-// last of the head's contributors (acquire-release arrival counter, no
-// waiting) merges all partials into out = acc / l.
-__device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, int keff,
-                                        int64_t wid, int64_t NW, int64_t T,
-                                        const float (&O)[16][4], float m_ref, float l_part,
-                                        int lane)
+// A warp is done with head cs.bh: write its partial (m, l, acc[128]) into
+// the head's slot for this worker; the combine kernel merges the slots.
+__device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, int64_t wid,
+                                        int64_t NW, int64_t T, const float (&O)[8][4],
+                                        float m_ref, float l_part, int lane)
 {
-    const int q4 = lane & 3;
-    const int64_t h0 = int64_t(cs.bh) * a.topk;
-    const int64_t k_first = owner(h0, T, NW);
-    const int64_t k_last = owner(h0 + (keff > 0 ? keff : 1) - 1, T, NW);
-    const int n_contrib = int(k_last - k_first + 1);
+    const int64_t k_first = owner(int64_t(cs.bh) * a.topk, T, NW);
     float *pp = a.part + (int64_t(cs.bh) * a.n_split + (wid - k_first)) * kPartStride;
-    float lw = lane < 4 ? l_part : 0.0f;  // lanes 4-7 repeat lanes 0-3's weights
+    float lw = lane < 4 ? l_part : 0.0f;  // lanes 0-3 hold all 16 keys of every stage
     lw += __shfl_xor_sync(0xffffffffu, lw, 1);
     lw += __shfl_xor_sync(0xffffffffu, lw, 2);
+    if ((lane & 3) == 0) {  // lane 4g: dims 16 mt + g and 16 mt + g + 8, hi + lo columns
+        const int g = lane >> 2;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const float o = O[j][e] + __shfl_xor_sync(0xffffffffu, O[j][e], 4);  // hi + lo rows
-            if (lane < 4) pp[4 + 8 * j + 2 * q4 + e] = o;
+        for (int mt = 0; mt < 8; ++mt) {
+            pp[4 + 16 * mt + g] = O[mt][0] + O[mt][1];
+            pp[4 + 16 * mt + g + 8] = O[mt][2] + O[mt][3];
         }
     }
     if (lane == 0) {
         pp[0] = m_ref;
         pp[1] = lw;
     }
-    __syncwarp();  // the warp's partial writes happen before lane 0's release
-    unsigned last = 0;
-    if (lane == 0) {
-        uint32_t prev;
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                     : "=r"(prev)
-                     : "l"(a.cnt_attn + cs.bh)
-                     : "memory");
-        last = prev == uint32_t(n_contrib - 1);
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) return;
-    __threadfence();  // (last contributor only) every lane reads after the acquire
-    // merge: the global maximum first, then the rescaled sums, loads batched
-    const float *pc = a.part + int64_t(cs.bh) * a.n_split * kPartStride;
-    float M = -INFINITY;
-    for (int c = 0; c < n_contrib; ++c) M = fmaxf(M, __ldcg(pc + c * kPartStride));
-    float L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int c = 0; c < n_contrib; ++c) {
-            const float *q = pc + c * kPartStride;
-            const float mc = __ldcg(q);
-            const float w = mc == -INFINITY ? 0.0f : fast_exp2(mc - M);
-            L += __ldcg(q + 1) * w;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) A[i] += __ldcg(q + 4 + lane + 32 * i) * w;
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        a.out[int64_t(cs.bh) * kD + lane + 32 * i] = L > 0.0f ? A[i] / L : 0.0f;
 }
 
 }  // namespace tc
@@ -577,7 +527,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     extern __shared__ __align__(128) uint8_t smem[];  // [warp][kRingW][K | V], then indices
     __shared__ int32_t rows_s[kTcWarps][kRingW][kSub];
     pdl_trigger();
-    pdl_wait();  // the selected index lists
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = int64_t(a.B) * a.H_q * a.topk;
@@ -590,22 +539,41 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     const uint8_t *Vg = static_cast<const uint8_t *>(a.V);
     const uint32_t wring = smem_addr(smem) + uint32_t(warp * kRingW * kStageBytes);
     int32_t *idx_s = reinterpret_cast<int32_t *>(smem + kRingBytes);
+    const int64_t beg = wid * T / NW, end = (wid + 1) * T / NW;
 
-    // the CTA's slice of the index list (the first kIdxCap of it), coalesced
+    // The walkers read only seq_len, a step input: set them up while the
+    // selection kernel is still running.
+    Walker<kSub> prod, cons;
+    if (wid < NW) {
+        prod.init(&a, beg, end);
+        cons.init(&a, beg, end);
+    }
+    pdl_wait();  // the selected index lists
+
+    // the CTA's slice of the index list (the first kIdxCap of it): all loads
+    // of a thread first, then the shared-memory stores
     if (cta_beg < cta_end) {
         const int64_t n_s = cta_end - cta_beg < kIdxCap ? cta_end - cta_beg : kIdxCap;
-        for (int64_t i = tid; i < n_s; i += kThreads) idx_s[i] = __ldg(a.idx + cta_beg + i);
+        constexpr int kPer = kIdxCap / kThreads;
+        static_assert(kIdxCap % kThreads == 0, "whole rounds of the slice load");
+        int32_t v[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int64_t i = tid + int64_t(u) * kThreads;
+            v[u] = i < n_s ? __ldg(a.idx + cta_beg + i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int64_t i = tid + int64_t(u) * kThreads;
+            if (i < n_s) idx_s[i] = v[u];
+        }
     }
     __syncthreads();
     if (wid >= NW) return;
-    const int64_t beg = wid * T / NW, end = (wid + 1) * T / NW;
     auto index_of = [&](int64_t x) {  // flat row -> key index
         return x - cta_beg < kIdxCap ? idx_s[x - cta_beg] : __ldg(a.idx + x);
     };
 
-    Walker<kSub> prod, cons;
-    prod.init(&a, beg, end);
-    cons.init(&a, beg, end);
     int64_t prod_x = beg;  // flat row of the producer walker's position
     int n_issued = 0;
     const int p = lane & 15, rb = lane >> 4;  // lane = piece p of rows rb, rb+2, ...
@@ -643,10 +611,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     for (int i = 0; i < kRingW - 1; ++i) issue_next();
 
     const int g4 = lane >> 2, q4 = lane & 3;   // mma fragment coordinates
-    const int part = g4 & 1;                    // lanes 0-3: hi row, 4-7: lo row
+    const int part = g4 & 1;                    // lanes 0-3: hi column, 4-7: lo column
     const LaneOffsets lo(lane);
-    uint32_t qa[8][2];
-    float O[16][4];
+    uint32_t qb[8][2];  // B operand of S^T: columns q_hi (lanes 0-3), q_lo (lanes 4-7)
+    float O[8][4];
     float m_ref = -INFINITY, l_part = 0.0f;
     int cur_bh = -1;
     Stage cs;
@@ -660,14 +628,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
                 if (lane < 8) {
                     const float2 x = __ldg(reinterpret_cast<const float2 *>(q + d0));
                     const float2 y = __ldg(reinterpret_cast<const float2 *>(q + d0 + 8));
-                    qa[kt][0] = pack2(split(x.x * a.scale_log2, part), split(x.y * a.scale_log2, part));
-                    qa[kt][1] = pack2(split(y.x * a.scale_log2, part), split(y.y * a.scale_log2, part));
+                    qb[kt][0] = pack2(split(x.x * a.scale_log2, part), split(x.y * a.scale_log2, part));
+                    qb[kt][1] = pack2(split(y.x * a.scale_log2, part), split(y.y * a.scale_log2, part));
                 } else {
-                    qa[kt][0] = qa[kt][1] = 0u;
+                    qb[kt][0] = qb[kt][1] = 0u;
                 }
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
+            for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
             m_ref = -INFINITY;
             l_part = 0.0f;
         }
@@ -676,12 +644,84 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
         __syncwarp();
         const int slot = s % kRingW;
         issue_next();
-        attend_stage(cs.n, wring + uint32_t(slot * kStageBytes), rows_s[warp][slot], qa, lo, O,
+        attend_stage(cs.n, wring + uint32_t(slot * kStageBytes), rows_s[warp][slot], qb, lo, O,
                      m_ref, l_part, lane);
 
-        if (cs.last) publish(a, cs, cons.keff, wid, NW, T, O, m_ref, l_part, lane);
+        if (cs.last) publish(a, cs, wid, NW, T, O, m_ref, l_part, lane);
     }
     cp_async_wait<0>();
+}
+
+// ------------------------------------------------------------------------
+// Combine: one warp per head merges the partials of the head's contributors
+// (workers k_first..k_last of the stream-K split) into out = acc / l.  It
+// runs as its own launch behind the attention kernel (programmatic
+// dependent launch: its CTAs are resident early and wait for the attention
+// grid to finish), so no attention worker waits for another or merges at
+// the end of its range.  The contributor count depends only on seq_len (a
+// step input), so it is known before the wait; after it, all loads of a
+// round of kCombineRound partials (lane c: m and l of contributor c; every
+// lane: its 4 output dims of each partial) are issued together, one
+// dependent memory round trip per round.
+constexpr int kCombineWarps = 4;
+constexpr int kCombineRound = 16;
+
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(AttendArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t bh = int64_t(blockIdx.x) * kCombineWarps + (threadIdx.x >> 5);
+    const bool live = bh < int64_t(a.B) * a.H_q;
+    int n_contrib = 0;
+    if (live) {
+        const int64_t T = int64_t(a.B) * a.H_q * a.topk, NW = a.n_workers;
+        const int b = int(bh / a.H_q);
+        const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);
+        const int64_t keff = int64_t(a.topk) < len ? int64_t(a.topk) : len;
+        const int64_t h0 = bh * a.topk;
+        n_contrib = int(owner(h0 + (keff > 0 ? keff : 1) - 1, T, NW) - owner(h0, T, NW) + 1);
+    }
+    pdl_wait();  // every partial is written
+    if (!live) return;
+    const float *pc = a.part + bh * a.n_split * kPartStride;
+    float M = -INFINITY, L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int c0 = 0; c0 < n_contrib; c0 += kCombineRound) {
+        const int c = c0 + lane;
+        const bool mine = lane < kCombineRound && c < n_contrib;
+        const float mc = mine ? __ldcg(pc + c * kPartStride) : -INFINITY;
+        const float lc = mine ? __ldcg(pc + c * kPartStride + 1) : 0.0f;
+        float acc[kCombineRound][4];
+#pragma unroll
+        for (int j = 0; j < kCombineRound; ++j) {
+            const float *q = pc + (c0 + j) * kPartStride + 4 + lane;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[j][i] = c0 + j < n_contrib ? __ldcg(q + 32 * i) : 0.0f;
+        }
+        float mr = mc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+        const float Mn = fmaxf(M, mr);
+        if (Mn == -INFINITY) continue;  // warp-uniform: no weight yet
+        if (M != Mn) {
+            const float r = M == -INFINITY ? 0.0f : exp2f(M - Mn);
+            L *= r;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) A[i] *= r;
+            M = Mn;
+        }
+        const float wc = mc == -INFINITY ? 0.0f : exp2f(mc - M);
+        float lw = lc * wc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+        L += lw;
+#pragma unroll
+        for (int j = 0; j < kCombineRound; ++j) {
+            const float w = __shfl_sync(0xffffffffu, wc, j);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) A[i] = fmaf(acc[j][i], w, A[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a.out[bh * kD + lane + 32 * i] = L > 0.0f ? A[i] / L : 0.0f;
 }
 
 template <typename Kernel>
@@ -697,6 +737,17 @@ cudaError_t occupancy_grid(Kernel kernel, int threads, size_t smem, int64_t *gri
     return e;
 }
 
+cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s)
+{
+    const int64_t heads = int64_t(a.B) * a.H_q;
+    // the same carveout as the attention kernel, so its CTAs can join the
+    // SMs without a shared-memory reconfiguration
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(combine_kernel), 0))
+        return e;
+    return launch_pdl(combine_kernel, dim3(unsigned(ceil_div(heads, kCombineWarps))),
+                      dim3(32 * kCombineWarps), 0, s, a);
+}
+
 }  // namespace
 
 cudaError_t launch_attend(const AttendArgs &args, bool bf16, cudaStream_t s)
@@ -710,8 +761,10 @@ cudaError_t launch_attend(const AttendArgs &args, bool bf16, cudaStream_t s)
         if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
         if (NW > T) NW = T;
         a.n_workers = NW;
-        return launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
-                          dim3(tc::kThreads), tc::kSmem, s, a);
+        if (cudaError_t e = launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
+                                       dim3(tc::kThreads), tc::kSmem, s, a))
+            return e;
+        return launch_combine(a, s);
     }
     constexpr size_t kSmemF32 = size_t(kRing) * Rows<false>::kSlotBytes;
     if (cudaError_t e = occupancy_grid(attend_simt_kernel<false>, kAttnThreads, kSmemF32, &P))
@@ -719,8 +772,10 @@ cudaError_t launch_attend(const AttendArgs &args, bool bf16, cudaStream_t s)
     if (P > kAttnMaxWorkers) P = kAttnMaxWorkers;
     if (P > T) P = T;
     a.n_workers = P;
-    return launch_pdl(attend_simt_kernel<false>, dim3(unsigned(P)), dim3(kAttnThreads), kSmemF32,
-                      s, a);
+    if (cudaError_t e = launch_pdl(attend_simt_kernel<false>, dim3(unsigned(P)),
+                                   dim3(kAttnThreads), kSmemF32, s, a))
+        return e;
+    return launch_combine(a, s);
 }
 
 }  // namespace hata

@@ -159,7 +159,6 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
         x = a.q[bh * kD + j];
         if (a.hist)
             for (int64_t t = j; t < a.hist_row_words; t += kD) a.hist[bh * a.hist_row_words + t] = 0u;
-        if (a.cnt_attn && j == 0) a.cnt_attn[bh] = 0u;
         if (a.flags && h == 0 && g == 0 && j == 0) {
             const int64_t sl = a.seq_len[b];
             uint32_t f = 0;

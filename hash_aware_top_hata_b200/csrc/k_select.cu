@@ -149,13 +149,13 @@ __device__ __forceinline__ void head_threshold(const SelectArgs &a, size_t bh, i
 __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
 {
     pdl_trigger();
-    pdl_wait();  // distances and tile histograms of the scoring kernel
     const int tile = blockIdx.x;
     const size_t bh = blockIdx.y;
     const int b = int(bh) / a.H_q;
-    const int len = int(clamp_len(a.seq_len[b], a.max_seq_len, a.n_cap));
+    const int len = int(clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap));  // step input
     const int tid = threadIdx.x;
     const int k_eff = a.topk < len ? a.topk : len;
+    pdl_wait();  // distances and tile histograms of the scoring kernel
     int32_t *idx = a.idx + bh * a.topk;
 
     __shared__ int2 scan_s[kWarps + 1];
