@@ -16,11 +16,11 @@ constexpr int kRbit = 128;      // hash bits (rbit = 128 on the HATA page)
 constexpr int kWords = kRbit / 32;
 constexpr int kBins = kRbit + 1;        // Hamming distances 0..128
 constexpr int kChunk = 4096;            // tokens per scoring / selection chunk
-constexpr int kScoreThreads = 256;
+constexpr int kScoreThreads = 1024;
 constexpr int kScoreHeads = 8;          // query heads scored per code load (one CTA)
 constexpr int kAttnThreads = 128;
 constexpr int kHistStride = 132;        // u32 per (head, tile) histogram row (129 bins)
-constexpr int kTile = 32768;            // tokens per histogram tile / selection tile
+constexpr int kTile = 36864;            // tokens per histogram tile / selection tile (9 x 4096)
 constexpr int kPartStride = 132;        // f32 per (head, chunk) partial: m, l, -, -, acc[128]
 constexpr int kPrepRows = 4;            // rows hashed together by one prep CTA
 constexpr uint8_t kDistPad = 255;       // distance stored past seq_len
@@ -46,7 +46,7 @@ inline int attn_max_contributors(int64_t BH, int topk)
 struct DecodeLayout {
     int64_t n_chunks = 0;   // 4096-token chunks of max_seq_len
     int64_t dist_row = 0;   // bytes per (b, h_q) distance row
-    int64_t n_tiles = 0;    // 32K-token histogram tiles of a distance row
+    int64_t n_tiles = 0;    // 36K-token histogram tiles of a distance row
     int zgroups = 0;        // ceil(G / kScoreHeads)
     int n_split = 0;        // attention partial slots per head
     size_t off_flags = 0, off_qcodes = 0, off_dist = 0, off_hist = 0, off_idx = 0,

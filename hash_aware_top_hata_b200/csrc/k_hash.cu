@@ -127,6 +127,7 @@ constexpr int kPrepThreads = kD * kPrepRows;
 template <bool BF16>
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
 {
+    pdl_trigger();  // the scoring kernel's setup (step inputs only) may start now
     const int h = blockIdx.y;
     const int r = threadIdx.x / kD, j = threadIdx.x % kD;
     const int nq = a.q ? a.B * a.G : 0;

@@ -28,12 +28,14 @@
 //
 // Per query head the kernel stores the u8 distance row (32 lanes write 32
 // consecutive bytes per store; the row stays L2-resident for the selection
-// kernel) and counts a 129-bin histogram per (head, 32K-token tile) in
+// kernel) and counts a 129-bin histogram per (head, 36K-token tile) in
 // shared memory; a range touches at most kMaxKeys (slab, tile) pairs.  At
 // the end of its range the CTA adds the non-zero bins into the tile
 // histograms in global memory (zeroed by the prep kernel), one reduction
 // per bin, so the selection kernel finds both the boundary distance and the
 // counts before any tile from them.
+#include <algorithm>
+
 #include "hata_internal.cuh"
 #include "tma.cuh"
 
@@ -43,8 +45,9 @@ namespace {
 constexpr int kWarps = kScoreThreads / 32;  // 8
 constexpr int kUnit = 128;                  // tokens per warp step
 constexpr int kRing = 2;                    // units per warp ring
-constexpr int kTileUnits = kTile / kUnit;   // 256
-constexpr int kMaxKeys = 3;                 // (slab, tile) histograms per CTA range
+constexpr int kTileUnits = kTile / kUnit;   // 288
+constexpr int kMaxKeys = 8;                 // (slab, tile) histograms per CTA range
+constexpr int kMaxRange = 2048;             // units per CTA range
 
 __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
 {
@@ -53,29 +56,22 @@ __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_
     return l < n_cap ? l : n_cap;
 }
 
-__device__ __forceinline__ int hamming128(const uint4 &k, const uint4 &q)
+// dist(k, q) with the XOR-ed words x_w = k_w ^ q_w, summed bit position by
+// bit position with a full adder and a half adder:
+//   x0 + x1 + x2 = s + 2c,  s = x0 ^ x1 ^ x2,  c = maj(x0, x1, x2)
+//   s + x3       = o + 2e,  o = s ^ x3,        e = s & x3
+// so dist = popc(o) + 2 (popc(c) + popc(e)).  s and o depend on the key only
+// through k0 ^ k1 ^ k2 and k0 ^ k1 ^ k2 ^ k3 (k012, k0123, shared by every
+// head of the group) and on the query through q012, q0123 (qd).
+__device__ __forceinline__ int hamming128(const uint4 &k, uint32_t k012, uint32_t k0123,
+                                          const uint4 &q, const uint2 &qd)
 {
-    const uint32_t x0 = k.x ^ q.x, x1 = k.y ^ q.y, x2 = k.z ^ q.z, x3 = k.w ^ q.w;
-    const uint32_t s = x0 ^ x1 ^ x2;
+    const uint32_t x0 = k.x ^ q.x, x1 = k.y ^ q.y, x2 = k.z ^ q.z;
     const uint32_t c = (x0 & x1) | (x2 & (x0 ^ x1));
-    const uint32_t ones = s ^ x3, c2 = s & x3;
-    return __popc(ones) + 2 * __popc(c ^ c2) + 4 * __popc(c & c2);
+    const uint32_t o = k0123 ^ qd.y;
+    const uint32_t e = (k012 ^ qd.x) & (k.w ^ q.w);
+    return __popc(o) + 2 * (__popc(c) + __popc(e));
 }
-
-// One (b, h_kv, head group) slab.
-struct Slab {
-    int b, h, ng;
-    int64_t len;
-    size_t bh0;  // b * H_q + first query head of the group
-};
-
-template <int GB>
-struct ScoreSmem {
-    uint4 ring[kWarps][kRing][kUnit];        // 32 KB of staged codes
-    uint4 qs[kMaxKeys][GB];                  // query codes of each key's slab
-    uint32_t hist[kMaxKeys][GB][kHistStride];
-    uint8_t tile[kWarps][GB < 4 ? 4 : (GB + 3) / 4 * 4][kUnit];  // a unit's distances
-};
 
 // Histogram increment: one shared-memory reduction, no return value.
 __device__ __forceinline__ void red_shared_add1(uint32_t addr)
@@ -88,16 +84,24 @@ __device__ __forceinline__ void red_shared_add1(uint32_t addr)
 // bin d of head g (base hb).  kFull: all 128 tokens hold keys; otherwise the
 // tokens from nv on get the pad byte and no count.
 template <int GB, bool kFull>
-__device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *qs, int ng,
-                                           uint32_t tb, uint32_t hb, int lane, int nv)
+__device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *qs,
+                                           const uint2 *qd, int ng, uint32_t tb, uint32_t hb,
+                                           int lane, int nv)
 {
+    uint32_t k012[4], k0123[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        k012[i] = cur[i].x ^ cur[i].y ^ cur[i].z;
+        k0123[i] = k012[i] ^ cur[i].w;
+    }
 #pragma unroll
     for (int g = 0; g < GB; ++g) {
         if (g < ng) {
             const uint4 q = qs[g];
+            const uint2 qx = qd[g];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t d = uint32_t(hamming128(cur[i], q));
+                const uint32_t d = uint32_t(hamming128(cur[i], k012[i], k0123[i], q, qx));
                 const uint32_t t = tb + uint32_t(g * kUnit + 32 * i);
                 if (kFull || lane + 32 * i < nv) {
                     asm volatile("st.shared.u8 [%0], %1;" ::"r"(t), "r"(d) : "memory");
@@ -111,137 +115,148 @@ __device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *q
     }
 }
 
+// A (slab, tile) histogram key of the CTA range: where its rows live.
+struct KeyInfo {
+    uint4 q[kScoreHeads];  // query codes of the slab's heads
+    uint2 qd[kScoreHeads]; // their q0 ^ q1 ^ q2 and q0 ^ q1 ^ q2 ^ q3
+    int64_t code0;         // first code (uint4 index) of the slab
+    int64_t dist0;         // first distance byte of head 0 of the slab
+    int len, ng, slab, pad;
+};
+
 template <int GB>
-__global__ void __launch_bounds__(kScoreThreads, 4) score_kernel(ScoreArgs a)
+struct ScoreSmem {
+    uint4 ring[kWarps][kRing][kUnit];           // 2 KB per unit
+    KeyInfo key[kMaxKeys];
+    uint32_t hist[kMaxKeys][GB][kHistStride];
+    uint8_t tile[kWarps][GB < 4 ? 4 : (GB + 3) / 4 * 4][kUnit];  // a unit's distances
+    uint32_t unit[kMaxRange];                   // per unit of the range: key << 28 | unit in slab
+    int next;                                   // units of the range handed out
+};
+
+template <int GB>
+__global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ScoreSmem<GB> &S = *reinterpret_cast<ScoreSmem<GB> *>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_trigger();
-    pdl_wait();  // query codes, the appended key code and cleared histograms
 
     const int nu = int(a.dist_row / kUnit);  // units per slab (pads included)
     const int n_tiles = int(a.n_tiles);
     const int n_units = int(int64_t(a.B) * a.H_kv * a.zgroups * nu);
     const int f_beg = int(int64_t(blockIdx.x) * n_units / gridDim.x);
     const int f_end = int(int64_t(blockIdx.x + 1) * n_units / gridDim.x);
-    if (f_beg >= f_end) return;
-
-    auto slab_of = [&](int s) {
-        Slab r;
-        const int z = s % a.zgroups;
-        const int bh = s / a.zgroups;
-        r.h = bh % a.H_kv;
-        r.b = bh / a.H_kv;
-        r.len = clamp_len(__ldg(a.seq_len + r.b), a.max_seq_len, a.n_cap);
-        const int g0 = z * kScoreHeads;
-        r.ng = min(GB, a.G - g0);
-        r.bh0 = size_t(r.b) * a.H_q + size_t(r.h) * a.G + g0;
-        return r;
+    auto key_of = [&](int f) {
+        const int slab = f / nu;
+        return slab * n_tiles + (f - slab * nu) / kTileUnits;
     };
-    auto key_of = [&](int slab, int uis) { return slab * n_tiles + uis / kTileUnits; };
-    int k_lo, k_hi;
-    {
-        const int s0 = f_beg / nu, s1 = (f_end - 1) / nu;
-        k_lo = key_of(s0, f_beg - s0 * nu);
-        k_hi = key_of(s1, f_end - 1 - s1 * nu);
-    }
+    const int k_lo = key_of(f_beg), k_hi = key_of(f_end - 1);
+    const int n_keys = k_hi - k_lo + 1;
 
-    for (int i = tid; i < kMaxKeys * GB * kHistStride; i += kScoreThreads)
+    // ---- before the dependency wait: the range's keys (seq_len is a step
+    // input), cleared histograms, the unit counter ----
+    for (int i = tid; i < n_keys * GB * kHistStride; i += kScoreThreads)
         (&S.hist[0][0][0])[i] = 0u;
-    if (tid < kMaxKeys * GB * 4) {  // query codes of every key's slab
-        const int kk = tid / (GB * 4), g = (tid / 4) % GB, w = tid & 3;
-        uint32_t v = 0u;
-        if (k_lo + kk <= k_hi) {
-            const Slab r = slab_of((k_lo + kk) / n_tiles);
-            if (g < r.ng) v = __ldg(a.qcodes + (r.bh0 + g) * kWords + w);
-        }
-        reinterpret_cast<uint32_t *>(&S.qs[kk][g])[w] = v;
+    if (tid < n_keys) {
+        const int slab = (k_lo + tid) / n_tiles;
+        const int z = slab % a.zgroups, bh = slab / a.zgroups;
+        const int h = bh % a.H_kv, b = bh / a.H_kv;
+        const int g0 = z * kScoreHeads;
+        KeyInfo &K = S.key[tid];
+        K.len = int(clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap));
+        K.ng = min(GB, a.G - g0);
+        K.slab = slab;
+        K.code0 = (int64_t(b) * a.H_kv + h) * a.n_cap;
+        K.dist0 = (int64_t(b) * a.H_q + int64_t(h) * a.G + g0) * a.dist_row;
+    }
+    for (int u = tid; u < f_end - f_beg; u += kScoreThreads) {
+        const int f = f_beg + u, slab = f / nu;
+        S.unit[u] = uint32_t(key_of(f) - k_lo) << 28 | uint32_t(f - slab * nu);
+    }
+    if (tid == 0) S.next = 0;
+    pdl_wait();  // query codes, the appended key code and cleared tile histograms
+    if (tid < n_keys * GB) {
+        const int kk = tid / GB, g = tid % GB;
+        const int slab = (k_lo + kk) / n_tiles;
+        const int z = slab % a.zgroups, bh = slab / a.zgroups;
+        const int h = bh % a.H_kv, b = bh / a.H_kv;
+        const int g0 = z * kScoreHeads;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (g < min(GB, a.G - g0))
+            v = __ldg(reinterpret_cast<const uint4 *>(a.qcodes) +
+                      (size_t(b) * a.H_q + size_t(h) * a.G + g0 + g));
+        S.key[kk].q[g] = v;
+        const uint32_t q012 = v.x ^ v.y ^ v.z;
+        S.key[kk].qd[g] = make_uint2(q012, q012 ^ v.w);
     }
     __syncthreads();
 
+    // ---- units of the range go to warps on demand (one shared counter):
+    // the oldest warps of the SM, which the scheduler favours, take more,
+    // and every warp finishes within about one unit of the others ----
     const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes);
-    const int my_first = f_beg + warp;
-    const int my_n = my_first < f_end ? (f_end - 1 - my_first) / kWarps + 1 : 0;
-    constexpr int kStep = kWarps * kUnit;  // tokens between a warp's units
-
-    // ---- load side: unit j into ring slot j % kRing, kRing-1 units ahead.
-    // l_src points at token t0 + lane of the next unit, l_left = len - t0;
-    // both advance by kStep per unit and are rebuilt at a slab change.
-    int l_slab = my_first / nu, l_uis = my_first - l_slab * nu;
-    const uint4 *l_src = codes;
-    int l_left = 0;
-    auto l_rebuild = [&]() {
-        const Slab r = slab_of(l_slab);
-        l_src = codes + (int64_t(r.b) * a.H_kv + r.h) * a.n_cap + int64_t(l_uis) * kUnit + lane;
-        l_left = int(r.len - int64_t(l_uis) * kUnit);
+    const int n_range = f_end - f_beg;
+    auto grab = [&]() {
+        int u = 0;
+        if (lane == 0) u = atomicAdd(&S.next, 1);
+        return __shfl_sync(0xffffffffu, u, 0);
     };
-    l_rebuild();
-    auto issue = [&](int j) {
+    // issue the copies of unit u (range-relative) into ring slot `slot`
+    auto issue = [&](int u, int slot) {
         asm volatile("" ::: "memory");  // earlier reads of the ring stay before the copies
-        if (j < my_n) {
-            const uint32_t dst = smem_addr(&S.ring[warp][j % kRing][lane]);
+        if (u < n_range) {
+            const uint32_t e = S.unit[u];
+            const int uis = int(e & 0x0fffffffu);
+            const KeyInfo &K = S.key[e >> 28];
+            const int left = K.len - uis * kUnit;
+            const uint4 *src = codes + K.code0 + int64_t(uis) * kUnit + lane;
+            const uint32_t dst = smem_addr(&S.ring[warp][slot][lane]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const bool ok = lane + 32 * i < l_left;  // zero fill past len, no read
-                cp_async16_zfill(dst + 512u * i, ok ? l_src + 32 * i : codes, ok ? 16u : 0u);
-            }
-            l_uis += kWarps;
-            l_src += kStep;
-            l_left -= kStep;
-            if (l_uis >= nu) {
-                do {
-                    l_uis -= nu;
-                    ++l_slab;
-                } while (l_uis >= nu);
-                if (j + 1 < my_n) l_rebuild();
+                const bool ok = lane + 32 * i < left;  // zero fill past len, no read
+                cp_async16_zfill(dst + 512u * i, ok ? src + 32 * i : codes, ok ? 16u : 0u);
             }
         }
         cp_async_commit();
     };
-    for (int j = 0; j < kRing - 1; ++j) issue(j);
-
-    // ---- compute side: c_row = distance row of head 0 at t0, c_left = len - t0
-    int c_slab = my_first / nu, c_uis = my_first - c_slab * nu;
-    uint8_t *c_row = a.dist;
-    int c_left = 0, c_ng = 0, c_kbase = 0;
-    auto c_rebuild = [&]() {
-        const Slab r = slab_of(c_slab);
-        c_row = a.dist + r.bh0 * a.dist_row + int64_t(c_uis) * kUnit;
-        c_left = int(r.len - int64_t(c_uis) * kUnit);
-        c_ng = r.ng;
-        c_kbase = c_slab * n_tiles - k_lo;
-    };
-    c_rebuild();
     // lane l stores 16 bytes of head (g0 + l / 8) of a unit: its offset in
-    // the rows, fixed for the whole range
+    // the rows
     const int64_t lane_off = int64_t(lane >> 3) * a.dist_row + (lane & 7) * 16;
     const uint32_t tb = smem_addr(&S.tile[warp][0][0]) + uint32_t(lane);
 
-    for (int j = 0; j < my_n; ++j) {
-        issue(j + kRing - 1);
-        cp_async_wait<kRing - 1>();  // this lane's copies of unit j have landed
+    int u_cur = grab();
+    issue(u_cur, 0);
+    for (int j = 0; u_cur < n_range; ++j) {
+        const int u_next = grab();
+        issue(u_next, (j + 1) % kRing);
+        cp_async_wait<kRing - 1>();  // this lane's copies of the current unit have landed
         uint4 cur[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) cur[i] = S.ring[warp][j % kRing][lane + 32 * i];
-        const int kk = c_kbase + (c_uis >> 8);  // kTileUnits = 256 units per tile
+        const uint32_t e = S.unit[u_cur];
+        const int uis = int(e & 0x0fffffffu), kk = int(e >> 28);
+        const KeyInfo &K = S.key[kk];
+        const int c_left = K.len - uis * kUnit;
+        uint8_t *c_row = a.dist + K.dist0 + int64_t(uis) * kUnit;
         if (c_left <= 0) {
             // past seq_len: pad bytes only (4 per lane, 128 per head)
 #pragma unroll
             for (int g = 0; g < GB; ++g)
-                if (g < c_ng)
-                    reinterpret_cast<uint32_t *>(c_row + g * a.dist_row)[lane] = 0xffffffffu;
+                if (g < K.ng) reinterpret_cast<uint32_t *>(c_row + g * a.dist_row)[lane] = 0xffffffffu;
         } else {
             const uint32_t hb = smem_addr(&S.hist[kk][0][0]);
-            if (c_left >= kUnit)
-                score_unit<GB, true>(cur, S.qs[kk], c_ng, tb, hb, lane, kUnit);
+            if (c_left >= kUnit && K.ng == GB)
+                score_unit<GB, true>(cur, K.q, K.qd, GB, tb, hb, lane, kUnit);
+            else if (c_left >= kUnit)
+                score_unit<GB, true>(cur, K.q, K.qd, K.ng, tb, hb, lane, kUnit);
             else
-                score_unit<GB, false>(cur, S.qs[kk], c_ng, tb, hb, lane, c_left);
+                score_unit<GB, false>(cur, K.q, K.qd, K.ng, tb, hb, lane, c_left);
             __syncwarp();
             // the tile to the rows: lane l stores 16 bytes of head g0 + l / 8
 #pragma unroll
             for (int g0 = 0; g0 < GB; g0 += 4) {
-                if (g0 + (lane >> 3) < c_ng) {
+                if (g0 + (lane >> 3) < K.ng) {
                     const uint4 v = *reinterpret_cast<const uint4 *>(
                         &S.tile[warp][g0 + (lane >> 3)][(lane & 7) * 16]);
                     __stcg(reinterpret_cast<uint4 *>(c_row + g0 * a.dist_row + lane_off), v);
@@ -249,31 +264,35 @@ __global__ void __launch_bounds__(kScoreThreads, 4) score_kernel(ScoreArgs a)
             }
             __syncwarp();  // the tile is rewritten by the next unit
         }
-        c_uis += kWarps;
-        c_row += kStep;
-        c_left -= kStep;
-        if (c_uis >= nu) {
-            do {
-                c_uis -= nu;
-                ++c_slab;
-            } while (c_uis >= nu);
-            if (j + 1 < my_n) c_rebuild();
-        }
+        u_cur = u_next;
     }
     cp_async_wait<0>();
 
     // ---- publish: add the non-zero bins of every touched (slab, tile) ----
     __syncthreads();
-    const int n_keys = k_hi - k_lo + 1;
     for (int i = tid; i < n_keys * GB * kBins; i += kScoreThreads) {
         const int kk = i / (GB * kBins), g = (i / kBins) % GB, t = i % kBins;
         const uint32_t v = S.hist[kk][g][t];
-        if (v == 0u) continue;
+        if (v == 0u || g >= S.key[kk].ng) continue;
         const int key = k_lo + kk;
-        const Slab r = slab_of(key / n_tiles);
-        if (g < r.ng)
-            atomicAdd(a.hist + ((r.bh0 + g) * size_t(n_tiles) + key % n_tiles) * kHistStride + t, v);
+        atomicAdd(a.hist + (size_t(S.key[kk].dist0 / a.dist_row + g) * size_t(n_tiles) +
+                            key % n_tiles) * kHistStride + t,
+                  v);
     }
+}
+
+// Most (slab, tile) keys any CTA range touches when the U units are cut into
+// P ranges (keys are numbered in flat unit order, so a range [f0, f1) touches
+// key_of(f1 - 1) - key_of(f0) + 1 of them).
+inline int64_t max_keys_per_range(int64_t U, int64_t P, int64_t nu, int64_t n_tiles)
+{
+    auto key_of = [&](int64_t f) { return (f / nu) * n_tiles + (f % nu) / kTileUnits; };
+    int64_t m = 0;
+    for (int64_t c = 0; c < P; ++c) {
+        const int64_t f0 = c * U / P, f1 = (c + 1) * U / P;
+        if (f1 > f0) m = std::max(m, key_of(f1 - 1) - key_of(f0) + 1);
+    }
+    return m;
 }
 
 template <int GB>
@@ -288,17 +307,15 @@ cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_kernel<GB>,
                                                           kScoreThreads, sizeof(ScoreSmem<GB>));
     if (e != cudaSuccess) return e;
-    // One range per resident CTA, unless ranges would touch more than
-    // kMaxKeys = 3 (slab, tile) pairs.  Slabs of >= kTileUnits units: a range
-    // of <= kTileUnits units meets at most the end of one tile, a short last
-    // tile and the start of the next slab.  Shorter slabs are one key each:
-    // a range of <= 2 * nu units meets at most three of them.
+    // One range per resident CTA (one per SM); more ranges only if a range
+    // would touch more than kMaxKeys (slab, tile) histograms.
     const int64_t nu = a.dist_row / kUnit;
     const int64_t units = int64_t(a.B) * a.H_kv * a.zgroups * nu;
-    const int64_t max_range = nu >= kTileUnits ? kTileUnits : (kMaxKeys - 1) * nu;
-    int64_t P = int64_t(per_sm > 0 ? per_sm : 1) * sms;
-    if (P * max_range < units) P = ceil_div(units, max_range);
-    if (P > units) P = units;
+    const int64_t wave = int64_t(per_sm > 0 ? per_sm : 1) * sms;
+    int64_t P = wave < units ? wave : units;
+    while (P < units && (ceil_div(units, P) > kMaxRange ||
+                         max_keys_per_range(units, P, nu, a.n_tiles) > kMaxKeys))
+        P = P + wave < units ? P + wave : units;
     return launch_pdl(score_kernel<GB>, dim3(unsigned(P)), dim3(kScoreThreads), sizeof(ScoreSmem<GB>),
                       s, a);
 }

@@ -10,7 +10,7 @@
 //   S     = {n : dist[n] < T}  +  the r = k_eff - #(dist < T) lowest-index
 //           keys with dist[n] == T.
 //
-// Grid: (32K-token tile, b * H_q + h_q), 256 threads, each thread owning 128
+// Grid: (36K-token tile, b * H_q + h_q), 288 threads, each thread owning 128
 // consecutive distances (eight 16-byte loads, issued first).  Warp 0 sums
 // the head's tile histograms (written by the scoring kernel) while they are
 // in flight: the total gives T and r, the tiles before this one the keys
@@ -27,7 +27,7 @@
 namespace hata {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 288;  // 9 warps x 128 distances = one tile
 constexpr int kWarps = kThreads / 32;
 constexpr int kPer = 128;                               // distances per thread
 constexpr int kPieces = kPer / 16;                      // 16-byte loads per thread
@@ -286,7 +286,7 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t s)
 {
     if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(select_kernel), 0))
         return e;
-    // one CTA per (32K-token tile, head)
+    // one CTA per (36K-token tile, head)
     const dim3 grid(static_cast<unsigned>(ceil_div(a.max_seq_len, kTile)),
                     static_cast<unsigned>(int64_t(a.B) * a.H_q));
     return launch_pdl(select_kernel, grid, dim3(kThreads), 0, s, a);
