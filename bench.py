@@ -277,23 +277,22 @@ def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, w
     kn_h = w.k_new[t0:t0 + K_steps].cpu().pin_memory()
     vn_h = w.v_new[t0:t0 + K_steps].cpu().pin_memory()
     out_h = torch.empty((K_steps, B, Hq, 128)).pin_memory()
-    q_d, kn_d, vn_d = (torch.empty_like(x[0], device=dev) for x in (q_h, kn_h, vn_h))
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K_steps)]
+    # the step's inputs and its output stay in pinned host memory: the
+    # library's kernels read q, k_new, v_new over the bus and write out back
+    # (the public call with host pointers, no separate copy operations)
     for i in range(K_steps):
         flush()
         e2e_ev[i][0].record(stream)
-        q_d.copy_(q_h[i], non_blocking=True)
-        kn_d.copy_(kn_h[i], non_blocking=True)
-        vn_d.copy_(vn_h[i], non_blocking=True)
-        H.hata_decode_step(q_d, w.W_H, codes, w.K, w.V, seq[t0 + i], w.n_cap, cfg.topk, scale,
-                           ws, out, k_new=kn_d, v_new=vn_d)
-        out_h[i].copy_(out, non_blocking=True)
+        H.hata_decode_step(q_h[i], w.W_H, codes, w.K, w.V, seq[t0 + i], w.n_cap, cfg.topk, scale,
+                           ws, out_h[i], k_new=kn_h[i], v_new=vn_h[i])
         e2e_ev[i][1].record(stream)
+        e2e_ev[i][1].synchronize()  # a caller reads each step's output before the next
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(world, statistics.mean(a.elapsed_time(b) for a, b in e2e_ev))
-    h2d = q_d.numel() * 4 + (kn_d.numel() + vn_d.numel()) * kv_elt
-    d2h = out.numel() * 4
+    h2d = q_h[0].numel() * 4 + (kn_h[0].numel() + vn_h[0].numel()) * kv_elt
+    d2h = out_h[0].numel() * 4
 
     # ---- dense decode attention at the same shape (context for the speedup) ----
     dws = torch.empty(H.hata_dense_workspace_size(B, Hq, Hkv, w.n_cap), dtype=torch.uint8,

@@ -144,9 +144,9 @@ hata_status_t hata_append_code(const void *k_new, hata_dtype_t kv_dtype, const f
     if (B <= 0 || H_kv <= 0 || int64_t(B) * H_kv > (int64_t(1) << 24) || H_kv > 65535)
         return fail(HATA_ERR_INVALID_ARG, "B=%d H_kv=%d out of range", B, H_kv);
     if (n_cap <= 0) return fail(HATA_ERR_INVALID_ARG, "n_cap=%lld", (long long)n_cap);
-    if (!aligned(k_new, 4) || !aligned(codes, 16) || !aligned(pos, 4) || !aligned(W_H, 16) ||
+    if (!aligned(k_new, 16) || !aligned(codes, 16) || !aligned(pos, 4) || !aligned(W_H, 16) ||
         (err_flags && !aligned(err_flags, 4)))
-        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer");
+        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer (k_new, codes, W_H: 16 B)");
     PrepArgs a{};
     a.k_new = k_new;
     a.W = W_H;
@@ -199,10 +199,10 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
         return fail(HATA_ERR_INVALID_ARG, "scale must be finite");
     if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(codes, 16) ||
         !aligned(out, 16) || !aligned(W_H, 16) || !aligned(seq_len, 4) ||
-        (k_new && !aligned(k_new, 4)) || (v_new && !aligned(v_new, 4)) ||
+        (k_new && !aligned(k_new, 16)) || (v_new && !aligned(v_new, 16)) ||
         (sel_idx && !aligned(sel_idx, 4)) || (q_codes && !aligned(q_codes, 16)))
         return fail(HATA_ERR_INVALID_ARG,
-                    "misaligned pointer (q, W_H, K, V, codes, out, q_codes: 16 B)");
+                    "misaligned pointer (q, W_H, K, V, codes, out, k_new, v_new, q_codes: 16 B)");
     if (!aligned(workspace, 256)) return fail(HATA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     DecodeLayout L;
     if (!decode_layout(B, H_q, H_kv, max_seq_len, topk, &L))
@@ -231,8 +231,10 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
 
     if ((e = ev.record(0)) != cudaSuccess) return cuda_fail(e, "event record");
 
+    float *q_dev = reinterpret_cast<float *>(ws + L.off_q);
     PrepArgs p{};
     p.q = q;
+    p.q_copy = q_dev;
     p.k_new = k_new;
     p.v_new = v_new;
     p.W = W_H;
@@ -290,7 +292,7 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     if ((e = ev.record(3)) != cudaSuccess) return cuda_fail(e, "event record");
 
     AttendArgs aa{};
-    aa.q = q;
+    aa.q = q_dev;
     aa.K = K;
     aa.V = V;
     aa.seq_len = seq_len;

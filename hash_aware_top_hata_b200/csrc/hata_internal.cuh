@@ -49,7 +49,7 @@ struct DecodeLayout {
     int64_t n_tiles = 0;    // 36K-token histogram tiles of a distance row
     int zgroups = 0;        // ceil(G / kScoreHeads)
     int n_split = 0;        // attention partial slots per head
-    size_t off_flags = 0, off_qcodes = 0, off_dist = 0, off_hist = 0, off_idx = 0,
+    size_t off_flags = 0, off_qcodes = 0, off_q = 0, off_dist = 0, off_hist = 0, off_idx = 0,
            off_part = 0, total = 0;
 };
 
@@ -72,6 +72,7 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
     size_t o = 256;
     L->off_flags = o;      o = align_up(o + 4 * size_t(B), 256);
     L->off_qcodes = o;     o = align_up(o + 16 * size_t(BH), 256);
+    L->off_q = o;          o = align_up(o + 4 * kD * size_t(BH), 256);  // q, read once per step
     L->off_dist = o;       o = align_up(o + size_t(BH) * L->dist_row, 256);
     L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * L->n_tiles * kHistStride, 256);
     L->off_idx = o;        o = align_up(o + 4 * size_t(BH) * topk, 256);
@@ -82,7 +83,8 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
 
 // ------------------------------------------------------------------ args --
 struct PrepArgs {
-    const float *q;          // [B][H_q][128] or null (append only)
+    const float *q;          // [B][H_q][128] or null (append only); device or mapped host
+    float *q_copy;           // [B][H_q][128] device copy of q for the attention, or null
     const void *k_new;       // [B][H_kv][128] or null
     const void *v_new;       // [B][H_kv][128] or null
     const float *W;          // [H_kv][128][128]

@@ -37,15 +37,6 @@ __device__ __forceinline__ float load_x(const void *base, int64_t i)
     return reinterpret_cast<const float *>(base)[i];
 }
 
-template <bool BF16>
-__device__ __forceinline__ void store_x(void *base, int64_t i, const void *src, int64_t si)
-{
-    if (BF16)
-        reinterpret_cast<uint16_t *>(base)[i] = reinterpret_cast<const uint16_t *>(src)[si];
-    else
-        reinterpret_cast<float *>(base)[i] = reinterpret_cast<const float *>(src)[si];
-}
-
 // Column j of one head's W_H into registers.
 __device__ __forceinline__ void load_w_column(const float *__restrict__ Wh, int j, float (&w)[kD])
 {
@@ -153,11 +144,30 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
         cp_async_commit();
     }
 
-    float x = 0.0f;
+    // the row itself: its first warp reads it with 16-byte (q, fp32 keys) or
+    // 8-byte (bf16 keys) loads -- q and k_new may be host memory, where few
+    // wide requests cost much less than many narrow ones
+    if (j < 32 && row < rows) {
+        float4 v;
+        if (row < nq) {
+            const size_t bh = size_t(row / a.G) * a.H_q + h * a.G + row % a.G;
+            v = reinterpret_cast<const float4 *>(a.q + bh * kD)[j];
+            if (a.q_copy) reinterpret_cast<float4 *>(a.q_copy + bh * kD)[j] = v;
+        } else {
+            const int64_t e0 = (int64_t(row - nq) * a.H_kv + h) * kD;
+            if (BF16) {
+                const uint2 u = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.k_new) + e0)[j];
+                v = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+            } else {
+                v = reinterpret_cast<const float4 *>(static_cast<const float *>(a.k_new) + e0)[j];
+            }
+        }
+        reinterpret_cast<float4 *>(xs + r * kD)[j] = v;
+    }
     if (row < nq) {
         const int b = row / a.G, g = row % a.G, hq = h * a.G + g;
         const size_t bh = size_t(b) * a.H_q + hq;
-        x = a.q[bh * kD + j];
         if (a.hist)
             for (int64_t t = j; t < a.hist_row_words; t += kD) a.hist[bh * a.hist_row_words + t] = 0u;
         if (a.flags && h == 0 && g == 0 && j == 0) {
@@ -167,11 +177,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
             if (a.k_new && (sl - 1 < 0 || sl - 1 >= a.n_cap)) f |= HATA_FLAG_POS_RANGE;
             a.flags[b] = f;
         }
-    } else if (row < rows) {
-        const int b = row - nq;
-        x = load_x<BF16>(a.k_new, (int64_t(b) * a.H_kv + h) * kD + j);
     }
-    xs[r * kD + j] = x;
     cp_async_wait<0>();
     __syncthreads();
 
@@ -215,9 +221,22 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
             const int64_t crow = (int64_t(b) * a.H_kv + h) * a.n_cap + pos;
             if ((j & 31) == 0) a.codes[crow * kWords + (j >> 5)] = word;
             if (a.v_new) {
-                const int64_t src = (int64_t(b) * a.H_kv + h) * kD + j;
-                store_x<BF16>(a.K, crow * kD + j, a.k_new, src);
-                store_x<BF16>(a.V, crow * kD + j, a.v_new, src);
+                // K from the staged row (a bf16 key is the upper half of its
+                // fp32 widening: exact); V copied by the row's first warp
+                const float xk = xs[r * kD + j];
+                if (BF16)
+                    static_cast<uint16_t *>(a.K)[crow * kD + j] = uint16_t(__float_as_uint(xk) >> 16);
+                else
+                    static_cast<float *>(a.K)[crow * kD + j] = xk;
+                if (j < 32) {
+                    const int64_t e0 = (int64_t(b) * a.H_kv + h) * kD;
+                    if (BF16)
+                        reinterpret_cast<uint2 *>(static_cast<uint16_t *>(a.V) + crow * kD)[j] =
+                            reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.v_new) + e0)[j];
+                    else
+                        reinterpret_cast<float4 *>(static_cast<float *>(a.V) + crow * kD)[j] =
+                            reinterpret_cast<const float4 *>(static_cast<const float *>(a.v_new) + e0)[j];
+                }
             }
         } else if (a.err_word && j == 0) {
             atomicOr(a.err_word, HATA_FLAG_POS_RANGE);

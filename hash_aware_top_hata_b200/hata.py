@@ -111,7 +111,7 @@ def _kv_code(t: torch.Tensor) -> int:
     raise TypeError(f"K/V must be bfloat16 or float32, got {t.dtype}")
 
 
-def _need(t: torch.Tensor, name: str, dtype=None, ndim=None, cuda=True) -> None:
+def _need(t: torch.Tensor, name: str, dtype=None, ndim=None, cuda=True, host_ok=False) -> None:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if dtype is not None and t.dtype != dtype:
@@ -120,8 +120,9 @@ def _need(t: torch.Tensor, name: str, dtype=None, ndim=None, cuda=True) -> None:
         raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if cuda and not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+    if cuda and not t.is_cuda and not (host_ok and t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor" +
+                         (" or a pinned host tensor" if host_ok else ""))
 
 
 # ------------------------------------------------------------------ API --
@@ -182,18 +183,20 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
     q [B][H_q][128] fp32, K/V [B][H_kv][n_cap][128], seq_len [B] int32,
     workspace uint8 of hata_decode_workspace_size bytes, out [B][H_q][128] fp32.
     Optional: k_new/v_new [B][H_kv][128], sel_idx [B][H_q][topk] int32,
-    q_codes [B][H_q][4] int32, dist [B][H_q][row] uint8, events: 5 torch.cuda.Event."""
-    _need(q, "q", torch.float32, 3)
+    q_codes [B][H_q][4] int32, dist [B][H_q][row] uint8, events: 5 torch.cuda.Event.
+    q, k_new, v_new and out may also be pinned host tensors: the kernels read
+    and write them over the bus once per step (no separate copies)."""
+    _need(q, "q", torch.float32, 3, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
     _need(K, "K", ndim=4)
     _need(V, "V", ndim=4)
     _need(seq_len, "seq_len", torch.int32, 1)
     _need(workspace, "workspace", torch.uint8)
-    _need(out, "out", torch.float32, 3)
+    _need(out, "out", torch.float32, 3, host_ok=True)
     for t, name in ((k_new, "k_new"), (v_new, "v_new")):
         if t is not None:
-            _need(t, name, K.dtype, 3)
+            _need(t, name, K.dtype, 3, host_ok=True)
     if sel_idx is not None:
         _need(sel_idx, "sel_idx", torch.int32, 3)
     if q_codes is not None:
@@ -227,16 +230,16 @@ def hata_decode_step_noalloc(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Te
     caller workspace, for callers that cannot allocate device memory (see
     include/hata.h).  Calls on one device share that scratch: keep them
     ordered on one stream."""
-    _need(q, "q", torch.float32, 3)
+    _need(q, "q", torch.float32, 3, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
     _need(K, "K", ndim=4)
     _need(V, "V", ndim=4)
     _need(seq_len, "seq_len", torch.int32, 1)
-    _need(out, "out", torch.float32, 3)
+    _need(out, "out", torch.float32, 3, host_ok=True)
     for t, name in ((k_new, "k_new"), (v_new, "v_new")):
         if t is not None:
-            _need(t, name, K.dtype, 3)
+            _need(t, name, K.dtype, 3, host_ok=True)
     if sel_idx is not None:
         _need(sel_idx, "sel_idx", torch.int32, 3)
     if q_codes is not None:

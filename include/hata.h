@@ -27,6 +27,7 @@
  *       codes  [B][H_kv][n_cap][r/32] uint32, bit j in word j/32 at bit j%32
  *                                   (least significant first), 16-byte aligned
  *       q, out [B][H_q][d] fp32, 16-byte aligned
+ *       k_new, v_new [B][H_kv][d] (kv_dtype), 16-byte aligned
  *     Query head h_q uses KV head h_q / (H_q / H_kv) (grouped-query attention);
  *     its code is made with that KV head's W_H so that codes are comparable.
  *   - Hash arithmetic: the projection of bit j is the fp32 chain
@@ -126,7 +127,11 @@ int64_t hata_dist_row_bytes(int64_t max_seq_len);
  *      boundary bucket to the lower token index;
  *   4. out[b][h_q] = sum_{n in S} softmax_n(scale * q.K[n]) V[n]  (fp32
  *      accumulation, exact softmax over S only).  seq_len[b] == 0 gives 0.
- * Arguments:
+ * Arguments (q, k_new, v_new and out may be device memory or page-locked host
+ * memory that the device can address (any cudaHostAlloc / cudaMallocHost
+ * block under unified addressing): each is read, or written, once per step by
+ * the kernels themselves, so a step with host inputs and output needs no
+ * separate copy operations; every other buffer is device memory):
  *   q         [B][H_q][d] fp32
  *   W_H       [H_kv][d][r] fp32, 16-byte aligned
  *   codes     [B][H_kv][n_cap][r/32]; written only by the optional append

@@ -321,3 +321,33 @@ def test_full_size_sampled_heads(name):
             assert needles <= set(got[1][b, hq].tolist())
     del w, dec
     torch.cuda.empty_cache()
+
+
+def test_host_buffers_match_device_buffers():
+    """q, k_new, v_new and out in pinned host memory: the kernels read and
+    write them directly; the step's output, selection and appended caches are
+    bit-identical to the same step with device buffers."""
+    cfg = wl.scaled(wl.CONFIGS["llama31_8b_gqa_128k"], N=7000, topk=120, B=2)
+    w = wl.make_workload(cfg, 4242, device="cuda", steps=1)
+    res = []
+    for host in (False, True):
+        codes = torch.zeros((cfg.B, cfg.H_kv, w.n_cap, 4), dtype=torch.int32, device="cuda")
+        H.hata_hash_keys(w.K, w.W_H, codes, 0, cfg.N)
+        K, V = w.K.clone(), w.V.clone()
+        ws = torch.empty(H.hata_decode_workspace_size(cfg.B, cfg.H_q, cfg.H_kv, w.n_cap, cfg.topk),
+                         dtype=torch.uint8, device="cuda")
+        sel = torch.empty((cfg.B, cfg.H_q, cfg.topk), dtype=torch.int32, device="cuda")
+        sl = torch.full((cfg.B,), cfg.N + 1, dtype=torch.int32, device="cuda")
+        q, kn, vn = w.q[0], w.k_new[0], w.v_new[0]
+        if host:
+            q, kn, vn = q.cpu().pin_memory(), kn.cpu().pin_memory(), vn.cpu().pin_memory()
+            out = torch.full((cfg.B, cfg.H_q, 128), float("nan")).pin_memory()
+        else:
+            out = torch.full((cfg.B, cfg.H_q, 128), float("nan"), device="cuda")
+        H.hata_decode_step(q, w.W_H, codes, K, V, sl, w.n_cap, cfg.topk, SCALE, ws, out,
+                           k_new=kn, v_new=vn, sel_idx=sel)
+        torch.cuda.synchronize()
+        H.hata_workspace_check(ws)
+        res.append((out.cpu(), sel.cpu(), codes.cpu(), K[:, :, cfg.N].cpu(), V[:, :, cfg.N].cpu()))
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
