@@ -74,7 +74,7 @@ __device__ __forceinline__ uint32_t to_token_order(uint32_t m)
 __device__ __forceinline__ void head_threshold(const SelectArgs &a, size_t bh, int k_eff, int tile,
                                                int lane, int *out)
 {
-    constexpr int kRegTiles = 8;  // rows held in registers: one round trip to L2
+    constexpr int kRegTiles = 4;  // rows held in registers per round
     const uint32_t *hrow = a.hist + bh * size_t(a.n_tiles) * kHistStride;
     const int n_tiles = int(a.n_tiles);
     auto row_bins = [&](int t, uint32_t (&v)[5]) {
@@ -82,32 +82,27 @@ __device__ __forceinline__ void head_threshold(const SelectArgs &a, size_t bh, i
         for (int e = 0; e < 5; ++e)
             v[e] = lane * 5 + e < kBins ? __ldg(hrow + t * kHistStride + lane * 5 + e) : 0u;
     };
-    uint32_t rv[kRegTiles][5];
-#pragma unroll
-    for (int t = 0; t < kRegTiles; ++t) {
-        if (t < n_tiles) {
-            row_bins(t, rv[t]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 5; ++e) rv[t][e] = 0u;
-        }
-    }
     uint32_t tot[5] = {0u, 0u, 0u, 0u, 0u}, pre[5] = {0u, 0u, 0u, 0u, 0u};
+    // rounds of kRegTiles rows: all loads of a round are issued before any
+    // is summed, so a round costs one round trip to L2
+    for (int t0 = 0; t0 < n_tiles; t0 += kRegTiles) {
+        uint32_t rv[kRegTiles][5];
 #pragma unroll
-    for (int t = 0; t < kRegTiles; ++t)
+        for (int t = 0; t < kRegTiles; ++t) {
+            if (t0 + t < n_tiles) {
+                row_bins(t0 + t, rv[t]);
+            } else {
 #pragma unroll
-        for (int e = 0; e < 5; ++e) {
-            tot[e] += rv[t][e];
-            pre[e] += t < tile ? rv[t][e] : 0u;
+                for (int e = 0; e < 5; ++e) rv[t][e] = 0u;
+            }
         }
-    for (int t = kRegTiles; t < n_tiles; ++t) {  // long contexts only
-        uint32_t v[5];
-        row_bins(t, v);
 #pragma unroll
-        for (int e = 0; e < 5; ++e) {
-            tot[e] += v[e];
-            pre[e] += t < tile ? v[e] : 0u;
-        }
+        for (int t = 0; t < kRegTiles; ++t)
+#pragma unroll
+            for (int e = 0; e < 5; ++e) {
+                tot[e] += rv[t][e];
+                pre[e] += t0 + t < tile ? rv[t][e] : 0u;
+            }
     }
     const uint32_t run = tot[0] + tot[1] + tot[2] + tot[3] + tot[4];
     uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
@@ -171,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     const int my0 = tile * kTile + tid * kPer;
     // ---- warp 0 first finds T, #(dist < T) and the keys below T / at T in
     // the tiles before this one from the head's tile histograms (one round
-    // trip to L2 for up to kRegTiles tiles), ahead of its own distance loads;
+    // trip to L2 per 4 tiles), ahead of its own distance loads;
     // the other warps' distance loads are in flight meanwhile ----
     if (tid < 32) head_threshold(a, bh, k_eff, tile, tid, s_thr);
     // the warp's 4 KB arrive by coalesced 16-byte copies (lane l: bytes
