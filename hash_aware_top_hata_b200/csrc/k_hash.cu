@@ -25,7 +25,6 @@
 namespace hata {
 namespace {
 
-constexpr int kPrefillRowsPerCta = 128;
 
 template <bool BF16>
 __device__ __forceinline__ float load_x(const void *base, int64_t i)
@@ -37,70 +36,113 @@ __device__ __forceinline__ float load_x(const void *base, int64_t i)
     return reinterpret_cast<const float *>(base)[i];
 }
 
-// Column j of one head's W_H into registers.
-__device__ __forceinline__ void load_w_column(const float *__restrict__ Wh, int j, float (&w)[kD])
-{
-#pragma unroll
-    for (int i = 0; i < kD; ++i) w[i] = __ldg(Wh + i * kRbit + j);
-}
-
-// xs: [kD][R] floats (row r of the group in column r); w: column j of W_H
-// (j = threadIdx.x) in registers.  Returns, for every row, the ballot of this
-// warp's 32 bits = code word (threadIdx.x / 32).
-template <int R>
-__device__ __forceinline__ void hash_group(const float *__restrict__ xs, const float (&w)[kD],
-                                           uint32_t (&words)[R])
-{
-    float acc[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kD; ++i) {
-#pragma unroll
-        for (int r4 = 0; r4 < R / 4; ++r4) {
-            const float4 x = reinterpret_cast<const float4 *>(xs + i * R)[r4];
-            acc[4 * r4 + 0] = __fmaf_rn(x.x, w[i], acc[4 * r4 + 0]);
-            acc[4 * r4 + 1] = __fmaf_rn(x.y, w[i], acc[4 * r4 + 1]);
-            acc[4 * r4 + 2] = __fmaf_rn(x.z, w[i], acc[4 * r4 + 2]);
-            acc[4 * r4 + 3] = __fmaf_rn(x.w, w[i], acc[4 * r4 + 3]);
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) words[r] = __ballot_sync(0xffffffffu, acc[r] > 0.0f);
-}
-
 // -------------------------------------------------------------- prefill --
-template <bool BF16>
-__global__ void __launch_bounds__(kD) hash_prefill_kernel(const void *__restrict__ K,
-                                                          int64_t n_cap,
-                                                          const float *__restrict__ W,
-                                                          uint32_t *__restrict__ codes,
-                                                          int H_kv, int64_t pos0, int64_t n)
+// Register-blocked: a CTA stages its head's W_H in shared memory once and
+// walks its rows in passes of kPfPass rows; warp w takes 8 rows of a pass,
+// lane l the output bits 4l..4l+3 of each, so a lane holds 32 accumulators,
+// each the fp32 chain acc = fmaf(x_i, W[i][j], acc) over i = 0..127 in order.
+// Per step i a lane reads its 4 W values (one 16-byte load; the warp reads
+// W's row i contiguously) and the 8 row values (two broadcast loads), then
+// issues 16 paired FMAs over row pairs: fma.rn.f32x2 performs two IEEE fp32
+// fused multiply-adds, each rounded to nearest, so every chain is the one
+// the scalar form computes (it halves the issue slots, not the FMA work).
+// 96 KB of shared memory: two CTAs, 16 warps, per SM.
+constexpr int kPfWarps = 8;
+constexpr int kPfThreads = 32 * kPfWarps;
+constexpr int kPfRows = 8;                   // rows per warp and pass
+constexpr int kPfPass = kPfWarps * kPfRows;  // rows per CTA and pass
+constexpr int kPfRowsPerCta = 16 * kPfPass;  // 1024 rows per CTA
+
+struct PfSmem {
+    float W[kD * kRbit];                     // this head's W_H, [i][j]
+    float x[kPfWarps][kD][kPfRows];          // each warp's rows, [i][row]
+};
+
+// acc (two fp32 chains) += x (pair) * w (pair), element by element
+__device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t x, uint64_t w)
 {
-    constexpr int R = kPrepRows;
-    const int h = blockIdx.y, b = blockIdx.z, j = threadIdx.x;
-    const int64_t g_begin = int64_t(blockIdx.x) * kPrefillRowsPerCta;
-    const int64_t g_end = min(g_begin + kPrefillRowsPerCta, n);
-    const int64_t slab = (int64_t(b) * H_kv + h) * n_cap;  // row index of token 0
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(w));
+}
 
-    float w[kD];
-    load_w_column(W + size_t(h) * kD * kRbit, j, w);
-    __shared__ __align__(16) float xs[kD * R];
+__device__ __forceinline__ uint64_t dup2(float v)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
+}
 
-    for (int64_t g0 = g_begin; g0 < g_end; g0 += R) {
-        __syncthreads();
+template <bool BF16>
+__global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void *__restrict__ K,
+                                                                    int64_t n_cap,
+                                                                    const float *__restrict__ W,
+                                                                    uint32_t *__restrict__ codes,
+                                                                    int H_kv, int64_t pos0, int64_t n)
+{
+    extern __shared__ __align__(16) uint8_t pf_raw[];
+    PfSmem &S = *reinterpret_cast<PfSmem *>(pf_raw);
+    const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t g_begin = int64_t(blockIdx.x) * kPfRowsPerCta;
+    const int64_t g_end = min(g_begin + kPfRowsPerCta, n);
+    const int64_t slab = (int64_t(b) * H_kv + h) * n_cap + pos0;  // row index of row 0
+    {
+        const float *Wh = W + size_t(h) * kD * kRbit;
+        const uint32_t base = smem_addr(S.W);
+        for (int c = tid; c < kD * kRbit / 4; c += kPfThreads)
+            cp_async16_zfill(base + 16u * c, Wh + 4 * c, 16u);
+        cp_async_commit();
+    }
+    // staging: lane l holds row (l & 7) of its warp at steps i = 4k + (l >> 3)
+    // (eight lanes write one 32-byte run); the next pass's values are loaded
+    // into registers while a pass computes
+    const int sr = lane & 7, si = lane >> 3;
+    float xv[kD / 4];
+    auto fetch = [&](int64_t g0) {
+        const int64_t t = g0 + warp * kPfRows + sr;
+        const bool ok = t < g_end;
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int64_t t = g0 + r;
-            xs[j * R + r] = (t < g_end) ? load_x<BF16>(K, (slab + pos0 + t) * kD + j) : 0.0f;
+        for (int k = 0; k < kD / 4; ++k) xv[k] = ok ? load_x<BF16>(K, (slab + t) * kD + 4 * k + si) : 0.0f;
+    };
+    fetch(g_begin);
+    for (int64_t g0 = g_begin; g0 < g_end; g0 += kPfPass) {
+        __syncthreads();  // the previous pass is done with the rows
+#pragma unroll
+        for (int k = 0; k < kD / 4; ++k) S.x[warp][4 * k + si][sr] = xv[k];
+        cp_async_wait<0>();
+        __syncthreads();
+        if (g0 + kPfPass < g_end) fetch(g0 + kPfPass);
+        uint64_t acc[kPfRows / 2][4];  // [row pair][column]
+#pragma unroll
+        for (int p = 0; p < kPfRows / 2; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0ull;
+        const float4 *wrow = reinterpret_cast<const float4 *>(S.W) + lane;  // W[0][4l..4l+3]
+        const ulonglong2 *xrow = reinterpret_cast<const ulonglong2 *>(&S.x[warp][0][0]);
+#pragma unroll 4
+        for (int i = 0; i < kD; ++i) {
+            const float4 w = wrow[i * (kRbit / 4)];
+            const uint64_t w0 = dup2(w.x), w1 = dup2(w.y), w2 = dup2(w.z), w3 = dup2(w.w);
+            const ulonglong2 xa = xrow[i * 2], xb = xrow[i * 2 + 1];  // rows (0,1) (2,3) | (4,5) (6,7)
+            const uint64_t xp[4] = {xa.x, xa.y, xb.x, xb.y};
+#pragma unroll
+            for (int p = 0; p < kPfRows / 2; ++p) {
+                ffma2(acc[p][0], xp[p], w0);
+                ffma2(acc[p][1], xp[p], w1);
+                ffma2(acc[p][2], xp[p], w2);
+                ffma2(acc[p][3], xp[p], w3);
+            }
         }
-        __syncthreads();
-        uint32_t words[R];
-        hash_group<R>(xs, w, words);
-        if ((j & 31) == 0) {
+        // bits 4l..4l+3 of each row -> word l / 8 (bit 4 (l % 8) + c)
 #pragma unroll
-            for (int r = 0; r < R; ++r)
-                if (g0 + r < g_end) codes[(slab + pos0 + g0 + r) * kWords + (j >> 5)] = words[r];
+        for (int r = 0; r < kPfRows; ++r) {
+            const int p = r >> 1, sh = 32 * (r & 1);
+            uint32_t v = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                v |= (__uint_as_float(uint32_t(acc[p][c] >> sh)) > 0.0f ? 1u : 0u) << c;
+            v <<= 4 * (lane & 7);
+            v |= __shfl_xor_sync(0xffffffffu, v, 1);
+            v |= __shfl_xor_sync(0xffffffffu, v, 2);
+            v |= __shfl_xor_sync(0xffffffffu, v, 4);
+            const int64_t t = g0 + warp * kPfRows + r;
+            if ((lane & 7) == 0 && t < g_end) codes[(slab + t) * kWords + (lane >> 3)] = v;
         }
     }
 }
@@ -250,11 +292,15 @@ cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const f
                                 uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
                                 cudaStream_t s)
 {
-    const dim3 grid(unsigned(ceil_div(n, kPrefillRowsPerCta)), unsigned(H_kv), unsigned(B));
+    constexpr size_t kSmem = sizeof(PfSmem);
+    const void *fn = bf16 ? reinterpret_cast<const void *>(hash_prefill_kernel<true>)
+                          : reinterpret_cast<const void *>(hash_prefill_kernel<false>);
+    if (cudaError_t e = ensure_smem_attr(fn, kSmem)) return e;
+    const dim3 grid(unsigned(ceil_div(n, kPfRowsPerCta)), unsigned(H_kv), unsigned(B));
     if (bf16)
-        hash_prefill_kernel<true><<<grid, kD, 0, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
+        hash_prefill_kernel<true><<<grid, kPfThreads, kSmem, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
     else
-        hash_prefill_kernel<false><<<grid, kD, 0, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
+        hash_prefill_kernel<false><<<grid, kPfThreads, kSmem, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
     return cudaGetLastError();
 }
 
