@@ -473,10 +473,10 @@ def run_hata(args, world, rank, local):
     H.hata_workspace_check(ws)
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
 
-    # per-kernel breakdown (untimed pass): events between the four kernels
-    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K_steps)]
-    for e5 in kevs:  # torch creates the CUDA event on first record; the library needs handles
-        for e in e5:
+    # per-kernel breakdown (untimed pass): events between the five kernels
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K_steps)]
+    for e6 in kevs:  # torch creates the CUDA event on first record; the library needs handles
+        for e in e6:
             e.record(stream)
     torch.cuda.synchronize()
     for i in range(K_steps):
@@ -487,7 +487,8 @@ def run_hata(args, world, rank, local):
     score_ms = [e[1].elapsed_time(e[2]) for e in kevs]
     select_ms = [e[2].elapsed_time(e[3]) for e in kevs]
     attend_ms = [e[3].elapsed_time(e[4]) for e in kevs]
-    split_ms = [e[0].elapsed_time(e[4]) for e in kevs]
+    combine_ms = [e[4].elapsed_time(e[5]) for e in kevs]
+    split_ms = [e[0].elapsed_time(e[5]) for e in kevs]
     ms = statistics.mean(step_ms)
     ms_max = max_over_ranks(world, ms)
 
@@ -526,6 +527,7 @@ def run_hata(args, world, rank, local):
                        "score": round(score_s * 1e6, 2),
                        "select": round(statistics.mean(select_ms) * 1e3, 2),
                        "attend": round(attend_s * 1e6, 2),
+                       "combine": round(statistics.mean(combine_ms) * 1e3, 2),
                        "sum_with_events": round(statistics.mean(split_ms) * 1e3, 2),
                        "score_gbs": round(code_bytes / score_s / 1e9, 1)},
         "dense_us": _num(dense_ms * 1e3, 1),

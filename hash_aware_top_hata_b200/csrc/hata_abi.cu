@@ -312,6 +312,8 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     if ((e = launch_attend(aa, kv_dtype == HATA_DT_BF16, s)) != cudaSuccess)
         return cuda_fail(e, "attend launch");
     if ((e = ev.record(4)) != cudaSuccess) return cuda_fail(e, "event record");
+    if ((e = launch_combine(aa, s)) != cudaSuccess) return cuda_fail(e, "combine launch");
+    if ((e = ev.record(5)) != cudaSuccess) return cuda_fail(e, "event record");
     return ok();
 }
 

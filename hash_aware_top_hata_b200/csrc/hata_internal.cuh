@@ -214,7 +214,8 @@ cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const f
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
-cudaError_t launch_attend(const AttendArgs &a, bool bf16, cudaStream_t s);
+cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s);  // sets a.n_workers
+cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s);
 cudaError_t launch_dense(const DenseArgs &a, bool bf16, cudaStream_t s);
 
 }  // namespace hata

@@ -737,6 +737,33 @@ cudaError_t occupancy_grid(Kernel kernel, int threads, size_t smem, int64_t *gri
     return e;
 }
 
+}  // namespace
+
+cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
+{
+    const int64_t T = int64_t(a.B) * a.H_q * a.topk;
+    int64_t P = 0;
+    if (bf16) {
+        if (cudaError_t e = occupancy_grid(attend_tc_kernel, tc::kThreads, tc::kSmem, &P)) return e;
+        int64_t NW = P * tc::kTcWarps;
+        if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
+        if (NW > T) NW = T;
+        a.n_workers = NW;
+        return launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
+                          dim3(tc::kThreads), tc::kSmem, s, a);
+    }
+    constexpr size_t kSmemF32 = size_t(kRing) * Rows<false>::kSlotBytes;
+    if (cudaError_t e = occupancy_grid(attend_simt_kernel<false>, kAttnThreads, kSmemF32, &P))
+        return e;
+    if (P > kAttnMaxWorkers) P = kAttnMaxWorkers;
+    if (P > T) P = T;
+    a.n_workers = P;
+    return launch_pdl(attend_simt_kernel<false>, dim3(unsigned(P)), dim3(kAttnThreads), kSmemF32,
+                      s, a);
+}
+
+// The merge of the split heads: launched right behind launch_attend (whose
+// call sets a.n_workers), with programmatic dependent launch.
 cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s)
 {
     const int64_t heads = int64_t(a.B) * a.H_q;
@@ -746,36 +773,6 @@ cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s)
         return e;
     return launch_pdl(combine_kernel, dim3(unsigned(ceil_div(heads, kCombineWarps))),
                       dim3(32 * kCombineWarps), 0, s, a);
-}
-
-}  // namespace
-
-cudaError_t launch_attend(const AttendArgs &args, bool bf16, cudaStream_t s)
-{
-    AttendArgs a = args;
-    const int64_t T = int64_t(a.B) * a.H_q * a.topk;
-    int64_t P = 0;
-    if (bf16) {
-        if (cudaError_t e = occupancy_grid(attend_tc_kernel, tc::kThreads, tc::kSmem, &P)) return e;
-        int64_t NW = P * tc::kTcWarps;
-        if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
-        if (NW > T) NW = T;
-        a.n_workers = NW;
-        if (cudaError_t e = launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
-                                       dim3(tc::kThreads), tc::kSmem, s, a))
-            return e;
-        return launch_combine(a, s);
-    }
-    constexpr size_t kSmemF32 = size_t(kRing) * Rows<false>::kSlotBytes;
-    if (cudaError_t e = occupancy_grid(attend_simt_kernel<false>, kAttnThreads, kSmemF32, &P))
-        return e;
-    if (P > kAttnMaxWorkers) P = kAttnMaxWorkers;
-    if (P > T) P = T;
-    a.n_workers = P;
-    if (cudaError_t e = launch_pdl(attend_simt_kernel<false>, dim3(unsigned(P)),
-                                   dim3(kAttnThreads), kSmemF32, s, a))
-        return e;
-    return launch_combine(a, s);
 }
 
 }  // namespace hata

@@ -183,7 +183,7 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
     q [B][H_q][128] fp32, K/V [B][H_kv][n_cap][128], seq_len [B] int32,
     workspace uint8 of hata_decode_workspace_size bytes, out [B][H_q][128] fp32.
     Optional: k_new/v_new [B][H_kv][128], sel_idx [B][H_q][topk] int32,
-    q_codes [B][H_q][4] int32, dist [B][H_q][row] uint8, events: 5 torch.cuda.Event.
+    q_codes [B][H_q][4] int32, dist [B][H_q][row] uint8, events: 6 torch.cuda.Event.
     q, k_new, v_new and out may also be pinned host tensors: the kernels read
     and write them over the bus once per step (no separate copies)."""
     _need(q, "q", torch.float32, 3, host_ok=True)
@@ -209,9 +209,9 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
     H_kv, n_cap = K.shape[1], K.shape[2]
     ev = None
     if events is not None:
-        if len(events) != 5:
-            raise ValueError("events: give 5 torch.cuda.Event (recorded around the 4 kernels)")
-        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+        if len(events) != 6:
+            raise ValueError("events: give 6 torch.cuda.Event (recorded around the 5 kernels)")
+        ev = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events])
     _check(lib().hata_decode_step(
         _ptr(q), _ptr(W_H), _ptr(codes), _ptr(K), _ptr(V), _kv_code(K), n_cap, _ptr(seq_len),
         max_seq_len, _ptr(k_new), _ptr(v_new), B, H_q, H_kv, d, W_H.shape[2], topk,
@@ -252,9 +252,9 @@ def hata_decode_step_noalloc(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Te
     H_kv, n_cap = K.shape[1], K.shape[2]
     ev = None
     if events is not None:
-        if len(events) != 5:
-            raise ValueError("events: give 5 torch.cuda.Event (recorded around the 4 kernels)")
-        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+        if len(events) != 6:
+            raise ValueError("events: give 6 torch.cuda.Event (recorded around the 5 kernels)")
+        ev = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events])
     _check(lib().hata_decode_step_noalloc(
         _ptr(q), _ptr(W_H), _ptr(codes), _ptr(K), _ptr(V), _kv_code(K), n_cap, _ptr(seq_len),
         max_seq_len, _ptr(k_new), _ptr(v_new), B, H_q, H_kv, d, W_H.shape[2], topk,

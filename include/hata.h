@@ -150,9 +150,10 @@ int64_t hata_dist_row_bytes(int64_t max_seq_len);
  *             Hamming distances (0..128); positions seq_len[b] ..
  *             hata_dist_row_bytes(max_seq_len)-1 hold 255;
  *             dist_row_bytes >= hata_dist_row_bytes(max_seq_len), multiple of 16
- *   events    optional array of 5 cudaEvent_t recorded on `stream` before the
- *             first kernel and after each of the four kernels (prep, score,
- *             select, attend) -- a profiling hook
+ *   events    optional array of 6 cudaEvent_t recorded on `stream` before the
+ *             first kernel and after each of the five kernels (prep, score,
+ *             select, attend, combine) -- a profiling hook (an event between
+ *             two kernels keeps the second from starting early)
  */
 hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
                                void *V, hata_dtype_t kv_dtype, int64_t n_cap,
