@@ -324,9 +324,9 @@ def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, w
 
 def more_legs(cfg, w, codes, ws, out, seq, flush, stream, t0, K_steps):
     """Labelled side measurements of the same workload: warm-L2 step time,
-    needle recall, prefill key encoding against the FP32 peak, torch SDPA
-    dense decode, and K_steps consecutive decode steps replayed from one
-    CUDA Graph."""
+    needle recall, the step with the K/V caches in host memory, prefill key
+    encoding against the FP32 peak, torch SDPA dense decode, and K_steps
+    consecutive decode steps replayed from one CUDA Graph."""
     B, Hq, Hkv, N, G = cfg.B, cfg.H_q, cfg.H_kv, cfg.N, cfg.G
     scale = 1.0 / math.sqrt(128)
     dev = out.device
@@ -361,6 +361,29 @@ def more_legs(cfg, w, codes, ws, out, seq, flush, stream, t0, K_steps):
                 hits += len(nd & got)
                 total += len(nd)
         res["needle_recall"] = round(hits / max(total, 1), 4)
+
+    # ---- HATA-off: the K/V caches in pinned host memory; a step reads only
+    # the selected rows over the bus (the codes stay on the device) ----
+    try:
+        Kh, Vh = w.K.cpu().pin_memory(), w.V.cpu().pin_memory()
+        kh_ev = [ev_pair() for _ in range(3)]
+        for i in range(5):
+            flush()
+            if i >= 2:
+                kh_ev[i - 2][0].record(stream)
+            H.hata_decode_step(w.q[t0 + i], w.W_H, codes, Kh, Vh, seq[t0 + i], w.n_cap, cfg.topk,
+                               scale, ws, out, k_new=w.k_new[t0 + i], v_new=w.v_new[t0 + i])
+            if i >= 2:
+                kh_ev[i - 2][1].record(stream)
+        torch.cuda.synchronize()
+        t_kh = statistics.median(a.elapsed_time(b) for a, b in kh_ev) / 1e3
+        row_bytes = B * Hq * cfg.topk * 2 * w.K.shape[-1] * w.K.element_size()
+        res["kv_host"] = {"us_per_step": round(t_kh * 1e6, 1),
+                          "selected_row_gbs": round(row_bytes / t_kh / 1e9, 2),
+                          "selected_row_bytes": row_bytes}
+        del Kh, Vh
+    except RuntimeError as e:  # pinned host memory unavailable
+        res["kv_host"] = {"unavailable": str(e).splitlines()[0][:120]}
 
     # ---- prefill key encoding (hata_hash_keys over the whole cache) ----
     pe = [ev_pair() for _ in range(3)]
@@ -427,7 +450,7 @@ def run_hata(args, world, rank, local):
     cfg = bench_config(args)
     K_steps, W_steps = args.steps, args.warmup
     G_steps = min(K_steps, 16)  # side legs: warm-L2 steps and the CUDA Graph
-    total_steps = W_steps + 3 * K_steps + G_steps + 1
+    total_steps = W_steps + 3 * K_steps + G_steps + 6  # + the host-cache leg's 5 steps
     seed = wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config) + 1000 * rank
     dev = torch.device("cuda", torch.cuda.current_device())
     w = wl.make_workload(cfg, seed, device=dev, steps=total_steps)

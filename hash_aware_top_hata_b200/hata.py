@@ -139,8 +139,9 @@ def hata_hash_keys(K: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, pos0
                    n: int | None = None, stream=None) -> None:
     """Prefill: codes[b, h, pos0:pos0+n] = hash(K[b, h, pos0:pos0+n]).
     K [B][H_kv][n_cap][128] bf16/fp32, W_H [H_kv][128][128] fp32,
-    codes [B][H_kv][n_cap][4] int32 (uint32 bit patterns)."""
-    _need(K, "K", ndim=4)
+    codes [B][H_kv][n_cap][4] int32 (uint32 bit patterns).  K may be a pinned
+    host tensor (a cache kept in host memory)."""
+    _need(K, "K", ndim=4, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
     B, H, n_cap, d = K.shape
@@ -189,8 +190,8 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
     _need(q, "q", torch.float32, 3, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
-    _need(K, "K", ndim=4)
-    _need(V, "V", ndim=4)
+    _need(K, "K", ndim=4, host_ok=True)
+    _need(V, "V", ndim=4, host_ok=True)
     _need(seq_len, "seq_len", torch.int32, 1)
     _need(workspace, "workspace", torch.uint8)
     _need(out, "out", torch.float32, 3, host_ok=True)
@@ -233,8 +234,8 @@ def hata_decode_step_noalloc(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Te
     _need(q, "q", torch.float32, 3, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
-    _need(K, "K", ndim=4)
-    _need(V, "V", ndim=4)
+    _need(K, "K", ndim=4, host_ok=True)
+    _need(V, "V", ndim=4, host_ok=True)
     _need(seq_len, "seq_len", torch.int32, 1)
     _need(out, "out", torch.float32, 3, host_ok=True)
     for t, name in ((k_new, "k_new"), (v_new, "v_new")):
@@ -285,8 +286,8 @@ def hata_dense_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_len
     """Dense decode attention over keys 0..seq_len[b]-1 (the full-attention
     baseline)."""
     _need(q, "q", torch.float32, 3)
-    _need(K, "K", ndim=4)
-    _need(V, "V", ndim=4)
+    _need(K, "K", ndim=4, host_ok=True)
+    _need(V, "V", ndim=4, host_ok=True)
     _need(seq_len, "seq_len", torch.int32, 1)
     _need(workspace, "workspace", torch.uint8)
     _need(out, "out", torch.float32, 3)

@@ -131,7 +131,10 @@ int64_t hata_dist_row_bytes(int64_t max_seq_len);
  * memory that the device can address (any cudaHostAlloc / cudaMallocHost
  * block under unified addressing): each is read, or written, once per step by
  * the kernels themselves, so a step with host inputs and output needs no
- * separate copy operations; every other buffer is device memory):
+ * separate copy operations.  K and V may be page-locked host memory too (the
+ * caches kept off the device): a step then reads only the selected rows,
+ * 2 * topk rows per query head, across the bus.  Every other buffer is
+ * device memory):
  *   q         [B][H_q][d] fp32
  *   W_H       [H_kv][d][r] fp32, 16-byte aligned
  *   codes     [B][H_kv][n_cap][r/32]; written only by the optional append

@@ -351,3 +351,30 @@ def test_host_buffers_match_device_buffers():
         res.append((out.cpu(), sel.cpu(), codes.cpu(), K[:, :, cfg.N].cpu(), V[:, :, cfg.N].cpu()))
     for a, b in zip(*res):
         assert torch.equal(a, b)
+
+
+def test_host_resident_kv_cache_matches_device():
+    """K and V kept in pinned host memory (only the selected rows cross the
+    bus each step): output, selection and the appended rows are identical to
+    the same step on device-resident caches."""
+    cfg = wl.scaled(wl.CONFIGS["llama31_8b_gqa_128k"], N=5000, topk=96, B=2)
+    w = wl.make_workload(cfg, 5151, device="cuda", steps=1)
+    res = []
+    for host in (False, True):
+        K, V = w.K.clone(), w.V.clone()
+        if host:
+            K, V = K.cpu().pin_memory(), V.cpu().pin_memory()
+        codes = torch.zeros((cfg.B, cfg.H_kv, w.n_cap, 4), dtype=torch.int32, device="cuda")
+        H.hata_hash_keys(K, w.W_H, codes, 0, cfg.N)
+        ws = torch.empty(H.hata_decode_workspace_size(cfg.B, cfg.H_q, cfg.H_kv, w.n_cap, cfg.topk),
+                         dtype=torch.uint8, device="cuda")
+        sel = torch.empty((cfg.B, cfg.H_q, cfg.topk), dtype=torch.int32, device="cuda")
+        out = torch.empty((cfg.B, cfg.H_q, 128), device="cuda")
+        sl = torch.full((cfg.B,), cfg.N + 1, dtype=torch.int32, device="cuda")
+        H.hata_decode_step(w.q[0], w.W_H, codes, K, V, sl, w.n_cap, cfg.topk, SCALE, ws, out,
+                           k_new=w.k_new[0], v_new=w.v_new[0], sel_idx=sel)
+        torch.cuda.synchronize()
+        H.hata_workspace_check(ws)
+        res.append((out.cpu(), sel.cpu(), codes.cpu(), K[:, :, cfg.N].cpu(), V[:, :, cfg.N].cpu()))
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
