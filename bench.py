@@ -520,8 +520,9 @@ def run_hata(args, world, rank, local):
     if not args.no_extras:
         e2e_ms, h2d, d2h, dense_ms = extras(args, cfg, w, codes, ws, out, seq, flush, stream,
                                             W_steps, K_steps, world)
-        side = more_legs(cfg, w, codes, ws, out, seq, flush, stream, W_steps + 3 * K_steps,
-                         G_steps)
+        if rank == 0:  # no collectives inside; only rank 0 prints the line
+            side = more_legs(cfg, w, codes, ws, out, seq, flush, stream, W_steps + 3 * K_steps,
+                             G_steps)
     # ---- roofline ----
     peak, peak_kind = measured_peaks()
     kv_row = 128 * kv_elt
