@@ -135,6 +135,8 @@ struct AttendArgs {
     int64_t n_cap, max_seq_len;
     int B, H_q, H_kv, G, topk, n_split;
     int64_t n_workers;       // stream-K workers (set by the launcher)
+    int head_per_cta;        // 1: a CTA's warps cover one whole head and merge it in shared
+                             // memory (no combine launch); set by the launcher
     float scale_log2;        // scale * log2(e)
 };
 

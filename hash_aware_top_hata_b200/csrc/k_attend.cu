@@ -494,14 +494,10 @@ __device__ __forceinline__ void attend_stage(int n, uint32_t Ks, const int32_t *
     }
 }
 
-// A warp is done with head cs.bh: write its partial (m, l, acc[128]) into
-// the head's slot for this worker; the combine kernel merges the slots.
-__device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, int64_t wid,
-                                        int64_t NW, int64_t T, const float (&O)[8][4],
-                                        float m_ref, float l_part, int lane)
+// Write a warp's partial (m, l, acc[128]) to pp (global or shared).
+__device__ __forceinline__ void store_partial(float *pp, const float (&O)[8][4], float m_ref,
+                                              float l_part, int lane)
 {
-    const int64_t k_first = owner(int64_t(cs.bh) * a.topk, T, NW);
-    float *pp = a.part + (int64_t(cs.bh) * a.n_split + (wid - k_first)) * kPartStride;
     float lw = lane < 4 ? l_part : 0.0f;  // lanes 0-3 hold all 16 keys of every stage
     lw += __shfl_xor_sync(0xffffffffu, lw, 1);
     lw += __shfl_xor_sync(0xffffffffu, lw, 2);
@@ -519,6 +515,17 @@ __device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, in
     }
 }
 
+// A warp is done with head cs.bh: write its partial into the head's slot
+// for this worker; the combine kernel merges the slots.
+__device__ __forceinline__ void publish(const AttendArgs &a, const Stage &cs, int64_t wid,
+                                        int64_t NW, int64_t T, const float (&O)[8][4],
+                                        float m_ref, float l_part, int lane)
+{
+    const int64_t k_first = owner(int64_t(cs.bh) * a.topk, T, NW);
+    store_partial(a.part + (int64_t(cs.bh) * a.n_split + (wid - k_first)) * kPartStride, O,
+                  m_ref, l_part, lane);
+}
+
 }  // namespace tc
 
 __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a)
@@ -526,6 +533,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     using namespace tc;
     extern __shared__ __align__(128) uint8_t smem[];  // [warp][kRingW][K | V], then indices
     __shared__ int32_t rows_s[kTcWarps][kRingW][kSub];
+    __shared__ __align__(16) float part_s[kTcWarps][kPartStride];  // head-per-CTA partials
     pdl_trigger();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -548,6 +556,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
         prod.init(&a, beg, end);
         cons.init(&a, beg, end);
     }
+    if (a.head_per_cta)  // a warp with no row of the head leaves an empty partial
+        for (int i = lane; i < kPartStride; i += 32) part_s[warp][i] = i == 0 ? -INFINITY : 0.0f;
+    __syncwarp();
     pdl_wait();  // the selected index lists
 
     // the CTA's slice of the index list (the first kIdxCap of it): all loads
@@ -647,9 +658,33 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
         attend_stage(cs.n, wring + uint32_t(slot * kStageBytes), rows_s[warp][slot], qb, lo, O,
                      m_ref, l_part, lane);
 
-        if (cs.last) publish(a, cs, wid, NW, T, O, m_ref, l_part, lane);
+        if (cs.last) {
+            if (a.head_per_cta)
+                store_partial(part_s[warp], O, m_ref, l_part, lane);
+            else
+                publish(a, cs, wid, NW, T, O, m_ref, l_part, lane);
+        }
     }
     cp_async_wait<0>();
+    if (a.head_per_cta) {
+        // the CTA holds all of head blockIdx.x: merge its warps' partials
+        __syncthreads();
+        if (tid < kD) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, part_s[w][0]);
+            float L = 0.0f, A = 0.0f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kTcWarps; ++w) {
+                    const float wt = part_s[w][0] == -INFINITY ? 0.0f : exp2f(part_s[w][0] - M);
+                    L = fmaf(part_s[w][1], wt, L);
+                    A = fmaf(part_s[w][4 + tid], wt, A);
+                }
+            }
+            a.out[int64_t(blockIdx.x) * kD + tid] = L > 0.0f ? A / L : 0.0f;
+        }
+    }
 }
 
 // ------------------------------------------------------------------------
@@ -748,6 +783,11 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
         int64_t NW = P * tc::kTcWarps;
         if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
         if (NW > T) NW = T;
+        // Heads that nearly fill one wave of CTAs: a CTA per head, merged in
+        // shared memory, saves the combine launch and its completion gap.
+        const int64_t heads = int64_t(a.B) * a.H_q;
+        a.head_per_cta = heads * 5 >= P * 4 && heads <= P && a.topk >= 16 * tc::kTcWarps;
+        if (a.head_per_cta) NW = heads * tc::kTcWarps;
         a.n_workers = NW;
         return launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
                           dim3(tc::kThreads), tc::kSmem, s, a);
@@ -758,6 +798,7 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
     if (P > kAttnMaxWorkers) P = kAttnMaxWorkers;
     if (P > T) P = T;
     a.n_workers = P;
+    a.head_per_cta = 0;
     return launch_pdl(attend_simt_kernel<false>, dim3(unsigned(P)), dim3(kAttnThreads), kSmemF32,
                       s, a);
 }
@@ -766,6 +807,7 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
 // call sets a.n_workers), with programmatic dependent launch.
 cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s)
 {
+    if (a.head_per_cta) return cudaSuccess;  // merged inside the attention CTAs
     const int64_t heads = int64_t(a.B) * a.H_q;
     // the same carveout as the attention kernel, so its CTAs can join the
     // SMs without a shared-memory reconfiguration

@@ -378,3 +378,25 @@ def test_host_resident_kv_cache_matches_device():
         res.append((out.cpu(), sel.cpu(), codes.cpu(), K[:, :, cfg.N].cpu(), V[:, :, cfg.N].cpu()))
     for a, b in zip(*res):
         assert torch.equal(a, b)
+
+
+def test_decode_head_per_cta_merge():
+    """128 query heads (about one wave of attention CTAs): every head is
+    gathered by one CTA and merged in shared memory; the oracle still
+    decides, including short rows (k_eff < topk) and an empty one."""
+    cfg = wl.scaled(wl.CONFIGS["llama31_8b_gqa_128k"], N=3000, topk=160, B=4)
+    w = wl.make_workload(cfg, 8181, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk)
+    lens = [cfg.N, 100, 0, 2500]  # full, k_eff = len < topk, empty, partial
+    slabs = host_slabs(w, [(b, hq // cfg.G) for b in range(cfg.B) for hq in (0, 7, 31)])
+    got = dec.step(w.q[0], lens)
+    Wn = w.W_H.cpu().numpy()
+    for b in range(cfg.B):
+        for hq in (0, 7, 31):
+            n = lens[b]
+            if n == 0:
+                assert np.all(got[0][b, hq] == 0) and np.all(got[1][b, hq] == -1)
+                continue
+            h = hq // cfg.G
+            want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n, cfg.topk)
+            compare_head(got, want, b, hq, n, dec.drow)
