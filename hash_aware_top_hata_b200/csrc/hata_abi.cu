@@ -175,6 +175,21 @@ int64_t hata_dist_row_bytes(int64_t max_seq_len)
     return max_seq_len <= 0 ? 0 : ceil_div(max_seq_len, kChunk) * kChunk;
 }
 
+int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
+{
+    if (B <= 0 || H_q <= 0 || topk <= 0 || !valid_dtype(kv_dtype)) {
+        fail(HATA_ERR_INVALID_ARG, "B=%d H_q=%d topk=%d kv_dtype=%d", B, H_q, topk,
+             int(kv_dtype));
+        return -1;
+    }
+    int n = 0;
+    if (cudaError_t e = attend_launch_count(B, H_q, topk, kv_dtype == HATA_DT_BF16, &n)) {
+        cuda_fail(e, "occupancy query");
+        return -1;
+    }
+    return 3 + n;
+}
+
 hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
                                void *V, hata_dtype_t kv_dtype, int64_t n_cap,
                                const int32_t *seq_len, int64_t max_seq_len, const void *k_new,

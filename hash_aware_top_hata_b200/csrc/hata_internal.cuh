@@ -218,6 +218,9 @@ cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
 cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s);  // sets a.n_workers
 cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s);
+// Kernels launch_attend + launch_combine issue for these sizes on the current
+// device: 1 when the heads are merged inside the attention CTAs, else 2.
+cudaError_t attend_launch_count(int B, int H_q, int topk, bool bf16, int *n);
 cudaError_t launch_dense(const DenseArgs &a, bool bf16, cudaStream_t s);
 
 }  // namespace hata

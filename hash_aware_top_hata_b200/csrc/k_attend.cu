@@ -772,7 +772,25 @@ cudaError_t occupancy_grid(Kernel kernel, int threads, size_t smem, int64_t *gri
     return e;
 }
 
+// Heads that nearly fill one wave of P CTAs: a CTA per head, merged in
+// shared memory, saves the combine launch and its completion gap.
+bool head_per_cta(int B, int H_q, int topk, int64_t P)
+{
+    const int64_t heads = int64_t(B) * H_q;
+    return heads * 5 >= P * 4 && heads <= P && topk >= 16 * tc::kTcWarps;
+}
+
 }  // namespace
+
+cudaError_t attend_launch_count(int B, int H_q, int topk, bool bf16, int *n)
+{
+    int64_t P = 0;
+    *n = 2;
+    if (!bf16) return cudaSuccess;
+    if (cudaError_t e = occupancy_grid(attend_tc_kernel, tc::kThreads, tc::kSmem, &P)) return e;
+    if (head_per_cta(B, H_q, topk, P)) *n = 1;
+    return cudaSuccess;
+}
 
 cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
 {
@@ -783,11 +801,8 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
         int64_t NW = P * tc::kTcWarps;
         if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
         if (NW > T) NW = T;
-        // Heads that nearly fill one wave of CTAs: a CTA per head, merged in
-        // shared memory, saves the combine launch and its completion gap.
-        const int64_t heads = int64_t(a.B) * a.H_q;
-        a.head_per_cta = heads * 5 >= P * 4 && heads <= P && a.topk >= 16 * tc::kTcWarps;
-        if (a.head_per_cta) NW = heads * tc::kTcWarps;
+        a.head_per_cta = head_per_cta(a.B, a.H_q, a.topk, P);
+        if (a.head_per_cta) NW = int64_t(a.B) * a.H_q * tc::kTcWarps;
         a.n_workers = NW;
         return launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
                           dim3(tc::kThreads), tc::kSmem, s, a);

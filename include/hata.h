@@ -116,6 +116,13 @@ size_t hata_decode_workspace_size(int B, int H_q, int H_kv, int64_t max_seq_len,
  * have at least: max_seq_len rounded up to the scoring chunk (4096). */
 int64_t hata_dist_row_bytes(int64_t max_seq_len);
 
+/* Number of kernels one hata_decode_step with these sizes launches on the
+ * current device (prep, score, select, attention and, unless the heads are
+ * merged inside the attention CTAs, the combine kernel): 4 or 5.  Returns -1
+ * (hata_last_error says why) for invalid sizes or if the device query fails.
+ * Host-only; launches nothing. */
+int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype);
+
 /* ------------------------------------------------------------------------
  * hata_decode_step -- one decode step of HATA for every (b, h_q) (Figure 2):
  *   0. optional append: if k_new != NULL its rows are hashed into

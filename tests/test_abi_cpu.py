@@ -125,3 +125,14 @@ def test_workspace_check_rejects_bad_workspace():
     assert H.lib().hata_workspace_check(NULL, 4096, ctypes.byref(flags), NULL) == \
         H.HATA_ERR_INVALID_ARG
     assert flags.value == 0
+
+
+def test_decode_kernel_launches_host_logic():
+    L = H.lib()
+    # fp32 caches take the SIMT attention kernel, always followed by the combine
+    assert H.hata_decode_kernel_launches(4, 32, 2048, torch.float32) == 5
+    for bad in ((0, 32, 2048, H.HATA_DT_BF16), (4, 0, 2048, H.HATA_DT_BF16),
+                (4, 32, 0, H.HATA_DT_BF16), (4, 32, 2048, 9)):
+        assert L.hata_decode_kernel_launches(*bad) == -1
+    with pytest.raises(H.HataError):
+        H.hata_decode_kernel_launches(4, 32, -1, torch.bfloat16)

@@ -400,3 +400,11 @@ def test_decode_head_per_cta_merge():
             h = hq // cfg.G
             want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n, cfg.topk)
             compare_head(got, want, b, hq, n, dec.drow)
+
+
+def test_decode_kernel_launch_count():
+    """128 heads at topk 2048 fill about one wave of attention CTAs (merged
+    in-CTA, no combine kernel); 32 heads do not."""
+    assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 4
+    assert H.hata_decode_kernel_launches(1, 32, 2048, torch.bfloat16) == 5
+    assert H.hata_decode_kernel_launches(4, 32, 100, torch.bfloat16) == 5  # too few rows per warp
