@@ -427,16 +427,35 @@ struct LaneOffsets {
 // g + 8, columns 2t and 2t + 1: only lanes with t == 0 see the two live
 // columns.  O[mt] in those lanes: dims 16 mt + g (O[mt][0] + O[mt][1]) and
 // 16 mt + g + 8 (O[mt][2] + O[mt][3]).
-__device__ __forceinline__ void attend_stage(int n, uint32_t Ks, const int32_t *rows,
+// The B operand of S^T = K Q^T for query row q (pre-scaled by scale_log2):
+// column 0 (lanes 0-3) holds bf16(q), column 1 (lanes 4-7) the remainder
+// q - bf16(q); the other columns are zero.
+__device__ __forceinline__ void load_query(const float *q, float scale_log2, int lane,
+                                           uint32_t (&qb)[8][2])
+{
+    const int part = (lane >> 2) & 1, q4 = lane & 3;
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) {
+        const int d0 = 16 * kt + 2 * q4;
+        if (lane < 8) {
+            const float2 x = __ldg(reinterpret_cast<const float2 *>(q + d0));
+            const float2 y = __ldg(reinterpret_cast<const float2 *>(q + d0 + 8));
+            qb[kt][0] = pack2(split(x.x * scale_log2, part), split(x.y * scale_log2, part));
+            qb[kt][1] = pack2(split(y.x * scale_log2, part), split(y.y * scale_log2, part));
+        } else {
+            qb[kt][0] = qb[kt][1] = 0u;
+        }
+    }
+}
+
+// vmask: bit j set if key j of the stage holds a row.
+__device__ __forceinline__ void attend_stage(uint32_t vmask, uint32_t Ks,
                                              const uint32_t (&qb)[8][2], const LaneOffsets &lo,
                                              float (&O)[8][4], float &m_ref, float &l_part,
                                              int lane)
 {
     const uint32_t Vs = Ks + kSub * kRowB;
     const int g = lane >> 2, t = lane & 3;
-    // keys of the stage that hold a row
-    const uint32_t vmask =
-        __ballot_sync(0xffffffffu, lane < kSub && lane < n && rows[lane < kSub ? lane : 0] >= 0);
     // ---- S^T = K Q^T: even / odd k-tiles in separate accumulators ----
     float S[2][4];
 #pragma unroll
@@ -533,7 +552,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     using namespace tc;
     extern __shared__ __align__(128) uint8_t smem[];  // [warp][kRingW][K | V], then indices
     __shared__ int32_t rows_s[kTcWarps][kRingW][kSub];
-    __shared__ __align__(16) float part_s[kTcWarps][kPartStride];  // head-per-CTA partials
     pdl_trigger();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -556,9 +574,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
         prod.init(&a, beg, end);
         cons.init(&a, beg, end);
     }
-    if (a.head_per_cta)  // a warp with no row of the head leaves an empty partial
-        for (int i = lane; i < kPartStride; i += 32) part_s[warp][i] = i == 0 ? -INFINITY : 0.0f;
-    __syncwarp();
     pdl_wait();  // the selected index lists
 
     // the CTA's slice of the index list (the first kIdxCap of it): all loads
@@ -621,8 +636,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     };
     for (int i = 0; i < kRingW - 1; ++i) issue_next();
 
-    const int g4 = lane >> 2, q4 = lane & 3;   // mma fragment coordinates
-    const int part = g4 & 1;                    // lanes 0-3: hi column, 4-7: lo column
     const LaneOffsets lo(lane);
     uint32_t qb[8][2];  // B operand of S^T: columns q_hi (lanes 0-3), q_lo (lanes 4-7)
     float O[8][4];
@@ -632,19 +645,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
     for (int s = 0; cons.next(cs); ++s) {
         if (cs.bh != cur_bh) {  // a new head: its query as hi/lo bf16 rows, fresh state
             cur_bh = cs.bh;
-            const float *q = a.q + int64_t(cs.bh) * kD;
-#pragma unroll
-            for (int kt = 0; kt < 8; ++kt) {
-                const int d0 = 16 * kt + 2 * q4;
-                if (lane < 8) {
-                    const float2 x = __ldg(reinterpret_cast<const float2 *>(q + d0));
-                    const float2 y = __ldg(reinterpret_cast<const float2 *>(q + d0 + 8));
-                    qb[kt][0] = pack2(split(x.x * a.scale_log2, part), split(x.y * a.scale_log2, part));
-                    qb[kt][1] = pack2(split(y.x * a.scale_log2, part), split(y.y * a.scale_log2, part));
-                } else {
-                    qb[kt][0] = qb[kt][1] = 0u;
-                }
-            }
+            load_query(a.q + int64_t(cs.bh) * kD, a.scale_log2, lane, qb);
 #pragma unroll
             for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
             m_ref = -INFINITY;
@@ -655,35 +656,130 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
         __syncwarp();
         const int slot = s % kRingW;
         issue_next();
-        attend_stage(cs.n, wring + uint32_t(slot * kStageBytes), rows_s[warp][slot], qb, lo, O,
-                     m_ref, l_part, lane);
+        const int32_t *rows = rows_s[warp][slot];
+        const uint32_t vmask = __ballot_sync(
+            0xffffffffu, lane < kSub && lane < cs.n && rows[lane < kSub ? lane : 0] >= 0);
+        attend_stage(vmask, wring + uint32_t(slot * kStageBytes), qb, lo, O, m_ref, l_part, lane);
 
-        if (cs.last) {
-            if (a.head_per_cta)
-                store_partial(part_s[warp], O, m_ref, l_part, lane);
-            else
-                publish(a, cs, wid, NW, T, O, m_ref, l_part, lane);
-        }
+        if (cs.last) publish(a, cs, wid, NW, T, O, m_ref, l_part, lane);
     }
     cp_async_wait<0>();
-    if (a.head_per_cta) {
-        // the CTA holds all of head blockIdx.x: merge its warps' partials
-        __syncthreads();
-        if (tid < kD) {
-            float M = -INFINITY;
+}
+
+// Head-per-CTA form, for heads that fill about one wave of CTAs: CTA bh
+// attends the whole selected list of head bh.  Warp w takes the w-th eighth
+// of the list (plain index arithmetic, no walker), the gather addresses are
+// one multiply-add from the slab's base, and the warps' partials are merged
+// in shared memory, so no combine launch follows.  Needs topk <= kIdxCap.
+__global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs a)
+{
+    using namespace tc;
+    extern __shared__ __align__(128) uint8_t smem[];  // [warp][kRingW][K | V], then indices
+    __shared__ __align__(16) float part_s[kTcWarps][kPartStride];
+    pdl_trigger();
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / a.H_q, h = (bh - b * a.H_q) / a.G;
+    // seq_len is a step input: everything up to the wait overlaps the selection
+    const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);
+    const int keff = int(int64_t(a.topk) < len ? int64_t(a.topk) : len);
+    const int r0 = int(int64_t(warp) * a.topk / kTcWarps);
+    int r1 = int(int64_t(warp + 1) * a.topk / kTcWarps);
+    r1 = r1 < keff ? r1 : keff;
+    const int n_rows = r1 > r0 ? r1 - r0 : 0;
+    const int n_st = (n_rows + kSub - 1) / kSub;
+
+    const int p = lane & 15, rh = lane >> 4;  // 16-byte piece p of rows 8 rh .. 8 rh + 7
+    const int64_t slab = (int64_t(b) * a.H_kv + h) * a.n_cap;
+    const uint8_t *Kp = static_cast<const uint8_t *>(a.K) + slab * kRowB + p * 16;
+    const uint8_t *Vp = static_cast<const uint8_t *>(a.V) + slab * kRowB + p * 16;
+    const uint32_t wring = smem_addr(smem) + uint32_t(warp * kRingW * kStageBytes);
+    int32_t *idx_s = reinterpret_cast<int32_t *>(smem + kRingBytes);
+    uint32_t doff[8];
 #pragma unroll
-            for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, part_s[w][0]);
-            float L = 0.0f, A = 0.0f;
-            if (M != -INFINITY) {
+    for (int u = 0; u < 8; ++u) doff[u] = swz(8 * rh + u, p);
+    // a warp with no row of the head leaves an empty partial
+    for (int i = lane; i < kPartStride; i += 32) part_s[warp][i] = i == 0 ? -INFINITY : 0.0f;
+    __syncwarp();
+    pdl_wait();  // the selected index lists
+
+    {  // the head's list (its first keff entries): all loads first, then the stores
+        const int32_t *src = a.idx + int64_t(bh) * a.topk;
+        constexpr int kPer = kIdxCap / kThreads;
+        int32_t v[kPer];
 #pragma unroll
-                for (int w = 0; w < kTcWarps; ++w) {
-                    const float wt = part_s[w][0] == -INFINITY ? 0.0f : exp2f(part_s[w][0] - M);
-                    L = fmaf(part_s[w][1], wt, L);
-                    A = fmaf(part_s[w][4 + tid], wt, A);
-                }
-            }
-            a.out[int64_t(blockIdx.x) * kD + tid] = L > 0.0f ? A / L : 0.0f;
+        for (int u = 0; u < kPer; ++u) {
+            const int i = tid + u * kThreads;
+            v[u] = i < keff ? __ldg(src + i) : -1;
         }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = tid + u * kThreads;
+            if (i < keff) idx_s[i] = v[u];
+        }
+    }
+    __syncthreads();
+
+    // stage s of this warp (rows r0 + 16 s ...) into ring slot s % kRingW;
+    // always commits one group
+    auto issue = [&](int s) {
+        if (s < n_st) {
+            const uint32_t Ks = wring + uint32_t((s % kRingW) * kStageBytes);
+            const uint32_t Vs = Ks + kSub * kRowB;
+            const int x0 = r0 + s * kSub + 8 * rh;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int32_t row = x0 + u < r1 ? idx_s[x0 + u] : -1;
+                // the selection never yields an index outside [0, len); the
+                // check keeps a corrupted list from steering a copy outside
+                // the cache.  Rows without a key are zero-filled.
+                const bool ok = row >= 0 && row < len;
+                const int64_t off = ok ? int64_t(row) * kRowB : 0;
+                cp_async16_zfill(Ks + doff[u], Kp + off, ok ? 16u : 0u);
+                cp_async16_zfill(Vs + doff[u], Vp + off, ok ? 16u : 0u);
+            }
+        }
+        cp_async_commit();
+    };
+    for (int i = 0; i < kRingW - 1; ++i) issue(i);
+
+    const LaneOffsets lo(lane);
+    uint32_t qb[8][2];
+    load_query(a.q + int64_t(bh) * kD, a.scale_log2, lane, qb);
+    float O[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
+    float m_ref = -INFINITY, l_part = 0.0f;
+
+    for (int s = 0; s < n_st; ++s) {
+        cp_async_wait<kRingW - 2>();
+        __syncwarp();
+        issue(s + kRingW - 1);
+        const int x = r0 + s * kSub + lane;
+        const int32_t row = lane < kSub && x < r1 ? idx_s[x] : -1;
+        const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0 && row < len);
+        attend_stage(vmask, wring + uint32_t((s % kRingW) * kStageBytes), qb, lo, O, m_ref,
+                     l_part, lane);
+    }
+    cp_async_wait<0>();
+    if (n_st > 0) store_partial(part_s[warp], O, m_ref, l_part, lane);
+
+    // merge the warps' partials of the head
+    __syncthreads();
+    if (tid < kD) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, part_s[w][0]);
+        float L = 0.0f, A = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kTcWarps; ++w) {
+                const float wt = part_s[w][0] == -INFINITY ? 0.0f : exp2f(part_s[w][0] - M);
+                L = fmaf(part_s[w][1], wt, L);
+                A = fmaf(part_s[w][4 + tid], wt, A);
+            }
+        }
+        a.out[int64_t(bh) * kD + tid] = L > 0.0f ? A / L : 0.0f;
     }
 }
 
@@ -777,7 +873,8 @@ cudaError_t occupancy_grid(Kernel kernel, int threads, size_t smem, int64_t *gri
 bool head_per_cta(int B, int H_q, int topk, int64_t P)
 {
     const int64_t heads = int64_t(B) * H_q;
-    return heads * 5 >= P * 4 && heads <= P && topk >= 16 * tc::kTcWarps;
+    return heads * 5 >= P * 4 && heads <= P && topk >= 16 * tc::kTcWarps &&
+           topk <= tc::kIdxCap;
 }
 
 }  // namespace
@@ -802,7 +899,14 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
         if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
         if (NW > T) NW = T;
         a.head_per_cta = head_per_cta(a.B, a.H_q, a.topk, P);
-        if (a.head_per_cta) NW = int64_t(a.B) * a.H_q * tc::kTcWarps;
+        if (a.head_per_cta) {
+            a.n_workers = 0;
+            if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(attend_head_kernel),
+                                                 tc::kSmem))
+                return e;
+            return launch_pdl(attend_head_kernel, dim3(unsigned(int64_t(a.B) * a.H_q)),
+                              dim3(tc::kThreads), tc::kSmem, s, a);
+        }
         a.n_workers = NW;
         return launch_pdl(attend_tc_kernel, dim3(unsigned(ceil_div(NW, tc::kTcWarps))),
                           dim3(tc::kThreads), tc::kSmem, s, a);
