@@ -512,6 +512,8 @@ def run_hata(args, world, rank, local):
     attend_ms = [e[3].elapsed_time(e[4]) for e in kevs]
     combine_ms = [e[4].elapsed_time(e[5]) for e in kevs]
     n_launch = H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.topk, w.K.dtype)
+    # four launches: one CTA per head, merged in shared memory
+    attend_kernel = "attend_head_kernel" if n_launch == 4 else "attend_tc_kernel"
     split_ms = [e[0].elapsed_time(e[5]) for e in kevs]
     ms = statistics.mean(step_ms)
     ms_max = max_over_ranks(world, ms)
@@ -539,10 +541,10 @@ def run_hata(args, world, rank, local):
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian q/K/V, 2% planted keys, N(0,1/128) W_H)",
         "config": config_dict(cfg, "flushed before every timed step (512 MiB read)"),
-        "roofline": {"bound": "hbm", "kernel": "attend (gather + softmax)",
+        "roofline": {"bound": "hbm", "kernel": f"{attend_kernel} (gather + softmax)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(cfg, "attend_tc_kernel",
+                     "traffic": profiled_traffic(cfg, attend_kernel,
                                                  "hash_aware_top_hata_b200/csrc/k_attend.cu"),
                      "peak_kind": peak_kind, "algorithmic_bytes_per_launch": attend_bytes},
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
