@@ -20,8 +20,7 @@
 // thread its output position, and the ties a thread may take follow from
 // the ties before it: taken_before = min(ties_before, room).  Indices are
 // written straight to the head's list, ascending.
-#include "block_scan.cuh"
-#include "hata_internal.cuh"
+#include "select_common.cuh"
 #include "tma.cuh"
 
 namespace hata {
@@ -39,106 +38,6 @@ __device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_
     int64_t l = sl < 0 ? 0 : sl;
     l = l < max_len ? l : max_len;
     return l < n_cap ? l : n_cap;
-}
-
-// Byte-wise zero test of four distances (bytes of w: 0..128 or the pad
-// 255) against T4 (one value in every byte), plain integer logic: bit 7 of
-// each byte of the result is set iff the byte equals T; the other bits are
-// zero.  x = d ^ T is zero iff equal; (x & 0x7f) + 0x7f sets bit 7 iff the
-// low seven bits of x are not all zero (no carry out).
-__device__ __forceinline__ uint32_t byte_eq_mask(uint32_t w, uint32_t T4)
-{
-    const uint32_t x = w ^ T4;
-    const uint32_t t = (x & 0x7f7f7f7fu) + 0x7f7f7f7fu;
-    return ~(t | x) & 0x80808080u;
-}
-
-// Mask word of 32 distances, bit 8e + w <-> distance 4w + e; the same bits
-// in token order (bit 4w + e).  Only words that select something need it.
-__device__ __forceinline__ uint32_t to_token_order(uint32_t m)
-{
-    uint32_t t = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        // bits w, w+8, w+16, w+24 -> bits 21..24 (the products do not overlap)
-        const uint32_t x = (m >> w) & 0x01010101u;
-        t |= ((x * 0x00204081u) >> 21 & 0xfu) << (4 * w);
-    }
-    return t;
-}
-
-// T = the smallest distance t with #(dist <= t) >= k_eff, #(dist < T), and
-// the keys below T and at T in the tiles before `tile`, from head bh's tile
-// histograms.  One warp; lane l owns bins 5l .. 5l+4; out: {T, #(< T),
-// below-T before the tile, at-T before the tile}.
-__device__ __forceinline__ void head_threshold(const SelectArgs &a, size_t bh, int k_eff, int tile,
-                                               int lane, int *out)
-{
-    constexpr int kRegTiles = 4;  // rows held in registers per round
-    const uint32_t *hrow = a.hist + bh * size_t(a.n_tiles) * kHistStride;
-    const int n_tiles = int(a.n_tiles);
-    auto row_bins = [&](int t, uint32_t (&v)[5]) {
-#pragma unroll
-        for (int e = 0; e < 5; ++e)
-            v[e] = lane * 5 + e < kBins ? __ldg(hrow + t * kHistStride + lane * 5 + e) : 0u;
-    };
-    uint32_t tot[5] = {0u, 0u, 0u, 0u, 0u}, pre[5] = {0u, 0u, 0u, 0u, 0u};
-    // rounds of kRegTiles rows: all loads of a round are issued before any
-    // is summed, so a round costs one round trip to L2
-    for (int t0 = 0; t0 < n_tiles; t0 += kRegTiles) {
-        uint32_t rv[kRegTiles][5];
-#pragma unroll
-        for (int t = 0; t < kRegTiles; ++t) {
-            if (t0 + t < n_tiles) {
-                row_bins(t0 + t, rv[t]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < 5; ++e) rv[t][e] = 0u;
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < kRegTiles; ++t)
-#pragma unroll
-            for (int e = 0; e < 5; ++e) {
-                tot[e] += rv[t][e];
-                pre[e] += t0 + t < tile ? rv[t][e] : 0u;
-            }
-    }
-    const uint32_t run = tot[0] + tot[1] + tot[2] + tot[3] + tot[4];
-    uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
-    int Tl = -1;
-    uint32_t less_l = 0;
-#pragma unroll
-    for (int e = 0; e < 5; ++e) {
-        if (Tl < 0 && lane * 5 + e < kBins && acc + tot[e] >= uint32_t(k_eff)) {
-            Tl = lane * 5 + e;
-            less_l = acc;
-        }
-        acc += tot[e];
-    }
-    // cumulative counts are monotone: the lowest lane that found a bin holds T
-    const unsigned found = __ballot_sync(0xffffffffu, Tl >= 0);
-    const int src = found ? __ffs(int(found)) - 1 : 0;
-    const int T = found ? __shfl_sync(0xffffffffu, Tl, src) : 128;  // unreachable fallback
-    const int n_less = found ? __shfl_sync(0xffffffffu, int(less_l), src) : 0;
-    int l = 0, q = 0;
-#pragma unroll
-    for (int e = 0; e < 5; ++e) {
-        const int bin = lane * 5 + e;
-        l += bin < T ? int(pre[e]) : 0;
-        q += bin == T ? int(pre[e]) : 0;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        l += __shfl_xor_sync(0xffffffffu, l, o);
-        q += __shfl_xor_sync(0xffffffffu, q, o);
-    }
-    if (lane == 0) {
-        out[0] = T;
-        out[1] = n_less;
-        out[2] = l;
-        out[3] = q;
-    }
 }
 
 __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
@@ -168,7 +67,9 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     // the tiles before this one from the head's tile histograms (one round
     // trip to L2 per 4 tiles), ahead of its own distance loads;
     // the other warps' distance loads are in flight meanwhile ----
-    if (tid < 32) head_threshold(a, bh, k_eff, tile, tid, s_thr);
+    if (tid < 32)
+        head_threshold(a.hist + bh * size_t(a.n_tiles) * kHistStride, int(a.n_tiles), k_eff,
+                       tile, tid, s_thr);
     // the warp's 4 KB arrive by coalesced 16-byte copies (lane l: bytes
     // 16l .. 16l+15 of each 512-byte block) into a swizzled shared tile,
     // piece v of thread t at t*128 + 16*(v ^ (t & 7)), so that each thread
@@ -201,11 +102,6 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
         return;  // every key of the head is placed before this tile (CTA-uniform)
 
     // ---- masks: group m = pieces 2m, 2m+1 = distances 32m .. 32m+31 ----
-    // "< T" and "<= T" from one (d | 0x80) per byte: (d | 0x80) - t never
-    // borrows for t <= 128, so only T = 128 (where "<= T" means "not the pad
-    // 255") needs the zero-byte test.  Ties = "<= T" and not "< T".  Flags
-    // move into the packed word with a multiply-high and an add (a right
-    // shift of the word so far; the bits never overlap).
     const uint32_t T4 = uint32_t(T) * 0x01010101u, T4p = T4 + 0x01010101u;
     uint32_t lt_bits[kGroups], eq_bits[kGroups];
     int n_lt = 0, n_eq = 0;
@@ -213,20 +109,11 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     for (int m = 0; m < kGroups; ++m) {
         const uint32_t dw[8] = {dv[2 * m].x,     dv[2 * m].y,     dv[2 * m].z,     dv[2 * m].w,
                                 dv[2 * m + 1].x, dv[2 * m + 1].y, dv[2 * m + 1].z, dv[2 * m + 1].w};
-        uint32_t lb = 0, le = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            const uint32_t wh = dw[w] | 0x80808080u;
-            const uint32_t lt = ~(dw[w] | (wh - T4)) & 0x80808080u;
-            const uint32_t lq = T < 128 ? ~(dw[w] | (wh - T4p)) & 0x80808080u
-                                        : ~byte_eq_mask(dw[w], 0xffffffffu) & 0x80808080u;
-            // flag of byte e: bit 8e + 7 of word w -> bit 8e + w of the group
-            lb = __umulhi(lb, 0x80000000u) + lt;
-            le = __umulhi(le, 0x80000000u) + lq;
-        }
-        lt_bits[m] = lb;
-        eq_bits[m] = le & ~lb;
-        n_lt += __popc(lb);
+        if (T < 128)
+            group_masks<false>(dw, T4, T4p, lt_bits[m], eq_bits[m]);
+        else
+            group_masks<true>(dw, T4, T4p, lt_bits[m], eq_bits[m]);
+        n_lt += __popc(lt_bits[m]);
         n_eq += __popc(eq_bits[m]);
     }
 
@@ -238,41 +125,11 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     int my_take = take_tile - before.y;
     my_take = my_take < 0 ? 0 : (my_take > n_eq ? n_eq : my_take);
 
-    int pos = less_before + (ties_before < r_ties ? ties_before : r_ties) + before.x + taken_before;
-#pragma unroll
-    for (int m = 0; m < kGroups; ++m) {
-        uint32_t sel = lt_bits[m];
-        if (my_take > 0 && eq_bits[m]) {
-            const int ne = __popc(eq_bits[m]);
-            if (my_take >= ne) {  // every tie of this word
-                sel |= eq_bits[m];
-                my_take -= ne;
-            } else {              // the lowest-index my_take ties
-                uint32_t eqt = to_token_order(eq_bits[m]), kept = 0u;
-                for (; my_take > 0; --my_take) {
-                    kept |= eqt & (0u - eqt);
-                    eqt &= eqt - 1u;
-                }
-                uint32_t selt = to_token_order(sel) | kept;
-                while (selt) {
-                    const int e = __ffs(int(selt)) - 1;
-                    selt &= selt - 1u;
-                    if (pos < a.topk) idx[pos] = my0 + 32 * m + e;
-                    ++pos;
-                }
-                continue;
-            }
-        }
-        if (sel) {
-            uint32_t selt = to_token_order(sel);
-            while (selt) {
-                const int e = __ffs(int(selt)) - 1;
-                selt &= selt - 1u;
-                if (pos < a.topk) idx[pos] = my0 + 32 * m + e;
-                ++pos;
-            }
-        }
-    }
+    const int pos =
+        less_before + (ties_before < r_ties ? ties_before : r_ties) + before.x + taken_before;
+    emit_selected(lt_bits, eq_bits, my_take, pos, my0, [&](int p, int tok) {
+        if (p < a.topk) idx[p] = tok;
+    });
 }
 
 }  // namespace

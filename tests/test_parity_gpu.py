@@ -408,3 +408,23 @@ def test_decode_kernel_launch_count():
     assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 4
     assert H.hata_decode_kernel_launches(1, 32, 2048, torch.bfloat16) == 5
     assert H.hata_decode_kernel_launches(4, 32, 100, torch.bfloat16) == 5  # too few rows per warp
+
+
+def test_one_wave_of_heads_ties_across_tiles():
+    """128 heads (one attention CTA per head): a run of identical keys forms
+    the boundary bucket across selection tiles, and the lower-index ties
+    must win; lengths cover a full row, a partial one and k_eff = len."""
+    cfg = wl.Config("tie-fused", 4, 32, 8, 20000, 3000, "bf16", 0.0, 0.0, 0, 1)
+    w = wl.make_workload(cfg, 53, device="cuda", steps=1)
+    w.K[:, :, 3000:14000] = w.K[:, :, 7:8].clone()
+    heads = [(b, hq) for b in range(cfg.B) for hq in (0, 5, 31)]
+    slabs = host_slabs(w, sorted({(b, hq // cfg.G) for b, hq in heads}))
+    dec = GpuDecoder(w, cfg.topk)
+    assert H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.topk, torch.bfloat16) == 4
+    lens = [cfg.N, 17001, 2999, 19999]
+    got = dec.step(w.q[0], lens)
+    Wn = w.W_H.cpu().numpy()
+    for b, hq in heads:
+        h = hq // cfg.G
+        want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), lens[b], cfg.topk)
+        compare_head(got, want, b, hq, lens[b], dec.drow)
