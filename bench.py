@@ -324,9 +324,10 @@ def extras(args, cfg, w, codes, ws, out, seq, flush, stream, W_steps, K_steps, w
 
 def more_legs(cfg, w, codes, ws, out, seq, flush, stream, t0, K_steps):
     """Labelled side measurements of the same workload: warm-L2 step time,
-    needle recall, the step with the K/V caches in host memory, prefill key
-    encoding against the FP32 peak, torch SDPA dense decode, and K_steps
-    consecutive decode steps replayed from one CUDA Graph."""
+    needle recall, the step with the K/V caches in host memory, the step
+    with 64- and 32-bit codes, prefill key encoding against the FP32 peak,
+    torch SDPA dense decode, and K_steps consecutive decode steps replayed
+    from one CUDA Graph."""
     B, Hq, Hkv, N, G = cfg.B, cfg.H_q, cfg.H_kv, cfg.N, cfg.G
     scale = 1.0 / math.sqrt(128)
     dev = out.device
@@ -384,6 +385,28 @@ def more_legs(cfg, w, codes, ws, out, seq, flush, stream, t0, K_steps):
         del Kh, Vh
     except RuntimeError as e:  # pinned host memory unavailable
         res["kv_host"] = {"unavailable": str(e).splitlines()[0][:120]}
+
+    # ---- narrower codes (the page's r = 64 / 32 ablation): the same step
+    # with r-bit codes from the leading r columns of W_H ----
+    res["narrow_codes"] = {}
+    for r in (64, 32):
+        Wr = w.W_H[:, :, :r].contiguous()
+        codes_r = torch.empty((B, Hkv, w.n_cap, r // 32), dtype=torch.int32, device=dev)
+        H.hata_hash_keys(w.K, Wr, codes_r, 0, N)
+        nr_ev = [ev_pair() for _ in range(3)]
+        for i in range(5):
+            flush()
+            if i >= 2:
+                nr_ev[i - 2][0].record(stream)
+            H.hata_decode_step(w.q[t0 + i], Wr, codes_r, w.K, w.V, seq[t0 + i], w.n_cap,
+                               cfg.topk, scale, ws, out, k_new=w.k_new[t0 + i],
+                               v_new=w.v_new[t0 + i])
+            if i >= 2:
+                nr_ev[i - 2][1].record(stream)
+        torch.cuda.synchronize()
+        res["narrow_codes"][f"r{r}_us_per_step"] = round(
+            statistics.median(a.elapsed_time(b) for a, b in nr_ev) * 1e3, 1)
+        del codes_r
 
     # ---- prefill key encoding (hata_hash_keys over the whole cache) ----
     pe = [ev_pair() for _ in range(3)]

@@ -42,7 +42,8 @@ bool valid_dtype(hata_dtype_t t) { return t == HATA_DT_BF16 || t == HATA_DT_F32;
 hata_status_t check_dims(int d, int r)
 {
     if (d != kD) return fail(HATA_ERR_UNSUPPORTED, "head_dim d=%d: only %d is supported", d, kD);
-    if (r != kRbit) return fail(HATA_ERR_UNSUPPORTED, "hash bits r=%d: only %d is supported", r, kRbit);
+    if (r != 32 && r != 64 && r != kRbit)
+        return fail(HATA_ERR_UNSUPPORTED, "hash bits r=%d: 32, 64 or %d are supported", r, kRbit);
     return HATA_OK;
 }
 
@@ -130,7 +131,7 @@ hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t n_cap
     if (n == 0) return ok();
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = launch_hash_prefill(K, kv_dtype == HATA_DT_BF16, n_cap, W_H, codes, B,
-                                              H_kv, pos0, n, s);
+                                              H_kv, pos0, n, r / 32, s);
     return e == cudaSuccess ? ok() : cuda_fail(e, "hash_keys launch");
 }
 
@@ -160,6 +161,7 @@ hata_status_t hata_append_code(const void *k_new, hata_dtype_t kv_dtype, const f
     a.H_kv = H_kv;
     a.G = 1;
     a.kv_bf16 = kv_dtype == HATA_DT_BF16;
+    a.words = r / 32;
     const cudaError_t e = launch_prep(a, B, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "append_code launch");
 }
@@ -269,6 +271,7 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     p.H_kv = H_kv;
     p.G = G;
     p.kv_bf16 = kv_dtype == HATA_DT_BF16;
+    p.words = r / 32;
     if ((e = launch_prep(p, B * G + (k_new ? B : 0), s)) != cudaSuccess)
         return cuda_fail(e, "prep launch");
     if ((e = ev.record(1)) != cudaSuccess) return cuda_fail(e, "event record");
@@ -288,6 +291,7 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     sa.H_kv = H_kv;
     sa.G = G;
     sa.zgroups = L.zgroups;
+    sa.words = r / 32;
     if ((e = launch_score(sa, s)) != cudaSuccess) return cuda_fail(e, "score launch");
     if ((e = ev.record(2)) != cudaSuccess) return cuda_fail(e, "event record");
 

@@ -12,9 +12,9 @@
 namespace hata {
 
 constexpr int kD = 128;         // head_dim (the page's models all use 128)
-constexpr int kRbit = 128;      // hash bits (rbit = 128 on the HATA page)
+constexpr int kRbit = 128;      // widest hash (rbit = 128 on the HATA page; 32 and 64 too)
 constexpr int kWords = kRbit / 32;
-constexpr int kBins = kRbit + 1;        // Hamming distances 0..128
+constexpr int kBins = kRbit + 1;        // Hamming distances 0..128 (fewer bins used below)
 constexpr int kChunk = 4096;            // tokens per scoring / selection chunk
 constexpr int kScoreThreads = 1024;
 constexpr int kScoreHeads = 8;          // query heads scored per code load (one CTA)
@@ -87,12 +87,12 @@ struct PrepArgs {
     float *q_copy;           // [B][H_q][128] device copy of q for the attention, or null
     const void *k_new;       // [B][H_kv][128] or null
     const void *v_new;       // [B][H_kv][128] or null
-    const float *W;          // [H_kv][128][128]
-    uint32_t *codes;         // [B][H_kv][n_cap][4]
+    const float *W;          // [H_kv][128][r]
+    uint32_t *codes;         // [B][H_kv][n_cap][r/32]
     void *K, *V;             // caches, written only if v_new
     const int32_t *pos;      // explicit append positions [B] (append API) or null
     const int32_t *seq_len;  // decode: append at seq_len[b]-1, flags
-    uint32_t *q_out;         // [B][H_q][4]
+    uint32_t *q_out;         // [B][H_q][r/32]
     uint32_t *flags;         // per-b flag words (decode) or null
     uint32_t *err_word;      // single OR-ed word (append API) or null
     uint32_t *hist;          // [B][H_q][hist_row_words] zeroed (decode) or null
@@ -101,17 +101,19 @@ struct PrepArgs {
     int64_t n_cap, max_seq_len;
     int B, H_q, H_kv, G;
     int kv_bf16;
+    int words;               // r / 32: code words per token (1, 2 or 4)
 };
 
 struct ScoreArgs {
-    const uint32_t *qcodes;  // [B][H_q][4]
-    const uint32_t *codes;   // [B][H_kv][n_cap][4]
+    const uint32_t *qcodes;  // [B][H_q][r/32]
+    const uint32_t *codes;   // [B][H_kv][n_cap][r/32]
     const int32_t *seq_len;
     uint8_t *dist;           // [B][H_q][dist_row]
     int64_t dist_row;
     uint32_t *hist;          // [B][H_q][n_tiles][kHistStride], zeroed by prep
     int64_t n_cap, max_seq_len, n_tiles;
     int B, H_q, H_kv, G, zgroups;
+    int words;               // r / 32 (1, 2 or 4)
 };
 
 struct SelectArgs {
@@ -212,7 +214,7 @@ cudaError_t ensure_smem_attr(const void *func, size_t bytes);
 // Launchers (each returns the cudaGetLastError() of its launch).
 cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const float *W,
                                 uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
-                                cudaStream_t s);
+                                int words, cudaStream_t s);
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);

@@ -53,8 +53,9 @@ constexpr int kPfRows = 8;                   // rows per warp and pass
 constexpr int kPfPass = kPfWarps * kPfRows;  // rows per CTA and pass
 constexpr int kPfRowsPerCta = 16 * kPfPass;  // 1024 rows per CTA
 
+template <int R>
 struct PfSmem {
-    float W[kD * kRbit];                     // this head's W_H, [i][j]
+    float W[kD * R];                         // this head's W_H, [i][j]
     float x[kPfWarps][kD][kPfRows];          // each warp's rows, [i][row]
 };
 
@@ -71,7 +72,7 @@ __device__ __forceinline__ uint64_t dup2(float v)
     return r;
 }
 
-template <bool BF16>
+template <bool BF16, int R>
 __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void *__restrict__ K,
                                                                     int64_t n_cap,
                                                                     const float *__restrict__ W,
@@ -79,15 +80,16 @@ __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void 
                                                                     int H_kv, int64_t pos0, int64_t n)
 {
     extern __shared__ __align__(16) uint8_t pf_raw[];
-    PfSmem &S = *reinterpret_cast<PfSmem *>(pf_raw);
+    PfSmem<R> &S = *reinterpret_cast<PfSmem<R> *>(pf_raw);
+    constexpr int kBL = R / 32, kLPW = 32 / kBL;  // bits per lane, lanes per code word
     const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t g_begin = int64_t(blockIdx.x) * kPfRowsPerCta;
     const int64_t g_end = min(g_begin + kPfRowsPerCta, n);
     const int64_t slab = (int64_t(b) * H_kv + h) * n_cap + pos0;  // row index of row 0
     {
-        const float *Wh = W + size_t(h) * kD * kRbit;
+        const float *Wh = W + size_t(h) * kD * R;
         const uint32_t base = smem_addr(S.W);
-        for (int c = tid; c < kD * kRbit / 4; c += kPfThreads)
+        for (int c = tid; c < kD * R / 4; c += kPfThreads)
             cp_async16_zfill(base + 16u * c, Wh + 4 * c, 16u);
         cp_async_commit();
     }
@@ -110,59 +112,67 @@ __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void 
         cp_async_wait<0>();
         __syncthreads();
         if (g0 + kPfPass < g_end) fetch(g0 + kPfPass);
-        uint64_t acc[kPfRows / 2][4];  // [row pair][column]
+        uint64_t acc[kPfRows / 2][kBL];  // [row pair][column]
 #pragma unroll
-        for (int p = 0; p < kPfRows / 2; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0ull;
-        const float4 *wrow = reinterpret_cast<const float4 *>(S.W) + lane;  // W[0][4l..4l+3]
+        for (int p = 0; p < kPfRows / 2; ++p)
+#pragma unroll
+            for (int c = 0; c < kBL; ++c) acc[p][c] = 0ull;
+        const float *wrow = S.W + kBL * lane;  // W[0][kBL l ..]
         const ulonglong2 *xrow = reinterpret_cast<const ulonglong2 *>(&S.x[warp][0][0]);
 #pragma unroll 4
         for (int i = 0; i < kD; ++i) {
-            const float4 w = wrow[i * (kRbit / 4)];
-            const uint64_t w0 = dup2(w.x), w1 = dup2(w.y), w2 = dup2(w.z), w3 = dup2(w.w);
+            // this lane's kBL values of W's row i (one 4-, 8- or 16-byte load)
+            float wv[kBL];
+            if constexpr (kBL == 4) {
+                const float4 w = *reinterpret_cast<const float4 *>(wrow + i * R);
+                wv[0] = w.x, wv[1] = w.y, wv[2] = w.z, wv[3] = w.w;
+            } else if constexpr (kBL == 2) {
+                const float2 w = *reinterpret_cast<const float2 *>(wrow + i * R);
+                wv[0] = w.x, wv[1] = w.y;
+            } else {
+                wv[0] = wrow[i * R];
+            }
             const ulonglong2 xa = xrow[i * 2], xb = xrow[i * 2 + 1];  // rows (0,1) (2,3) | (4,5) (6,7)
             const uint64_t xp[4] = {xa.x, xa.y, xb.x, xb.y};
 #pragma unroll
-            for (int p = 0; p < kPfRows / 2; ++p) {
-                ffma2(acc[p][0], xp[p], w0);
-                ffma2(acc[p][1], xp[p], w1);
-                ffma2(acc[p][2], xp[p], w2);
-                ffma2(acc[p][3], xp[p], w3);
+            for (int c = 0; c < kBL; ++c) {
+                const uint64_t w2 = dup2(wv[c]);
+#pragma unroll
+                for (int p = 0; p < kPfRows / 2; ++p) ffma2(acc[p][c], xp[p], w2);
             }
         }
-        // bits 4l..4l+3 of each row -> word l / 8 (bit 4 (l % 8) + c)
+        // bits kBL l .. kBL l + kBL - 1 of each row -> word l / kLPW, bit kBL (l % kLPW) + c
 #pragma unroll
         for (int r = 0; r < kPfRows; ++r) {
             const int p = r >> 1, sh = 32 * (r & 1);
             uint32_t v = 0;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < kBL; ++c)
                 v |= (__uint_as_float(uint32_t(acc[p][c] >> sh)) > 0.0f ? 1u : 0u) << c;
-            v <<= 4 * (lane & 7);
-            v |= __shfl_xor_sync(0xffffffffu, v, 1);
-            v |= __shfl_xor_sync(0xffffffffu, v, 2);
-            v |= __shfl_xor_sync(0xffffffffu, v, 4);
+            v <<= kBL * (lane % kLPW);
+#pragma unroll
+            for (int o = 1; o < kLPW; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
             const int64_t t = g0 + warp * kPfRows + r;
-            if ((lane & 7) == 0 && t < g_end) codes[(slab + t) * kWords + (lane >> 3)] = v;
+            if (lane % kLPW == 0 && t < g_end) codes[(slab + t) * (R / 32) + lane / kLPW] = v;
         }
     }
 }
 
 // --------------------------------------------------------- decode prep --
 // Rows of KV head h: B*G query rows (b-major), then B appended-key rows.
-// A CTA takes kPrepRows rows of one head with 128 threads per row (thread j
+// A CTA takes kPrepRows rows of one head with r threads per row (thread j
 // of a row owns bit j).  The head's W_H is staged once in shared memory
 // (asynchronous 16-byte copies by all threads) next to the rows, so every
 // step of a chain reads its two operands from shared memory at addresses
 // known in advance: the loads run ahead of the dependent FMAs instead of
 // exposing their latency at each of the 128 steps.
-constexpr int kPrepThreads = kD * kPrepRows;
-
-template <bool BF16>
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
+template <bool BF16, int R>
+__global__ void __launch_bounds__(R * kPrepRows) prep_kernel(PrepArgs a)
 {
+    constexpr int kPrepThreads = R * kPrepRows;
     pdl_trigger();  // the scoring kernel's setup (step inputs only) may start now
     const int h = blockIdx.y;
-    const int r = threadIdx.x / kD, j = threadIdx.x % kD;
+    const int r = threadIdx.x / R, j = threadIdx.x % R;
     const int nq = a.q ? a.B * a.G : 0;
     const int nk = a.k_new ? a.B : 0;
     const int rows = nq + nk;
@@ -176,12 +186,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
     if (r0 >= rows) return;
 
     extern __shared__ __align__(16) float smem[];
-    float *ws = smem;                  // [kD][kRbit]: this head's W_H
-    float *xs = smem + kD * kRbit;     // [kPrepRows][kD]: the rows
+    float *ws = smem;                  // [kD][R]: this head's W_H
+    float *xs = smem + kD * R;         // [kPrepRows][kD]: the rows
     {
-        const float *Wh = a.W + size_t(h) * kD * kRbit;
+        const float *Wh = a.W + size_t(h) * kD * R;
         const uint32_t base = smem_addr(ws);
-        for (int c = threadIdx.x; c < kD * kRbit / 4; c += kPrepThreads)
+        for (int c = threadIdx.x; c < kD * R / 4; c += kPrepThreads)
             cp_async16_zfill(base + 16u * c, Wh + 4 * c, 16u);
         cp_async_commit();
     }
@@ -211,7 +221,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
         const int b = row / a.G, g = row % a.G, hq = h * a.G + g;
         const size_t bh = size_t(b) * a.H_q + hq;
         if (a.hist)
-            for (int64_t t = j; t < a.hist_row_words; t += kD) a.hist[bh * a.hist_row_words + t] = 0u;
+            for (int64_t t = j; t < a.hist_row_words; t += R) a.hist[bh * a.hist_row_words + t] = 0u;
         if (a.flags && h == 0 && g == 0 && j == 0) {
             const int64_t sl = a.seq_len[b];
             uint32_t f = 0;
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
             xv[4 * k] = v.x, xv[4 * k + 1] = v.y, xv[4 * k + 2] = v.z, xv[4 * k + 3] = v.w;
         }
 #pragma unroll
-        for (int k = 0; k < kBlk; ++k) wv[k] = ws[(i0 + k) * kRbit + j];
+        for (int k = 0; k < kBlk; ++k) wv[k] = ws[(i0 + k) * R + j];
     };
     float acc = 0.0f;
     fetch(0, xa, wa);
@@ -254,22 +264,25 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
         if ((j & 31) == 0) {
             const int b = row / a.G, g = row % a.G;
             const size_t bh = size_t(b) * a.H_q + h * a.G + g;
-            a.q_out[bh * kWords + (j >> 5)] = word;
+            a.q_out[bh * (R / 32) + (j >> 5)] = word;
         }
     } else if (row < rows) {
         const int b = row - nq;
         const int64_t pos = a.pos ? int64_t(a.pos[b]) : int64_t(a.seq_len[b]) - 1;
         if (pos >= 0 && pos < a.n_cap) {
             const int64_t crow = (int64_t(b) * a.H_kv + h) * a.n_cap + pos;
-            if ((j & 31) == 0) a.codes[crow * kWords + (j >> 5)] = word;
+            if ((j & 31) == 0) a.codes[crow * (R / 32) + (j >> 5)] = word;
             if (a.v_new) {
                 // K from the staged row (a bf16 key is the upper half of its
                 // fp32 widening: exact); V copied by the row's first warp
-                const float xk = xs[r * kD + j];
-                if (BF16)
-                    static_cast<uint16_t *>(a.K)[crow * kD + j] = uint16_t(__float_as_uint(xk) >> 16);
-                else
-                    static_cast<float *>(a.K)[crow * kD + j] = xk;
+                for (int e = j; e < kD; e += R) {
+                    const float xk = xs[r * kD + e];
+                    if (BF16)
+                        static_cast<uint16_t *>(a.K)[crow * kD + e] =
+                            uint16_t(__float_as_uint(xk) >> 16);
+                    else
+                        static_cast<float *>(a.K)[crow * kD + e] = xk;
+                }
                 if (j < 32) {
                     const int64_t e0 = (int64_t(b) * a.H_kv + h) * kD;
                     if (BF16)
@@ -288,34 +301,56 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
 
 }  // namespace
 
+template <bool BF16, int R>
+cudaError_t launch_hash_prefill_t(const void *K, int64_t n_cap, const float *W, uint32_t *codes,
+                                  int B, int H_kv, int64_t pos0, int64_t n, cudaStream_t s)
+{
+    constexpr size_t kSmem = sizeof(PfSmem<R>);
+    if (cudaError_t e = ensure_smem_attr(
+            reinterpret_cast<const void *>(hash_prefill_kernel<BF16, R>), kSmem))
+        return e;
+    const dim3 grid(unsigned(ceil_div(n, kPfRowsPerCta)), unsigned(H_kv), unsigned(B));
+    hash_prefill_kernel<BF16, R><<<grid, kPfThreads, kSmem, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const float *W,
                                 uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
-                                cudaStream_t s)
+                                int words, cudaStream_t s)
 {
-    constexpr size_t kSmem = sizeof(PfSmem);
-    const void *fn = bf16 ? reinterpret_cast<const void *>(hash_prefill_kernel<true>)
-                          : reinterpret_cast<const void *>(hash_prefill_kernel<false>);
-    if (cudaError_t e = ensure_smem_attr(fn, kSmem)) return e;
-    const dim3 grid(unsigned(ceil_div(n, kPfRowsPerCta)), unsigned(H_kv), unsigned(B));
-    if (bf16)
-        hash_prefill_kernel<true><<<grid, kPfThreads, kSmem, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
-    else
-        hash_prefill_kernel<false><<<grid, kPfThreads, kSmem, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
+    switch (words * 2 + (bf16 ? 1 : 0)) {
+    case 8 + 1: return launch_hash_prefill_t<true, 128>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 8: return launch_hash_prefill_t<false, 128>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 4 + 1: return launch_hash_prefill_t<true, 64>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 4: return launch_hash_prefill_t<false, 64>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 2 + 1: return launch_hash_prefill_t<true, 32>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 2: return launch_hash_prefill_t<false, 32>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <bool BF16, int R>
+cudaError_t launch_prep_t(const PrepArgs &a, int rows_per_head, cudaStream_t s)
+{
+    constexpr size_t kSmem = sizeof(float) * (kD * R + kD * kPrepRows);
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(prep_kernel<BF16, R>), kSmem))
+        return e;
+    const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRows)), unsigned(a.H_kv));
+    prep_kernel<BF16, R><<<grid, R * kPrepRows, kSmem, s>>>(a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s)
 {
-    constexpr size_t kSmem = sizeof(float) * (kD * kRbit + kD * kPrepRows);
-    const void *fn = a.kv_bf16 ? reinterpret_cast<const void *>(prep_kernel<true>)
-                               : reinterpret_cast<const void *>(prep_kernel<false>);
-    if (cudaError_t e = ensure_smem_attr(fn, kSmem)) return e;
-    const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRows)), unsigned(a.H_kv));
-    if (a.kv_bf16)
-        prep_kernel<true><<<grid, kPrepThreads, kSmem, s>>>(a);
-    else
-        prep_kernel<false><<<grid, kPrepThreads, kSmem, s>>>(a);
-    return cudaGetLastError();
+    switch (a.words * 2 + (a.kv_bf16 ? 1 : 0)) {
+    case 8 + 1: return launch_prep_t<true, 128>(a, rows_per_head, s);
+    case 8: return launch_prep_t<false, 128>(a, rows_per_head, s);
+    case 4 + 1: return launch_prep_t<true, 64>(a, rows_per_head, s);
+    case 4: return launch_prep_t<false, 64>(a, rows_per_head, s);
+    case 2 + 1: return launch_prep_t<true, 32>(a, rows_per_head, s);
+    case 2: return launch_prep_t<false, 32>(a, rows_per_head, s);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace hata

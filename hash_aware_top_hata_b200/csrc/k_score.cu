@@ -73,6 +73,17 @@ __device__ __forceinline__ int hamming128(const uint4 &k, uint32_t k012, uint32_
     return __popc(o) + 2 * (__popc(c) + __popc(e));
 }
 
+// dist(k, q) for codes of W words (r = 32 W bits): the carry-save form for
+// W = 4, plain population counts of the XOR-ed words otherwise.
+template <int W>
+__device__ __forceinline__ int hamming_w(const uint4 &k, uint32_t k012, uint32_t k0123,
+                                         const uint4 &q, const uint2 &qd)
+{
+    if constexpr (W == 4) return hamming128(k, k012, k0123, q, qd);
+    if constexpr (W == 2) return __popc(k.x ^ q.x) + __popc(k.y ^ q.y);
+    return __popc(k.x ^ q.x);
+}
+
 // Histogram increment: one shared-memory reduction, no return value.
 __device__ __forceinline__ void red_shared_add1(uint32_t addr)
 {
@@ -83,7 +94,7 @@ __device__ __forceinline__ void red_shared_add1(uint32_t addr)
 // g*128 + 32i of the warp's tile (base tb = tile + lane) and one count in
 // bin d of head g (base hb).  kFull: all 128 tokens hold keys; otherwise the
 // tokens from nv on get the pad byte and no count.
-template <int GB, bool kFull>
+template <int GB, int W, bool kFull>
 __device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *qs,
                                            const uint2 *qd, int ng, uint32_t tb, uint32_t hb,
                                            int lane, int nv)
@@ -91,8 +102,8 @@ __device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *q
     uint32_t k012[4], k0123[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        k012[i] = cur[i].x ^ cur[i].y ^ cur[i].z;
-        k0123[i] = k012[i] ^ cur[i].w;
+        k012[i] = W == 4 ? cur[i].x ^ cur[i].y ^ cur[i].z : 0u;
+        k0123[i] = W == 4 ? k012[i] ^ cur[i].w : 0u;
     }
 #pragma unroll
     for (int g = 0; g < GB; ++g) {
@@ -101,7 +112,7 @@ __device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *q
             const uint2 qx = qd[g];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t d = uint32_t(hamming128(cur[i], k012[i], k0123[i], q, qx));
+                const uint32_t d = uint32_t(hamming_w<W>(cur[i], k012[i], k0123[i], q, qx));
                 const uint32_t t = tb + uint32_t(g * kUnit + 32 * i);
                 if (kFull || lane + 32 * i < nv) {
                     asm volatile("st.shared.u8 [%0], %1;" ::"r"(t), "r"(d) : "memory");
@@ -134,7 +145,7 @@ struct ScoreSmem {
     int next;                                   // units of the range handed out
 };
 
-template <int GB>
+template <int GB, int W>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -182,10 +193,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
         const int z = slab % a.zgroups, bh = slab / a.zgroups;
         const int h = bh % a.H_kv, b = bh / a.H_kv;
         const int g0 = z * kScoreHeads;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (g < min(GB, a.G - g0))
-            v = __ldg(reinterpret_cast<const uint4 *>(a.qcodes) +
-                      (size_t(b) * a.H_q + size_t(h) * a.G + g0 + g));
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);  // words past W stay zero
+        if (g < min(GB, a.G - g0)) {
+            const uint32_t *qp = a.qcodes + (size_t(b) * a.H_q + size_t(h) * a.G + g0 + g) * W;
+            if constexpr (W == 4) {
+                v = __ldg(reinterpret_cast<const uint4 *>(qp));
+            } else {
+                v.x = __ldg(qp);
+                if constexpr (W == 2) v.y = __ldg(qp + 1);
+            }
+        }
         S.key[kk].q[g] = v;
         const uint32_t q012 = v.x ^ v.y ^ v.z;
         S.key[kk].qd[g] = make_uint2(q012, q012 ^ v.w);
@@ -195,7 +212,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
     // ---- units of the range go to warps on demand (one shared counter):
     // the oldest warps of the SM, which the scheduler favours, take more,
     // and every warp finishes within about one unit of the others ----
-    const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes);
+    const uint32_t *codes = a.codes;  // W words per token
     const int n_range = f_end - f_beg;
     auto grab = [&]() {
         int u = 0;
@@ -210,12 +227,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
             const int uis = int(e & 0x0fffffffu);
             const KeyInfo &K = S.key[e >> 28];
             const int left = K.len - uis * kUnit;
-            const uint4 *src = codes + K.code0 + int64_t(uis) * kUnit + lane;
+            // token t of the unit -> ring slot t (16 bytes; W words used)
+            const uint32_t *src = codes + (K.code0 + int64_t(uis) * kUnit + lane) * W;
             const uint32_t dst = smem_addr(&S.ring[warp][slot][lane]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const bool ok = lane + 32 * i < left;  // zero fill past len, no read
-                cp_async16_zfill(dst + 512u * i, ok ? src + 32 * i : codes, ok ? 16u : 0u);
+                cp_async_zfill<4 * W>(dst + 512u * i, ok ? src + 32 * W * i : codes,
+                                      ok ? 4u * W : 0u);
             }
         }
         cp_async_commit();
@@ -247,11 +266,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
         } else {
             const uint32_t hb = smem_addr(&S.hist[kk][0][0]);
             if (c_left >= kUnit && K.ng == GB)
-                score_unit<GB, true>(cur, K.q, K.qd, GB, tb, hb, lane, kUnit);
+                score_unit<GB, W, true>(cur, K.q, K.qd, GB, tb, hb, lane, kUnit);
             else if (c_left >= kUnit)
-                score_unit<GB, true>(cur, K.q, K.qd, K.ng, tb, hb, lane, kUnit);
+                score_unit<GB, W, true>(cur, K.q, K.qd, K.ng, tb, hb, lane, kUnit);
             else
-                score_unit<GB, false>(cur, K.q, K.qd, K.ng, tb, hb, lane, c_left);
+                score_unit<GB, W, false>(cur, K.q, K.qd, K.ng, tb, hb, lane, c_left);
             __syncwarp();
             // the tile to the rows: lane l stores 16 bytes of head g0 + l / 8
 #pragma unroll
@@ -295,16 +314,16 @@ inline int64_t max_keys_per_range(int64_t U, int64_t P, int64_t nu, int64_t n_ti
     return m;
 }
 
-template <int GB>
+template <int GB, int W>
 cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
 {
-    const void *fn = reinterpret_cast<const void *>(score_kernel<GB>);
+    const void *fn = reinterpret_cast<const void *>(score_kernel<GB, W>);
     if (cudaError_t e = ensure_smem_attr(fn, sizeof(ScoreSmem<GB>))) return e;
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_kernel<GB>,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_kernel<GB, W>,
                                                           kScoreThreads, sizeof(ScoreSmem<GB>));
     if (e != cudaSuccess) return e;
     // One range per resident CTA (one per SM); more ranges only if a range
@@ -316,7 +335,7 @@ cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
     while (P < units && (ceil_div(units, P) > kMaxRange ||
                          max_keys_per_range(units, P, nu, a.n_tiles) > kMaxKeys))
         P = P + wave < units ? P + wave : units;
-    return launch_pdl(score_kernel<GB>, dim3(unsigned(P)), dim3(kScoreThreads), sizeof(ScoreSmem<GB>),
+    return launch_pdl(score_kernel<GB, W>, dim3(unsigned(P)), dim3(kScoreThreads), sizeof(ScoreSmem<GB>),
                       s, a);
 }
 
@@ -325,16 +344,33 @@ cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s)
 {
     const int gb = a.G < kScoreHeads ? a.G : kScoreHeads;
-    switch (gb) {
-    case 1: return launch_score_t<1>(a, s);
-    case 2: return launch_score_t<2>(a, s);
-    case 3: return launch_score_t<3>(a, s);
-    case 4: return launch_score_t<4>(a, s);
-    case 5: return launch_score_t<5>(a, s);
-    case 6: return launch_score_t<6>(a, s);
-    case 7: return launch_score_t<7>(a, s);
-    default: return launch_score_t<8>(a, s);
+    if (a.words == 4) {
+        switch (gb) {
+        case 1: return launch_score_t<1, 4>(a, s);
+        case 2: return launch_score_t<2, 4>(a, s);
+        case 3: return launch_score_t<3, 4>(a, s);
+        case 4: return launch_score_t<4, 4>(a, s);
+        case 5: return launch_score_t<5, 4>(a, s);
+        case 6: return launch_score_t<6, 4>(a, s);
+        case 7: return launch_score_t<7, 4>(a, s);
+        default: return launch_score_t<8, 4>(a, s);
+        }
     }
+    // narrower codes: groups of 3, 5-7 heads take the next wider instance
+    // (its unused head slots are skipped)
+    if (a.words == 2) {
+        if (gb == 1) return launch_score_t<1, 2>(a, s);
+        if (gb == 2) return launch_score_t<2, 2>(a, s);
+        if (gb <= 4) return launch_score_t<4, 2>(a, s);
+        return launch_score_t<8, 2>(a, s);
+    }
+    if (a.words == 1) {
+        if (gb == 1) return launch_score_t<1, 1>(a, s);
+        if (gb == 2) return launch_score_t<2, 1>(a, s);
+        if (gb <= 4) return launch_score_t<4, 1>(a, s);
+        return launch_score_t<8, 1>(a, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace hata

@@ -75,25 +75,44 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     // piece v of thread t at t*128 + 16*(v ^ (t & 7)), so that each thread
     // then reads its own 128 bytes without bank conflicts
     const uint32_t sbase = smem_addr(dist_s);
-    const int wbase = (tid >> 5) * 32 * kPer;  // this warp's first byte in the tile
-#pragma unroll
-    for (int k = 0; k < kPieces; ++k) {
-        const int byte = wbase + k * 512 + (tid & 31) * 16;
-        const int t = byte >> 7, v = (byte >> 4) & 7;
-        const int64_t g = int64_t(tile) * kTile + byte;
-        const bool in = g < a.dist_row;  // past the row: no read (padding below)
-        cp_async16_zfill(sbase + uint32_t(t * kPer + 16 * (v ^ (t & 7))), in ? drow + g : drow,
-                         in ? 16u : 0u);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncwarp();
+    const int lane = tid & 31, wbase = (tid >> 5) * 32 * kPer;  // the warp's first byte
+    const bool full = int64_t(tile + 1) * kTile <= a.dist_row;    // CTA-uniform
     uint4 dv[kPieces];
+    if (full) {
+        // copy k: byte wbase + 512 k + 16 lane = thread t = wbase/128 + 4k + lane/8, piece
+        // lane & 7; t & 7 = lane/8 + 4 (k & 1), so odd copies flip address bit 6
+        const uint8_t *src = drow + int64_t(tile) * kTile + wbase + 16 * lane;
+        const uint32_t o0 = uint32_t(wbase + 128 * (lane >> 3) + 16 * ((lane & 7) ^ (lane >> 3)));
+        const uint32_t d0 = sbase + o0, d1 = sbase + (o0 ^ 64u);
 #pragma unroll
-    for (int v = 0; v < kPieces; ++v)
-        dv[v] = my0 + 16 * v < a.dist_row
-                    ? *reinterpret_cast<const uint4 *>(dist_s + tid * kPer + 16 * (v ^ (tid & 7)))
-                    : make_uint4(~0u, ~0u, ~0u, ~0u);
+        for (int k = 0; k < kPieces; ++k)
+            cp_async16_zfill((k & 1 ? d1 : d0) + 512u * k, src + 512 * k, 16u);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        const uint8_t *mine = dist_s + tid * kPer;
+#pragma unroll
+        for (int v = 0; v < kPieces; ++v)
+            dv[v] = *reinterpret_cast<const uint4 *>(mine + 16 * (v ^ (tid & 7)));
+    } else {  // the row's last tile: pieces past the row read as padding
+#pragma unroll
+        for (int k = 0; k < kPieces; ++k) {
+            const int byte = wbase + k * 512 + lane * 16;
+            const int t = byte >> 7, v = (byte >> 4) & 7;
+            const int64_t g = int64_t(tile) * kTile + byte;
+            const bool in = g < a.dist_row;
+            cp_async16_zfill(sbase + uint32_t(t * kPer + 16 * (v ^ (t & 7))), in ? drow + g : drow,
+                             in ? 16u : 0u);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+#pragma unroll
+        for (int v = 0; v < kPieces; ++v)
+            dv[v] = my0 + 16 * v < a.dist_row
+                        ? *reinterpret_cast<const uint4 *>(dist_s + tid * kPer + 16 * (v ^ (tid & 7)))
+                        : make_uint4(~0u, ~0u, ~0u, ~0u);
+    }
     __syncthreads();
     const int T = s_thr[0], n_less = s_thr[1], lp = s_thr[2], tp = s_thr[3];
     const int r_ties = k_eff - n_less;  // boundary keys taken over the whole head

@@ -1,6 +1,6 @@
-// select_common.cuh -- the pieces of the histogram top-k shared by the
-// selection kernel (one CTA per 36K-token tile of a head) and the fused
-// selection inside the head-per-CTA attention kernel (one CTA per head).
+// select_common.cuh -- the pieces of the histogram top-k of the selection
+// kernel (one CTA per 36K-token tile of a head): the threshold from the tile
+// histograms, the byte-wise masks and the ordered emission.
 //
 // HATA review page (arXiv 2506.02572), major comment 1 (Algorithm 3): the
 // top-k runs over Hamming scores that take only 129 values; the boundary
@@ -140,6 +140,24 @@ __device__ __forceinline__ void head_threshold(const uint32_t *hrow, int n_tiles
     }
 }
 
+// Store the tokens of the set bits of sel (bit 8e + w <-> token tok + 4w + e)
+// at positions pos + (their rank in token order), without transposing the
+// word: the rank of a bit is the number of set bits of lower tokens (lower w,
+// or the same w and lower e).
+template <class Put>
+__device__ __forceinline__ void put_ranked(uint32_t sel, int pos, int tok, Put &put)
+{
+    uint32_t rest = sel;
+    while (rest) {
+        const int bit = __ffs(int(rest)) - 1;
+        rest &= rest - 1u;
+        const int w = bit & 7, e = bit >> 3;
+        const uint32_t lower =
+            ((1u << w) - 1u) * 0x01010101u | ((0x01010101u << w) & ((1u << (8 * e)) - 1u));
+        put(pos + __popc(sel & lower), tok + 4 * w + e);
+    }
+}
+
 // Emit a thread's selected tokens in ascending order: group m (tokens
 // tok0 + 32 m ...) selects every "< T" key and, while my_take lasts, its
 // ties at T from the lowest index up.  put(pos, token) stores one entry;
@@ -173,12 +191,8 @@ __device__ __forceinline__ void emit_selected(const uint32_t (&lt_bits)[kGroupsN
             }
         }
         if (sel) {
-            uint32_t selt = to_token_order(sel);
-            while (selt) {
-                const int e = __ffs(int(selt)) - 1;
-                selt &= selt - 1u;
-                put(pos++, tok0 + 32 * m + e);
-            }
+            put_ranked(sel, pos, tok0 + 32 * m, put);
+            pos += __popc(sel);
         }
     }
 }

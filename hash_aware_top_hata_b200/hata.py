@@ -126,6 +126,13 @@ def _need(t: torch.Tensor, name: str, dtype=None, ndim=None, cuda=True, host_ok=
                          (" or a pinned host tensor" if host_ok else ""))
 
 
+def _need_code_words(codes: torch.Tensor, W_H: torch.Tensor) -> None:
+    """codes [..][r/32] must match W_H [H_kv][d][r]."""
+    if W_H.dim() != 3 or codes.shape[-1] * 32 != W_H.shape[2]:
+        raise ValueError(f"codes {tuple(codes.shape)} hold {codes.shape[-1]} words per token; "
+                         f"W_H {tuple(W_H.shape)} gives r/32 words")
+
+
 # ------------------------------------------------------------------ API --
 
 def hata_abi_version() -> int:
@@ -145,6 +152,7 @@ def hata_hash_keys(K: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, pos0
     _need(K, "K", ndim=4, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
+    _need_code_words(codes, W_H)
     B, H, n_cap, d = K.shape
     n = n_cap - pos0 if n is None else n
     _check(lib().hata_hash_keys(_ptr(K), _kv_code(K), n_cap, _ptr(W_H), _ptr(codes), B, H,
@@ -158,6 +166,7 @@ def hata_append_code(k_new: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor
     _need(k_new, "k_new", ndim=3)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
+    _need_code_words(codes, W_H)
     _need(pos, "pos", torch.int32, 1)
     if err_flags is not None:
         _need(err_flags, "err_flags", torch.int32)
@@ -201,6 +210,7 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
     _need(q, "q", torch.float32, 3, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
+    _need_code_words(codes, W_H)
     _need(K, "K", ndim=4, host_ok=True)
     _need(V, "V", ndim=4, host_ok=True)
     _need(seq_len, "seq_len", torch.int32, 1)
@@ -245,6 +255,7 @@ def hata_decode_step_noalloc(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Te
     _need(q, "q", torch.float32, 3, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
+    _need_code_words(codes, W_H)
     _need(K, "K", ndim=4, host_ok=True)
     _need(V, "V", ndim=4, host_ok=True)
     _need(seq_len, "seq_len", torch.int32, 1)

@@ -19,8 +19,10 @@
  *     caller; the library never allocates, frees or keeps them.  Work is
  *     enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
  *     and the call returns without synchronising, except where noted.
- *   - d (head_dim) and r (hash bits) must both be 128 (HATA_ERR_UNSUPPORTED
- *     otherwise).
+ *   - d (head_dim) must be 128; r (hash bits) 128, the page's width, or 32 /
+ *     64, the narrower widths of its ablation (HATA_ERR_UNSUPPORTED
+ *     otherwise).  r = 256 is not offered: its distances 0..256 do not fit
+ *     the byte-wide distance row next to the pad value 255.
  *   - Layouts are dense row-major:
  *       W_H    [H_kv][d][r]        fp32; bit j of a code is [sum_i x_i W_H[i][j] > 0]
  *       K, V   [B][H_kv][n_cap][d] bf16 or fp32 (kv_dtype), 16-byte aligned
@@ -56,7 +58,7 @@ extern "C" {
 typedef enum hata_status {
     HATA_OK = 0,
     HATA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, small workspace */
-    HATA_ERR_UNSUPPORTED = 2,   /* d != 128, r != 128, H_q not a multiple of H_kv */
+    HATA_ERR_UNSUPPORTED = 2,   /* d != 128, r not 32/64/128, H_q not a multiple of H_kv */
     HATA_ERR_CUDA = 3,          /* a CUDA launch or copy failed */
     HATA_ERR_DEVICE_CHECK = 4   /* a device-side range check fired (see the flags) */
 } hata_status_t;
@@ -157,7 +159,7 @@ int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
  *             slots past |S| set to -1
  *   q_codes   optional [B][H_q][r/32] uint32: the query codes
  *   dist, dist_row_bytes  optional [B][H_q][dist_row_bytes] uint8: the
- *             Hamming distances (0..128); positions seq_len[b] ..
+ *             Hamming distances (0..r); positions seq_len[b] ..
  *             hata_dist_row_bytes(max_seq_len)-1 hold 255;
  *             dist_row_bytes >= hata_dist_row_bytes(max_seq_len), multiple of 16
  *   events    optional array of 6 cudaEvent_t recorded on `stream` before the

@@ -52,14 +52,17 @@ class GpuDecoder:
     """Owns the device code cache and workspace of one workload."""
 
     def __init__(self, w: wl.Workload, topk: int, max_seq_len: int | None = None,
-                 prefill: int | None = None):
+                 prefill: int | None = None, r: int = 128):
         cfg = w.cfg
         self.w = w
         self.topk = topk
+        self.r = r
+        # r < 128: the leading r columns of the workload's projection
+        self.W = w.W_H if r == 128 else w.W_H[:, :, :r].contiguous()
         self.max_seq_len = max_seq_len or w.n_cap
-        self.codes = torch.full((cfg.B, cfg.H_kv, w.n_cap, 4), -1, dtype=torch.int32,
+        self.codes = torch.full((cfg.B, cfg.H_kv, w.n_cap, r // 32), -1, dtype=torch.int32,
                                 device="cuda")
-        H.hata_hash_keys(w.K, w.W_H, self.codes, 0, cfg.N if prefill is None else prefill)
+        H.hata_hash_keys(w.K, self.W, self.codes, 0, cfg.N if prefill is None else prefill)
         self.ws = torch.empty(H.hata_decode_workspace_size(cfg.B, cfg.H_q, cfg.H_kv,
                                                            self.max_seq_len, topk),
                               dtype=torch.uint8, device="cuda")
@@ -70,10 +73,10 @@ class GpuDecoder:
         B, Hq = cfg.B, cfg.H_q
         out = torch.full((B, Hq, 128), float("nan"), device="cuda")
         sel = torch.full((B, Hq, self.topk), -7, dtype=torch.int32, device="cuda")
-        qc = torch.zeros((B, Hq, 4), dtype=torch.int32, device="cuda")
+        qc = torch.zeros((B, Hq, self.r // 32), dtype=torch.int32, device="cuda")
         dist = torch.full((B, Hq, self.drow), 77, dtype=torch.uint8, device="cuda")
         sl = torch.tensor(seq_len, dtype=torch.int32, device="cuda")
-        H.hata_decode_step(q, self.w.W_H, self.codes, self.w.K, self.w.V, sl, self.max_seq_len,
+        H.hata_decode_step(q, self.W, self.codes, self.w.K, self.w.V, sl, self.max_seq_len,
                            self.topk, SCALE, self.ws, out, k_new=k_new, v_new=v_new,
                            sel_idx=sel, q_codes=qc, dist=dist)
         flags = H.hata_workspace_check(self.ws)

@@ -62,7 +62,8 @@ def decode(**over):
     (dict(seq_len=NULL), H.HATA_ERR_INVALID_ARG),
     (dict(ws=NULL), H.HATA_ERR_INVALID_ARG),
     (dict(d=64), H.HATA_ERR_UNSUPPORTED),
-    (dict(r=64), H.HATA_ERR_UNSUPPORTED),
+    (dict(r=96), H.HATA_ERR_UNSUPPORTED),
+    (dict(r=256), H.HATA_ERR_UNSUPPORTED),
     (dict(H_q=3), H.HATA_ERR_UNSUPPORTED),
     (dict(B=0), H.HATA_ERR_INVALID_ARG),
     (dict(topk=0), H.HATA_ERR_INVALID_ARG),

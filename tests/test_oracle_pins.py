@@ -364,3 +364,38 @@ def test_needles_are_selected_on_synthetic_workload():
     needles = set(w.planted[0, 0].tolist())
     assert needles <= set(idx.tolist())
     del torch
+
+
+# --------------------------------------------------- narrower codes (r) ---
+# The page's ablation also runs r = 32 and 64 bits: code bit j depends on
+# column j of W_H alone, so a narrower code is the leading words of the wide
+# one, and the Hamming range is 0..r.
+
+@pytest.mark.parametrize("r", [32, 64])
+def test_narrow_code_is_prefix_of_wide_code(r):
+    W = RNG.standard_normal((128, 128)).astype(np.float32) / math.sqrt(128)
+    for _ in range(20):
+        x = RNG.standard_normal(128).astype(np.float32)
+        wide = oracle.hash_vec(x, W)
+        narrow = oracle.hash_vec(x, np.ascontiguousarray(W[:, :r]))
+        assert narrow.shape == (r // 32,)
+        assert np.array_equal(narrow, wide[: r // 32])
+        # and each bit is the sign of its own projection (fp64 reference,
+        # well away from zero)
+        proj = x.astype(np.float64) @ W[:, :r].astype(np.float64)
+        bits = np.unpackbits(narrow.view(np.uint8), bitorder="little")
+        sure = np.abs(proj) > 1e-4
+        assert np.array_equal(bits[sure], (proj[sure] > 0).astype(np.uint8))
+
+
+@pytest.mark.parametrize("r", [32, 64])
+def test_narrow_hamming_range_and_brute_force(r):
+    w = r // 32
+    codes = RNG.integers(0, 2**32, (200, w), dtype=np.uint64).astype(np.uint32)
+    q = RNG.integers(0, 2**32, w, dtype=np.uint64).astype(np.uint32)
+    d = oracle.hamming_all(q, codes)
+    ub = np.unpackbits(codes.view(np.uint8), axis=-1)
+    uq = np.unpackbits(q.view(np.uint8))
+    assert np.array_equal(d, (ub != uq[None, :]).sum(-1))
+    assert oracle.hamming(q, ~q) == r and oracle.hamming(q, q) == 0
+    assert d.min() >= 0 and d.max() <= r

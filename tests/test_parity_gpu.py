@@ -65,11 +65,56 @@ def test_append_code_and_position_check():
     assert int(err.item()) == H.HATA_FLAG_POS_RANGE
 
 
+@pytest.mark.parametrize("r", [32, 64])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_hash_keys_narrow_codes_bit_exact(r, dtype):
+    """r = 32 / 64 bit codes (the page's ablation widths), r/32 words per
+    token, against the oracle with the same r columns."""
+    g = torch.Generator(device="cuda").manual_seed(13 + r)
+    B, Hkv, n_cap, pos0, n = 2, 3, 3001, 5, 2990
+    K = _kv(dtype, (B, Hkv, n_cap, 128), g)
+    W = torch.randn((Hkv, 128, r), generator=g, device="cuda") / math.sqrt(128)
+    K[0, 1, 7] = 0
+    codes = torch.full((B, Hkv, n_cap, r // 32), -1, dtype=torch.int32, device="cuda")
+    H.hata_hash_keys(K, W, codes, pos0, n)
+    got = to_np_codes(codes)
+    want = oracle.hash_keys(wl.to_numpy_kv(K), W.cpu().numpy(), pos0=pos0, n=n)
+    assert want.shape[-1] == r // 32
+    assert np.array_equal(got[:, :, pos0:pos0 + n], want[:, :, pos0:pos0 + n])
+    assert np.all(got[:, :, :pos0] == 0xFFFFFFFF) and np.all(got[:, :, pos0 + n:] == 0xFFFFFFFF)
+    assert np.all(got[0, 1, 7] == 0)
+    # a code buffer of the wrong width is refused by the binding
+    with pytest.raises(ValueError):
+        H.hata_hash_keys(K, W, torch.zeros((B, Hkv, n_cap, 4), dtype=torch.int32,
+                                           device="cuda"), 0, 1)
+
+
+@pytest.mark.parametrize("r", [32, 64])
+def test_append_code_narrow(r):
+    g = torch.Generator(device="cuda").manual_seed(14 + r)
+    B, Hkv, n_cap = 2, 3, 50
+    k_new = _kv("f32", (B, Hkv, 128), g)
+    W = torch.randn((Hkv, 128, r), generator=g, device="cuda") / math.sqrt(128)
+    codes = torch.zeros((B, Hkv, n_cap, r // 32), dtype=torch.int32, device="cuda")
+    pos = torch.tensor([3, 49], dtype=torch.int32, device="cuda")
+    H.hata_append_code(k_new, W, codes, pos)
+    got = to_np_codes(codes)
+    kn = wl.to_numpy_kv(k_new)
+    Wh = W.cpu().numpy()
+    for b, p in ((0, 3), (1, 49)):
+        for h in range(Hkv):
+            assert np.array_equal(got[b, h, p], oracle.hash_vec(kn[b, h], Wh[h]))
+    got[0, :, 3] = 0
+    got[1, :, 49] = 0
+    assert np.all(got == 0)
+
+
 # ---------------------------------------------------------------- decode --
 
-def run_and_check(cfg, seed, steps, topk=None, heads=None, n_cap=None):
+def run_and_check(cfg, seed, steps, topk=None, heads=None, n_cap=None, r=128):
     """Decode `steps` steps (each appends one token) on the GPU and compare
-    the given heads (default: all) with the oracle after every step."""
+    the given heads (default: all) with the oracle after every step; r-bit
+    codes from the leading r columns of the workload's W_H."""
     topk = cfg.topk if topk is None else topk
     w = wl.make_workload(cfg, seed, device="cuda", steps=steps, n_cap=n_cap)
     G = cfg.G
@@ -77,8 +122,8 @@ def run_and_check(cfg, seed, steps, topk=None, heads=None, n_cap=None):
         heads = [(b, hq) for b in range(cfg.B) for hq in range(cfg.H_q)]
     pairs = sorted({(b, hq // G) for b, hq in heads})
     slabs = host_slabs(w, pairs)
-    Wn = w.W_H.cpu().numpy()
-    dec = GpuDecoder(w, topk)
+    dec = GpuDecoder(w, topk, r=r)
+    Wn = dec.W.cpu().numpy()
     worst = 0.0
     for t in range(steps):
         pos = [cfg.N + t] * cfg.B
@@ -119,6 +164,21 @@ def test_decode_scaled_configs(name):
     if cfg.needles:
         cfg = wl.dataclasses.replace(cfg, needles=16)
     run_and_check(cfg, seed=wl.SEED_BASE + wl.CONFIG_ORDER.index(name), steps=2)
+
+
+NARROW = [("llama31_8b_gqa_128k", dict(N=10000, topk=156, B=2)),  # stream-K attention
+          ("llama31_8b_gqa_128k", dict(N=6000, topk=300, B=4)),   # one CTA per head
+          ("qwen_gqa_b32_32k", dict(N=5000, topk=94, B=3)),       # 7 heads per KV head
+          ("tiny_mha_4k", dict(N=4096))]                          # fp32 K/V
+
+
+@pytest.mark.parametrize("r", [32, 64])
+@pytest.mark.parametrize("case", range(len(NARROW)))
+def test_decode_narrow_codes(r, case):
+    """The whole decode step with r = 32 / 64 bit codes (distances 0..r)."""
+    name, kw = NARROW[case]
+    cfg = wl.scaled(wl.CONFIGS[name], **kw)
+    run_and_check(cfg, seed=wl.SEED_BASE + 40 + case, steps=2, r=r)
 
 
 def test_decode_tiny_config_full_size():
