@@ -22,7 +22,6 @@ constexpr int kAttnThreads = 128;
 constexpr int kHistStride = 132;        // u32 per (head, tile) histogram row (129 bins)
 constexpr int kTile = 36864;            // tokens per histogram tile / selection tile (9 x 4096)
 constexpr int kPartStride = 132;        // f32 per (head, chunk) partial: m, l, -, -, acc[128]
-constexpr int kPrepRows = 4;            // rows hashed together by one prep CTA
 constexpr uint8_t kDistPad = 255;       // distance stored past seq_len
 constexpr uint32_t kWsMagic = 0x48415441u;  // "HATA"
 

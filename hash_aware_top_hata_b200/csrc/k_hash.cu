@@ -160,69 +160,73 @@ __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void 
 
 // --------------------------------------------------------- decode prep --
 // Rows of KV head h: B*G query rows (b-major), then B appended-key rows.
-// A CTA takes kPrepRows rows of one head with r threads per row (thread j
-// of a row owns bit j).  The head's W_H is staged once in shared memory
-// (asynchronous 16-byte copies by all threads) next to the rows, so every
-// step of a chain reads its two operands from shared memory at addresses
-// known in advance: the loads run ahead of the dependent FMAs instead of
-// exposing their latency at each of the 128 steps.
+// A CTA takes kPrepRowsCta rows of one head and one 32-bit word of their
+// codes: warp = row, lane = bit 32 cb + lane (cb = blockIdx.z), so the CTA
+// stages only its 32 columns of the head's W_H (16 KB, asynchronous 16-byte
+// copies by all threads) next to its rows, and a warp ballot gives the
+// word.  Every step of a chain reads its two operands from shared memory at
+// addresses known in advance: the loads run ahead of the dependent FMAs
+// instead of exposing their latency at each of the 128 steps.  The side
+// jobs of a row (the device copy of q, the appended K/V rows, the flags)
+// fall to the CTAs of word 0; the histogram rows are cleared by all words.
+constexpr int kPrepRowsCta = 8;
+constexpr int kPrepThreads = 32 * kPrepRowsCta;
+
 template <bool BF16, int R>
-__global__ void __launch_bounds__(R * kPrepRows) prep_kernel(PrepArgs a)
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
 {
-    constexpr int kPrepThreads = R * kPrepRows;
     pdl_trigger();  // the scoring kernel's setup (step inputs only) may start now
-    const int h = blockIdx.y;
-    const int r = threadIdx.x / R, j = threadIdx.x % R;
+    const int h = blockIdx.y, cb = blockIdx.z;
+    const int r = threadIdx.x >> 5, lane = threadIdx.x & 31, j = 32 * cb + lane;
     const int nq = a.q ? a.B * a.G : 0;
     const int nk = a.k_new ? a.B : 0;
     const int rows = nq + nk;
-    const int r0 = blockIdx.x * kPrepRows;
+    const int r0 = blockIdx.x * kPrepRowsCta;
     const int row = r0 + r;
 
-    if (a.ws_header && blockIdx.x == 0 && h == 0 && threadIdx.x == 0) {
+    if (a.ws_header && blockIdx.x == 0 && h == 0 && cb == 0 && threadIdx.x == 0) {
         a.ws_header[0] = kWsMagic;
         a.ws_header[1] = uint32_t(a.B);
     }
     if (r0 >= rows) return;
 
-    extern __shared__ __align__(16) float smem[];
-    float *ws = smem;                  // [kD][R]: this head's W_H
-    float *xs = smem + kD * R;         // [kPrepRows][kD]: the rows
+    __shared__ __align__(16) float ws[kD][32];             // columns 32 cb .. of W_H
+    __shared__ __align__(16) float xs[kPrepRowsCta][kD];   // the rows
     {
-        const float *Wh = a.W + size_t(h) * kD * R;
-        const uint32_t base = smem_addr(ws);
-        for (int c = threadIdx.x; c < kD * R / 4; c += kPrepThreads)
-            cp_async16_zfill(base + 16u * c, Wh + 4 * c, 16u);
+        const float *Wh = a.W + size_t(h) * kD * R + 32 * cb;
+        const uint32_t base = smem_addr(&ws[0][0]);
+        for (int c = threadIdx.x; c < kD * 8; c += kPrepThreads)  // row c / 8, piece c % 8
+            cp_async16_zfill(base + 16u * c, Wh + size_t(c >> 3) * R + 4 * (c & 7), 16u);
         cp_async_commit();
     }
 
-    // the row itself: its first warp reads it with 16-byte (q, fp32 keys) or
+    // the row itself: its warp reads it with 16-byte (q, fp32 keys) or
     // 8-byte (bf16 keys) loads -- q and k_new may be host memory, where few
     // wide requests cost much less than many narrow ones
-    if (j < 32 && row < rows) {
+    if (row < rows) {
         float4 v;
         if (row < nq) {
             const size_t bh = size_t(row / a.G) * a.H_q + h * a.G + row % a.G;
-            v = reinterpret_cast<const float4 *>(a.q + bh * kD)[j];
-            if (a.q_copy) reinterpret_cast<float4 *>(a.q_copy + bh * kD)[j] = v;
+            v = reinterpret_cast<const float4 *>(a.q + bh * kD)[lane];
+            if (a.q_copy && cb == 0) reinterpret_cast<float4 *>(a.q_copy + bh * kD)[lane] = v;
         } else {
             const int64_t e0 = (int64_t(row - nq) * a.H_kv + h) * kD;
             if (BF16) {
-                const uint2 u = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.k_new) + e0)[j];
+                const uint2 u = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.k_new) + e0)[lane];
                 v = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
                                 __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
             } else {
-                v = reinterpret_cast<const float4 *>(static_cast<const float *>(a.k_new) + e0)[j];
+                v = reinterpret_cast<const float4 *>(static_cast<const float *>(a.k_new) + e0)[lane];
             }
         }
-        reinterpret_cast<float4 *>(xs + r * kD)[j] = v;
+        reinterpret_cast<float4 *>(&xs[r][0])[lane] = v;
     }
     if (row < nq) {
         const int b = row / a.G, g = row % a.G, hq = h * a.G + g;
         const size_t bh = size_t(b) * a.H_q + hq;
         if (a.hist)
             for (int64_t t = j; t < a.hist_row_words; t += R) a.hist[bh * a.hist_row_words + t] = 0u;
-        if (a.flags && h == 0 && g == 0 && j == 0) {
+        if (a.flags && h == 0 && g == 0 && cb == 0 && lane == 0) {
             const int64_t sl = a.seq_len[b];
             uint32_t f = 0;
             if (sl < 0 || sl > a.max_seq_len || sl > a.n_cap) f |= HATA_FLAG_SEQ_LEN_RANGE;
@@ -232,11 +236,12 @@ __global__ void __launch_bounds__(R * kPrepRows) prep_kernel(PrepArgs a)
     }
     cp_async_wait<0>();
     __syncthreads();
+    if (row >= rows) return;  // warp-uniform; no barrier follows
 
     // the fixed-order chain acc = fmaf(x_i, W[i][j], acc), i = 0..127
     // (operands of block i0 + 16 are loaded before block i0 is multiplied in)
     constexpr int kBlk = 16;
-    const float4 *xr = reinterpret_cast<const float4 *>(xs + r * kD);
+    const float4 *xr = reinterpret_cast<const float4 *>(&xs[r][0]);
     float xa[kBlk], wa[kBlk], xb[kBlk], wb[kBlk];
     auto fetch = [&](int i0, float (&xv)[kBlk], float (&wv)[kBlk]) {
 #pragma unroll
@@ -245,7 +250,7 @@ __global__ void __launch_bounds__(R * kPrepRows) prep_kernel(PrepArgs a)
             xv[4 * k] = v.x, xv[4 * k + 1] = v.y, xv[4 * k + 2] = v.z, xv[4 * k + 3] = v.w;
         }
 #pragma unroll
-        for (int k = 0; k < kBlk; ++k) wv[k] = ws[(i0 + k) * R + j];
+        for (int k = 0; k < kBlk; ++k) wv[k] = ws[i0 + k][lane];
     };
     float acc = 0.0f;
     fetch(0, xa, wa);
@@ -261,39 +266,38 @@ __global__ void __launch_bounds__(R * kPrepRows) prep_kernel(PrepArgs a)
     const uint32_t word = __ballot_sync(0xffffffffu, acc > 0.0f);
 
     if (row < nq) {
-        if ((j & 31) == 0) {
+        if (lane == 0) {
             const int b = row / a.G, g = row % a.G;
             const size_t bh = size_t(b) * a.H_q + h * a.G + g;
-            a.q_out[bh * (R / 32) + (j >> 5)] = word;
+            a.q_out[bh * (R / 32) + cb] = word;
         }
-    } else if (row < rows) {
+    } else {
         const int b = row - nq;
         const int64_t pos = a.pos ? int64_t(a.pos[b]) : int64_t(a.seq_len[b]) - 1;
         if (pos >= 0 && pos < a.n_cap) {
             const int64_t crow = (int64_t(b) * a.H_kv + h) * a.n_cap + pos;
-            if ((j & 31) == 0) a.codes[crow * (R / 32) + (j >> 5)] = word;
-            if (a.v_new) {
+            if (lane == 0) a.codes[crow * (R / 32) + cb] = word;
+            if (a.v_new && cb == 0) {
                 // K from the staged row (a bf16 key is the upper half of its
-                // fp32 widening: exact); V copied by the row's first warp
-                for (int e = j; e < kD; e += R) {
-                    const float xk = xs[r * kD + e];
+                // fp32 widening: exact); V copied by the row's warp
+#pragma unroll
+                for (int e = lane; e < kD; e += 32) {
+                    const float xk = xs[r][e];
                     if (BF16)
                         static_cast<uint16_t *>(a.K)[crow * kD + e] =
                             uint16_t(__float_as_uint(xk) >> 16);
                     else
                         static_cast<float *>(a.K)[crow * kD + e] = xk;
                 }
-                if (j < 32) {
-                    const int64_t e0 = (int64_t(b) * a.H_kv + h) * kD;
-                    if (BF16)
-                        reinterpret_cast<uint2 *>(static_cast<uint16_t *>(a.V) + crow * kD)[j] =
-                            reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.v_new) + e0)[j];
-                    else
-                        reinterpret_cast<float4 *>(static_cast<float *>(a.V) + crow * kD)[j] =
-                            reinterpret_cast<const float4 *>(static_cast<const float *>(a.v_new) + e0)[j];
-                }
+                const int64_t e0 = (int64_t(b) * a.H_kv + h) * kD;
+                if (BF16)
+                    reinterpret_cast<uint2 *>(static_cast<uint16_t *>(a.V) + crow * kD)[lane] =
+                        reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(a.v_new) + e0)[lane];
+                else
+                    reinterpret_cast<float4 *>(static_cast<float *>(a.V) + crow * kD)[lane] =
+                        reinterpret_cast<const float4 *>(static_cast<const float *>(a.v_new) + e0)[lane];
             }
-        } else if (a.err_word && j == 0) {
+        } else if (a.err_word && cb == 0 && lane == 0) {
             atomicOr(a.err_word, HATA_FLAG_POS_RANGE);
         }
     }
@@ -332,11 +336,9 @@ cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const f
 template <bool BF16, int R>
 cudaError_t launch_prep_t(const PrepArgs &a, int rows_per_head, cudaStream_t s)
 {
-    constexpr size_t kSmem = sizeof(float) * (kD * R + kD * kPrepRows);
-    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(prep_kernel<BF16, R>), kSmem))
-        return e;
-    const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRows)), unsigned(a.H_kv));
-    prep_kernel<BF16, R><<<grid, R * kPrepRows, kSmem, s>>>(a);
+    const dim3 grid(unsigned(ceil_div(rows_per_head, kPrepRowsCta)), unsigned(a.H_kv),
+                    unsigned(R / 32));
+    prep_kernel<BF16, R><<<grid, kPrepThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
