@@ -6,19 +6,19 @@
 // Figure 2 caption (Algorithm 1: HashEncode(K) fills the code cache, rbit/32
 // words per token).
 //
-// One CTA of 128 threads hashes a group of rows against one KV head's W_H:
-// thread j owns output bit j, keeps column j of W_H in registers and runs
-// the fp32 chain acc = fmaf(x_i, W[i][j], acc), i = 0..127 ascending, for
-// every row of the group (rows staged in shared memory, read as broadcast
-// float4s).  A warp ballot packs bits 32w..32w+31 into code word w.  The
-// chain order is fixed, so codes are reproducible bit for bit by any
-// implementation that follows the same order (the CPU oracle does).
+// Every code bit j is the fp32 chain acc = fmaf(x_i, W[i][j], acc), i = 0..127
+// ascending, then acc > 0.  The chain order is fixed, so codes are
+// reproducible bit for bit by any implementation that follows the same
+// order (the CPU oracle does).  r = 128 bits (the page's width), or 32 / 64
+// (the narrower widths of its ablation): r/32 code words per token.
 //
-// The projection is 16K FMAs per row: on the FP32 pipes, not the tensor
-// cores, whose accumulation order is unspecified and would break bit-exact
-// codes.  At decode time the kernel also appends the new key's code (and
-// optionally its K/V rows) and clears the per-step counters the scoring
-// kernel accumulates into.
+// Two kernels: the prefill hash (register-blocked over 8 rows per warp, the
+// head's W_H in shared memory) for hata_hash_keys, and the decode prep
+// (one 32-bit code word of 8 rows per CTA) that hashes the step's queries,
+// appends the new key's code (and optionally its K/V rows) and clears the
+// per-step counters the scoring kernel accumulates into.  The projection
+// is 16K FMAs per row at r = 128: on the FP32 pipes, not the tensor cores,
+// whose accumulation order is unspecified and would break bit-exact codes.
 #include "hata_internal.cuh"
 #include "tma.cuh"
 
