@@ -25,6 +25,8 @@
 //
 // i.e. three population counts instead of four: POPC issues at an eighth of
 // the integer-logic rate on sm_100a, and it is what bounds the arithmetic.
+// Codes of 32 or 64 bits (the ablation widths) take 4- or 8-byte copies
+// into the same 16-byte ring slots and one or two population counts.
 //
 // Per query head the kernel stores the u8 distance row (32 lanes write 32
 // consecutive bytes per store; the row stays L2-resident for the selection
