@@ -126,8 +126,8 @@ hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t n_cap
     if (n_cap <= 0 || pos0 < 0 || n < 0 || pos0 > n_cap || n > n_cap - pos0)
         return fail(HATA_ERR_INVALID_ARG, "positions [%lld, %lld) outside the cache of %lld",
                     (long long)pos0, (long long)(pos0 + n), (long long)n_cap);
-    if (!aligned(K, 16) || !aligned(codes, 16) || !aligned(W_H, 4))
-        return fail(HATA_ERR_INVALID_ARG, "K and codes must be 16-byte aligned");
+    if (!aligned(K, 16) || !aligned(codes, 16) || !aligned(W_H, 16))  // 16-byte copies of W_H
+        return fail(HATA_ERR_INVALID_ARG, "K, codes and W_H must be 16-byte aligned");
     if (n == 0) return ok();
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = launch_hash_prefill(K, kv_dtype == HATA_DT_BF16, n_cap, W_H, codes, B,

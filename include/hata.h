@@ -24,7 +24,8 @@
  *     otherwise).  r = 256 is not offered: its distances 0..256 do not fit
  *     the byte-wide distance row next to the pad value 255.
  *   - Layouts are dense row-major:
- *       W_H    [H_kv][d][r]        fp32; bit j of a code is [sum_i x_i W_H[i][j] > 0]
+ *       W_H    [H_kv][d][r]        fp32, 16-byte aligned; bit j of a code is
+ *                                   [sum_i x_i W_H[i][j] > 0]
  *       K, V   [B][H_kv][n_cap][d] bf16 or fp32 (kv_dtype), 16-byte aligned
  *       codes  [B][H_kv][n_cap][r/32] uint32, bit j in word j/32 at bit j%32
  *                                   (least significant first), 16-byte aligned

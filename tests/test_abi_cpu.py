@@ -98,6 +98,8 @@ def test_hash_and_append_reject_on_host():
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
     bad = list(ok_args); bad[4] = FAKE + 4
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[3] = FAKE + 4   # W_H is copied in 16-byte pieces
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
     bad = list(ok_args); bad[0] = NULL
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
     # n == 0 is a valid no-op that enqueues nothing
