@@ -4,22 +4,24 @@
 // top-k indices select K/V for attention, which the page runs as a fused
 // gather + FlashAttention over the selected keys.
 //
-// Persistent, stream-K style.  The selected rows of all heads form one flat
-// space of B*H_q*topk rows (head bh owns [bh*topk, bh*topk + k_eff)); CTA k of
-// P owns the contiguous range [k*T/P, (k+1)*T/P), so every CTA moves the
-// same number of bytes whatever the distance distribution, and a head is
-// shared by at most a few CTAs.  Each CTA walks its range in stages of up to
-// 32 rows through a 4-deep ring in shared memory: while it computes stage s
-// the 16-byte cp.async copies of stages s+1..s+3 are in flight (for bf16,
-// 16 lanes per 256-byte row; on B200 this random-row gather runs at the
-// streaming HBM bandwidth, where one bulk-copy request per row reaches only
-// half of it).  Every 16-lane half-warp takes rows, computes q.k in fp32
-// with the softmax scale and log2(e) folded into q, and keeps an online
-// softmax state (m, l, acc[8 per lane]).  When a CTA leaves a head, its
-// eight half-warp states merge into one partial (m, l, acc[128]) in the
-// head's slot for that CTA.  A separate combine launch (chained by
-// programmatic dependent launch) merges each head's slots into
-// out = acc / l, so no worker waits for another or merges behind the others.
+// The selected rows of all heads form one flat space of B*H_q*topk rows
+// (head bh owns [bh*topk, bh*topk + k_eff)).  Three kernels walk it:
+//   * attend_tc_kernel (bf16 K/V): every warp is a stream-K worker over an
+//     equal, contiguous slice of the flat space, gathering 16 rows per stage
+//     through a private 3-stage ring of 16-byte cp.async copies and running
+//     each stage on the tensor cores (mma.sync, keys along M, q and the
+//     softmax weights as hi/lo bf16 pairs); when a warp leaves a head it
+//     writes one partial (m, l, acc[128]) into the head's slot for it;
+//   * attend_head_kernel (bf16, heads filling about one wave of CTAs): one
+//     CTA per head, warp w takes the w-th eighth of the head's list, and the
+//     eight partials merge in shared memory (no combine launch);
+//   * attend_simt_kernel (fp32 K/V): CTA-level stream-K on the CUDA cores,
+//     16 lanes per row, a 4-deep ring of up to 32 rows.
+// combine_kernel, chained behind the stream-K kernels by programmatic
+// dependent launch, merges each head's partials into out = acc / l, so no
+// worker waits for another.  The random 256-byte row gathers of K and V
+// peak at ~5.0 TB/s on B200 (one bulk-copy request per row reaches about
+// half of that), which bounds all three.
 #include <cuda_bf16.h>
 
 #include "hata_internal.cuh"
