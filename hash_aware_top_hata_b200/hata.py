@@ -146,8 +146,8 @@ def hata_status_string(status: int) -> str:
 def hata_hash_keys(K: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, pos0: int = 0,
                    n: int | None = None, stream=None) -> None:
     """Prefill: codes[b, h, pos0:pos0+n] = hash(K[b, h, pos0:pos0+n]).
-    K [B][H_kv][n_cap][128] bf16/fp32, W_H [H_kv][128][128] fp32,
-    codes [B][H_kv][n_cap][4] int32 (uint32 bit patterns).  K may be a pinned
+    K [B][H_kv][n_cap][128] bf16/fp32, W_H [H_kv][128][r] fp32 (r = 32, 64 or 128),
+    codes [B][H_kv][n_cap][r/32] int32 (uint32 bit patterns).  K may be a pinned
     host tensor (a cache kept in host memory)."""
     _need(K, "K", ndim=4, host_ok=True)
     _need(W_H, "W_H", torch.float32, 3)
@@ -204,7 +204,7 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
     q [B][H_q][128] fp32, K/V [B][H_kv][n_cap][128], seq_len [B] int32,
     workspace uint8 of hata_decode_workspace_size bytes, out [B][H_q][128] fp32.
     Optional: k_new/v_new [B][H_kv][128], sel_idx [B][H_q][topk] int32,
-    q_codes [B][H_q][4] int32, dist [B][H_q][row] uint8, events: 6 torch.cuda.Event.
+    q_codes [B][H_q][r/32] int32, dist [B][H_q][row] uint8, events: 6 torch.cuda.Event.
     q, k_new, v_new and out may also be pinned host tensors: the kernels read
     and write them over the bus once per step (no separate copies)."""
     _need(q, "q", torch.float32, 3, host_ok=True)
