@@ -26,6 +26,15 @@ constexpr uint8_t kDistPad = 255;       // distance stored past seq_len
 constexpr uint32_t kWsMagic = 0x48415441u;  // "HATA"
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// A batch row's sequence length as the kernels use it: seq_len[b] clamped to
+// [0, min(max_len, n_cap)] (an out-of-range length is also flagged by prep).
+__device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
+{
+    int64_t l = sl < 0 ? 0 : sl;
+    l = l < max_len ? l : max_len;
+    return l < n_cap ? l : n_cap;
+}
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kAttnMaxWorkers = 4096;   // upper bound of the attention stream-K workers

@@ -36,13 +36,6 @@ constexpr int kStageRows = 32;
 constexpr int kRing = 4;
 constexpr int kRowsPerHalf = kStageRows / kHalves;  // 4
 
-__device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
-{
-    int64_t l = sl < 0 ? 0 : sl;
-    l = l < max_len ? l : max_len;
-    return l < n_cap ? l : n_cap;
-}
-
 template <bool BF16>
 struct Rows {
     static constexpr int kRowBytes = kD * (BF16 ? 2 : 4);

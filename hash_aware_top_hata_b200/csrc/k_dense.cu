@@ -20,13 +20,6 @@ constexpr int kHalves = kWarps * 2;
 constexpr int kU = 4;  // rows per half-warp per round
 constexpr int kHeads = kDenseHeads;
 
-__device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
-{
-    int64_t l = sl < 0 ? 0 : sl;
-    l = l < max_len ? l : max_len;
-    return l < n_cap ? l : n_cap;
-}
-
 template <bool BF16>
 __device__ __forceinline__ void load8(const void *base, int64_t elem, float (&f)[8])
 {

@@ -51,13 +51,6 @@ constexpr int kTileUnits = kTile / kUnit;   // 288
 constexpr int kMaxKeys = 8;                 // (slab, tile) histograms per CTA range
 constexpr int kMaxRange = 2048;             // units per CTA range
 
-__device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
-{
-    int64_t l = sl < 0 ? 0 : sl;
-    l = l < max_len ? l : max_len;
-    return l < n_cap ? l : n_cap;
-}
-
 // dist(k, q) with the XOR-ed words x_w = k_w ^ q_w, summed bit position by
 // bit position with a full adder and a half adder:
 //   x0 + x1 + x2 = s + 2c,  s = x0 ^ x1 ^ x2,  c = maj(x0, x1, x2)

@@ -33,13 +33,6 @@ constexpr int kPieces = kPer / 16;                      // 16-byte loads per thr
 constexpr int kGroups = kPer / 32;                      // 32-distance mask words
 static_assert(kThreads * kPer == kTile, "a CTA covers one histogram tile per pass");
 
-__device__ __forceinline__ int64_t clamp_len(int32_t sl, int64_t max_len, int64_t n_cap)
-{
-    int64_t l = sl < 0 ? 0 : sl;
-    l = l < max_len ? l : max_len;
-    return l < n_cap ? l : n_cap;
-}
-
 __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
 {
     pdl_trigger();
