@@ -37,19 +37,39 @@ MUTANTS = {
 }
 
 
+def _argsets(fn) -> list[dict]:
+    """The keyword sets pytest would call a pin with (from its parametrize
+    marks; a pin without marks runs once with no arguments)."""
+    sets = [dict()]
+    for mark in getattr(fn, "pytestmark", []):
+        if mark.name != "parametrize":
+            continue
+        names = [n.strip() for n in mark.args[0].split(",")] if isinstance(mark.args[0], str) \
+            else list(mark.args[0])
+        combos = []
+        for values in mark.args[1]:
+            values = values if len(names) > 1 else (values,)
+            combos.append(dict(zip(names, values)))
+        sets = [dict(a, **b) for a in sets for b in combos]
+    return sets
+
+
 def _run_pins() -> int:
     failures = 0
     for name, fn in inspect.getmembers(pins, inspect.isfunction):
         if not name.startswith("test_"):
             continue
-        argsets = [dict(kv="f32"), dict(kv="bf16")] if "kv" in inspect.signature(fn).parameters \
-            else [dict()]
-        for kw in argsets:
+        for kw in _argsets(fn):
             try:
                 fn(**kw)
             except Exception:
                 failures += 1
     return failures
+
+
+def test_pins_pass_on_the_real_oracle():
+    """Without this, a pin that cannot run at all would 'catch' every mutant."""
+    assert _run_pins() == 0
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
