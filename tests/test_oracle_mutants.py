@@ -34,6 +34,9 @@ MUTANTS = {
     "softmax not normalised": ("out[i] /= l;", "out[i] /= 1.0;"),
     "bf16 widened from the low half": ("uint32_t u = ((uint32_t)h) << 16;",
                                        "uint32_t u = ((uint32_t)h);"),
+    "bf16 cache rows strided as 4-byte elements": (
+        "row * d * (dtype == ORACLE_DT_BF16 ? 2 : 4);",
+        "row * d * (dtype == ORACLE_DT_BF16 ? 4 : 4);"),
 }
 
 

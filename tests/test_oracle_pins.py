@@ -125,16 +125,24 @@ def test_hash_bf16_input_is_exact_widening():
         assert np.array_equal(oracle.hash_vec(bits, W), oracle.hash_vec(widen(bits), W))
 
 
-def test_hash_keys_layout():
+@pytest.mark.parametrize("kv", ["f32", "bf16"])
+def test_hash_keys_layout(kv):
     """Algorithm 1: codes[b][h][t] is the hash of K[b][h][t] with head h's W_H,
-    for t in [pos0, pos0+n) only."""
+    for t in [pos0, pos0+n) only.  A bf16 cache is read as 2-byte rows whose
+    values widen exactly to fp32, so its codes are the fp64 projection signs
+    of the widened values (a wrong row stride or widening reads other keys)."""
     B, H, n_cap, d, r = 2, 3, 9, 128, 128
     K = RNG.standard_normal((B, H, n_cap, d)).astype(np.float32)
+    if kv == "bf16":
+        K = bf16_round_bits(K)
+        Kf = widen(K)
+    else:
+        Kf = K
     W = (RNG.standard_normal((H, d, r)) / math.sqrt(d)).astype(np.float32)
     codes = oracle.hash_keys(K, W, pos0=2, n=5)
     for b, h, t in itertools.product(range(B), range(H), range(n_cap)):
         if 2 <= t < 7:
-            proj = K[b, h, t].astype(np.float64) @ W[h]
+            proj = Kf[b, h, t].astype(np.float64) @ W[h]
             assert np.array_equal(codes[b, h, t], pack_bits_le(proj > 0))
         else:
             assert np.all(codes[b, h, t] == 0)
