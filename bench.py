@@ -528,6 +528,7 @@ def run_hata(args, world, rank, local):
     for i in range(K_steps):
         flush()
         step(W_steps + K_steps + i, kevs[i])
+        H.hata_workspace_check(ws)  # every step of this untimed pass is checked
     torch.cuda.synchronize()
     prep_ms = [e[0].elapsed_time(e[1]) for e in kevs]
     score_ms = [e[1].elapsed_time(e[2]) for e in kevs]
@@ -535,8 +536,10 @@ def run_hata(args, world, rank, local):
     attend_ms = [e[3].elapsed_time(e[4]) for e in kevs]
     combine_ms = [e[4].elapsed_time(e[5]) for e in kevs]
     n_launch = H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.topk, w.K.dtype)
+    fused = n_launch == 3
     # four launches: one CTA per head, merged in shared memory
-    attend_kernel = "attend_head_kernel" if n_launch == 4 else "attend_tc_kernel"
+    attend_kernel = ("fused_select_attend_kernel" if fused else
+                     "attend_head_kernel" if n_launch == 4 else "attend_tc_kernel")
     split_ms = [e[0].elapsed_time(e[5]) for e in kevs]
     ms = statistics.mean(step_ms)
     ms_max = max_over_ranks(world, ms)
@@ -556,32 +559,47 @@ def run_hata(args, world, rank, local):
     code_bytes = B * Hkv * (N + W_steps + K_steps // 2) * 16  # every code once per KV head
     attend_s = statistics.mean(attend_ms) / 1e3
     score_s = statistics.mean(score_ms) / 1e3
-    achieved = attend_bytes / attend_s / 1e9
     step_bytes = attend_bytes + code_bytes
+    fused_s = statistics.mean(select_ms) / 1e3  # fused step: the selection + attention kernel
+    if fused:
+        # the selection + attention kernel moves the selected K/V rows
+        roof_bytes, roof_s = attend_bytes, fused_s
+        roof_src = "hash_aware_top_hata_b200/csrc/k_fused.cu"
+        roof_what = "fused_select_attend_kernel (top-k + gather + softmax)"
+    else:
+        roof_bytes, roof_s = attend_bytes, attend_s
+        roof_src = "hash_aware_top_hata_b200/csrc/k_attend.cu"
+        roof_what = f"{attend_kernel} (gather + softmax)"
+    achieved = roof_bytes / roof_s / 1e9
     line = {
         "metric": METRIC, "value": round(ms_max * 1e3, 2), "unit": UNIT, "n_gpus": world,
         "steps": K_steps, "warmup": W_steps, "ms_per_step": round(ms_max, 5),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian q/K/V, 2% planted keys, N(0,1/128) W_H)",
         "config": config_dict(cfg, "flushed before every timed step (512 MiB read)"),
-        "roofline": {"bound": "hbm", "kernel": f"{attend_kernel} (gather + softmax)",
+        "roofline": {"bound": "hbm", "kernel": roof_what,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(cfg, attend_kernel,
-                                                 "hash_aware_top_hata_b200/csrc/k_attend.cu"),
-                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": attend_bytes},
+                     "traffic": profiled_traffic(cfg, attend_kernel, roof_src),
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": roof_bytes},
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
                           "frac_of_measured": round(step_bytes / (ms / 1e3) / 1e9 / peak, 4),
                           "frac_of_8000": round(step_bytes / (ms / 1e3) / 1e9 / 8000.0, 4)},
-        "kernels_us": {"prep": round(statistics.mean(prep_ms) * 1e3, 2),
-                       "score": round(score_s * 1e6, 2),
-                       "select": round(statistics.mean(select_ms) * 1e3, 2),
-                       "attend": round(attend_s * 1e6, 2),
-                       # null: the heads were merged inside the attention CTAs
-                       "combine": (round(statistics.mean(combine_ms) * 1e3, 2)
-                                   if n_launch == 5 else None),
-                       "sum_with_events": round(statistics.mean(split_ms) * 1e3, 2),
-                       "score_gbs": round(code_bytes / score_s / 1e9, 1)},
+        "kernels_us": ({"prep": round(statistics.mean(prep_ms) * 1e3, 2),
+                        "score": round(score_s * 1e6, 2),
+                        "select_attend": round(fused_s * 1e6, 2),
+                        "sum_with_events": round(statistics.mean(split_ms) * 1e3, 2),
+                        "score_gbs": round(code_bytes / score_s / 1e9, 1)}
+                       if fused else
+                       {"prep": round(statistics.mean(prep_ms) * 1e3, 2),
+                        "score": round(score_s * 1e6, 2),
+                        "select": round(statistics.mean(select_ms) * 1e3, 2),
+                        "attend": round(attend_s * 1e6, 2),
+                        # null: the heads were merged inside the attention CTAs
+                        "combine": (round(statistics.mean(combine_ms) * 1e3, 2)
+                                    if n_launch == 5 else None),
+                        "sum_with_events": round(statistics.mean(split_ms) * 1e3, 2),
+                        "score_gbs": round(code_bytes / score_s / 1e9, 1)}),
         "dense_us": _num(dense_ms * 1e3, 1),
         "speedup_vs_dense": _num(dense_ms / ms, 2),
         "e2e": {"value": _num(e2e_ms * 1e3, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -614,10 +632,16 @@ def main():
     ap.add_argument("--topk", type=int, default=0, help="override the top-k budget")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e, dense and CPU legs (profiling runs)")
+    ap.add_argument("--decode-mode", default="auto", choices=["auto", "multi_kernel", "fused"],
+                    help="step implementation: auto (the library's choice), the multi-kernel "
+                         "step or the fused step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup(args)
+    if args.impl == "hata":
+        H.hata_set_decode_mode({"auto": H.HATA_MODE_AUTO, "fused": H.HATA_MODE_FUSED,
+                                "multi_kernel": H.HATA_MODE_MULTI_KERNEL}[args.decode_mode])
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)

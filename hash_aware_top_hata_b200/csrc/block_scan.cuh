@@ -42,14 +42,23 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *scratch, int *to
 
 namespace hata {
 
-// Exclusive prefix sums of two counters (a, b) over the block at once, in
-// threadIdx.x order; *ta / *tb get the block sums.  scratch: >= NT/32 + 1
-// int2 of shared memory.  Every thread must call it; two block barriers,
-// plus one at the end so that scratch may be reused right after.
-template <int NT>
+// Exclusive prefix sums of two counters (a, b) over the first NT threads of
+// the block at once, in threadIdx.x order; *ta / *tb get the sums.  scratch:
+// >= NT/32 + 1 int2 of shared memory.  Every one of the NT threads must call
+// it.  BAR = 0 synchronises with __syncthreads (NT = the block size); any
+// other BAR with the named barrier BAR over those NT threads, so that other
+// warps of the block may run unrelated work meanwhile.  Two barriers, plus
+// one at the end so that scratch may be reused right after.
+template <int NT, int BAR = 0>
 __device__ __forceinline__ int2 block_exclusive_scan2(int a, int b, int2 *scratch, int *ta, int *tb)
 {
     constexpr int NW = NT / 32;
+    auto sync = [] {
+        if constexpr (BAR == 0)
+            __syncthreads();
+        else
+            asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+    };
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int ia = a, ib = b;
 #pragma unroll
@@ -59,7 +68,7 @@ __device__ __forceinline__ int2 block_exclusive_scan2(int a, int b, int2 *scratc
         if (lane >= o) { ia += na; ib += nb; }
     }
     if (lane == 31) scratch[warp] = make_int2(ia, ib);
-    __syncthreads();
+    sync();
     if (warp == 0) {
         const int2 w = lane < NW ? scratch[lane] : make_int2(0, 0);
         int wa = w.x, wb = w.y;
@@ -72,11 +81,11 @@ __device__ __forceinline__ int2 block_exclusive_scan2(int a, int b, int2 *scratc
         if (lane < NW) scratch[lane] = make_int2(wa - w.x, wb - w.y);
         if (lane == NW - 1) scratch[NW] = make_int2(wa, wb);
     }
-    __syncthreads();
+    sync();
     const int2 base = scratch[warp];
     *ta = scratch[NW].x;
     *tb = scratch[NW].y;
-    __syncthreads();
+    sync();
     return make_int2(base.x + ia - a, base.y + ib - b);
 }
 

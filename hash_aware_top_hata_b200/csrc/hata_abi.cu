@@ -1,6 +1,7 @@
 // hata_abi.cu -- the extern "C" boundary of libhata: argument checks on the
 // host, workspace carving, and the launch sequence of each entry point on the
 // caller's stream.  Every check runs before anything is enqueued.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -14,6 +15,26 @@ using namespace hata;
 namespace {
 
 thread_local char g_err[512];
+
+// Process-wide settings (hata_set_decode_mode / hata_set_wait_limit_ns).
+std::atomic<int> g_mode{HATA_MODE_AUTO};
+std::atomic<uint64_t> g_wait_ns{1000000000ull};
+
+#ifndef HATA_SEL_LAG
+#define HATA_SEL_LAG 2
+#endif
+
+// Which step HATA_MODE_AUTO picks for bf16 caches (the faster one on B200).
+constexpr bool kAutoFused = false;
+
+// The fused step serves bf16 K/V caches when asked for (or chosen by AUTO);
+// fp32 caches always take the multi-kernel step.
+bool use_fused(hata_dtype_t kv_dtype)
+{
+    const int m = g_mode.load();
+    return kv_dtype == HATA_DT_BF16 &&
+           (m == HATA_MODE_FUSED || (m == HATA_MODE_AUTO && kAutoFused));
+}
 
 hata_status_t fail(hata_status_t st, const char *fmt, ...)
 {
@@ -98,7 +119,7 @@ cudaError_t ensure_smem_attr(const void *func, size_t bytes)
 
 extern "C" {
 
-int hata_abi_version(void) { return 1; }
+int hata_abi_version(void) { return 2; }
 
 const char *hata_status_string(int status)
 {
@@ -114,8 +135,25 @@ const char *hata_status_string(int status)
 
 const char *hata_last_error(void) { return g_err; }
 
-hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t n_cap,
-                             const float *W_H, uint32_t *codes, int B, int H_kv, int64_t pos0,
+hata_status_t hata_set_decode_mode(int mode)
+{
+    if (mode != HATA_MODE_AUTO && mode != HATA_MODE_MULTI_KERNEL && mode != HATA_MODE_FUSED)
+        return fail(HATA_ERR_INVALID_ARG, "decode mode %d", mode);
+    g_mode.store(mode);
+    return ok();
+}
+
+int hata_get_decode_mode(void) { return g_mode.load(); }
+
+hata_status_t hata_set_wait_limit_ns(uint64_t ns)
+{
+    g_wait_ns.store(ns);
+    return ok();
+}
+
+hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t k_stride_b,
+                             int64_t k_stride_h, int64_t k_stride_n, const float *W_H,
+                             uint32_t *codes, int64_t n_cap, int B, int H_kv, int64_t pos0,
                              int64_t n, int d, int r, void *stream)
 {
     if (hata_status_t st = check_dims(d, r)) return st;
@@ -126,12 +164,20 @@ hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t n_cap
     if (n_cap <= 0 || pos0 < 0 || n < 0 || pos0 > n_cap || n > n_cap - pos0)
         return fail(HATA_ERR_INVALID_ARG, "positions [%lld, %lld) outside the cache of %lld",
                     (long long)pos0, (long long)(pos0 + n), (long long)n_cap);
-    if (!aligned(K, 16) || !aligned(codes, 16) || !aligned(W_H, 16))  // 16-byte copies of W_H
-        return fail(HATA_ERR_INVALID_ARG, "K, codes and W_H must be 16-byte aligned");
+    if (k_stride_b < 0 || k_stride_h < 0 || k_stride_n < d)
+        return fail(HATA_ERR_INVALID_ARG,
+                    "K strides (%lld, %lld, %lld): non-negative, and rows of d elements must not "
+                    "overlap (k_stride_n >= d)",
+                    (long long)k_stride_b, (long long)k_stride_h, (long long)k_stride_n);
+    const size_t elt = kv_dtype == HATA_DT_BF16 ? 2 : 4;
+    if (!aligned(K, elt) || !aligned(codes, 16) || !aligned(W_H, 16))  // 16-byte copies of W_H
+        return fail(HATA_ERR_INVALID_ARG,
+                    "K must be aligned to its element, codes and W_H to 16 bytes");
     if (n == 0) return ok();
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t e = launch_hash_prefill(K, kv_dtype == HATA_DT_BF16, n_cap, W_H, codes, B,
-                                              H_kv, pos0, n, r / 32, s);
+    const KStrides ks{k_stride_b, k_stride_h, k_stride_n};
+    const cudaError_t e = launch_hash_prefill(K, kv_dtype == HATA_DT_BF16, ks, n_cap, W_H, codes,
+                                              B, H_kv, pos0, n, r / 32, s);
     return e == cudaSuccess ? ok() : cuda_fail(e, "hash_keys launch");
 }
 
@@ -184,6 +230,7 @@ int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
              int(kv_dtype));
         return -1;
     }
+    if (use_fused(kv_dtype)) return 3;  // prep, score, the selection + attention kernel
     int n = 0;
     if (cudaError_t e = attend_launch_count(B, H_q, topk, kv_dtype == HATA_DT_BF16, &n)) {
         cuda_fail(e, "occupancy query");
@@ -263,6 +310,9 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     p.flags = flags;
     p.hist = hist;
     p.hist_row_words = L.n_tiles * kHistStride;
+    const bool fused = use_fused(kv_dtype);
+    uint32_t *sync = reinterpret_cast<uint32_t *>(ws + L.off_sync);
+    p.sync = fused ? sync : nullptr;
     p.ws_header = reinterpret_cast<uint32_t *>(ws);
     p.n_cap = n_cap;
     p.max_seq_len = max_seq_len;
@@ -294,6 +344,42 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     sa.words = r / 32;
     if ((e = launch_score(sa, s)) != cudaSuccess) return cuda_fail(e, "score launch");
     if ((e = ev.record(2)) != cudaSuccess) return cuda_fail(e, "event record");
+
+    if (fused) {
+        FusedArgs fa{};
+        fa.seq_len = seq_len;
+        fa.q = q_dev;
+        fa.K = K;
+        fa.V = V;
+        fa.dist = dst;
+        fa.hist = hist;
+        fa.idx = idx;
+        fa.part = reinterpret_cast<float *>(ws + L.off_part);
+        fa.out = out;
+        fa.sel_done = sync;
+        fa.head_cnt = sync + int64_t(B) * H_q;
+        fa.flags = flags;
+        fa.abort_word = sync + 2 * int64_t(B) * H_q;
+        fa.dist_row = drow;
+        fa.dist_len = L.dist_row;
+        fa.n_cap = n_cap;
+        fa.max_seq_len = max_seq_len;
+        fa.n_tiles = int(L.n_tiles);
+        fa.B = B;
+        fa.H_q = H_q;
+        fa.H_kv = H_kv;
+        fa.G = G;
+        fa.topk = topk;
+        fa.n_seg = L.n_seg;
+        fa.scale_log2 = scale * 1.4426950408889634f;
+        fa.spin_limit_ns = g_wait_ns.load();
+        if ((e = launch_fused(fa, s)) != cudaSuccess) return cuda_fail(e, "fused launch");
+        // one kernel does the work of the select, attend and combine kernels:
+        // its end is recorded for all three
+        for (int i = 3; i <= 5; ++i)
+            if ((e = ev.record(i)) != cudaSuccess) return cuda_fail(e, "event record");
+        return ok();
+    }
 
     SelectArgs se{};
     se.seq_len = seq_len;

@@ -20,8 +20,10 @@ constexpr int kScoreThreads = 1024;
 constexpr int kScoreHeads = 8;          // query heads scored per code load (one CTA)
 constexpr int kAttnThreads = 128;
 constexpr int kHistStride = 132;        // u32 per (head, tile) histogram row (129 bins)
-constexpr int kTile = 36864;            // tokens per histogram tile / selection tile (9 x 4096)
+constexpr int kTile = 32768;            // tokens per histogram tile / selection tile (8 x 4096)
 constexpr int kPartStride = 132;        // f32 per (head, chunk) partial: m, l, -, -, acc[128]
+constexpr int kFSeg = 112;              // selected rows per attention item, fused step
+                                        // (16 per attention warp)
 constexpr uint8_t kDistPad = 255;       // distance stored past seq_len
 constexpr uint32_t kWsMagic = 0x48415441u;  // "HATA"
 
@@ -54,11 +56,12 @@ inline int attn_max_contributors(int64_t BH, int topk)
 struct DecodeLayout {
     int64_t n_chunks = 0;   // 4096-token chunks of max_seq_len
     int64_t dist_row = 0;   // bytes per (b, h_q) distance row
-    int64_t n_tiles = 0;    // 36K-token histogram tiles of a distance row
+    int64_t n_tiles = 0;    // 32K-token histogram / selection tiles of a distance row
     int zgroups = 0;        // ceil(G / kScoreHeads)
-    int n_split = 0;        // attention partial slots per head
+    int n_split = 0;        // attention partial slots per head (multi-kernel step)
+    int n_seg = 0;          // attention items per head (fused step)
     size_t off_flags = 0, off_qcodes = 0, off_q = 0, off_dist = 0, off_hist = 0, off_idx = 0,
-           off_part = 0, total = 0;
+           off_part = 0, off_sync = 0, total = 0;
 };
 
 inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
@@ -77,6 +80,11 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
     // the scoring kernel numbers its 128-token units with 32-bit integers
     if (int64_t(B) * H_kv * L->zgroups * (L->dist_row / 128) >= (int64_t(1) << 31)) return false;
     L->n_split = attn_max_contributors(BH, topk);
+    L->n_seg = int(ceil_div(topk, kFSeg));
+    // the fused step numbers its selection and attention items with 32-bit
+    // integers too
+    if (BH * L->n_seg >= (int64_t(1) << 31) || BH * L->n_tiles >= (int64_t(1) << 31)) return false;
+    const int64_t parts = L->n_split > L->n_seg ? L->n_split : L->n_seg;
     size_t o = 256;
     L->off_flags = o;      o = align_up(o + 4 * size_t(B), 256);
     L->off_qcodes = o;     o = align_up(o + 16 * size_t(BH), 256);
@@ -84,7 +92,10 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
     L->off_dist = o;       o = align_up(o + size_t(BH) * L->dist_row, 256);
     L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * L->n_tiles * kHistStride, 256);
     L->off_idx = o;        o = align_up(o + 4 * size_t(BH) * topk, 256);
-    L->off_part = o;       o = align_up(o + 4 * size_t(BH) * L->n_split * kPartStride, 256);
+    L->off_part = o;       o = align_up(o + 4 * size_t(BH) * parts * kPartStride, 256);
+    // fused-step counters: selection tiles done and attention items published
+    // per head, then the step's abort word (all zeroed by prep every step)
+    L->off_sync = o;       o = align_up(o + 4 * size_t(2 * BH + 1), 256);
     L->total = o;
     return true;
 }
@@ -105,6 +116,8 @@ struct PrepArgs {
     uint32_t *err_word;      // single OR-ed word (append API) or null
     uint32_t *hist;          // [B][H_q][hist_row_words] zeroed (decode) or null
     int64_t hist_row_words;  // n_tiles * kHistStride
+    uint32_t *sync;          // fused-step counters zeroed (decode, fused step) or null:
+                             // [B][H_q] twice, then one abort word
     uint32_t *ws_header;     // {magic, B} written (decode) or null
     int64_t n_cap, max_seq_len;
     int B, H_q, H_kv, G;
@@ -148,6 +161,33 @@ struct AttendArgs {
     int head_per_cta;        // 1: a CTA's warps cover one whole head and merge it in shared
                              // memory (no combine launch); set by the launcher
     float scale_log2;        // scale * log2(e)
+};
+
+// The fused step's selection + attention kernel (after prep and the scoring
+// kernel): selection warps turn the distance rows into index lists, attention
+// warps gather and attend the heads selected so far, one publisher warp per
+// CTA hands results between CTAs.
+struct FusedArgs {
+    const int32_t *seq_len;
+    const float *q;          // [B][H_q][128] device copy written by prep
+    const void *K, *V;       // bf16 [B][H_kv][n_cap][128]
+    const uint8_t *dist;     // [B][H_q][dist_row] (scoring kernel)
+    const uint32_t *hist;    // [B][H_q][n_tiles][kHistStride] (scoring kernel)
+    int32_t *idx;            // [B][H_q][topk]
+    float *part;             // [B][H_q][n_seg][kPartStride]
+    float *out;              // [B][H_q][128]
+    uint32_t *sel_done;      // [B][H_q] selection tiles done, zeroed by prep
+    uint32_t *head_cnt;      // [B][H_q] attention items published, zeroed by prep
+    uint32_t *flags;         // per-b flag words: a wait that gives up ORs TIMEOUT into [0]
+    uint32_t *abort_word;    // this step's "someone gave up" word, zeroed by prep
+    int64_t dist_row;        // stride of the distance rows (bytes)
+    int64_t dist_len;        // bytes of each row the scoring kernel wrote: max_seq_len
+                             // rounded up to kChunk
+    int64_t n_cap, max_seq_len;
+    int n_tiles;             // kTile tiles of dist_len
+    int B, H_q, H_kv, G, topk, n_seg;
+    float scale_log2;
+    uint64_t spin_limit_ns;  // bound of every wait
 };
 
 struct DenseArgs {
@@ -220,9 +260,13 @@ hata_status_t report_error(hata_status_t st, const char *msg);
 cudaError_t ensure_smem_attr(const void *func, size_t bytes);
 
 // Launchers (each returns the cudaGetLastError() of its launch).
-cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const float *W,
-                                uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
-                                int words, cudaStream_t s);
+// Element strides of a key cache K[b][h][t][i] (i contiguous).
+struct KStrides {
+    int64_t b, h, n;
+};
+cudaError_t launch_hash_prefill(const void *K, bool bf16, KStrides ks, int64_t n_cap,
+                                const float *W, uint32_t *codes, int B, int H_kv, int64_t pos0,
+                                int64_t n, int words, cudaStream_t s);
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s);
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
@@ -232,5 +276,6 @@ cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s);
 // device: 1 when the heads are merged inside the attention CTAs, else 2.
 cudaError_t attend_launch_count(int B, int H_q, int topk, bool bf16, int *n);
 cudaError_t launch_dense(const DenseArgs &a, bool bf16, cudaStream_t s);
+cudaError_t launch_fused(const FusedArgs &a, cudaStream_t s);
 
 }  // namespace hata

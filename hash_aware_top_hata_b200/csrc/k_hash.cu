@@ -20,7 +20,7 @@
 // is 16K FMAs per row at r = 128: on the FP32 pipes, not the tensor cores,
 // whose accumulation order is unspecified and would break bit-exact codes.
 #include "hata_internal.cuh"
-#include "tma.cuh"
+#include "async_copy.cuh"
 
 namespace hata {
 namespace {
@@ -74,7 +74,7 @@ __device__ __forceinline__ uint64_t dup2(float v)
 
 template <bool BF16, int R>
 __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void *__restrict__ K,
-                                                                    int64_t n_cap,
+                                                                    KStrides ks, int64_t n_cap,
                                                                     const float *__restrict__ W,
                                                                     uint32_t *__restrict__ codes,
                                                                     int H_kv, int64_t pos0, int64_t n)
@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void 
     const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t g_begin = int64_t(blockIdx.x) * kPfRowsPerCta;
     const int64_t g_end = min(g_begin + kPfRowsPerCta, n);
-    const int64_t slab = (int64_t(b) * H_kv + h) * n_cap + pos0;  // row index of row 0
+    const int64_t slab = (int64_t(b) * H_kv + h) * n_cap + pos0;  // code row of row 0
+    const int64_t kbase = int64_t(b) * ks.b + int64_t(h) * ks.h + pos0 * ks.n;  // K element of row 0
     {
         const float *Wh = W + size_t(h) * kD * R;
         const uint32_t base = smem_addr(S.W);
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void 
         const int64_t t = g0 + warp * kPfRows + sr;
         const bool ok = t < g_end;
 #pragma unroll
-        for (int k = 0; k < kD / 4; ++k) xv[k] = ok ? load_x<BF16>(K, (slab + t) * kD + 4 * k + si) : 0.0f;
+        for (int k = 0; k < kD / 4; ++k) xv[k] = ok ? load_x<BF16>(K, kbase + t * ks.n + 4 * k + si) : 0.0f;
     };
     fetch(g_begin);
     for (int64_t g0 = g_begin; g0 < g_end; g0 += kPfPass) {
@@ -226,6 +227,14 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
         const size_t bh = size_t(b) * a.H_q + hq;
         if (a.hist)
             for (int64_t t = j; t < a.hist_row_words; t += R) a.hist[bh * a.hist_row_words + t] = 0u;
+        if (a.sync && cb == 0 && lane == 0) {
+            // the fused step's counters: selection tiles done and attention
+            // items published of this head
+            const size_t BH = size_t(a.B) * a.H_q;
+            a.sync[bh] = 0u;
+            a.sync[BH + bh] = 0u;
+            if (bh == 0) a.sync[2 * BH] = 0u;  // the step's abort word
+        }
         if (a.flags && h == 0 && g == 0 && cb == 0 && lane == 0) {
             const int64_t sl = a.seq_len[b];
             uint32_t f = 0;
@@ -306,29 +315,30 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepArgs a)
 }  // namespace
 
 template <bool BF16, int R>
-cudaError_t launch_hash_prefill_t(const void *K, int64_t n_cap, const float *W, uint32_t *codes,
-                                  int B, int H_kv, int64_t pos0, int64_t n, cudaStream_t s)
+cudaError_t launch_hash_prefill_t(const void *K, KStrides ks, int64_t n_cap, const float *W,
+                                  uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
+                                  cudaStream_t s)
 {
     constexpr size_t kSmem = sizeof(PfSmem<R>);
     if (cudaError_t e = ensure_smem_attr(
             reinterpret_cast<const void *>(hash_prefill_kernel<BF16, R>), kSmem))
         return e;
     const dim3 grid(unsigned(ceil_div(n, kPfRowsPerCta)), unsigned(H_kv), unsigned(B));
-    hash_prefill_kernel<BF16, R><<<grid, kPfThreads, kSmem, s>>>(K, n_cap, W, codes, H_kv, pos0, n);
+    hash_prefill_kernel<BF16, R><<<grid, kPfThreads, kSmem, s>>>(K, ks, n_cap, W, codes, H_kv, pos0, n);
     return cudaGetLastError();
 }
 
-cudaError_t launch_hash_prefill(const void *K, bool bf16, int64_t n_cap, const float *W,
-                                uint32_t *codes, int B, int H_kv, int64_t pos0, int64_t n,
-                                int words, cudaStream_t s)
+cudaError_t launch_hash_prefill(const void *K, bool bf16, KStrides ks, int64_t n_cap,
+                                const float *W, uint32_t *codes, int B, int H_kv, int64_t pos0,
+                                int64_t n, int words, cudaStream_t s)
 {
     switch (words * 2 + (bf16 ? 1 : 0)) {
-    case 8 + 1: return launch_hash_prefill_t<true, 128>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
-    case 8: return launch_hash_prefill_t<false, 128>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
-    case 4 + 1: return launch_hash_prefill_t<true, 64>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
-    case 4: return launch_hash_prefill_t<false, 64>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
-    case 2 + 1: return launch_hash_prefill_t<true, 32>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
-    case 2: return launch_hash_prefill_t<false, 32>(K, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 8 + 1: return launch_hash_prefill_t<true, 128>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 8: return launch_hash_prefill_t<false, 128>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 4 + 1: return launch_hash_prefill_t<true, 64>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 4: return launch_hash_prefill_t<false, 64>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 2 + 1: return launch_hash_prefill_t<true, 32>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 2: return launch_hash_prefill_t<false, 32>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -30,7 +30,7 @@
 //
 // Per query head the kernel stores the u8 distance row (32 lanes write 32
 // consecutive bytes per store; the row stays L2-resident for the selection
-// kernel) and counts a 129-bin histogram per (head, 36K-token tile) in
+// kernel) and counts a 129-bin histogram per (head, 32K-token tile) in
 // shared memory; a range touches at most kMaxKeys (slab, tile) pairs.  At
 // the end of its range the CTA adds the non-zero bins into the tile
 // histograms in global memory (zeroed by the prep kernel), one reduction
@@ -39,7 +39,8 @@
 #include <algorithm>
 
 #include "hata_internal.cuh"
-#include "tma.cuh"
+#include "async_copy.cuh"
+#include "score_common.cuh"
 
 namespace hata {
 namespace {
@@ -47,37 +48,9 @@ namespace {
 constexpr int kWarps = kScoreThreads / 32;  // 8
 constexpr int kUnit = 128;                  // tokens per warp step
 constexpr int kRing = 2;                    // units per warp ring
-constexpr int kTileUnits = kTile / kUnit;   // 288
+constexpr int kTileUnits = kTile / kUnit;   // 256
 constexpr int kMaxKeys = 8;                 // (slab, tile) histograms per CTA range
 constexpr int kMaxRange = 2048;             // units per CTA range
-
-// dist(k, q) with the XOR-ed words x_w = k_w ^ q_w, summed bit position by
-// bit position with a full adder and a half adder:
-//   x0 + x1 + x2 = s + 2c,  s = x0 ^ x1 ^ x2,  c = maj(x0, x1, x2)
-//   s + x3       = o + 2e,  o = s ^ x3,        e = s & x3
-// so dist = popc(o) + 2 (popc(c) + popc(e)).  s and o depend on the key only
-// through k0 ^ k1 ^ k2 and k0 ^ k1 ^ k2 ^ k3 (k012, k0123, shared by every
-// head of the group) and on the query through q012, q0123 (qd).
-__device__ __forceinline__ int hamming128(const uint4 &k, uint32_t k012, uint32_t k0123,
-                                          const uint4 &q, const uint2 &qd)
-{
-    const uint32_t x0 = k.x ^ q.x, x1 = k.y ^ q.y, x2 = k.z ^ q.z;
-    const uint32_t c = (x0 & x1) | (x2 & (x0 ^ x1));
-    const uint32_t o = k0123 ^ qd.y;
-    const uint32_t e = (k012 ^ qd.x) & (k.w ^ q.w);
-    return __popc(o) + 2 * (__popc(c) + __popc(e));
-}
-
-// dist(k, q) for codes of W words (r = 32 W bits): the carry-save form for
-// W = 4, plain population counts of the XOR-ed words otherwise.
-template <int W>
-__device__ __forceinline__ int hamming_w(const uint4 &k, uint32_t k012, uint32_t k0123,
-                                         const uint4 &q, const uint2 &qd)
-{
-    if constexpr (W == 4) return hamming128(k, k012, k0123, q, qd);
-    if constexpr (W == 2) return __popc(k.x ^ q.x) + __popc(k.y ^ q.y);
-    return __popc(k.x ^ q.x);
-}
 
 // Histogram increment: one shared-memory reduction, no return value.
 __device__ __forceinline__ void red_shared_add1(uint32_t addr)

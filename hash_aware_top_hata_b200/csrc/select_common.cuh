@@ -71,15 +71,19 @@ __device__ __forceinline__ void group_masks(const uint32_t (&dw)[8], uint32_t T4
 // the keys below T and at T in the tiles before `tile`, from one head's
 // tile histograms (hrow: n_tiles rows of kHistStride words).  One warp;
 // lane l owns bins 5l .. 5l+4; out: {T, #(< T), below-T before the tile,
-// at-T before the tile}.
+// at-T before the tile}.  kCoherent: the rows were written by the running
+// kernel itself (loads through L2 only); otherwise by an earlier kernel.
+template <bool kCoherent = false, int kRegTiles = 4>  // kRegTiles: rows per round
 __device__ __forceinline__ void head_threshold(const uint32_t *hrow, int n_tiles, int k_eff,
                                                int tile, int lane, int *out)
 {
-    constexpr int kRegTiles = 4;  // rows held in registers per round
     auto row_bins = [&](int t, uint32_t (&v)[5]) {
 #pragma unroll
         for (int e = 0; e < 5; ++e)
-            v[e] = lane * 5 + e < kBins ? __ldg(hrow + t * kHistStride + lane * 5 + e) : 0u;
+            v[e] = lane * 5 + e < kBins
+                       ? (kCoherent ? __ldcg(hrow + t * kHistStride + lane * 5 + e)
+                                    : __ldg(hrow + t * kHistStride + lane * 5 + e))
+                       : 0u;
     };
     uint32_t tot[5] = {0u, 0u, 0u, 0u, 0u}, pre[5] = {0u, 0u, 0u, 0u, 0u};
     // rounds of kRegTiles rows: all loads of a round are issued before any

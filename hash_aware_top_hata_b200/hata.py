@@ -29,6 +29,9 @@ HATA_FLAG_SEQ_LEN_RANGE = 1
 HATA_FLAG_POS_RANGE = 2
 HATA_FLAG_TIMEOUT = 4
 HATA_NOALLOC_WORKSPACE_BYTES = 64 << 20
+HATA_MODE_AUTO = 0
+HATA_MODE_MULTI_KERNEL = 1
+HATA_MODE_FUSED = 2
 D = 128
 RBIT = 128
 
@@ -46,7 +49,7 @@ _SIGS = {
     "hata_abi_version": ([], I),
     "hata_status_string": ([I], ctypes.c_char_p),
     "hata_last_error": ([], ctypes.c_char_p),
-    "hata_hash_keys": ([P, I, I64, P, P, I, I, I64, I64, I, I, P], I),
+    "hata_hash_keys": ([P, I, I64, I64, I64, P, P, I64, I, I, I64, I64, I, I, P], I),
     "hata_append_code": ([P, I, P, P, I64, P, I, I, I, I, P, P], I),
     "hata_decode_workspace_size": ([I, I, I, I64, I], U64),
     "hata_dist_row_bytes": ([I64], I64),
@@ -58,6 +61,9 @@ _SIGS = {
     "hata_workspace_check": ([P, U64, P, P], I),
     "hata_dense_workspace_size": ([I, I, I, I64], U64),
     "hata_dense_decode": ([P, P, P, I, I64, P, I64, I, I, I, I, F, P, U64, P, P], I),
+    "hata_set_decode_mode": ([I], I),
+    "hata_get_decode_mode": ([], I),
+    "hata_set_wait_limit_ns": ([ctypes.c_uint64], I),
 }
 
 
@@ -146,17 +152,29 @@ def hata_status_string(status: int) -> str:
 def hata_hash_keys(K: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, pos0: int = 0,
                    n: int | None = None, stream=None) -> None:
     """Prefill: codes[b, h, pos0:pos0+n] = hash(K[b, h, pos0:pos0+n]).
-    K [B][H_kv][n_cap][128] bf16/fp32, W_H [H_kv][128][r] fp32 (r = 32, 64 or 128),
-    codes [B][H_kv][n_cap][r/32] int32 (uint32 bit patterns).  K may be a pinned
-    host tensor (a cache kept in host memory)."""
-    _need(K, "K", ndim=4, host_ok=True)
+    K [B][H_kv][n_cap][128] bf16/fp32, any strides with the last dimension
+    contiguous (a strided view of a larger cache is hashed in place),
+    W_H [H_kv][128][r] fp32 (r = 32, 64 or 128), codes [B][H_kv][n_cap][r/32]
+    int32 (uint32 bit patterns).  K may be a pinned host tensor (a cache kept
+    in host memory)."""
+    if not isinstance(K, torch.Tensor) or K.dim() != 4:
+        raise ValueError("K must be a 4-dim tensor [B][H_kv][n_cap][d]")
+    if K.stride(3) != 1:
+        raise ValueError("K's last dimension must be contiguous")
+    if not K.is_cuda and not K.is_pinned():
+        raise ValueError("K must be a CUDA tensor or a pinned host tensor")
     _need(W_H, "W_H", torch.float32, 3)
     _need(codes, "codes", torch.int32, 4)
     _need_code_words(codes, W_H)
     B, H, n_cap, d = K.shape
+    if codes.shape[:3] != (B, H, n_cap):
+        raise ValueError(f"codes {tuple(codes.shape)} must be [B][H_kv][n_cap][r/32] of K "
+                         f"{tuple(K.shape)}")
     n = n_cap - pos0 if n is None else n
-    _check(lib().hata_hash_keys(_ptr(K), _kv_code(K), n_cap, _ptr(W_H), _ptr(codes), B, H,
-                                pos0, n, d, W_H.shape[2], _stream(stream)), "hata_hash_keys")
+    sb, sh, sn, _ = K.stride()
+    _check(lib().hata_hash_keys(_ptr(K), _kv_code(K), sb, sh, sn, _ptr(W_H), _ptr(codes), n_cap,
+                                B, H, pos0, n, d, W_H.shape[2], _stream(stream)),
+           "hata_hash_keys")
 
 
 def hata_append_code(k_new: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor,
@@ -283,6 +301,21 @@ def hata_decode_step_noalloc(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Te
         max_seq_len, _ptr(k_new), _ptr(v_new), B, H_q, H_kv, d, W_H.shape[2], topk,
         float(scale), _ptr(out), _ptr(sel_idx), _ptr(q_codes), _ptr(dist), drow, ev,
         _stream(stream)), "hata_decode_step_noalloc")
+
+
+def hata_set_decode_mode(mode: int) -> None:
+    """HATA_MODE_AUTO (the library's choice), HATA_MODE_MULTI_KERNEL or
+    HATA_MODE_FUSED (the fused step for bf16 caches); process-wide."""
+    _check(lib().hata_set_decode_mode(int(mode)), "hata_set_decode_mode")
+
+
+def hata_get_decode_mode() -> int:
+    return int(lib().hata_get_decode_mode())
+
+
+def hata_set_wait_limit_ns(ns: int) -> None:
+    """Bound of every wait of the fused step (default 1 s); process-wide."""
+    _check(lib().hata_set_wait_limit_ns(int(ns)), "hata_set_wait_limit_ns")
 
 
 def hata_workspace_check(workspace: torch.Tensor, stream=None) -> int:

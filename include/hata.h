@@ -72,7 +72,9 @@ typedef enum hata_dtype {
 /* Device-side check flags (OR-ed into the error word). */
 #define HATA_FLAG_SEQ_LEN_RANGE 1u  /* seq_len[b] < 0, > max_seq_len or > n_cap: clamped */
 #define HATA_FLAG_POS_RANGE     2u  /* an append position outside [0, n_cap): skipped  */
-#define HATA_FLAG_TIMEOUT       4u  /* a bounded wait on an asynchronous copy gave up  */
+#define HATA_FLAG_TIMEOUT       4u  /* a bounded wait of the fused decode step gave up:
+                                       its results are not valid (see
+                                       hata_set_wait_limit_ns)                         */
 
 /* ABI revision; bumps whenever a signature below changes. */
 int hata_abi_version(void);
@@ -88,13 +90,19 @@ const char *hata_last_error(void);
  * hata_hash_keys -- prefill (Algorithm 1: KH <- HashEncode(K); Kcache_H <- KH).
  * Hashes the keys of positions [pos0, pos0 + n) of every (b, h_kv) of the
  * key cache K with W_H[h_kv] and writes codes[b][h_kv][pos0 .. pos0+n).
- *   K      [B][H_kv][n_cap][d] (kv_dtype)   read
+ *   K      (kv_dtype) read: element [b][h][t][i] at
+ *          K + b*k_stride_b + h*k_stride_h + t*k_stride_n + i (element
+ *          strides; i contiguous), so a strided or paged view of a larger
+ *          cache is hashed in place.  The dense [B][H_kv][n_cap][d] cache is
+ *          (n_cap*H_kv*d, n_cap*d, d).  Aligned to its element size.
  *   W_H    [H_kv][d][r] fp32                read
  *   codes  [B][H_kv][n_cap][r/32] uint32    written at the hashed positions only
- * Requires 0 <= pos0, n >= 0, pos0 + n <= n_cap.  n == 0 enqueues nothing. */
-hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t n_cap,
-                             const float *W_H, uint32_t *codes, int B, int H_kv,
-                             int64_t pos0, int64_t n, int d, int r, void *stream);
+ * Requires 0 <= pos0, n >= 0, pos0 + n <= n_cap, strides >= 0 and
+ * k_stride_n >= d.  n == 0 enqueues nothing. */
+hata_status_t hata_hash_keys(const void *K, hata_dtype_t kv_dtype, int64_t k_stride_b,
+                             int64_t k_stride_h, int64_t k_stride_n, const float *W_H,
+                             uint32_t *codes, int64_t n_cap, int B, int H_kv, int64_t pos0,
+                             int64_t n, int d, int r, void *stream);
 
 /* ------------------------------------------------------------------------
  * hata_append_code -- decode-time growth of the key code cache (the decode
@@ -120,11 +128,41 @@ size_t hata_decode_workspace_size(int B, int H_q, int H_kv, int64_t max_seq_len,
 int64_t hata_dist_row_bytes(int64_t max_seq_len);
 
 /* Number of kernels one hata_decode_step with these sizes launches on the
- * current device (prep, score, select, attention and, unless the heads are
- * merged inside the attention CTAs, the combine kernel): 4 or 5.  Returns -1
- * (hata_last_error says why) for invalid sizes or if the device query fails.
- * Host-only; launches nothing. */
+ * current device in the current mode (hata_set_decode_mode): 3 for the fused
+ * step (prep, score, the persistent selection + attention kernel); for the
+ * multi-kernel step prep, score, select, attention and, unless the heads are
+ * merged inside the attention CTAs, the combine kernel: 4 or 5.  Returns -1 (hata_last_error says why) for invalid sizes or if the
+ * device query fails.  Host-only; launches nothing. */
 int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype);
+
+/* ------------------------------------------------------------------------
+ * Step implementation.  Two implementations give the same codes, distances
+ * and indices bit for bit (outputs agree within the attention tolerance):
+ *   the multi-kernel step  prep, score, select, attention and (unless every
+ *                          head is merged inside its attention CTA) combine;
+ *   the fused step         prep, score, then ONE persistent kernel with one
+ *                          CTA per SM in which selection warps build the
+ *                          index lists while attention warps already gather
+ *                          and attend the heads selected so far (bf16 caches
+ *                          only; fp32 caches take the multi-kernel step).
+ *   HATA_MODE_AUTO          the library's choice (default)
+ *   HATA_MODE_MULTI_KERNEL  always the multi-kernel step
+ *   HATA_MODE_FUSED         the fused step for bf16 caches
+ * The mode is process-wide and read when a step is enqueued. */
+#define HATA_MODE_AUTO 0
+#define HATA_MODE_MULTI_KERNEL 1
+#define HATA_MODE_FUSED 2
+hata_status_t hata_set_decode_mode(int mode);
+int hata_get_decode_mode(void);
+
+/* Bound, in nanoseconds of wall time, of every wait of the fused step's
+ * persistent kernel on another warp or CTA (default 1 s; process-wide, read
+ * when a step is enqueued).  A wait that reaches it gives up: the kernel sets
+ * HATA_FLAG_TIMEOUT (reported by hata_workspace_check) and finishes without
+ * valid results instead of staying resident.  Its CTAs must all be resident
+ * at once to make progress, so a GPU shared with long-running kernels of
+ * other streams may need a longer bound. */
+hata_status_t hata_set_wait_limit_ns(uint64_t ns);
 
 /* ------------------------------------------------------------------------
  * hata_decode_step -- one decode step of HATA for every (b, h_q) (Figure 2):
@@ -166,7 +204,8 @@ int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
  *   events    optional array of 6 cudaEvent_t recorded on `stream` before the
  *             first kernel and after each of the five kernels (prep, score,
  *             select, attend, combine) -- a profiling hook (an event between
- *             two kernels keeps the second from starting early)
+ *             two kernels keeps the second from starting early).  In the
+ *             fused step events 2..5 are all recorded after the step kernel.
  */
 hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
                                void *V, hata_dtype_t kv_dtype, int64_t n_cap,

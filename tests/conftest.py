@@ -24,3 +24,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=["fused", "multi_kernel"])
+def decode_mode(request):
+    """Run a decode-step test under both step implementations: the fused
+    step (selection + attention in one persistent kernel) and the
+    multi-kernel step.
+    The process-wide mode is restored afterwards."""
+    from hash_aware_top_hata_b200 import hata as H
+    mode = H.HATA_MODE_FUSED if request.param == "fused" else H.HATA_MODE_MULTI_KERNEL
+    H.hata_set_decode_mode(mode)
+    yield request.param
+    H.hata_set_decode_mode(H.HATA_MODE_AUTO)

@@ -22,7 +22,7 @@ def test_library_exports_every_header_function():
     lib = H.lib()
     for n in names:
         assert hasattr(lib, n), n
-    assert H.hata_abi_version() == 1
+    assert H.hata_abi_version() == 2
 
 
 def test_status_strings():
@@ -89,27 +89,63 @@ def test_decode_step_rejects_on_host(over, status):
 
 def test_hash_and_append_reject_on_host():
     L = H.lib()
-    ok_args = [FAKE, 0, 4096, FAKE, FAKE, 1, 2, 0, 4096, 128, 128, NULL]
-    bad = list(ok_args); bad[10] = 96
+    # K, dtype, strides (b, h, n), W_H, codes, n_cap, B, H_kv, pos0, n, d, r, stream
+    dense = [4096 * 2 * 128, 4096 * 128, 128]
+    ok_args = [FAKE, 0, *dense, FAKE, FAKE, 4096, 1, 2, 0, 4096, 128, 128, NULL]
+    bad = list(ok_args); bad[13] = 96
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_UNSUPPORTED
-    bad = list(ok_args); bad[8] = 4097
+    bad = list(ok_args); bad[11] = 4097
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
-    bad = list(ok_args); bad[7] = -1
+    bad = list(ok_args); bad[10] = -1
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
-    bad = list(ok_args); bad[4] = FAKE + 4
+    bad = list(ok_args); bad[6] = FAKE + 4
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
-    bad = list(ok_args); bad[3] = FAKE + 4   # W_H is copied in 16-byte pieces
+    bad = list(ok_args); bad[5] = FAKE + 4   # W_H is copied in 16-byte pieces
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
     bad = list(ok_args); bad[0] = NULL
     assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    # strides: rows may not overlap, none negative; K aligned to its element
+    bad = list(ok_args); bad[4] = 64
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[2] = -1
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    bad = list(ok_args); bad[0] = FAKE + 1
+    assert L.hata_hash_keys(*bad) == H.HATA_ERR_INVALID_ARG
+    # a strided view (rows of a wider cache, an odd element offset) is fine
+    view = [FAKE + 2, 0, 9000 * 2 * 256, 9000 * 256, 256, FAKE, FAKE, 4096, 1, 2, 0, 0, 128,
+            128, NULL]
+    assert L.hata_hash_keys(*view) == H.HATA_OK
     # n == 0 is a valid no-op that enqueues nothing
-    zero = list(ok_args); zero[8] = 0
+    zero = list(ok_args); zero[11] = 0
     assert L.hata_hash_keys(*zero) == H.HATA_OK
     app = [FAKE, 0, FAKE, FAKE, 4096, FAKE, 1, 2, 128, 128, NULL, NULL]
     bad = list(app); bad[5] = NULL
     assert L.hata_append_code(*bad) == H.HATA_ERR_INVALID_ARG
     bad = list(app); bad[8] = 64
     assert L.hata_append_code(*bad) == H.HATA_ERR_UNSUPPORTED
+
+
+def test_binding_rejects_hash_keys_views_it_cannot_pass():
+    K = torch.zeros((1, 2, 64, 128), dtype=torch.bfloat16)
+    W = torch.zeros((2, 128, 128))
+    codes = torch.zeros((1, 2, 64, 4), dtype=torch.int32)
+    with pytest.raises(ValueError):                      # last dim not contiguous
+        H.hata_hash_keys(K.transpose(2, 3), W, codes)
+    with pytest.raises(ValueError):                      # host memory, not pinned
+        H.hata_hash_keys(K, W, codes)
+
+
+def test_decode_modes():
+    assert H.hata_get_decode_mode() == H.HATA_MODE_AUTO
+    assert H.lib().hata_set_decode_mode(7) == H.HATA_ERR_INVALID_ARG
+    for m in (H.HATA_MODE_MULTI_KERNEL, H.HATA_MODE_FUSED):
+        H.hata_set_decode_mode(m)
+        try:
+            assert H.hata_get_decode_mode() == m
+        finally:
+            H.hata_set_decode_mode(H.HATA_MODE_AUTO)
+    assert H.hata_get_decode_mode() == H.HATA_MODE_AUTO
+    assert H.lib().hata_set_wait_limit_ns(10**9) == H.HATA_OK
 
 
 def test_dense_rejects_on_host():
@@ -134,6 +170,12 @@ def test_decode_kernel_launches_host_logic():
     L = H.lib()
     # fp32 caches take the SIMT attention kernel, always followed by the combine
     assert H.hata_decode_kernel_launches(4, 32, 2048, torch.float32) == 5
+    # bf16 caches in the fused step: prep, score, the selection + attention kernel
+    H.hata_set_decode_mode(H.HATA_MODE_FUSED)
+    try:
+        assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 3
+    finally:
+        H.hata_set_decode_mode(H.HATA_MODE_AUTO)
     for bad in ((0, 32, 2048, H.HATA_DT_BF16), (4, 0, 2048, H.HATA_DT_BF16),
                 (4, 32, 0, H.HATA_DT_BF16), (4, 32, 2048, 9)):
         assert L.hata_decode_kernel_launches(*bad) == -1

@@ -46,6 +46,25 @@ def test_hash_keys_bit_exact(dtype):
     assert np.all((got[:, 1, pos0:pos0 + n, 2] >> 13) & 1 == 0)  # bit 77 = word 2, bit 13
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_hash_keys_strided_view(dtype):
+    """A key cache seen through a strided view of a larger buffer (extra
+    positions and channels around it, an odd element offset) is hashed in
+    place; the oracle hashes a dense copy."""
+    g = torch.Generator(device="cuda").manual_seed(15)
+    B, Hkv, n_cap, pos0, n = 2, 3, 1500, 7, 1480
+    big = _kv(dtype, (B, Hkv + 1, n_cap + 37, 256 + 8), g)
+    K = big[:, 1:, 5:5 + n_cap, 3:3 + 128]
+    assert not K.is_contiguous() and K.stride(3) == 1
+    W = torch.randn((Hkv, 128, 128), generator=g, device="cuda") / math.sqrt(128)
+    codes = torch.full((B, Hkv, n_cap, 4), -1, dtype=torch.int32, device="cuda")
+    H.hata_hash_keys(K, W, codes, pos0, n)
+    got = to_np_codes(codes)
+    want = oracle.hash_keys(wl.to_numpy_kv(K.contiguous()), W.cpu().numpy(), pos0=pos0, n=n)
+    assert np.array_equal(got[:, :, pos0:pos0 + n], want[:, :, pos0:pos0 + n])
+    assert np.all(got[:, :, :pos0] == 0xFFFFFFFF) and np.all(got[:, :, pos0 + n:] == 0xFFFFFFFF)
+
+
 def test_append_code_and_position_check():
     g = torch.Generator(device="cuda").manual_seed(12)
     B, Hkv, n_cap = 3, 2, 100
@@ -158,7 +177,7 @@ SCALED = {
 
 
 @pytest.mark.parametrize("name", wl.CONFIG_ORDER)
-def test_decode_scaled_configs(name):
+def test_decode_scaled_configs(name, decode_mode):
     kw = SCALED[name]
     cfg = wl.scaled(wl.CONFIGS[name], **kw)
     if cfg.needles:
@@ -174,7 +193,7 @@ NARROW = [("llama31_8b_gqa_128k", dict(N=10000, topk=156, B=2)),  # stream-K att
 
 @pytest.mark.parametrize("r", [32, 64])
 @pytest.mark.parametrize("case", range(len(NARROW)))
-def test_decode_narrow_codes(r, case):
+def test_decode_narrow_codes(r, case, decode_mode):
     """The whole decode step with r = 32 / 64 bit codes (distances 0..r)."""
     name, kw = NARROW[case]
     cfg = wl.scaled(wl.CONFIGS[name], **kw)
@@ -190,12 +209,12 @@ def test_decode_tiny_config_full_size():
 @pytest.mark.parametrize("N,topk", [(1, 1), (1, 5), (7, 3), (31, 31), (31, 64), (100, 1),
                                     (4095, 4095), (4096, 2), (4097, 4097), (8192, 300),
                                     (9000, 9000), (12345, 20000)])
-def test_decode_edge_sizes(N, topk):
+def test_decode_edge_sizes(N, topk, decode_mode):
     cfg = wl.Config("edge", 1, 4, 2, N, topk, "bf16", 0.0, 0.0, 0, 1)
     run_and_check(cfg, seed=31 + N, steps=1)
 
 
-def test_decode_ragged_batch_lengths():
+def test_decode_ragged_batch_lengths(decode_mode):
     """Sequences of one batch at different lengths, including an empty one."""
     cfg = wl.Config("ragged", 4, 4, 2, 9000, 70, "bf16", 0.0, 0.0, 0, 1)
     w = wl.make_workload(cfg, 41, device="cuda", steps=1)
@@ -217,7 +236,7 @@ def test_decode_ragged_batch_lengths():
             compare_head(got, want, b, hq, n, dec.drow)
 
 
-def test_all_equal_distances_take_lowest_indices():
+def test_all_equal_distances_take_lowest_indices(decode_mode):
     """Identical keys: every distance ties, so S = {0 .. k-1}."""
     cfg = wl.Config("ties", 1, 2, 1, 10000, 5000, "bf16", 0.0, 0.0, 0, 1)
     w = wl.make_workload(cfg, 51, device="cuda", steps=1)
@@ -228,7 +247,7 @@ def test_all_equal_distances_take_lowest_indices():
     assert np.all(dist[0, :, :cfg.N] == dist[0, :, :1])
 
 
-def test_tie_bucket_spanning_chunk_boundaries():
+def test_tie_bucket_spanning_chunk_boundaries(decode_mode):
     """A run of identical keys across chunk boundaries forms the boundary
     bucket; the lower-index ties must win, chunk by chunk."""
     cfg = wl.Config("tie-span", 1, 3, 1, 20000, 3000, "bf16", 0.0, 0.0, 0, 1)
@@ -243,7 +262,7 @@ def test_tie_bucket_spanning_chunk_boundaries():
         compare_head(got, want, 0, hq, cfg.N, dec.drow)
 
 
-def test_full_budget_equals_dense():
+def test_full_budget_equals_dense(decode_mode):
     """k >= seq_len selects every key: the sparse output equals dense softmax
     attention (the GPU dense kernel and the oracle's)."""
     cfg = wl.Config("dense", 2, 8, 2, 7000, 8000, "bf16", 0.0, 0.0, 0, 1)
@@ -286,7 +305,7 @@ def test_dense_kernel_matches_oracle_all_shapes():
                 assert np.max(np.abs(dout[b, hq] - ref)) <= ATOL, (B, Hq, Hkv, N, b, hq)
 
 
-def test_repeatable_bitwise():
+def test_repeatable_bitwise(decode_mode):
     """Two identical calls give bitwise identical results (no races)."""
     cfg = wl.scaled(wl.CONFIGS["qwen_gqa_b32_32k"], N=9000, topk=140, B=4)
     w = wl.make_workload(cfg, 71, device="cuda", steps=1)
@@ -342,48 +361,126 @@ def test_invalid_arguments_with_real_tensors():
     assert e.value.status == H.HATA_ERR_UNSUPPORTED
 
 
+def test_fused_wait_limit_reports_timeout_and_recovers():
+    """With a wait bound of 0 ns every wait of the fused step that is not
+    already satisfied gives up: the kernel finishes, HATA_FLAG_TIMEOUT is
+    reported, and the next step with the normal bound is correct again on
+    the same context and workspace."""
+    cfg = wl.Config("timeout", 2, 8, 2, 12000, 200, "bf16", 0.02, 0.3, 0, 1)
+    w = wl.make_workload(cfg, 93, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk)
+    out = torch.empty((2, 8, 128), device="cuda")
+    sl = torch.full((2,), cfg.N, dtype=torch.int32, device="cuda")
+    H.hata_set_wait_limit_ns(0)
+    try:
+        H.hata_decode_step(w.q[0], w.W_H, dec.codes, w.K, w.V, sl, dec.max_seq_len, cfg.topk,
+                           SCALE, dec.ws, out)
+        torch.cuda.synchronize()
+    finally:
+        H.hata_set_wait_limit_ns(10**9)
+    with pytest.raises(H.HataError) as e:
+        H.hata_workspace_check(dec.ws)
+    assert e.value.status == H.HATA_ERR_DEVICE_CHECK
+    assert "0x4" in str(e.value)
+    slabs = host_slabs(w, [(b, h) for b in range(2) for h in range(2)])
+    got = dec.step(w.q[0], [cfg.N] * 2)
+    Wn = w.W_H.cpu().numpy()
+    for b in range(2):
+        for hq in range(8):
+            want = oracle_head(slabs[(b, hq // 4)], Wn[hq // 4], w.q[0, b, hq].cpu().numpy(),
+                               cfg.N, cfg.topk)
+            compare_head(got, want, b, hq, cfg.N, dec.drow)
+
+
 # ------------------------------------------------------ full-size configs --
 
-FULL = {
-    "llama2_7b_mha_32k": [(0, 0), (0, 31)],
-    "llama31_8b_gqa_128k": [(0, 0), (3, 29)],
-    "qwen_gqa_b32_32k": [(0, 0), (31, 27)],
-    "needle_gqa_1m": [(0, 0), (0, 1)],
+# Sampled KV slabs of the full-size workloads; every query head of each
+# sampled slab is compared (the oracle hashes the slab's keys once).
+FULL_SLABS = {
+    "llama2_7b_mha_32k": [(0, h) for h in range(32)],   # MHA: all 32 heads
+    "llama31_8b_gqa_128k": [(0, 0), (3, 7)],
+    "qwen_gqa_b32_32k": [(0, 0), (31, 3)],
+    "needle_gqa_1m": [(0, 0), (0, 5)],
 }
 
 
-@pytest.mark.parametrize("name", list(FULL))
+def _oracle_slab_heads(cfg, w, slabs, Wn, b, h, n, got, drow, q, codes=None):
+    """Compare every query head of slab (b, h) with the oracle (codes: the
+    slab's key codes as the oracle hashed them, if already known)."""
+    for hq in range(h * cfg.G, (h + 1) * cfg.G):
+        want = oracle_head(slabs[(b, h)], Wn[h], q[b, hq].cpu().numpy(), n, cfg.topk, codes)
+        codes = want[0]
+        compare_head(got, want, b, hq, n, drow)
+        if cfg.needles and hq % cfg.G == 0:
+            needles = set(w.planted[b, h].tolist())
+            assert needles <= set(got[1][b, hq].tolist())
+    return codes
+
+
+@pytest.mark.parametrize("name", list(FULL_SLABS))
 def test_full_size_sampled_heads(name):
     """Full-size workloads in the launch configuration bench.py times; the
-    oracle recomputes sampled heads one by one.  For the needle workload the
-    needles of the group's first query head must all be selected."""
+    oracle recomputes every query head of the sampled KV slabs one by one.
+    For the needle workload the needles of the group's first query head must
+    all be selected."""
     cfg = wl.CONFIGS[name]
-    heads = FULL[name]
+    pairs = FULL_SLABS[name]
     w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(name), device="cuda",
                          steps=1)
-    pairs = sorted({(b, hq // cfg.G) for b, hq in heads})
     slabs = host_slabs(w, pairs)
     pos = [cfg.N] * cfg.B
     host_append(slabs, w, 0, pos)
     dec = GpuDecoder(w, cfg.topk)
     n = cfg.N + 1
-    got = dec.step(w.q[0], [n] * cfg.B, k_new=w.k_new[0], v_new=w.v_new[0])
+    # both step implementations (the append is the same token both times)
+    gots = []
+    for mode in (H.HATA_MODE_FUSED, H.HATA_MODE_MULTI_KERNEL):
+        H.hata_set_decode_mode(mode)
+        try:
+            gots.append(dec.step(w.q[0], [n] * cfg.B, k_new=w.k_new[0], v_new=w.v_new[0]))
+        finally:
+            H.hata_set_decode_mode(H.HATA_MODE_AUTO)
     Wn = w.W_H.cpu().numpy()
-    cache = {}
-    for b, hq in heads:
-        h = hq // cfg.G
-        want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n, cfg.topk,
-                           cache.get((b, h)))
-        cache[(b, h)] = want[0]
-        compare_head(got, want, b, hq, n, dec.drow)
-        if cfg.needles and hq % cfg.G == 0:
-            needles = set(w.planted[b, h].tolist())
-            assert needles <= set(got[1][b, hq].tolist())
+    gcodes = to_np_codes(dec.codes)
+    for b, h in pairs:
+        codes = None
+        for got in gots:
+            codes = _oracle_slab_heads(cfg, w, slabs, Wn, b, h, n, got, dec.drow, w.q[0], codes)
+        assert np.array_equal(gcodes[b, h, :n], codes), ("key codes", b, h)
     del w, dec
     torch.cuda.empty_cache()
 
 
-def test_host_buffers_match_device_buffers():
+def test_sixteen_appending_steps_full_size_qwen():
+    """The batched Qwen-shaped workload as the bench runs it: 16 consecutive
+    decode steps, each appending one key per sequence.  After the last step
+    the appended codes and K/V rows of all 16 positions, and every query
+    head of two sampled KV slabs, agree with the oracle."""
+    name = "qwen_gqa_b32_32k"
+    cfg = wl.CONFIGS[name]
+    steps = 16
+    pairs = [(0, 0), (31, 3)]
+    w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(name), device="cuda",
+                         steps=steps)
+    slabs = host_slabs(w, pairs)
+    dec = GpuDecoder(w, cfg.topk)
+    for t in range(steps):
+        pos = [cfg.N + t] * cfg.B
+        host_append(slabs, w, t, pos)
+        got = dec.step(w.q[t], [cfg.N + t + 1] * cfg.B, k_new=w.k_new[t], v_new=w.v_new[t])
+    n = cfg.N + steps
+    Wn = w.W_H.cpu().numpy()
+    gcodes = to_np_codes(dec.codes)
+    for b, h in pairs:
+        codes = _oracle_slab_heads(cfg, w, slabs, Wn, b, h, n, got, dec.drow, w.q[steps - 1])
+        assert np.array_equal(gcodes[b, h, :n], codes), ("key codes", b, h)
+        assert np.array_equal(wl.to_numpy_kv(w.K[b, h, cfg.N:n]), slabs[(b, h)].K[cfg.N:n])
+        assert np.array_equal(wl.to_numpy_kv(w.V[b, h, cfg.N:n]), slabs[(b, h)].V[cfg.N:n])
+    del w, dec
+    torch.cuda.empty_cache()
+
+
+def test_host_buffers_match_device_buffers(decode_mode):
     """q, k_new, v_new and out in pinned host memory: the kernels read and
     write them directly; the step's output, selection and appended caches are
     bit-identical to the same step with device buffers."""
@@ -413,7 +510,7 @@ def test_host_buffers_match_device_buffers():
         assert torch.equal(a, b)
 
 
-def test_host_resident_kv_cache_matches_device():
+def test_host_resident_kv_cache_matches_device(decode_mode):
     """K and V kept in pinned host memory (only the selected rows cross the
     bus each step): output, selection and the appended rows are identical to
     the same step on device-resident caches."""
@@ -438,9 +535,24 @@ def test_host_resident_kv_cache_matches_device():
         res.append((out.cpu(), sel.cpu(), codes.cpu(), K[:, :, cfg.N].cpu(), V[:, :, cfg.N].cpu()))
     for a, b in zip(*res):
         assert torch.equal(a, b)
+    # and the host-resident step agrees with the oracle on every head
+    slabs = host_slabs(w, [(b, h) for b in range(cfg.B) for h in range(cfg.H_kv)])
+    host_append(slabs, w, 0, [cfg.N] * cfg.B)
+    out_h, sel_h = res[1][0].numpy(), res[1][1].numpy()
+    Wn = w.W_H.cpu().numpy()
+    n = cfg.N + 1
+    for b in range(cfg.B):
+        for h in range(cfg.H_kv):
+            codes = None
+            for hq in range(h * cfg.G, (h + 1) * cfg.G):
+                want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n,
+                                   cfg.topk, codes)
+                codes = want[0]
+                np.testing.assert_array_equal(sel_h[b, hq], want[3])
+                assert np.max(np.abs(out_h[b, hq].astype(np.float64) - want[4])) <= ATOL
 
 
-def test_decode_head_per_cta_merge():
+def test_decode_head_per_cta_merge(decode_mode):
     """128 query heads (about one wave of attention CTAs): every head is
     gathered by one CTA and merged in shared memory; the oracle still
     decides, including short rows (k_eff < topk) and an empty one."""
@@ -463,14 +575,25 @@ def test_decode_head_per_cta_merge():
 
 
 def test_decode_kernel_launch_count():
-    """128 heads at topk 2048 fill about one wave of attention CTAs (merged
-    in-CTA, no combine kernel); 32 heads do not."""
-    assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 4
-    assert H.hata_decode_kernel_launches(1, 32, 2048, torch.bfloat16) == 5
-    assert H.hata_decode_kernel_launches(4, 32, 100, torch.bfloat16) == 5  # too few rows per warp
+    """Fused step: prep, score and one persistent selection + attention
+    kernel.  Multi-kernel step: 128
+    heads at topk 2048 fill about one wave of attention CTAs (merged in-CTA,
+    no combine kernel); 32 heads do not."""
+    H.hata_set_decode_mode(H.HATA_MODE_FUSED)
+    try:
+        assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 3
+    finally:
+        H.hata_set_decode_mode(H.HATA_MODE_AUTO)
+    H.hata_set_decode_mode(H.HATA_MODE_MULTI_KERNEL)
+    try:
+        assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 4
+        assert H.hata_decode_kernel_launches(1, 32, 2048, torch.bfloat16) == 5
+        assert H.hata_decode_kernel_launches(4, 32, 100, torch.bfloat16) == 5  # too few rows per warp
+    finally:
+        H.hata_set_decode_mode(H.HATA_MODE_AUTO)
 
 
-def test_one_wave_of_heads_ties_across_tiles():
+def test_one_wave_of_heads_ties_across_tiles(decode_mode):
     """128 heads (one attention CTA per head): a run of identical keys forms
     the boundary bucket across selection tiles, and the lower-index ties
     must win; lengths cover a full row, a partial one and k_eff = len."""
@@ -480,7 +603,8 @@ def test_one_wave_of_heads_ties_across_tiles():
     heads = [(b, hq) for b in range(cfg.B) for hq in (0, 5, 31)]
     slabs = host_slabs(w, sorted({(b, hq // cfg.G) for b, hq in heads}))
     dec = GpuDecoder(w, cfg.topk)
-    assert H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.topk, torch.bfloat16) == 4
+    assert H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.topk, torch.bfloat16) == (
+        4 if decode_mode == "multi_kernel" else 3)
     lens = [cfg.N, 17001, 2999, 19999]
     got = dec.step(w.q[0], lens)
     Wn = w.W_H.cpu().numpy()
@@ -491,7 +615,7 @@ def test_one_wave_of_heads_ties_across_tiles():
 
 
 @pytest.mark.parametrize("B", [1, 4])
-def test_decode_steps_replay_from_cuda_graph(B):
+def test_decode_steps_replay_from_cuda_graph(B, decode_mode):
     """Consecutive decode steps (each appending a token) captured once into a
     CUDA Graph and replayed give the same bits as the same steps run eagerly
     on an identical workload (B = 4: one attention CTA per head; B = 1:
@@ -532,3 +656,20 @@ def test_decode_steps_replay_from_cuda_graph(B):
     for x, y in zip(*outs):
         assert np.array_equal(x, y)
     assert np.all(outs[0][1][:, :, :, :cfg.topk] >= 0)  # every step selected a full list
+    # the replayed steps agree with the oracle (every head, every step)
+    w = wl.make_workload(cfg, 77, device="cuda", steps=steps)
+    slabs = host_slabs(w, [(b, h) for b in range(B) for h in range(cfg.H_kv)])
+    Wn = w.W_H.cpu().numpy()
+    g_out, g_sel = outs[1][0], outs[1][1]
+    for t in range(steps):
+        host_append(slabs, w, t, [cfg.N + t] * B)
+        n = cfg.N + t + 1
+        for b in range(B):
+            for h in range(cfg.H_kv):
+                codes = None
+                for hq in range(h * cfg.G, (h + 1) * cfg.G):
+                    want = oracle_head(slabs[(b, h)], Wn[h], w.q[t, b, hq].cpu().numpy(), n,
+                                       cfg.topk, codes)
+                    codes = want[0]
+                    np.testing.assert_array_equal(g_sel[t, b, hq], want[3])
+                    assert np.max(np.abs(g_out[t, b, hq].astype(np.float64) - want[4])) <= ATOL
