@@ -29,6 +29,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -99,7 +100,8 @@ class ClockSampler:
             time.sleep(0.002)
 
     def __enter__(self):
-        self._t.start()
+        if not self._t.is_alive() and not self._stop.is_set():
+            self._t.start()
         return self
 
     def __exit__(self, *exc):
@@ -146,51 +148,39 @@ def max_over_ranks(world, x: float) -> float:
 
 # ------------------------------------------------------------ oracle (CPU) --
 
-class OracleSample:
-    """A bounded sample of the workload for the CPU oracle: `n_heads` query
-    heads at context n_len, their slabs' key codes hashed once up front (the
-    decode step itself only hashes the query)."""
-
-    def __init__(self, cfg, w, n_heads: int, n_len: int):
-        import oracle
-        self.cfg, self.n_len = cfg, n_len
-        G = cfg.G
-        self.heads = [(b, hq) for b in range(cfg.B) for hq in range(cfg.H_q)][
-            :: max(1, cfg.B * cfg.H_q // n_heads)][:n_heads]
-        self.Wn = w.W_H.cpu().numpy()
-        self.slabs, self.codes = {}, {}
-        for b, hq in self.heads:
-            h = hq // G
-            if (b, h) not in self.slabs:
-                K = wl.to_numpy_kv(w.K[b, h, :n_len])
-                V = wl.to_numpy_kv(w.V[b, h, :n_len])
-                self.slabs[(b, h)] = (K, V)
-                self.codes[(b, h)] = oracle.hash_keys(K[None, None], self.Wn[h][None])[0, 0]
-        self.qs = {(b, hq): w.q[0, b, hq].cpu().numpy() for b, hq in self.heads}
-
-    def seconds_per_head(self) -> float:
-        """Time the oracle's decode step over the sample; seconds per head."""
-        import oracle
-        t0 = time.perf_counter()
-        for b, hq in self.heads:
-            h = hq // self.cfg.G
-            K, V = self.slabs[(b, h)]
-            oracle.decode_head(self.qs[(b, hq)], self.Wn[h], self.codes[(b, h)], K, V,
-                               self.n_len, self.cfg.topk, 1.0 / math.sqrt(128))
-        return (time.perf_counter() - t0) / len(self.heads)
-
-    def describe(self) -> str:
-        c = self.cfg
-        return (f"oracle decode (hash q, Hamming over {self.n_len} codes, sorted top-{c.topk}, "
-                f"fp64 attention) on {len(self.heads)} of {c.B * c.H_q} query heads, scaled to "
-                f"a full step; key codes hashed before timing")
+def oracle_step(cfg, w, workers=None):
+    """The CPU oracle on whole decode steps of the workload over the host
+    cores (oracle/pool.py): the prompt caches (generator values, never
+    written by the CUDA path) copied to the host, their key codes hashed by
+    the oracle's pool beforehand (untimed)."""
+    from oracle import pool
+    N = cfg.N
+    K = np.zeros((cfg.B, cfg.H_kv, w.n_cap, 128), wl.to_numpy_kv(w.K[:1, :1, :1]).dtype)
+    V = np.zeros_like(K)
+    K[:, :, :N] = wl.to_numpy_kv(w.K[:, :, :N])
+    V[:, :, :N] = wl.to_numpy_kv(w.V[:, :, :N])
+    ops = pool.OracleStep(K, V, w.W_H.cpu().numpy(), cfg.H_q, workers=workers)
+    del K, V
+    t_hash = ops.hash_prefix(N)
+    return ops, t_hash
 
 
-def oracle_sample(cfg, w, n_heads: int, n_len: int):
-    """Time the CPU oracle on `n_heads` query heads of the workload at
-    context n_len; returns (seconds per head, description)."""
-    s = OracleSample(cfg, w, n_heads, n_len)
-    return s.seconds_per_head(), s.describe()
+def oracle_step_time(cfg, w, ops, t: int):
+    """One oracle decode step t (append of the step's key and value at
+    position N + t, then every query head at context N + t + 1); seconds."""
+    t0 = time.perf_counter()
+    ops.append(wl.to_numpy_kv(w.k_new[t]), wl.to_numpy_kv(w.v_new[t]), cfg.N + t)
+    t_append = time.perf_counter() - t0
+    dt, _ = ops.step(w.q[t].cpu().numpy(), cfg.N + t + 1, cfg.topk, 1.0 / math.sqrt(128))
+    return t_append + dt
+
+
+def oracle_desc(cfg, ops) -> str:
+    from oracle import pool
+    return (f"CPU oracle, whole decode steps (append, then hash q, Hamming over "
+            f"{cfg.N + 1} codes, sorted top-{cfg.topk} and fp64 attention for all "
+            f"{cfg.B * cfg.H_q} query heads), one task per head on {ops.workers} processes "
+            f"({pool.cpu_model()}); prompt key codes hashed by the oracle beforehand, untimed")
 
 
 def bench_config(args):
@@ -206,19 +196,23 @@ def bench_config(args):
 
 
 def run_reference(args, world, rank):
-    """--impl reference: the CPU oracle, single-threaded, on the host cores."""
+    """--impl reference: the CPU oracle on whole decode steps of the same
+    workload, over all host cores (rank 0 only)."""
     if rank != 0:
         return
     cfg = bench_config(args)
-    w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config), device="cpu"
-                         if not torch.cuda.is_available() else "cuda", steps=1)
-    sample = OracleSample(cfg, w, n_heads=2, n_len=cfg.N)
-    heads_total = cfg.B * cfg.H_q
-    # each step times the same bounded sample (two heads) and scales it to a full step
-    for _ in range(args.warmup):
-        sample.seconds_per_head()
-    times = [sample.seconds_per_head() * heads_total for _ in range(args.steps)]
-    desc = sample.describe()
+    steps = args.warmup + args.steps
+    w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(args.config),
+                         device="cuda" if torch.cuda.is_available() else "cpu", steps=steps)
+    ops, _ = oracle_step(cfg, w)
+    try:
+        for t in range(args.warmup):
+            oracle_step_time(cfg, w, ops, t)
+        times = [oracle_step_time(cfg, w, ops, args.warmup + i) for i in range(args.steps)]
+        desc = oracle_desc(cfg, ops)
+        cores = ops.workers
+    finally:
+        ops.close()
     us = statistics.mean(times) * 1e6
     line = {
         "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": UNIT,
@@ -226,7 +220,7 @@ def run_reference(args, world, rank):
         "ms_per_step": round(us / 1e3, 3), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(cfg, "none (CPU)"),
-        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -469,6 +463,73 @@ def more_legs(cfg, w, codes, ws, out, seq, flush, stream, t0, K_steps):
     return res
 
 
+OTHER_WORKLOADS = ("llama2_7b_mha_32k", "qwen_gqa_b32_32k", "needle_gqa_1m")
+
+
+def other_workloads(args, dev):
+    """The other large workloads, each on its own (flushed L2 before every
+    step): microseconds per decode step and the step's roofline fraction;
+    the batched Qwen-shaped workload runs its 16 consecutive appending steps
+    (per-step figure), the million-token workload reports needle recall."""
+    res = {}
+    peak, _ = measured_peaks()
+    scale = 1.0 / math.sqrt(128)
+    flush_buf = torch.zeros(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+    for name in OTHER_WORKLOADS:
+        if name == args.config:
+            continue
+        cfg = wl.CONFIGS[name]
+        B, Hq, Hkv, N = cfg.B, cfg.H_q, cfg.H_kv, cfg.N
+        warm = 3
+        timed = cfg.steps if cfg.steps > 1 else 10
+        w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(name), device=dev,
+                             steps=warm + timed)
+        codes = torch.zeros((B, Hkv, w.n_cap, 4), dtype=torch.int32, device=dev)
+        H.hata_hash_keys(w.K, w.W_H, codes, 0, N)
+        ws = torch.empty(H.hata_decode_workspace_size(B, Hq, Hkv, w.n_cap, cfg.topk),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty((B, Hq, 128), device=dev)
+        sel = torch.empty((B, Hq, cfg.topk), dtype=torch.int32, device=dev)
+        seq = (N + 1 + torch.arange(warm + timed, dtype=torch.int32, device=dev))[:, None] \
+            .expand(warm + timed, B).contiguous()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(timed)]
+        for t in range(warm + timed):
+            torch.sum(flush_buf)
+            if t >= warm:
+                evs[t - warm][0].record(stream)
+            H.hata_decode_step(w.q[t], w.W_H, codes, w.K, w.V, seq[t], w.n_cap, cfg.topk, scale,
+                               ws, out, k_new=w.k_new[t], v_new=w.v_new[t], sel_idx=sel)
+            if t >= warm:
+                evs[t - warm][1].record(stream)
+        torch.cuda.synchronize()
+        H.hata_workspace_check(ws)
+        us = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
+        step_bytes = B * Hkv * (N + warm + timed // 2) * 16 + B * Hq * cfg.topk * 2 * 256
+        entry = {"us_per_step": round(us, 2), "steps": timed,
+                 "step_roofline_bytes": step_bytes,
+                 "step_frac_of_measured": round(step_bytes / (us * 1e-6) / 1e9 / peak, 4),
+                 "shape": f"B {B}, {Hq}/{Hkv} heads, context {N}, top-{cfg.topk}"}
+        if cfg.steps > 1:
+            entry["note"] = f"{timed} consecutive decode steps, each appending one key"
+        if cfg.needles > 0:
+            # needles kept in the last step's selection of each group's first
+            # query head (the head the needles point at)
+            sel_c = sel.cpu()
+            hits = total = 0
+            for b in range(B):
+                for h in range(Hkv):
+                    nd = set(x for x in w.planted[b, h].tolist() if x >= 0)
+                    hits += len(nd & set(sel_c[b, h * cfg.G].tolist()))
+                    total += len(nd)
+            entry["needle_recall"] = round(hits / max(total, 1), 4)
+        res[name] = entry
+        del w, codes, ws, out, sel
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_hata(args, world, rank, local):
     cfg = bench_config(args)
     K_steps, W_steps = args.steps, args.warmup
@@ -495,6 +556,8 @@ def run_hata(args, world, rank, local):
         H.hata_decode_step(w.q[t], w.W_H, codes, w.K, w.V, seq[t], w.n_cap, cfg.topk, scale,
                            ws, out, k_new=w.k_new[t], v_new=w.v_new[t], events=events)
 
+    # clocks are sampled from the warm-up on, through the timed region
+    clk = ClockSampler(local).__enter__()
     for t in range(W_steps):
         flush()
         step(t)
@@ -504,7 +567,7 @@ def run_hata(args, world, rank, local):
     # timed region: the step alone (no events between its kernels, so each
     # kernel's launch overlaps its predecessor), bracketed by two events
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
-    with ClockSampler(local) as clk:
+    with clk:
         barrier(world)
         torch.cuda.synchronize()
         wall0 = time.perf_counter()
@@ -601,7 +664,7 @@ def run_hata(args, world, rank, local):
                         "sum_with_events": round(statistics.mean(split_ms) * 1e3, 2),
                         "score_gbs": round(code_bytes / score_s / 1e9, 1)}),
         "dense_us": _num(dense_ms * 1e3, 1),
-        "speedup_vs_dense": _num(dense_ms / ms, 2),
+        "speedup_vs_dense": None,
         "e2e": {"value": _num(e2e_ms * 1e3, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "side": side,
@@ -610,10 +673,39 @@ def run_hata(args, world, rank, local):
         "clocks": clk.summary(),
         "wall_s_timed_region": round(wall, 4),
     }
+    # the speedup over dense decode attention at the same shape divides by
+    # the faster of this library's dense kernel and torch SDPA
+    sdpa_us = (side or {}).get("sdpa_dense_us")
+    dense_cands = [(dense_ms * 1e3, "hata_dense_decode")]
+    if sdpa_us:
+        dense_cands.append((sdpa_us, "torch SDPA (enable_gqa)"))
+    dense_cands = [c for c in dense_cands if c[0] == c[0]]
+    if dense_cands:
+        best_us, best_name = min(dense_cands)
+        line["speedup_vs_dense"] = round(best_us / (ms * 1e3), 2)
+        line["dense_baseline"] = {"us": round(best_us, 1), "impl": best_name}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_head, desc = oracle_sample(cfg, w, n_heads=args.cpu_heads, n_len=N)
-        line["cpu_baseline"] = {"value": round(per_head * B * Hq * 1e6, 1), "unit": UNIT,
-                                "cores": 1, "kind": "oracle", "sample": desc}
+        # the oracle on one whole step over every host core, and whole heads
+        # on one core (scaled to a step)
+        ops, t_hash = oracle_step(cfg, w)
+        try:
+            t_all = oracle_step_time(cfg, w, ops, 0)
+            heads = [(0, 0), (B - 1, Hq - 1)]
+            per_head = ops.one_core_seconds_per_head(w.q[1].cpu().numpy(), N + 1, cfg.topk,
+                                                     scale, heads)
+            line["cpu_baseline"] = {"value": round(t_all * 1e6, 1), "unit": UNIT,
+                                    "cores": ops.workers, "kind": "oracle",
+                                    "sample": oracle_desc(cfg, ops),
+                                    "one_core_us_per_step": round(per_head * B * Hq * 1e6, 1),
+                                    "one_core_sample": f"{len(heads)} whole heads on one core, "
+                                                       f"scaled to {B * Hq} heads",
+                                    "prompt_hash_s": round(t_hash, 2)}
+        finally:
+            ops.close()
+    if rank == 0 and world == 1 and not args.no_extras and not args.no_other_configs:
+        del w, codes, ws, flush_buf
+        torch.cuda.empty_cache()
+        line["other_workloads"] = other_workloads(args, dev)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -625,13 +717,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=wl.CONFIG_ORDER)
     ap.add_argument("--impl", default="hata", choices=["hata", "reference"])
-    ap.add_argument("--cpu-heads", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--context", type=int, default=0, help="override the context length")
     ap.add_argument("--batch", type=int, default=0, help="override the batch size")
     ap.add_argument("--topk", type=int, default=0, help="override the top-k budget")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e, dense and CPU legs (profiling runs)")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the side measurements of the other large workloads")
     ap.add_argument("--decode-mode", default="auto", choices=["auto", "multi_kernel", "fused"],
                     help="step implementation: auto (the library's choice), the multi-kernel "
                          "step or the fused step")

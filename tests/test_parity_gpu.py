@@ -371,6 +371,7 @@ def test_fused_wait_limit_reports_timeout_and_recovers():
     dec = GpuDecoder(w, cfg.topk)
     out = torch.empty((2, 8, 128), device="cuda")
     sl = torch.full((2,), cfg.N, dtype=torch.int32, device="cuda")
+    H.hata_set_decode_mode(H.HATA_MODE_FUSED)
     H.hata_set_wait_limit_ns(0)
     try:
         H.hata_decode_step(w.q[0], w.W_H, dec.codes, w.K, w.V, sl, dec.max_seq_len, cfg.topk,
@@ -383,7 +384,10 @@ def test_fused_wait_limit_reports_timeout_and_recovers():
     assert e.value.status == H.HATA_ERR_DEVICE_CHECK
     assert "0x4" in str(e.value)
     slabs = host_slabs(w, [(b, h) for b in range(2) for h in range(2)])
-    got = dec.step(w.q[0], [cfg.N] * 2)
+    try:
+        got = dec.step(w.q[0], [cfg.N] * 2)
+    finally:
+        H.hata_set_decode_mode(H.HATA_MODE_AUTO)
     Wn = w.W_H.cpu().numpy()
     for b in range(2):
         for hq in range(8):
@@ -572,6 +576,29 @@ def test_decode_head_per_cta_merge(decode_mode):
             h = hq // cfg.G
             want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n, cfg.topk)
             compare_head(got, want, b, hq, n, dec.drow)
+
+
+def test_decode_many_selected_rows(decode_mode):
+    """A thousand selected rows for each of 96 heads (every attention worker
+    takes rows of two heads, and heads are shared between workers), a
+    sequence shorter than the budget (k_eff < topk) and an empty one,
+    against the oracle."""
+    cfg = wl.Config("split", 3, 32, 8, 20000, 1000, "bf16", 0.02, 0.3, 0, 1)
+    w = wl.make_workload(cfg, 8282, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk)
+    lens = [cfg.N, 700, 0]
+    heads = [(b, hq) for b in range(2) for hq in range(0, 32, 3)] + [(2, 0), (2, 31)]
+    slabs = host_slabs(w, sorted({(b, hq // cfg.G) for b, hq in heads}))
+    got = dec.step(w.q[0], lens)
+    Wn = w.W_H.cpu().numpy()
+    for b, hq in heads:
+        n = lens[b]
+        if n == 0:
+            assert np.all(got[0][b, hq] == 0) and np.all(got[1][b, hq] == -1)
+            continue
+        h = hq // cfg.G
+        want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n, cfg.topk)
+        compare_head(got, want, b, hq, n, dec.drow)
 
 
 def test_decode_kernel_launch_count():
