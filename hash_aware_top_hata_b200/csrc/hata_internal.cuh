@@ -20,9 +20,9 @@ constexpr int kScoreThreads = 1024;
 constexpr int kScoreHeads = 8;          // query heads scored per code load (one CTA)
 constexpr int kAttnThreads = 128;
 constexpr int kHistStride = 132;        // u32 per (head, tile) histogram row (129 bins)
-constexpr int kTile = 32768;            // tokens per histogram tile / selection tile (8 x 4096)
+constexpr int kTile = 36864;            // tokens per histogram tile / selection tile (9 x 4096)
 constexpr int kPartStride = 132;        // f32 per (head, chunk) partial: m, l, -, -, acc[128]
-constexpr int kFSeg = 112;              // selected rows per attention item, fused step
+constexpr int kFSeg = 96;               // selected rows per attention item, fused step
                                         // (16 per attention warp)
 constexpr uint8_t kDistPad = 255;       // distance stored past seq_len
 constexpr uint32_t kWsMagic = 0x48415441u;  // "HATA"
@@ -56,7 +56,7 @@ inline int attn_max_contributors(int64_t BH, int topk)
 struct DecodeLayout {
     int64_t n_chunks = 0;   // 4096-token chunks of max_seq_len
     int64_t dist_row = 0;   // bytes per (b, h_q) distance row
-    int64_t n_tiles = 0;    // 32K-token histogram / selection tiles of a distance row
+    int64_t n_tiles = 0;    // 36K-token histogram / selection tiles of a distance row
     int zgroups = 0;        // ceil(G / kScoreHeads)
     int n_split = 0;        // attention partial slots per head (multi-kernel step)
     int n_seg = 0;          // attention items per head (fused step)

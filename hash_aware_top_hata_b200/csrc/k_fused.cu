@@ -11,11 +11,11 @@
 // selected set is unique.
 //
 // As separate kernels, the selection (latency-bound: a threshold from the
-// tile histograms, one block scan and an ordered compaction per 32K-token
+// tile histograms, one block scan and an ordered compaction per 36K-token
 // tile) runs while HBM idles, and the attention waits for all of it.  Here
 // one CTA per SM runs three kinds of warps at once:
 //
-//   * kSW selection warps (256 threads): the CTA's selection tiles, statically
+//   * kSW selection warps (288 threads): the CTA's selection tiles, statically
 //     assigned (tile i of the flat (head, tile) sequence to CTA i mod P, in
 //     head order), each the multi-kernel selection's arithmetic
 //     (select_common.cuh); a finished tile is handed to the publisher.
@@ -48,8 +48,8 @@
 namespace hata {
 namespace {
 
-constexpr int kSW = 8;                     // selection warps
-constexpr int kAW = 7;                     // attention warps
+constexpr int kSW = 9;                     // selection warps
+constexpr int kAW = 6;                     // attention warps
 constexpr int kPubWarp = kSW + kAW;        // the publisher
 constexpr int kThreads = 32 * (kSW + kAW + 1);
 // 16 warps: four per SM sub-partition (each holds a quarter of the register

@@ -30,7 +30,7 @@
 //
 // Per query head the kernel stores the u8 distance row (32 lanes write 32
 // consecutive bytes per store; the row stays L2-resident for the selection
-// kernel) and counts a 129-bin histogram per (head, 32K-token tile) in
+// kernel) and counts a 129-bin histogram per (head, 36K-token tile) in
 // shared memory; a range touches at most kMaxKeys (slab, tile) pairs.  At
 // the end of its range the CTA adds the non-zero bins into the tile
 // histograms in global memory (zeroed by the prep kernel), one reduction
@@ -48,7 +48,7 @@ namespace {
 constexpr int kWarps = kScoreThreads / 32;  // 8
 constexpr int kUnit = 128;                  // tokens per warp step
 constexpr int kRing = 2;                    // units per warp ring
-constexpr int kTileUnits = kTile / kUnit;   // 256
+constexpr int kTileUnits = kTile / kUnit;   // 288
 constexpr int kMaxKeys = 8;                 // (slab, tile) histograms per CTA range
 constexpr int kMaxRange = 2048;             // units per CTA range
 

@@ -10,7 +10,7 @@
 //   S     = {n : dist[n] < T}  +  the r = k_eff - #(dist < T) lowest-index
 //           keys with dist[n] == T.
 //
-// Grid: (32K-token tile, b * H_q + h_q), 256 threads, each thread owning 128
+// Grid: (36K-token tile, b * H_q + h_q), 288 threads, each thread owning 128
 // consecutive distances (eight 16-byte loads, issued first).  Warp 0 sums
 // the head's tile histograms (written by the scoring kernel) while they are
 // in flight: the total gives T and r, the tiles before this one the keys
@@ -26,7 +26,7 @@
 namespace hata {
 namespace {
 
-constexpr int kThreads = 256;  // 8 warps x 128 distances = one tile
+constexpr int kThreads = 288;  // 9 warps x 128 distances = one tile
 constexpr int kWarps = kThreads / 32;
 constexpr int kPer = 128;                               // distances per thread
 constexpr int kPieces = kPer / 16;                      // 16-byte loads per thread
