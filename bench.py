@@ -530,6 +530,133 @@ def other_workloads(args, dev):
     return res
 
 
+def wide_code_leg(dev, name="llama31_8b_gqa_128k"):
+    """The headline workload with 256-bit codes (the widest width of the
+    page's ablation): microseconds per decode step (flushed L2) and the
+    step's roofline fraction, whose code bytes double to 32 per key."""
+    cfg = wl.CONFIGS[name]
+    B, Hq, Hkv, N = cfg.B, cfg.H_q, cfg.H_kv, cfg.N
+    warm, timed = 3, 10
+    peak, _ = measured_peaks()
+    w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(name), device=dev,
+                         steps=warm + timed)
+    W = wl.projection(w.W_H, 256)
+    codes = torch.zeros((B, Hkv, w.n_cap, 8), dtype=torch.int32, device=dev)
+    H.hata_hash_keys(w.K, W, codes, 0, N)
+    ws = torch.empty(H.hata_decode_workspace_size(B, Hq, Hkv, w.n_cap, cfg.topk),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty((B, Hq, 128), device=dev)
+    flush_buf = torch.zeros(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+    seq = (N + 1 + torch.arange(warm + timed, dtype=torch.int32, device=dev))[:, None] \
+        .expand(warm + timed, B).contiguous()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(timed)]
+    for t in range(warm + timed):
+        torch.sum(flush_buf)
+        if t >= warm:
+            evs[t - warm][0].record(stream)
+        H.hata_decode_step(w.q[t], W, codes, w.K, w.V, seq[t], w.n_cap, cfg.topk,
+                           1.0 / math.sqrt(128), ws, out, k_new=w.k_new[t], v_new=w.v_new[t])
+        if t >= warm:
+            evs[t - warm][1].record(stream)
+    torch.cuda.synchronize()
+    H.hata_workspace_check(ws)
+    us = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
+    step_bytes = B * Hkv * (N + warm + timed // 2) * 32 + B * Hq * cfg.topk * 2 * 256
+    res = {"us_per_step": round(us, 2), "steps": timed, "r": 256,
+           "step_roofline_bytes": step_bytes,
+           "step_frac_of_measured": round(step_bytes / (us * 1e-6) / 1e9 / peak, 4),
+           "shape": f"{name} with 256-bit codes: B {B}, {Hq}/{Hkv} heads, context {N}, "
+                    f"top-{cfg.topk}"}
+    del w, codes, ws, out, flush_buf
+    torch.cuda.empty_cache()
+    return res
+
+
+def seqpar_leg(dev, ranks=8, name="needle_gqa_1m"):
+    """The million-token workload as a sequence-parallel step over `ranks`
+    emulated ranks on this one GPU: every rank's two local phases are timed
+    on its own contiguous shard (flushed L2 before each), the exchanges are
+    stacks of the ranks' buffers.  Reported: each phase's slowest rank and
+    the merge -- the kernel part of one sharded step's latency; the two
+    all-gathers of a few KB per head between GPUs are not in it (one GPU
+    here).  Needle recall of the union of the shard selections."""
+    cfg = wl.CONFIGS[name]
+    B, Hq, Hkv, N, k = cfg.B, cfg.H_q, cfg.H_kv, cfg.N, cfg.topk
+    scale = 1.0 / math.sqrt(128)
+    w = wl.make_workload(cfg, wl.SEED_BASE + wl.CONFIG_ORDER.index(name), device=dev, steps=1)
+    flush_buf = torch.zeros(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+    n = N // ranks
+    shards = []
+    for r in range(ranks):
+        K = w.K[:, :, r * n:(r + 1) * n].contiguous()
+        V = w.V[:, :, r * n:(r + 1) * n].contiguous()
+        codes = torch.zeros((B, Hkv, n, 4), dtype=torch.int32, device=dev)
+        H.hata_hash_keys(K, w.W_H, codes, 0, n)
+        ws = torch.empty(H.hata_decode_workspace_size(B, Hq, Hkv, n, k), dtype=torch.uint8,
+                         device=dev)
+        sl = torch.full((B,), n, dtype=torch.int32, device=dev)
+        shards.append((K, V, codes, ws, sl))
+    hist = torch.empty((ranks, B, Hq, H.HATA_SP_HIST_WORDS), dtype=torch.int32, device=dev)
+    part = torch.empty((ranks, B, Hq, H.HATA_SP_PART_WORDS), device=dev)
+    sel = torch.empty((ranks, B, Hq, k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, 128), device=dev)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    t1, t2, tm = [], [], []
+    for it in range(8):
+        e1 = [(ev(), ev()) for _ in range(ranks)]
+        e2 = [(ev(), ev()) for _ in range(ranks)]
+        em = (ev(), ev())
+        for r, (K, V, codes, ws, sl) in enumerate(shards):
+            torch.sum(flush_buf)
+            e1[r][0].record(stream)
+            H.hata_sp_score(w.q[0], w.W_H, codes, K, V, sl, n, k, ws, hist[r])
+            e1[r][1].record(stream)
+        for r, (K, V, codes, ws, sl) in enumerate(shards):
+            torch.sum(flush_buf)
+            e2[r][0].record(stream)
+            H.hata_sp_attend(hist, r, codes, K, V, sl, n, Hq, 128, k, scale, ws, part[r],
+                             sel_idx=sel[r])
+            e2[r][1].record(stream)
+        em[0].record(stream)
+        H.hata_sp_merge(part, out)
+        em[1].record(stream)
+        torch.cuda.synchronize()
+        if it >= 3:
+            t1.append(max(a.elapsed_time(b) for a, b in e1))
+            t2.append(max(a.elapsed_time(b) for a, b in e2))
+            tm.append(em[0].elapsed_time(em[1]))
+    for _, _, _, ws, _ in shards:
+        H.hata_workspace_check(ws)
+    sel_c = sel.cpu()
+    hits = total = 0
+    for b in range(B):
+        for h in range(Hkv):
+            got = set()
+            for r in range(ranks):
+                got |= {x + r * n for x in sel_c[r, b, h * cfg.G].tolist() if x >= 0}
+            nd = set(x for x in w.planted[b, h].tolist() if x >= 0)
+            hits += len(nd & got)
+            total += len(nd)
+    res = {"ranks_emulated": ranks, "tokens_per_rank": n,
+           "score_us_slowest_rank": round(statistics.mean(t1) * 1e3, 2),
+           "attend_us_slowest_rank": round(statistics.mean(t2) * 1e3, 2),
+           "merge_us": round(statistics.mean(tm) * 1e3, 2),
+           "kernel_us_per_step": round((statistics.mean(t1) + statistics.mean(t2)
+                                        + statistics.mean(tm)) * 1e3, 2),
+           "needle_recall": round(hits / max(total, 1), 4),
+           "note": "one GPU: shards run one after another, exchanges are buffer stacks; the "
+                   "NCCL all-gathers between GPUs are not timed"}
+    del w, shards, hist, part, sel, out, flush_buf
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_hata(args, world, rank, local):
     cfg = bench_config(args)
     K_steps, W_steps = args.steps, args.warmup
@@ -706,6 +833,8 @@ def run_hata(args, world, rank, local):
         del w, codes, ws, flush_buf
         torch.cuda.empty_cache()
         line["other_workloads"] = other_workloads(args, dev)
+        line["other_workloads"]["llama31_8b_gqa_128k_r256"] = wide_code_leg(dev)
+        line["other_workloads"]["needle_gqa_1m_seqpar8"] = seqpar_leg(dev)
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -20,19 +20,16 @@ thread_local char g_err[512];
 std::atomic<int> g_mode{HATA_MODE_AUTO};
 std::atomic<uint64_t> g_wait_ns{1000000000ull};
 
-#ifndef HATA_SEL_LAG
-#define HATA_SEL_LAG 2
-#endif
-
 // Which step HATA_MODE_AUTO picks for bf16 caches (the faster one on B200).
 constexpr bool kAutoFused = false;
 
-// The fused step serves bf16 K/V caches when asked for (or chosen by AUTO);
-// fp32 caches always take the multi-kernel step.
-bool use_fused(hata_dtype_t kv_dtype)
+// The fused step serves bf16 K/V caches with codes of up to 128 bits when
+// asked for (or chosen by AUTO); fp32 caches and 256-bit codes always take
+// the multi-kernel step.
+bool use_fused(hata_dtype_t kv_dtype, int r)
 {
     const int m = g_mode.load();
-    return kv_dtype == HATA_DT_BF16 &&
+    return kv_dtype == HATA_DT_BF16 && r <= kRbit &&
            (m == HATA_MODE_FUSED || (m == HATA_MODE_AUTO && kAutoFused));
 }
 
@@ -63,8 +60,9 @@ bool valid_dtype(hata_dtype_t t) { return t == HATA_DT_BF16 || t == HATA_DT_F32;
 hata_status_t check_dims(int d, int r)
 {
     if (d != kD) return fail(HATA_ERR_UNSUPPORTED, "head_dim d=%d: only %d is supported", d, kD);
-    if (r != 32 && r != 64 && r != kRbit)
-        return fail(HATA_ERR_UNSUPPORTED, "hash bits r=%d: 32, 64 or %d are supported", r, kRbit);
+    if (r != 32 && r != 64 && r != kRbit && r != kRbitWide)
+        return fail(HATA_ERR_UNSUPPORTED, "hash bits r=%d: 32, 64, %d or %d are supported", r,
+                    kRbit, kRbitWide);
     return HATA_OK;
 }
 
@@ -119,7 +117,7 @@ cudaError_t ensure_smem_attr(const void *func, size_t bytes)
 
 extern "C" {
 
-int hata_abi_version(void) { return 2; }
+int hata_abi_version(void) { return 3; }
 
 const char *hata_status_string(int status)
 {
@@ -230,7 +228,7 @@ int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
              int(kv_dtype));
         return -1;
     }
-    if (use_fused(kv_dtype)) return 3;  // prep, score, the selection + attention kernel
+    if (use_fused(kv_dtype, kRbit)) return 3;  // prep, score, the selection + attention kernel
     int n = 0;
     if (cudaError_t e = attend_launch_count(B, H_q, topk, kv_dtype == HATA_DT_BF16, &n)) {
         cuda_fail(e, "occupancy query");
@@ -239,66 +237,85 @@ int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
     return 3 + n;
 }
 
-hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
-                               void *V, hata_dtype_t kv_dtype, int64_t n_cap,
-                               const int32_t *seq_len, int64_t max_seq_len, const void *k_new,
-                               const void *v_new, int B, int H_q, int H_kv, int d, int r,
-                               int topk, float scale, void *workspace, size_t workspace_bytes,
-                               float *out, int32_t *sel_idx, uint32_t *q_codes, uint8_t *dist,
-                               int64_t dist_row_bytes, void *const *events, void *stream)
+}  // extern "C"
+
+namespace {
+
+// The checks every step entry point shares: sizes, the caches, the
+// workspace.  Fills the workspace layout.
+hata_status_t check_step(const uint32_t *codes, const void *K, const void *V,
+                         hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                         int64_t max_seq_len, int B, int H_q, int H_kv, int d, int r, int topk,
+                         void *workspace, size_t workspace_bytes, DecodeLayout *L)
 {
     if (hata_status_t st = check_dims(d, r)) return st;
     if (hata_status_t st = check_heads(B, H_q, H_kv)) return st;
-    if (!q || !W_H || !codes || !K || !V || !seq_len || !workspace || !out)
+    if (!codes || !K || !V || !seq_len || !workspace)
         return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
     if (!valid_dtype(kv_dtype)) return fail(HATA_ERR_INVALID_ARG, "bad kv_dtype %d", int(kv_dtype));
-    if (v_new && !k_new) return fail(HATA_ERR_INVALID_ARG, "v_new given without k_new");
     if (topk <= 0) return fail(HATA_ERR_INVALID_ARG, "topk=%d must be >= 1", topk);
     if (n_cap <= 0 || n_cap >= (int64_t(1) << 31))
         return fail(HATA_ERR_INVALID_ARG, "n_cap=%lld out of range", (long long)n_cap);
     if (max_seq_len <= 0 || max_seq_len > n_cap)
         return fail(HATA_ERR_INVALID_ARG, "max_seq_len=%lld must be in [1, n_cap=%lld]",
                     (long long)max_seq_len, (long long)n_cap);
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(codes, 16) || !aligned(seq_len, 4))
+        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer (K, V, codes: 16 B)");
+    if (!aligned(workspace, 256)) return fail(HATA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (!decode_layout(B, H_q, H_kv, max_seq_len, topk, L))
+        return fail(HATA_ERR_INVALID_ARG, "sizes out of range");
+    if (workspace_bytes < L->total)
+        return fail(HATA_ERR_INVALID_ARG, "workspace of %zu bytes < required %zu", workspace_bytes,
+                    L->total);
+    return HATA_OK;
+}
+
+hata_status_t check_scale(float scale)
+{
     if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
         return fail(HATA_ERR_INVALID_ARG, "scale must be finite");
-    if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(codes, 16) ||
-        !aligned(out, 16) || !aligned(W_H, 16) || !aligned(seq_len, 4) ||
-        (k_new && !aligned(k_new, 16)) || (v_new && !aligned(v_new, 16)) ||
-        (sel_idx && !aligned(sel_idx, 4)) || (q_codes && !aligned(q_codes, 16)))
-        return fail(HATA_ERR_INVALID_ARG,
-                    "misaligned pointer (q, W_H, K, V, codes, out, k_new, v_new, q_codes: 16 B)");
-    if (!aligned(workspace, 256)) return fail(HATA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    DecodeLayout L;
-    if (!decode_layout(B, H_q, H_kv, max_seq_len, topk, &L))
-        return fail(HATA_ERR_INVALID_ARG, "sizes out of range");
-    if (workspace_bytes < L.total)
-        return fail(HATA_ERR_INVALID_ARG, "workspace of %zu bytes < required %zu", workspace_bytes,
-                    L.total);
-    if (dist) {
-        if (!aligned(dist, 16) || dist_row_bytes % 16 || dist_row_bytes < L.dist_row)
-            return fail(HATA_ERR_INVALID_ARG,
-                        "dist must be 16-byte aligned with dist_row_bytes >= %lld, multiple of 16",
-                        (long long)L.dist_row);
-    }
+    return HATA_OK;
+}
 
-    char *ws = static_cast<char *>(workspace);
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+// Where a step's intermediate results live.
+struct StepBufs {
+    uint32_t *qc;      // query codes [B][H_q][r/32]
+    uint8_t *dist;     // distance rows
+    int64_t drow;      // their stride
+    int32_t *idx;      // index lists [B][H_q][topk]
+    uint32_t *flags, *hist;
+    float *q_dev;      // device copy of q
+};
+
+StepBufs step_bufs(char *ws, const DecodeLayout &L, uint32_t *q_codes, uint8_t *dist,
+                   int64_t dist_row_bytes, int32_t *sel_idx)
+{
+    StepBufs sb;
+    sb.qc = q_codes ? q_codes : reinterpret_cast<uint32_t *>(ws + L.off_qcodes);
+    sb.dist = dist ? dist : reinterpret_cast<uint8_t *>(ws + L.off_dist);
+    sb.drow = dist ? dist_row_bytes : L.dist_row;
+    sb.idx = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(ws + L.off_idx);
+    sb.flags = reinterpret_cast<uint32_t *>(ws + L.off_flags);
+    sb.hist = reinterpret_cast<uint32_t *>(ws + L.off_hist);
+    sb.q_dev = reinterpret_cast<float *>(ws + L.off_q);
+    return sb;
+}
+
+// The front of a step: prep (hash q, append, clear the histograms, flags),
+// then the scoring kernel.  Events 0..2 around them.
+hata_status_t enqueue_front(const float *q, const float *W_H, uint32_t *codes, void *K, void *V,
+                            hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                            int64_t max_seq_len, const void *k_new, const void *v_new, int B,
+                            int H_q, int H_kv, int r, const DecodeLayout &L, const StepBufs &sb,
+                            char *ws, uint32_t *sync, const Events &ev)
+{
+    const cudaStream_t s = ev.s;
     const int G = H_q / H_kv;
-    uint32_t *qc = q_codes ? q_codes : reinterpret_cast<uint32_t *>(ws + L.off_qcodes);
-    uint8_t *dst = dist ? dist : reinterpret_cast<uint8_t *>(ws + L.off_dist);
-    const int64_t drow = dist ? dist_row_bytes : L.dist_row;
-    int32_t *idx = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(ws + L.off_idx);
-    uint32_t *flags = reinterpret_cast<uint32_t *>(ws + L.off_flags);
-    uint32_t *hist = reinterpret_cast<uint32_t *>(ws + L.off_hist);
-    const Events ev{events, s};
     cudaError_t e;
-
     if ((e = ev.record(0)) != cudaSuccess) return cuda_fail(e, "event record");
-
-    float *q_dev = reinterpret_cast<float *>(ws + L.off_q);
     PrepArgs p{};
     p.q = q;
-    p.q_copy = q_dev;
+    p.q_copy = sb.q_dev;
     p.k_new = k_new;
     p.v_new = v_new;
     p.W = W_H;
@@ -306,13 +323,11 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     p.K = K;
     p.V = V;
     p.seq_len = seq_len;
-    p.q_out = qc;
-    p.flags = flags;
-    p.hist = hist;
-    p.hist_row_words = L.n_tiles * kHistStride;
-    const bool fused = use_fused(kv_dtype);
-    uint32_t *sync = reinterpret_cast<uint32_t *>(ws + L.off_sync);
-    p.sync = fused ? sync : nullptr;
+    p.q_out = sb.qc;
+    p.flags = sb.flags;
+    p.hist = sb.hist;
+    p.hist_row_words = L.n_tiles * hist_stride(r / 32);
+    p.sync = sync;
     p.ws_header = reinterpret_cast<uint32_t *>(ws);
     p.n_cap = n_cap;
     p.max_seq_len = max_seq_len;
@@ -327,12 +342,12 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     if ((e = ev.record(1)) != cudaSuccess) return cuda_fail(e, "event record");
 
     ScoreArgs sa{};
-    sa.qcodes = qc;
+    sa.qcodes = sb.qc;
     sa.codes = codes;
     sa.seq_len = seq_len;
-    sa.dist = dst;
-    sa.dist_row = drow;
-    sa.hist = hist;
+    sa.dist = sb.dist;
+    sa.dist_row = sb.drow;
+    sa.hist = sb.hist;
     sa.n_cap = n_cap;
     sa.max_seq_len = max_seq_len;
     sa.n_tiles = L.n_tiles;
@@ -344,23 +359,117 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     sa.words = r / 32;
     if ((e = launch_score(sa, s)) != cudaSuccess) return cuda_fail(e, "score launch");
     if ((e = ev.record(2)) != cudaSuccess) return cuda_fail(e, "event record");
+    return HATA_OK;
+}
+
+SelectArgs select_args(const StepBufs &sb, const uint32_t *codes, const int32_t *seq_len,
+                       int64_t n_cap, int64_t max_seq_len, const DecodeLayout &L, int B, int H_q,
+                       int H_kv, int r, int topk)
+{
+    SelectArgs se{};
+    se.seq_len = seq_len;
+    se.dist = sb.dist;
+    se.dist_row = sb.drow;
+    se.hist = sb.hist;
+    se.idx = sb.idx;
+    se.qcodes = sb.qc;
+    se.codes = codes;
+    se.n_cap = n_cap;
+    se.max_seq_len = max_seq_len;
+    se.n_tiles = L.n_tiles;
+    se.B = B;
+    se.H_q = H_q;
+    se.H_kv = H_kv;
+    se.G = H_q / H_kv;
+    se.topk = topk;
+    se.words = r / 32;
+    return se;
+}
+
+AttendArgs attend_args(const StepBufs &sb, const void *K, const void *V, const int32_t *seq_len,
+                       int64_t n_cap, int64_t max_seq_len, char *ws, const DecodeLayout &L, int B,
+                       int H_q, int H_kv, int topk, float scale, float *out)
+{
+    AttendArgs aa{};
+    aa.q = sb.q_dev;
+    aa.K = K;
+    aa.V = V;
+    aa.seq_len = seq_len;
+    aa.idx = sb.idx;
+    aa.part = reinterpret_cast<float *>(ws + L.off_part);
+    aa.flags = sb.flags;
+    aa.out = out;
+    aa.n_cap = n_cap;
+    aa.max_seq_len = max_seq_len;
+    aa.B = B;
+    aa.H_q = H_q;
+    aa.H_kv = H_kv;
+    aa.G = H_q / H_kv;
+    aa.topk = topk;
+    aa.n_split = L.n_split;
+    aa.scale_log2 = scale * 1.4426950408889634f;
+    return aa;
+}
+
+}  // namespace
+
+extern "C" {
+
+hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
+                               void *V, hata_dtype_t kv_dtype, int64_t n_cap,
+                               const int32_t *seq_len, int64_t max_seq_len, const void *k_new,
+                               const void *v_new, int B, int H_q, int H_kv, int d, int r,
+                               int topk, float scale, void *workspace, size_t workspace_bytes,
+                               float *out, int32_t *sel_idx, uint32_t *q_codes, uint8_t *dist,
+                               int64_t dist_row_bytes, void *const *events, void *stream)
+{
+    DecodeLayout L;
+    if (hata_status_t st = check_step(codes, K, V, kv_dtype, n_cap, seq_len, max_seq_len, B, H_q,
+                                      H_kv, d, r, topk, workspace, workspace_bytes, &L))
+        return st;
+    if (!q || !W_H || !out) return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (v_new && !k_new) return fail(HATA_ERR_INVALID_ARG, "v_new given without k_new");
+    if (hata_status_t st = check_scale(scale)) return st;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(W_H, 16) ||
+        (k_new && !aligned(k_new, 16)) || (v_new && !aligned(v_new, 16)) ||
+        (sel_idx && !aligned(sel_idx, 4)) || (q_codes && !aligned(q_codes, 16)))
+        return fail(HATA_ERR_INVALID_ARG,
+                    "misaligned pointer (q, W_H, K, V, codes, out, k_new, v_new, q_codes: 16 B)");
+    if (dist) {
+        if (!aligned(dist, 16) || dist_row_bytes % 16 || dist_row_bytes < L.dist_row)
+            return fail(HATA_ERR_INVALID_ARG,
+                        "dist must be 16-byte aligned with dist_row_bytes >= %lld, multiple of 16",
+                        (long long)L.dist_row);
+    }
+
+    char *ws = static_cast<char *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const StepBufs sb = step_bufs(ws, L, q_codes, dist, dist_row_bytes, sel_idx);
+    const Events ev{events, s};
+    const bool fused = use_fused(kv_dtype, r);
+    uint32_t *sync = reinterpret_cast<uint32_t *>(ws + L.off_sync);
+    if (hata_status_t st = enqueue_front(q, W_H, codes, K, V, kv_dtype, n_cap, seq_len,
+                                         max_seq_len, k_new, v_new, B, H_q, H_kv, r, L, sb, ws,
+                                         fused ? sync : nullptr, ev))
+        return st;
+    cudaError_t e;
 
     if (fused) {
         FusedArgs fa{};
         fa.seq_len = seq_len;
-        fa.q = q_dev;
+        fa.q = sb.q_dev;
         fa.K = K;
         fa.V = V;
-        fa.dist = dst;
-        fa.hist = hist;
-        fa.idx = idx;
+        fa.dist = sb.dist;
+        fa.hist = sb.hist;
+        fa.idx = sb.idx;
         fa.part = reinterpret_cast<float *>(ws + L.off_part);
         fa.out = out;
         fa.sel_done = sync;
         fa.head_cnt = sync + int64_t(B) * H_q;
-        fa.flags = flags;
+        fa.flags = sb.flags;
         fa.abort_word = sync + 2 * int64_t(B) * H_q;
-        fa.dist_row = drow;
+        fa.dist_row = sb.drow;
         fa.dist_len = L.dist_row;
         fa.n_cap = n_cap;
         fa.max_seq_len = max_seq_len;
@@ -368,7 +477,7 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
         fa.B = B;
         fa.H_q = H_q;
         fa.H_kv = H_kv;
-        fa.G = G;
+        fa.G = H_q / H_kv;
         fa.topk = topk;
         fa.n_seg = L.n_seg;
         fa.scale_log2 = scale * 1.4426950408889634f;
@@ -381,45 +490,99 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
         return ok();
     }
 
-    SelectArgs se{};
-    se.seq_len = seq_len;
-    se.dist = dst;
-    se.dist_row = drow;
-    se.hist = hist;
-    se.idx = idx;
-    se.n_cap = n_cap;
-    se.max_seq_len = max_seq_len;
-    se.n_tiles = L.n_tiles;
-    se.B = B;
-    se.H_q = H_q;
-    se.topk = topk;
+    const SelectArgs se =
+        select_args(sb, codes, seq_len, n_cap, max_seq_len, L, B, H_q, H_kv, r, topk);
     if ((e = launch_select(se, s)) != cudaSuccess) return cuda_fail(e, "select launch");
     if ((e = ev.record(3)) != cudaSuccess) return cuda_fail(e, "event record");
 
-    AttendArgs aa{};
-    aa.q = q_dev;
-    aa.K = K;
-    aa.V = V;
-    aa.seq_len = seq_len;
-    aa.idx = idx;
-    aa.part = reinterpret_cast<float *>(ws + L.off_part);
-    aa.flags = flags;
-    aa.out = out;
-    aa.n_cap = n_cap;
-    aa.max_seq_len = max_seq_len;
-    aa.B = B;
-    aa.H_q = H_q;
-    aa.H_kv = H_kv;
-    aa.G = G;
-    aa.topk = topk;
-    aa.n_split = L.n_split;
-    aa.scale_log2 = scale * 1.4426950408889634f;
+    AttendArgs aa = attend_args(sb, K, V, seq_len, n_cap, max_seq_len, ws, L, B, H_q, H_kv, topk,
+                                scale, out);
     if ((e = launch_attend(aa, kv_dtype == HATA_DT_BF16, s)) != cudaSuccess)
         return cuda_fail(e, "attend launch");
     if ((e = ev.record(4)) != cudaSuccess) return cuda_fail(e, "event record");
     if ((e = launch_combine(aa, s)) != cudaSuccess) return cuda_fail(e, "combine launch");
     if ((e = ev.record(5)) != cudaSuccess) return cuda_fail(e, "event record");
     return ok();
+}
+
+hata_status_t hata_sp_score(const float *q, const float *W_H, uint32_t *codes, void *K, void *V,
+                            hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                            int64_t max_seq_len, const void *k_new, const void *v_new, int B,
+                            int H_q, int H_kv, int d, int r, int topk, void *workspace,
+                            size_t workspace_bytes, uint32_t *hist_out, void *stream)
+{
+    DecodeLayout L;
+    if (hata_status_t st = check_step(codes, K, V, kv_dtype, n_cap, seq_len, max_seq_len, B, H_q,
+                                      H_kv, d, r, topk, workspace, workspace_bytes, &L))
+        return st;
+    if (!q || !W_H || !hist_out) return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (v_new && !k_new) return fail(HATA_ERR_INVALID_ARG, "v_new given without k_new");
+    if (!aligned(q, 16) || !aligned(W_H, 16) || !aligned(hist_out, 4) ||
+        (k_new && !aligned(k_new, 16)) || (v_new && !aligned(v_new, 16)))
+        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer (q, W_H, k_new, v_new: 16 B)");
+    char *ws = static_cast<char *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const StepBufs sb = step_bufs(ws, L, nullptr, nullptr, 0, nullptr);
+    const Events ev{nullptr, s};
+    if (hata_status_t st = enqueue_front(q, W_H, codes, K, V, kv_dtype, n_cap, seq_len,
+                                         max_seq_len, k_new, v_new, B, H_q, H_kv, r, L, sb, ws,
+                                         nullptr, ev))
+        return st;
+    const cudaError_t e = launch_sp_hist(sb.hist, L.n_tiles, hist_stride(r / 32),
+                                         int64_t(B) * H_q, hist_out, s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "histogram launch");
+}
+
+hata_status_t hata_sp_attend(const uint32_t *hist_all, int world, int rank,
+                             const uint32_t *codes, const void *K, const void *V,
+                             hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                             int64_t max_seq_len, int B, int H_q, int H_kv, int d, int r,
+                             int topk, float scale, void *workspace, size_t workspace_bytes,
+                             float *part_out, int32_t *sel_idx, void *stream)
+{
+    DecodeLayout L;
+    if (hata_status_t st = check_step(codes, K, V, kv_dtype, n_cap, seq_len, max_seq_len, B, H_q,
+                                      H_kv, d, r, topk, workspace, workspace_bytes, &L))
+        return st;
+    if (!hist_all || !part_out) return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (world < 1 || rank < 0 || rank >= world)
+        return fail(HATA_ERR_INVALID_ARG, "rank %d of world %d", rank, world);
+    if (hata_status_t st = check_scale(scale)) return st;
+    if (!aligned(hist_all, 4) || !aligned(part_out, 16) || (sel_idx && !aligned(sel_idx, 4)))
+        return fail(HATA_ERR_INVALID_ARG, "misaligned pointer (part_out: 16 B)");
+    char *ws = static_cast<char *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const StepBufs sb = step_bufs(ws, L, nullptr, nullptr, 0, sel_idx);
+    int32_t *k_head = reinterpret_cast<int32_t *>(ws + L.off_khead);
+    const int64_t BH = int64_t(B) * H_q;
+    cudaError_t e = launch_sp_quota(hist_all, world, rank, BH, topk, r + 1, k_head, s);
+    if (e != cudaSuccess) return cuda_fail(e, "quota launch");
+    SelectArgs se =
+        select_args(sb, codes, seq_len, n_cap, max_seq_len, L, B, H_q, H_kv, r, topk);
+    se.k_head = k_head;
+    if ((e = launch_select(se, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+    AttendArgs aa = attend_args(sb, K, V, seq_len, n_cap, max_seq_len, ws, L, B, H_q, H_kv, topk,
+                                scale, nullptr);
+    aa.k_head = k_head;
+    aa.part_out = part_out;
+    aa.n_split = L.n_split > L.n_seg ? L.n_split : L.n_seg;  // partial slots per head
+    e = kv_dtype == HATA_DT_BF16 ? launch_attend_split(aa, s) : launch_attend(aa, false, s);
+    if (e != cudaSuccess) return cuda_fail(e, "attend launch");
+    if ((e = launch_combine(aa, s)) != cudaSuccess) return cuda_fail(e, "combine launch");
+    return ok();
+}
+
+hata_status_t hata_sp_merge(const float *part_all, int world, int B, int H_q, float *out,
+                            void *stream)
+{
+    if (!part_all || !out) return fail(HATA_ERR_INVALID_ARG, "null pointer argument");
+    if (world < 1 || B <= 0 || H_q <= 0 || int64_t(B) * H_q > 65535)
+        return fail(HATA_ERR_INVALID_ARG, "world=%d B=%d H_q=%d", world, B, H_q);
+    if (!aligned(part_all, 16) || !aligned(out, 16))
+        return fail(HATA_ERR_INVALID_ARG, "part_all and out must be 16-byte aligned");
+    const cudaError_t e =
+        launch_sp_merge(part_all, world, int64_t(B) * H_q, out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "merge launch");
 }
 
 hata_status_t hata_workspace_check(void *workspace, size_t workspace_bytes, uint32_t *flags,

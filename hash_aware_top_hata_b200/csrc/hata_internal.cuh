@@ -12,19 +12,24 @@
 namespace hata {
 
 constexpr int kD = 128;         // head_dim (the page's models all use 128)
-constexpr int kRbit = 128;      // widest hash (rbit = 128 on the HATA page; 32 and 64 too)
-constexpr int kWords = kRbit / 32;
+constexpr int kRbit = 128;      // the page's hash width (rbit = 128)
+constexpr int kRbitWide = 256;  // widest hash of its ablation (32, 64 and 256 too)
 constexpr int kBins = kRbit + 1;        // Hamming distances 0..128 (fewer bins used below)
+constexpr int kBinsWide = kRbitWide + 1;  // distances 0..256 of the 256-bit codes
 constexpr int kChunk = 4096;            // tokens per scoring / selection chunk
 constexpr int kScoreThreads = 1024;
 constexpr int kScoreHeads = 8;          // query heads scored per code load (one CTA)
 constexpr int kAttnThreads = 128;
 constexpr int kHistStride = 132;        // u32 per (head, tile) histogram row (129 bins)
+constexpr int kHistStrideWide = 260;    // the same at r = 256 (257 bins); the workspace
+                                        // reserves rows of this size for every width
 constexpr int kTile = 36864;            // tokens per histogram tile / selection tile (9 x 4096)
 constexpr int kPartStride = 132;        // f32 per (head, chunk) partial: m, l, -, -, acc[128]
 constexpr int kFSeg = 96;               // selected rows per attention item, fused step
                                         // (16 per attention warp)
-constexpr uint8_t kDistPad = 255;       // distance stored past seq_len
+constexpr uint8_t kDistPad = 255;       // distance stored past seq_len; at r = 256 the
+                                        // stored distance saturates at 255 too
+constexpr int kSpHistWords = 260;       // sequence-parallel histogram row (HATA_SP_HIST_WORDS)
 constexpr uint32_t kWsMagic = 0x48415441u;  // "HATA"
 
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -61,8 +66,11 @@ struct DecodeLayout {
     int n_split = 0;        // attention partial slots per head (multi-kernel step)
     int n_seg = 0;          // attention items per head (fused step)
     size_t off_flags = 0, off_qcodes = 0, off_q = 0, off_dist = 0, off_hist = 0, off_idx = 0,
-           off_part = 0, off_sync = 0, total = 0;
+           off_part = 0, off_sync = 0, off_khead = 0, total = 0;
 };
+
+// Words per (head, tile) histogram row for r/32 = words code words.
+inline int hist_stride(int words) { return words == 8 ? kHistStrideWide : kHistStride; }
 
 inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
                           DecodeLayout *L)
@@ -87,15 +95,17 @@ inline bool decode_layout(int B, int H_q, int H_kv, int64_t max_seq_len, int top
     const int64_t parts = L->n_split > L->n_seg ? L->n_split : L->n_seg;
     size_t o = 256;
     L->off_flags = o;      o = align_up(o + 4 * size_t(B), 256);
-    L->off_qcodes = o;     o = align_up(o + 16 * size_t(BH), 256);
+    L->off_qcodes = o;     o = align_up(o + 32 * size_t(BH), 256);  // up to 8 words a head
     L->off_q = o;          o = align_up(o + 4 * kD * size_t(BH), 256);  // q, read once per step
     L->off_dist = o;       o = align_up(o + size_t(BH) * L->dist_row, 256);
-    L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * L->n_tiles * kHistStride, 256);
+    L->off_hist = o;       o = align_up(o + 4 * size_t(BH) * L->n_tiles * kHistStrideWide, 256);
     L->off_idx = o;        o = align_up(o + 4 * size_t(BH) * topk, 256);
     L->off_part = o;       o = align_up(o + 4 * size_t(BH) * parts * kPartStride, 256);
     // fused-step counters: selection tiles done and attention items published
     // per head, then the step's abort word (all zeroed by prep every step)
     L->off_sync = o;       o = align_up(o + 4 * size_t(2 * BH + 1), 256);
+    // sequence-parallel step: the keys each head selects from this shard
+    L->off_khead = o;      o = align_up(o + 4 * size_t(BH), 256);
     L->total = o;
     return true;
 }
@@ -115,7 +125,7 @@ struct PrepArgs {
     uint32_t *flags;         // per-b flag words (decode) or null
     uint32_t *err_word;      // single OR-ed word (append API) or null
     uint32_t *hist;          // [B][H_q][hist_row_words] zeroed (decode) or null
-    int64_t hist_row_words;  // n_tiles * kHistStride
+    int64_t hist_row_words;  // n_tiles * hist_stride(words)
     uint32_t *sync;          // fused-step counters zeroed (decode, fused step) or null:
                              // [B][H_q] twice, then one abort word
     uint32_t *ws_header;     // {magic, B} written (decode) or null
@@ -131,20 +141,25 @@ struct ScoreArgs {
     const int32_t *seq_len;
     uint8_t *dist;           // [B][H_q][dist_row]
     int64_t dist_row;
-    uint32_t *hist;          // [B][H_q][n_tiles][kHistStride], zeroed by prep
+    uint32_t *hist;          // [B][H_q][n_tiles][hist_stride(words)], zeroed by prep
     int64_t n_cap, max_seq_len, n_tiles;
     int B, H_q, H_kv, G, zgroups;
-    int words;               // r / 32 (1, 2 or 4)
+    int words;               // r / 32 (1, 2, 4 or 8)
 };
 
 struct SelectArgs {
     const int32_t *seq_len;
     const uint8_t *dist;
     int64_t dist_row;
-    const uint32_t *hist;    // [B][H_q][n_tiles][kHistStride]
+    const uint32_t *hist;    // [B][H_q][n_tiles][hist_stride(words)]
     int32_t *idx;            // [B][H_q][topk] ascending, -1 padded
+    const int32_t *k_head;   // [B][H_q] keys to select per head (sequence-parallel step;
+                             // written by the kernel before) or null: min(topk, len)
+    const uint32_t *qcodes;  // r = 256 only: [B][H_q][8] query codes and the key codes
+    const uint32_t *codes;   //   [B][H_kv][n_cap][8], for exact distances at 255 / 256
     int64_t n_cap, max_seq_len, n_tiles;
-    int B, H_q, topk;
+    int B, H_q, H_kv, G, topk;
+    int words;
 };
 
 struct AttendArgs {
@@ -160,6 +175,11 @@ struct AttendArgs {
     int64_t n_workers;       // stream-K workers (set by the launcher)
     int head_per_cta;        // 1: a CTA's warps cover one whole head and merge it in shared
                              // memory (no combine launch); set by the launcher
+    int head_split;          // > 0: head_split CTAs per head (the sequence-parallel step);
+                             // set by the launcher
+    const int32_t *k_head;   // [B][H_q] selected keys per head, or null: min(topk, len)
+    float *part_out;         // [B][H_q][kPartStride]: unnormalised (m, l, acc) per head
+                             // instead of out (the sequence-parallel step), or null
     float scale_log2;        // scale * log2(e)
 };
 
@@ -277,5 +297,19 @@ cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s);
 cudaError_t attend_launch_count(int B, int H_q, int topk, bool bf16, int *n);
 cudaError_t launch_dense(const DenseArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_fused(const FusedArgs &a, cudaStream_t s);
+// Sequence-parallel step: the attention of one shard's selected keys split
+// over several CTAs per head (bf16; fp32 caches take launch_attend with
+// a.k_head), partials merged by launch_combine into a.part_out.
+cudaError_t launch_attend_split(AttendArgs &a, cudaStream_t s);  // sets a.head_split
+// The per-head sum of the tile histograms: out[bh][0 .. kSpHistWords).
+cudaError_t launch_sp_hist(const uint32_t *hist, int64_t n_tiles, int stride, int64_t BH,
+                           uint32_t *out, cudaStream_t s);
+// Keys each head selects from shard `rank` of `world`, from every shard's
+// histogram (hist_all: [world][BH][kSpHistWords], `bins` = r + 1 used).
+cudaError_t launch_sp_quota(const uint32_t *hist_all, int world, int rank, int64_t BH, int topk,
+                            int bins, int32_t *k_head, cudaStream_t s);
+// out[bh] = merge of the world partials part_all[w][bh][kPartStride].
+cudaError_t launch_sp_merge(const float *part_all, int world, int64_t BH, float *out,
+                            cudaStream_t s);
 
 }  // namespace hata

@@ -24,6 +24,8 @@
 // half of that), which bounds all three.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "hata_internal.cuh"
 #include "async_copy.cuh"
 #include "attend_common.cuh"
@@ -455,6 +457,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_tc_kernel(AttendArgs a
 // of the list (plain index arithmetic, no walker), the gather addresses are
 // one multiply-add from the slab's base, and the warps' partials are merged
 // in shared memory, so no combine launch follows.  Needs topk <= kIdxCap.
+//
+// The sequence-parallel step runs the same kernel with head_split CTAs per
+// head (CTA c takes the c-th of head_split equal parts of the head's list,
+// whose length k_head the kernel before wrote) and unnormalised partials
+// out: into part_out directly (head_split = 1), or one per CTA into the
+// head's partial slots for combine_kernel.
 __global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs a)
 {
     using namespace tc;
@@ -463,15 +471,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs
     pdl_trigger();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, b = bh / a.H_q, h = (bh - b * a.H_q) / a.G;
+    const int split = a.head_split > 0 ? a.head_split : 1;
+    const int bh = int(blockIdx.x) / split, cs = int(blockIdx.x) - bh * split;
+    const int b = bh / a.H_q, h = (bh - b * a.H_q) / a.G;
     // seq_len is a step input: everything up to the wait overlaps the selection
     const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);
-    const int keff = int(int64_t(a.topk) < len ? int64_t(a.topk) : len);
-    const int r0 = int(int64_t(warp) * a.topk / kTcWarps);
-    int r1 = int(int64_t(warp + 1) * a.topk / kTcWarps);
-    r1 = r1 < keff ? r1 : keff;
-    const int n_rows = r1 > r0 ? r1 - r0 : 0;
-    const int n_st = (n_rows + kSub - 1) / kSub;
+    int keff = int(int64_t(a.topk) < len ? int64_t(a.topk) : len);
 
     const int p = lane & 15, rh = lane >> 4;  // 16-byte piece p of rows 8 rh .. 8 rh + 7
     const int64_t slab = (int64_t(b) * a.H_kv + h) * a.n_cap;
@@ -485,26 +490,35 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs
     // a warp with no row of the head leaves an empty partial
     for (int i = lane; i < kPartStride; i += 32) part_s[warp][i] = i == 0 ? -INFINITY : 0.0f;
     __syncwarp();
-    pdl_wait();  // the selected index lists
+    pdl_wait();  // the selected index lists (and k_head)
+    if (a.k_head) {
+        const int kh = __ldg(a.k_head + bh);
+        keff = kh < keff ? (kh > 0 ? kh : 0) : keff;
+    }
+    // this CTA's entries [c0, c1) of the head's list; warp w its w-th eighth
+    const int c0 = int(int64_t(cs) * keff / split), c1 = int(int64_t(cs + 1) * keff / split);
+    const int r0 = c0 + int(int64_t(warp) * (c1 - c0) / kTcWarps);
+    const int r1 = c0 + int(int64_t(warp + 1) * (c1 - c0) / kTcWarps);
+    const int n_st = (r1 - r0 + kSub - 1) / kSub;
 
-    {  // the head's list (its first keff entries): all loads first, then the stores
-        const int32_t *src = a.idx + int64_t(bh) * a.topk;
+    {  // the CTA's part of the list: all loads first, then the stores
+        const int32_t *src = a.idx + int64_t(bh) * a.topk + c0;
         constexpr int kPer = kIdxCap / kThreads;
         int32_t v[kPer];
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
             const int i = tid + u * kThreads;
-            v[u] = i < keff ? __ldg(src + i) : -1;
+            v[u] = i < c1 - c0 ? __ldg(src + i) : -1;
         }
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
             const int i = tid + u * kThreads;
-            if (i < keff) idx_s[i] = v[u];
+            if (i < c1 - c0) idx_s[i] = v[u];
         }
     }
     __syncthreads();
 
-    // stage s of this warp (rows r0 + 16 s ...) into ring slot s % kRingW;
+    // stage s of this warp (entries r0 + 16 s ...) into ring slot s % kRingW;
     // always commits one group
     auto issue = [&](int s) {
         if (s < n_st) {
@@ -513,7 +527,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs
             const int x0 = r0 + s * kSub + 8 * rh;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int32_t row = x0 + u < r1 ? idx_s[x0 + u] : -1;
+                const int32_t row = x0 + u < r1 ? idx_s[x0 + u - c0] : -1;
                 // the selection never yields an index outside [0, len); the
                 // check keeps a corrupted list from steering a copy outside
                 // the cache.  Rows without a key are zero-filled.
@@ -540,7 +554,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs
         __syncwarp();
         issue(s + kRingW - 1);
         const int x = r0 + s * kSub + lane;
-        const int32_t row = lane < kSub && x < r1 ? idx_s[x] : -1;
+        const int32_t row = lane < kSub && x < r1 ? idx_s[x - c0] : -1;
         const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0 && row < len);
         attend_stage(vmask, wring + uint32_t((s % kRingW) * kStageBytes), qb, lo, O, m_ref,
                      l_part, lane);
@@ -563,7 +577,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs
                 A = fmaf(part_s[w][4 + tid], wt, A);
             }
         }
-        a.out[int64_t(bh) * kD + tid] = L > 0.0f ? A / L : 0.0f;
+        if (a.part_out || split > 1) {  // an unnormalised partial (m, l, acc)
+            float *pp = split > 1 ? a.part + (int64_t(bh) * a.n_split + cs) * kPartStride
+                                  : a.part_out + int64_t(bh) * kPartStride;
+            if (tid == 0) {
+                pp[0] = M;
+                pp[1] = L;
+            }
+            pp[4 + tid] = A;
+        } else {
+            a.out[int64_t(bh) * kD + tid] = L > 0.0f ? A / L : 0.0f;
+        }
     }
 }
 
@@ -587,7 +611,9 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(AttendArgs 
     const int64_t bh = int64_t(blockIdx.x) * kCombineWarps + (threadIdx.x >> 5);
     const bool live = bh < int64_t(a.B) * a.H_q;
     int n_contrib = 0;
-    if (live) {
+    if (live && a.head_split > 0) {
+        n_contrib = a.head_split;  // one partial per CTA of the head
+    } else if (live) {
         const int64_t T = int64_t(a.B) * a.H_q * a.topk, NW = a.n_workers;
         const int b = int(bh / a.H_q);
         const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);
@@ -634,6 +660,16 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(AttendArgs 
 #pragma unroll
             for (int i = 0; i < 4; ++i) A[i] = fmaf(acc[j][i], w, A[i]);
         }
+    }
+    if (a.part_out) {  // the sequence-parallel step: this shard's unnormalised partial
+        float *pp = a.part_out + bh * kPartStride;
+        if (lane == 0) {
+            pp[0] = M;
+            pp[1] = L;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pp[4 + lane + 32 * i] = A[i];
+        return;
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) a.out[bh * kD + lane + 32 * i] = L > 0.0f ? A[i] / L : 0.0f;
@@ -683,6 +719,7 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
         if (NW > kAttnMaxWorkers) NW = kAttnMaxWorkers;
         if (NW > T) NW = T;
         a.head_per_cta = head_per_cta(a.B, a.H_q, a.topk, P);
+        a.head_split = 0;
         if (a.head_per_cta) {
             a.n_workers = 0;
             if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(attend_head_kernel),
@@ -702,8 +739,28 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
     if (P > T) P = T;
     a.n_workers = P;
     a.head_per_cta = 0;
+    a.head_split = 0;
     return launch_pdl(attend_simt_kernel<false>, dim3(unsigned(P)), dim3(kAttnThreads), kSmemF32,
                       s, a);
+}
+
+// The sequence-parallel step's attention (bf16): head_split CTAs per head,
+// enough to fill one wave of CTAs and to keep each CTA's part of a list
+// within kIdxCap; a.n_split (partial slots per head) bounds head_split.
+cudaError_t launch_attend_split(AttendArgs &a, cudaStream_t s)
+{
+    int64_t P = 0;
+    if (cudaError_t e = occupancy_grid(attend_head_kernel, tc::kThreads, tc::kSmem, &P)) return e;
+    const int64_t heads = int64_t(a.B) * a.H_q;
+    int64_t split = std::max(ceil_div(a.topk, tc::kIdxCap), ceil_div(P, heads));
+    if (split > a.n_split) split = a.n_split;
+    if (split * heads >= (int64_t(1) << 31) || ceil_div(a.topk, split) > tc::kIdxCap)
+        return cudaErrorInvalidValue;
+    a.head_split = int(split);
+    a.head_per_cta = split == 1;  // merged inside the CTA: no combine launch
+    a.n_workers = 0;
+    return launch_pdl(attend_head_kernel, dim3(unsigned(split * heads)), dim3(tc::kThreads),
+                      tc::kSmem, s, a);
 }
 
 // The merge of the split heads: launched right behind launch_attend (whose

@@ -9,8 +9,8 @@
 // Every code bit j is the fp32 chain acc = fmaf(x_i, W[i][j], acc), i = 0..127
 // ascending, then acc > 0.  The chain order is fixed, so codes are
 // reproducible bit for bit by any implementation that follows the same
-// order (the CPU oracle does).  r = 128 bits (the page's width), or 32 / 64
-// (the narrower widths of its ablation): r/32 code words per token.
+// order (the CPU oracle does).  r = 128 bits (the page's width), or 32 / 64 /
+// 256 (the other widths of its ablation): r/32 code words per token.
 //
 // Two kernels: the prefill hash (register-blocked over 8 rows per warp, the
 // head's W_H in shared memory) for hata_hash_keys, and the decode prep
@@ -122,9 +122,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) hash_prefill_kernel(const void 
         const ulonglong2 *xrow = reinterpret_cast<const ulonglong2 *>(&S.x[warp][0][0]);
 #pragma unroll 4
         for (int i = 0; i < kD; ++i) {
-            // this lane's kBL values of W's row i (one 4-, 8- or 16-byte load)
+            // this lane's kBL values of W's row i (4- to 32-byte loads)
             float wv[kBL];
-            if constexpr (kBL == 4) {
+            if constexpr (kBL == 8) {
+                const float4 w0 = *reinterpret_cast<const float4 *>(wrow + i * R);
+                const float4 w1 = *reinterpret_cast<const float4 *>(wrow + i * R + 4);
+                wv[0] = w0.x, wv[1] = w0.y, wv[2] = w0.z, wv[3] = w0.w;
+                wv[4] = w1.x, wv[5] = w1.y, wv[6] = w1.z, wv[7] = w1.w;
+            } else if constexpr (kBL == 4) {
                 const float4 w = *reinterpret_cast<const float4 *>(wrow + i * R);
                 wv[0] = w.x, wv[1] = w.y, wv[2] = w.z, wv[3] = w.w;
             } else if constexpr (kBL == 2) {
@@ -333,6 +338,8 @@ cudaError_t launch_hash_prefill(const void *K, bool bf16, KStrides ks, int64_t n
                                 int64_t n, int words, cudaStream_t s)
 {
     switch (words * 2 + (bf16 ? 1 : 0)) {
+    case 16 + 1: return launch_hash_prefill_t<true, 256>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
+    case 16: return launch_hash_prefill_t<false, 256>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
     case 8 + 1: return launch_hash_prefill_t<true, 128>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
     case 8: return launch_hash_prefill_t<false, 128>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
     case 4 + 1: return launch_hash_prefill_t<true, 64>(K, ks, n_cap, W, codes, B, H_kv, pos0, n, s);
@@ -355,6 +362,8 @@ cudaError_t launch_prep_t(const PrepArgs &a, int rows_per_head, cudaStream_t s)
 cudaError_t launch_prep(const PrepArgs &a, int rows_per_head, cudaStream_t s)
 {
     switch (a.words * 2 + (a.kv_bf16 ? 1 : 0)) {
+    case 16 + 1: return launch_prep_t<true, 256>(a, rows_per_head, s);
+    case 16: return launch_prep_t<false, 256>(a, rows_per_head, s);
     case 8 + 1: return launch_prep_t<true, 128>(a, rows_per_head, s);
     case 8: return launch_prep_t<false, 128>(a, rows_per_head, s);
     case 4 + 1: return launch_prep_t<true, 64>(a, rows_per_head, s);

@@ -36,6 +36,12 @@
 // histograms in global memory (zeroed by the prep kernel), one reduction
 // per bin, so the selection kernel finds both the boundary distance and the
 // counts before any tile from them.
+//
+// 256-bit codes (the widest of the ablation) take their own, plainer kernel
+// (score_wide_kernel below): distances 0..256 have 257 values, one more than
+// a byte holds, so the stored row saturates at 255 while the histogram keeps
+// all 257 bins exactly; the selection recomputes the exact distance of a
+// saturated key from the codes when the boundary reaches 255.
 #include <algorithm>
 
 #include "hata_internal.cuh"
@@ -307,10 +313,101 @@ cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
                       s, a);
 }
 
+// ------------------------------------------------------- r = 256 codes --
+// One CTA per (4096-token chunk, slab, group of <= 8 query heads); thread t
+// scores tokens 4t .. 4t+3 of each 1024-token quarter of the chunk (two
+// 16-byte halves of each 32-byte code, read once for all heads of the
+// group), stores the four distances of a head as one 32-bit word (a warp
+// writes 128 consecutive bytes) and counts them in a 257-bin shared
+// histogram per head, added to the chunk's tile histogram at the end.
+constexpr int kWideThreads = 256;
+constexpr int kWideQuarter = 4 * kWideThreads;  // tokens per pass
+static_assert(kChunk == 4 * kWideQuarter, "four passes cover a chunk");
+static_assert(kTile % kChunk == 0, "a chunk lies in one histogram tile");
+
+__global__ void __launch_bounds__(kWideThreads) score_wide_kernel(ScoreArgs a)
+{
+    __shared__ uint32_t hist[kScoreHeads][kHistStrideWide];
+    __shared__ uint4 qs[kScoreHeads][2];
+    __shared__ uint2 qd[kScoreHeads][2];
+    pdl_trigger();
+    const int tid = threadIdx.x;
+    const int chunk = blockIdx.x;
+    const int slab = blockIdx.y;  // (b * H_kv + h) * zgroups + z
+    const int z = slab % a.zgroups, bhk = slab / a.zgroups;
+    const int h = bhk % a.H_kv, b = bhk / a.H_kv;
+    const int g0 = z * kScoreHeads;
+    const int ng = min(kScoreHeads, a.G - g0);
+    const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);  // step input
+    for (int i = tid; i < kScoreHeads * kHistStrideWide; i += kWideThreads) (&hist[0][0])[i] = 0u;
+    const int64_t bh0 = int64_t(b) * a.H_q + int64_t(h) * a.G + g0;  // first head of the group
+    pdl_wait();  // query codes, the appended key code, cleared tile histograms
+    if (tid < 2 * ng) {
+        const int g = tid >> 1, half = tid & 1;
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.qcodes + (bh0 + g) * 8) + half);
+        qs[g][half] = v;
+        const uint32_t q012 = v.x ^ v.y ^ v.z;
+        qd[g][half] = make_uint2(q012, q012 ^ v.w);
+    }
+    __syncthreads();
+
+    const uint4 *code = reinterpret_cast<const uint4 *>(a.codes) +
+                        ((int64_t(b) * a.H_kv + h) * a.n_cap) * 2;
+    const int64_t t00 = int64_t(chunk) * kChunk;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int64_t t0 = t00 + pass * kWideQuarter + 4 * tid;  // this thread's first token
+        uint4 k[4][2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool in = t0 + i < len;
+            k[i][0] = in ? __ldg(code + (t0 + i) * 2) : make_uint4(0u, 0u, 0u, 0u);
+            k[i][1] = in ? __ldg(code + (t0 + i) * 2 + 1) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint32_t k012[4][2], k0123[4][2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                k012[i][hf] = k[i][hf].x ^ k[i][hf].y ^ k[i][hf].z;
+                k0123[i][hf] = k012[i][hf] ^ k[i][hf].w;
+            }
+        for (int g = 0; g < ng; ++g) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t byte = kDistPad;
+                if (t0 + i < len) {
+                    const int d = hamming128(k[i][0], k012[i][0], k0123[i][0], qs[g][0], qd[g][0]) +
+                                  hamming128(k[i][1], k012[i][1], k0123[i][1], qs[g][1], qd[g][1]);
+                    atomicAdd(&hist[g][d], 1u);
+                    byte = d < 255 ? uint32_t(d) : 255u;
+                }
+                word |= byte << (8 * i);
+            }
+            __stcg(reinterpret_cast<uint32_t *>(a.dist + (bh0 + g) * a.dist_row + t0), word);
+        }
+    }
+    __syncthreads();
+    // add the non-zero bins to the chunk's tile histograms
+    const int64_t tile = t00 / kTile;
+    for (int i = tid; i < ng * kBinsWide; i += kWideThreads) {
+        const int g = i / kBinsWide, t = i % kBinsWide;
+        const uint32_t v = hist[g][t];
+        if (v) atomicAdd(a.hist + ((bh0 + g) * a.n_tiles + tile) * kHistStrideWide + t, v);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s)
 {
+    if (a.words == 8) {
+        if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(score_wide_kernel), 0))
+            return e;
+        const dim3 grid(unsigned(a.dist_row / kChunk),
+                        unsigned(int64_t(a.B) * a.H_kv * a.zgroups));
+        return launch_pdl(score_wide_kernel, grid, dim3(kWideThreads), 0, s, a);
+    }
     const int gb = a.G < kScoreHeads ? a.G : kScoreHeads;
     if (a.words == 4) {
         switch (gb) {

@@ -20,6 +20,15 @@
 // thread its output position, and the ties a thread may take follow from
 // the ties before it: taken_before = min(ties_before, room).  Indices are
 // written straight to the head's list, ascending.
+//
+// 256-bit codes: the stored distance saturates at 255 (distances run to
+// 256), the tile histograms hold all 257 bins.  With T <= 254 the byte
+// compares stay exact (a stored 255 is above T); the rare T of 255 or 256
+// takes the exact distance of every saturated key from the codes.
+//
+// The sequence-parallel step passes k_head: the keys each head takes from
+// this shard, which makes the shard's selection its own top-k_head with the
+// same tie rule.
 #include "select_common.cuh"
 #include "async_copy.cuh"
 
@@ -33,7 +42,26 @@ constexpr int kPieces = kPer / 16;                      // 16-byte loads per thr
 constexpr int kGroups = kPer / 32;                      // 32-distance mask words
 static_assert(kThreads * kPer == kTile, "a CTA covers one histogram tile per pass");
 
-__global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
+// Exact distance of key `tok` of head bh's KV slab to the head's 256-bit
+// query code (q: its two 16-byte halves).
+__device__ __forceinline__ int exact_dist_wide(const SelectArgs &a, size_t bh, const uint4 (&q)[2],
+                                               int tok)
+{
+    const int b = int(bh) / a.H_q, h = (int(bh) - b * a.H_q) / a.G;
+    const uint4 *c = reinterpret_cast<const uint4 *>(a.codes) +
+                     ((int64_t(b) * a.H_kv + h) * a.n_cap + tok) * 2;
+    int d = 0;
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const uint4 k = __ldg(c + hf);
+        d += __popc(k.x ^ q[hf].x) + __popc(k.y ^ q[hf].y) + __popc(k.z ^ q[hf].z) +
+             __popc(k.w ^ q[hf].w);
+    }
+    return d;
+}
+
+template <bool kWide>
+__global__ void __launch_bounds__(kThreads, kWide ? 2 : 4) select_kernel(SelectArgs a)
 {
     pdl_trigger();
     const int tile = blockIdx.x;
@@ -41,8 +69,13 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     const int b = int(bh) / a.H_q;
     const int len = int(clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap));  // step input
     const int tid = threadIdx.x;
-    const int k_eff = a.topk < len ? a.topk : len;
+    int k_eff = a.topk < len ? a.topk : len;
     pdl_wait();  // distances and tile histograms of the scoring kernel
+    if (a.k_head) {  // written by the kernel before this one
+        const int kh = __ldg(a.k_head + bh);
+        k_eff = kh < k_eff ? (kh > 0 ? kh : 0) : k_eff;
+    }
+    constexpr int kStride = kWide ? kHistStrideWide : kHistStride;
     int32_t *idx = a.idx + bh * a.topk;
 
     __shared__ int2 scan_s[kWarps + 1];
@@ -61,8 +94,8 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     // trip to L2 per 4 tiles), ahead of its own distance loads;
     // the other warps' distance loads are in flight meanwhile ----
     if (tid < 32)
-        head_threshold(a.hist + bh * size_t(a.n_tiles) * kHistStride, int(a.n_tiles), k_eff,
-                       tile, tid, s_thr);
+        head_threshold<false, 4, kWide>(a.hist + bh * size_t(a.n_tiles) * kStride,
+                                        int(a.n_tiles), k_eff, tile, tid, s_thr);
     // the warp's 4 KB arrive by coalesced 16-byte copies (lane l: bytes
     // 16l .. 16l+15 of each 512-byte block) into a swizzled shared tile,
     // piece v of thread t at t*128 + 16*(v ^ (t & 7)), so that each thread
@@ -117,16 +150,48 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
     const uint32_t T4 = uint32_t(T) * 0x01010101u, T4p = T4 + 0x01010101u;
     uint32_t lt_bits[kGroups], eq_bits[kGroups];
     int n_lt = 0, n_eq = 0;
+    if (kWide && T >= 255) {
+        // the boundary reached the saturated byte: exact distances of the
+        // saturated keys (bit 8e + w of group m <-> distance 32 m + 4 w + e;
+        // keys at or past len never count)
+        uint4 q[2];
+        q[0] = __ldg(reinterpret_cast<const uint4 *>(a.qcodes) + bh * 2);
+        q[1] = __ldg(reinterpret_cast<const uint4 *>(a.qcodes) + bh * 2 + 1);
+        const uint8_t *mine = dist_s + tid * kPer;
 #pragma unroll
-    for (int m = 0; m < kGroups; ++m) {
-        const uint32_t dw[8] = {dv[2 * m].x,     dv[2 * m].y,     dv[2 * m].z,     dv[2 * m].w,
-                                dv[2 * m + 1].x, dv[2 * m + 1].y, dv[2 * m + 1].z, dv[2 * m + 1].w};
-        if (T < 128)
-            group_masks<false>(dw, T4, T4p, lt_bits[m], eq_bits[m]);
-        else
-            group_masks<true>(dw, T4, T4p, lt_bits[m], eq_bits[m]);
-        n_lt += __popc(lt_bits[m]);
-        n_eq += __popc(eq_bits[m]);
+        for (int m = 0; m < kGroups; ++m) {
+            uint32_t lt = 0u, eq = 0u;
+            for (int j = 0; j < 32; ++j) {
+                const int o = 32 * m + j, tok = my0 + o;
+                int d = 1 << 20;  // past len: never selected
+                if (tok < len) {
+                    d = mine[16 * ((o >> 4) ^ (tid & 7)) + (o & 15)];
+                    if (d == 255) d = exact_dist_wide(a, bh, q, tok);
+                }
+                const uint32_t bit = 1u << (8 * (j & 3) + (j >> 2));
+                lt |= d < T ? bit : 0u;
+                eq |= d == T ? bit : 0u;
+            }
+            lt_bits[m] = lt;
+            eq_bits[m] = eq;
+            n_lt += __popc(lt);
+            n_eq += __popc(eq);
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < kGroups; ++m) {
+            const uint32_t dw[8] = {dv[2 * m].x,     dv[2 * m].y,     dv[2 * m].z,
+                                    dv[2 * m].w,     dv[2 * m + 1].x, dv[2 * m + 1].y,
+                                    dv[2 * m + 1].z, dv[2 * m + 1].w};
+            if (kWide)
+                group_masks_any(dw, T4, lt_bits[m], eq_bits[m]);
+            else if (T < 128)
+                group_masks<false>(dw, T4, T4p, lt_bits[m], eq_bits[m]);
+            else
+                group_masks<true>(dw, T4, T4p, lt_bits[m], eq_bits[m]);
+            n_lt += __popc(lt_bits[m]);
+            n_eq += __popc(eq_bits[m]);
+        }
     }
 
     int tile_lt, tile_eq;
@@ -148,12 +213,12 @@ __global__ void __launch_bounds__(kThreads, 4) select_kernel(SelectArgs a)
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s)
 {
-    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(select_kernel), 0))
-        return e;
+    auto kernel = a.words == 8 ? select_kernel<true> : select_kernel<false>;
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kernel), 0)) return e;
     // one CTA per (36K-token tile, head)
     const dim3 grid(static_cast<unsigned>(ceil_div(a.max_seq_len, kTile)),
                     static_cast<unsigned>(int64_t(a.B) * a.H_q));
-    return launch_pdl(select_kernel, grid, dim3(kThreads), 0, s, a);
+    return launch_pdl(kernel, grid, dim3(kThreads), 0, s, a);
 }
 
 }  // namespace hata

@@ -3,8 +3,8 @@
 // histograms, the byte-wise masks and the ordered emission.
 //
 // HATA review page (arXiv 2506.02572), major comment 1 (Algorithm 3): the
-// top-k runs over Hamming scores that take only 129 values; the boundary
-// bucket goes to the lower token indices:
+// top-k runs over Hamming scores that take only r + 1 values (129 at the
+// page's r = 128); the boundary bucket goes to the lower token indices:
 //   k_eff = min(topk, len)
 //   T     = the smallest distance t with #(dist <= t) >= k_eff
 //   S     = {n : dist[n] < T}  +  the k_eff - #(dist < T) lowest-index keys
@@ -67,54 +67,79 @@ __device__ __forceinline__ void group_masks(const uint32_t (&dw)[8], uint32_t T4
     eq_out = le & ~lb;
 }
 
+// "< T" and "== T" masks of 32 consecutive distances for any T in 0..254
+// (the 256-bit codes, whose stored distances run 0..255): per-byte unsigned
+// compares, packed like group_masks.
+__device__ __forceinline__ void group_masks_any(const uint32_t (&dw)[8], uint32_t T4,
+                                                uint32_t &lt_out, uint32_t &eq_out)
+{
+    uint32_t lb = 0, lq = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        lb = __umulhi(lb, 0x80000000u) + (__vcmpltu4(dw[w], T4) & 0x80808080u);
+        lq = __umulhi(lq, 0x80000000u) + (__vcmpeq4(dw[w], T4) & 0x80808080u);
+    }
+    lt_out = lb;
+    eq_out = lq;
+}
+
 // T = the smallest distance t with #(dist <= t) >= k_eff, #(dist < T), and
 // the keys below T and at T in the tiles before `tile`, from one head's
-// tile histograms (hrow: n_tiles rows of kHistStride words).  One warp;
-// lane l owns bins 5l .. 5l+4; out: {T, #(< T), below-T before the tile,
-// at-T before the tile}.  kCoherent: the rows were written by the running
-// kernel itself (loads through L2 only); otherwise by an earlier kernel.
-template <bool kCoherent = false, int kRegTiles = 4>  // kRegTiles: rows per round
+// tile histograms (hrow: n_tiles rows of kHistStride words, or of
+// kHistStrideWide words for the 257 bins of 256-bit codes).  One warp; lane
+// l owns bins kBPL l .. kBPL l + kBPL - 1; out: {T, #(< T), below-T before
+// the tile, at-T before the tile}.  kCoherent: the rows were written by the
+// running kernel itself (loads through L2 only); otherwise by an earlier
+// kernel.
+template <bool kCoherent = false, int kRegTiles = 4, bool kWide = false>
 __device__ __forceinline__ void head_threshold(const uint32_t *hrow, int n_tiles, int k_eff,
                                                int tile, int lane, int *out)
 {
-    auto row_bins = [&](int t, uint32_t (&v)[5]) {
+    constexpr int kBPL = kWide ? 9 : 5;  // bins per lane: 32 lanes cover 257 / 129 bins
+    constexpr int kNB = kWide ? kBinsWide : kBins;
+    constexpr int kStride = kWide ? kHistStrideWide : kHistStride;
+    auto row_bins = [&](int t, uint32_t (&v)[kBPL]) {
 #pragma unroll
-        for (int e = 0; e < 5; ++e)
-            v[e] = lane * 5 + e < kBins
-                       ? (kCoherent ? __ldcg(hrow + t * kHistStride + lane * 5 + e)
-                                    : __ldg(hrow + t * kHistStride + lane * 5 + e))
+        for (int e = 0; e < kBPL; ++e)
+            v[e] = lane * kBPL + e < kNB
+                       ? (kCoherent ? __ldcg(hrow + t * kStride + lane * kBPL + e)
+                                    : __ldg(hrow + t * kStride + lane * kBPL + e))
                        : 0u;
     };
-    uint32_t tot[5] = {0u, 0u, 0u, 0u, 0u}, pre[5] = {0u, 0u, 0u, 0u, 0u};
+    uint32_t tot[kBPL], pre[kBPL];
+#pragma unroll
+    for (int e = 0; e < kBPL; ++e) tot[e] = pre[e] = 0u;
     // rounds of kRegTiles rows: all loads of a round are issued before any
     // is summed, so a round costs one round trip to L2
     for (int t0 = 0; t0 < n_tiles; t0 += kRegTiles) {
-        uint32_t rv[kRegTiles][5];
+        uint32_t rv[kRegTiles][kBPL];
 #pragma unroll
         for (int t = 0; t < kRegTiles; ++t) {
             if (t0 + t < n_tiles) {
                 row_bins(t0 + t, rv[t]);
             } else {
 #pragma unroll
-                for (int e = 0; e < 5; ++e) rv[t][e] = 0u;
+                for (int e = 0; e < kBPL; ++e) rv[t][e] = 0u;
             }
         }
 #pragma unroll
         for (int t = 0; t < kRegTiles; ++t)
 #pragma unroll
-            for (int e = 0; e < 5; ++e) {
+            for (int e = 0; e < kBPL; ++e) {
                 tot[e] += rv[t][e];
                 pre[e] += t0 + t < tile ? rv[t][e] : 0u;
             }
     }
-    const uint32_t run = tot[0] + tot[1] + tot[2] + tot[3] + tot[4];
+    uint32_t run = 0;
+#pragma unroll
+    for (int e = 0; e < kBPL; ++e) run += tot[e];
     uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
     int Tl = -1;
     uint32_t less_l = 0;
 #pragma unroll
-    for (int e = 0; e < 5; ++e) {
-        if (Tl < 0 && lane * 5 + e < kBins && acc + tot[e] >= uint32_t(k_eff)) {
-            Tl = lane * 5 + e;
+    for (int e = 0; e < kBPL; ++e) {
+        if (Tl < 0 && lane * kBPL + e < kNB && acc + tot[e] >= uint32_t(k_eff)) {
+            Tl = lane * kBPL + e;
             less_l = acc;
         }
         acc += tot[e];
@@ -122,12 +147,12 @@ __device__ __forceinline__ void head_threshold(const uint32_t *hrow, int n_tiles
     // cumulative counts are monotone: the lowest lane that found a bin holds T
     const unsigned found = __ballot_sync(0xffffffffu, Tl >= 0);
     const int src = found ? __ffs(int(found)) - 1 : 0;
-    const int T = found ? __shfl_sync(0xffffffffu, Tl, src) : 128;  // unreachable fallback
+    const int T = found ? __shfl_sync(0xffffffffu, Tl, src) : kNB - 1;  // unreachable fallback
     const int n_less = found ? __shfl_sync(0xffffffffu, int(less_l), src) : 0;
     int l = 0, q = 0;
 #pragma unroll
-    for (int e = 0; e < 5; ++e) {
-        const int bin = lane * 5 + e;
+    for (int e = 0; e < kBPL; ++e) {
+        const int bin = lane * kBPL + e;
         l += bin < T ? int(pre[e]) : 0;
         q += bin == T ? int(pre[e]) : 0;
     }

@@ -32,6 +32,8 @@ HATA_NOALLOC_WORKSPACE_BYTES = 64 << 20
 HATA_MODE_AUTO = 0
 HATA_MODE_MULTI_KERNEL = 1
 HATA_MODE_FUSED = 2
+HATA_SP_HIST_WORDS = 260
+HATA_SP_PART_WORDS = 132
 D = 128
 RBIT = 128
 
@@ -64,6 +66,10 @@ _SIGS = {
     "hata_set_decode_mode": ([I], I),
     "hata_get_decode_mode": ([], I),
     "hata_set_wait_limit_ns": ([ctypes.c_uint64], I),
+    "hata_sp_score": ([P, P, P, P, P, I, I64, P, I64, P, P, I, I, I, I, I, I, P, U64, P, P], I),
+    "hata_sp_attend": ([P, I, I, P, P, P, I, I64, P, I64, I, I, I, I, I, I, F, P, U64, P, P, P],
+                       I),
+    "hata_sp_merge": ([P, I, I, I, P, P], I),
 }
 
 
@@ -257,6 +263,72 @@ def hata_decode_step(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K:
         max_seq_len, _ptr(k_new), _ptr(v_new), B, H_q, H_kv, d, W_H.shape[2], topk,
         float(scale), _ptr(workspace), workspace.numel(), _ptr(out), _ptr(sel_idx),
         _ptr(q_codes), _ptr(dist), drow, ev, _stream(stream)), "hata_decode_step")
+
+
+def hata_sp_score(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor, K: torch.Tensor,
+                  V: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int, topk: int,
+                  workspace: torch.Tensor, hist_out: torch.Tensor,
+                  k_new: torch.Tensor | None = None, v_new: torch.Tensor | None = None,
+                  stream=None) -> None:
+    """Phase 1 of a sequence-parallel step on this rank's token shard (see
+    include/hata.h): hist_out [B][H_q][HATA_SP_HIST_WORDS] int32 receives the
+    shard's per-head histogram of Hamming distances."""
+    _need(q, "q", torch.float32, 3)
+    _need(W_H, "W_H", torch.float32, 3)
+    _need(codes, "codes", torch.int32, 4)
+    _need_code_words(codes, W_H)
+    _need(K, "K", ndim=4)
+    _need(V, "V", ndim=4)
+    _need(seq_len, "seq_len", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8)
+    _need(hist_out, "hist_out", torch.int32, 3)
+    for t, name in ((k_new, "k_new"), (v_new, "v_new")):
+        if t is not None:
+            _need(t, name, K.dtype, 3)
+    B, H_q, d = q.shape
+    if tuple(hist_out.shape) != (B, H_q, HATA_SP_HIST_WORDS):
+        raise ValueError(f"hist_out must be [{B}][{H_q}][{HATA_SP_HIST_WORDS}]")
+    H_kv, n_cap = K.shape[1], K.shape[2]
+    _check(lib().hata_sp_score(
+        _ptr(q), _ptr(W_H), _ptr(codes), _ptr(K), _ptr(V), _kv_code(K), n_cap, _ptr(seq_len),
+        max_seq_len, _ptr(k_new), _ptr(v_new), B, H_q, H_kv, d, W_H.shape[2], topk,
+        _ptr(workspace), workspace.numel(), _ptr(hist_out), _stream(stream)), "hata_sp_score")
+
+
+def hata_sp_attend(hist_all: torch.Tensor, rank: int, codes: torch.Tensor, K: torch.Tensor,
+                   V: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int, H_q: int, r: int,
+                   topk: int, scale: float, workspace: torch.Tensor, part_out: torch.Tensor,
+                   sel_idx: torch.Tensor | None = None, stream=None) -> None:
+    """Phase 2 of a sequence-parallel step: hist_all [world][B][H_q][HATA_SP_HIST_WORDS]
+    int32 (every rank's histograms, rank-major) -> part_out [B][H_q][HATA_SP_PART_WORDS]
+    fp32, this shard's unnormalised partial; sel_idx [B][H_q][topk] int32
+    optionally receives the shard-local selected positions."""
+    _need(hist_all, "hist_all", torch.int32, 4)
+    _need(codes, "codes", torch.int32, 4)
+    _need(K, "K", ndim=4)
+    _need(V, "V", ndim=4)
+    _need(seq_len, "seq_len", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8)
+    _need(part_out, "part_out", torch.float32, 3)
+    if sel_idx is not None:
+        _need(sel_idx, "sel_idx", torch.int32, 3)
+    world, B = hist_all.shape[0], hist_all.shape[1]
+    H_kv, n_cap, d = K.shape[1], K.shape[2], K.shape[3]
+    if tuple(part_out.shape) != (B, H_q, HATA_SP_PART_WORDS):
+        raise ValueError(f"part_out must be [{B}][{H_q}][{HATA_SP_PART_WORDS}]")
+    _check(lib().hata_sp_attend(
+        _ptr(hist_all), world, rank, _ptr(codes), _ptr(K), _ptr(V), _kv_code(K), n_cap,
+        _ptr(seq_len), max_seq_len, B, H_q, H_kv, d, r, topk, float(scale), _ptr(workspace),
+        workspace.numel(), _ptr(part_out), _ptr(sel_idx), _stream(stream)), "hata_sp_attend")
+
+
+def hata_sp_merge(part_all: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """Phase 3: part_all [world][B][H_q][HATA_SP_PART_WORDS] fp32 -> out [B][H_q][128]."""
+    _need(part_all, "part_all", torch.float32, 4)
+    _need(out, "out", torch.float32, 3)
+    world, B, H_q = part_all.shape[:3]
+    _check(lib().hata_sp_merge(_ptr(part_all), world, B, H_q, _ptr(out), _stream(stream)),
+           "hata_sp_merge")
 
 
 def hata_decode_step_noalloc(q: torch.Tensor, W_H: torch.Tensor, codes: torch.Tensor,

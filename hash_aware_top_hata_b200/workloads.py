@@ -18,7 +18,10 @@ RULER, InfiniteBench, NIAH) and trained hash weights are not available, so:
 * the million-token case instead plants 64 "needles" per KV head,
   key = 0.8 * u + 0.2 * N(0, 1), at random positions;
 * queries of later decode steps are q_t = q_0 + 0.25 * eps_t, and each step
-  appends one fresh N(0, 1) key and value per sequence and KV head.
+  appends one fresh N(0, 1) key and value per sequence and KV head;
+* the other code widths of the page's ablation use the leading r columns of
+  W_H (r = 32, 64), or W_H followed by r - 128 more N(0, 1/128) columns drawn
+  from their own seeded stream (r = 256): see ``projection``.
 """
 from __future__ import annotations
 
@@ -162,6 +165,18 @@ def make_workload(cfg: Config, seed: int, device="cpu", steps: int | None = None
     k_new = _randn((max(steps, 1), B, Hkv, D), g_s, device).to(kv_dtype)
     v_new = _randn((max(steps, 1), B, Hkv, D), g_s, device).to(kv_dtype)
     return Workload(cfg, n_cap, q, W_H, K, V, k_new, v_new, planted)
+
+
+def projection(W_H: torch.Tensor, r: int, seed: int = 20260256) -> torch.Tensor:
+    """The [H_kv][D][r] projection of an r-bit code from a workload's
+    [H_kv][D][128] W_H: its leading r columns for r <= 128, else W_H with
+    r - 128 further N(0, 1/D) columns appended (their own generator, seeded
+    `seed`, on W_H's device)."""
+    if r <= RBIT:
+        return W_H if r == RBIT else W_H[:, :, :r].contiguous()
+    g = _gen(W_H.device, seed)
+    extra = _randn((W_H.shape[0], D, r - RBIT), g, W_H.device) * (1.0 / math.sqrt(D))
+    return torch.cat([W_H, extra], dim=2).contiguous()
 
 
 def bf16_bits(t: torch.Tensor):

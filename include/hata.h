@@ -13,16 +13,18 @@
  *     cache Kcache_H, rbit/32 32-bit words per token; K and V fill the KV cache.
  *   Referee report, major comment 1 (Algorithm 3): top-k over 129 possible
  *     Hamming values; the choice inside the boundary bucket is left open.
+ *   "Assumptions & free parameters": rbit is a free parameter chosen by
+ *     ablation (accuracy grows from 32 to 128 bits, then levels off).
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers, allocated and owned by the
  *     caller; the library never allocates, frees or keeps them.  Work is
  *     enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
  *     and the call returns without synchronising, except where noted.
- *   - d (head_dim) must be 128; r (hash bits) 128, the page's width, or 32 /
- *     64, the narrower widths of its ablation (HATA_ERR_UNSUPPORTED
- *     otherwise).  r = 256 is not offered: its distances 0..256 do not fit
- *     the byte-wide distance row next to the pad value 255.
+ *   - d (head_dim) must be 128; r (hash bits) 128, the page's width, or 32,
+ *     64 or 256, the other widths of its ablation (HATA_ERR_UNSUPPORTED
+ *     otherwise).  At r = 256 the distances run 0..256; selections use them
+ *     exactly, while the optional byte-wide distance rows store min(d, 255).
  *   - Layouts are dense row-major:
  *       W_H    [H_kv][d][r]        fp32, 16-byte aligned; bit j of a code is
  *                                   [sum_i x_i W_H[i][j] > 0]
@@ -59,7 +61,7 @@ extern "C" {
 typedef enum hata_status {
     HATA_OK = 0,
     HATA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, small workspace */
-    HATA_ERR_UNSUPPORTED = 2,   /* d != 128, r not 32/64/128, H_q not a multiple of H_kv */
+    HATA_ERR_UNSUPPORTED = 2,   /* d != 128, r not 32/64/128/256, H_q not a multiple of H_kv */
     HATA_ERR_CUDA = 3,          /* a CUDA launch or copy failed */
     HATA_ERR_DEVICE_CHECK = 4   /* a device-side range check fired (see the flags) */
 } hata_status_t;
@@ -144,7 +146,8 @@ int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
  *                          CTA per SM in which selection warps build the
  *                          index lists while attention warps already gather
  *                          and attend the heads selected so far (bf16 caches
- *                          only; fp32 caches take the multi-kernel step).
+ *                          and r <= 128 only; other steps take the
+ *                          multi-kernel step).
  *   HATA_MODE_AUTO          the library's choice (default)
  *   HATA_MODE_MULTI_KERNEL  always the multi-kernel step
  *   HATA_MODE_FUSED         the fused step for bf16 caches
@@ -198,7 +201,8 @@ hata_status_t hata_set_wait_limit_ns(uint64_t ns);
  *             slots past |S| set to -1
  *   q_codes   optional [B][H_q][r/32] uint32: the query codes
  *   dist, dist_row_bytes  optional [B][H_q][dist_row_bytes] uint8: the
- *             Hamming distances (0..r); positions seq_len[b] ..
+ *             Hamming distances (0..r; min(d, 255) at r = 256); positions
+ *             seq_len[b] ..
  *             hata_dist_row_bytes(max_seq_len)-1 hold 255;
  *             dist_row_bytes >= hata_dist_row_bytes(max_seq_len), multiple of 16
  *   events    optional array of 6 cudaEvent_t recorded on `stream` before the
@@ -238,6 +242,10 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
  *     without ordering between them) race: order them on one stream.
  *   - hata_workspace_check cannot see this buffer; device-side flags of
  *     this entry point are not reported.
+ *   - The cached address belongs to the device's current context: after
+ *     cudaDeviceReset (or any other teardown of the primary context) the
+ *     library's device image is loaded again and the array may move, so
+ *     this entry point must not be called again in that process.
  * The call allocates nothing (no cudaMalloc / cudaFree / allocating
  * library routine). */
 #define HATA_NOALLOC_WORKSPACE_BYTES (64u << 20)
@@ -248,6 +256,56 @@ hata_status_t hata_decode_step_noalloc(const float *q, const float *W_H, uint32_
                                        int H_kv, int d, int r, int topk, float scale, float *out,
                                        int32_t *sel_idx, uint32_t *q_codes, uint8_t *dist,
                                        int64_t dist_row_bytes, void *const *events, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Sequence-parallel decode step (one head's keys sharded over ranks).
+ * The cached tokens of every (b, h_kv) are split into contiguous shards, one
+ * per rank, in rank order (rank w holds global tokens o_w .. o_w + len_w - 1
+ * with o_0 = 0 and o_{w+1} = o_w + len_w); each rank keeps its shard as an
+ * ordinary cache (positions 0 .. len_w - 1, seq_len[b] = len_w).  Algorithm
+ * 3's threshold top-k (referee report, major comment 1) needs only the
+ * shards' histograms of the r + 1 Hamming values, so a step is two local
+ * phases around two small exchanges that the caller runs (all-gathers over
+ * NCCL, for instance):
+ *   1. hata_sp_score   hash q (and append), score this shard, write its
+ *                      per-head histogram [B][H_q][HATA_SP_HIST_WORDS];
+ *      exchange        all-gather the histograms of every rank, rank-major:
+ *                      hist_all [world][B][H_q][HATA_SP_HIST_WORDS];
+ *   2. hata_sp_attend  from hist_all: the global threshold and this shard's
+ *                      share of the boundary ties (lower ranks, i.e. lower
+ *                      tokens, first), then the shard's selection and the
+ *                      attention over it, written as an unnormalised partial
+ *                      [B][H_q][HATA_SP_PART_WORDS] fp32: {m, l, -, -,
+ *                      acc[128]} with m in log2 units (scale * log2 e), the
+ *                      weights 2^(s - m), l their sum, acc the weighted sum
+ *                      of V rows (m = -inf, l = 0, acc = 0 when empty);
+ *      exchange        all-gather the partials: part_all [world][B][H_q][132];
+ *   3. hata_sp_merge   out = the log-sum-exp merge of the world partials.
+ * The union of the ranks' selections (shard positions + o_w) is the
+ * single-GPU selection of the whole sequence bit for bit, and out agrees
+ * with the single-GPU output within the attention tolerance.
+ * Phases 1 and 2 of a step use the same workspace (hata_decode_workspace_size
+ * of the same B, H_q, H_kv, max_seq_len, topk) and must be ordered on one
+ * stream; phase 2 reads the query codes, distances and tile histograms
+ * phase 1 left there.  A rank whose shard is empty passes seq_len 0.
+ * Only the rank that holds the newest token passes k_new / v_new. */
+#define HATA_SP_HIST_WORDS 260
+#define HATA_SP_PART_WORDS 132
+hata_status_t hata_sp_score(const float *q, const float *W_H, uint32_t *codes, void *K, void *V,
+                            hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                            int64_t max_seq_len, const void *k_new, const void *v_new, int B,
+                            int H_q, int H_kv, int d, int r, int topk, void *workspace,
+                            size_t workspace_bytes, uint32_t *hist_out, void *stream);
+/* sel_idx: optional [B][H_q][topk] int32, this shard's selected positions
+ * (shard-local, ascending), -1 after the last. */
+hata_status_t hata_sp_attend(const uint32_t *hist_all, int world, int rank,
+                             const uint32_t *codes, const void *K, const void *V,
+                             hata_dtype_t kv_dtype, int64_t n_cap, const int32_t *seq_len,
+                             int64_t max_seq_len, int B, int H_q, int H_kv, int d, int r,
+                             int topk, float scale, void *workspace, size_t workspace_bytes,
+                             float *part_out, int32_t *sel_idx, void *stream);
+hata_status_t hata_sp_merge(const float *part_all, int world, int B, int H_q, float *out,
+                            void *stream);
 
 /* ------------------------------------------------------------------------
  * hata_workspace_check -- synchronises `stream`, reads and clears the

@@ -22,7 +22,7 @@ def test_library_exports_every_header_function():
     lib = H.lib()
     for n in names:
         assert hasattr(lib, n), n
-    assert H.hata_abi_version() == 2
+    assert H.hata_abi_version() == 3
 
 
 def test_status_strings():
@@ -63,7 +63,8 @@ def decode(**over):
     (dict(ws=NULL), H.HATA_ERR_INVALID_ARG),
     (dict(d=64), H.HATA_ERR_UNSUPPORTED),
     (dict(r=96), H.HATA_ERR_UNSUPPORTED),
-    (dict(r=256), H.HATA_ERR_UNSUPPORTED),
+    (dict(r=512), H.HATA_ERR_UNSUPPORTED),
+    (dict(r=0), H.HATA_ERR_UNSUPPORTED),
     (dict(H_q=3), H.HATA_ERR_UNSUPPORTED),
     (dict(B=0), H.HATA_ERR_INVALID_ARG),
     (dict(topk=0), H.HATA_ERR_INVALID_ARG),
@@ -85,6 +86,69 @@ def decode(**over):
 def test_decode_step_rejects_on_host(over, status):
     assert decode(**over) == status
     assert H.lib().hata_last_error().decode() != ""
+
+
+def sp_score(**over):
+    """hata_sp_score through raw ctypes with fake pointers."""
+    args = dict(q=FAKE, W=FAKE, codes=FAKE, K=FAKE, V=FAKE, dt=0, n_cap=8192, seq_len=FAKE,
+                max_len=4096, k_new=NULL, v_new=NULL, B=1, H_q=4, H_kv=2, d=128, r=256, topk=64,
+                ws=FAKE, ws_bytes=1 << 40, hist=FAKE, stream=NULL)
+    args.update(over)
+    return H.lib().hata_sp_score(*args.values())
+
+
+def sp_attend(**over):
+    args = dict(hist_all=FAKE, world=2, rank=1, codes=FAKE, K=FAKE, V=FAKE, dt=0, n_cap=8192,
+                seq_len=FAKE, max_len=4096, B=1, H_q=4, H_kv=2, d=128, r=128, topk=64,
+                scale=0.088, ws=FAKE, ws_bytes=1 << 40, part=FAKE, sel=NULL, stream=NULL)
+    args.update(over)
+    return H.lib().hata_sp_attend(*args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(hist=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(hist=FAKE + 2), H.HATA_ERR_INVALID_ARG),
+    (dict(r=96), H.HATA_ERR_UNSUPPORTED),
+    (dict(topk=0), H.HATA_ERR_INVALID_ARG),
+    (dict(v_new=FAKE), H.HATA_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), H.HATA_ERR_INVALID_ARG),
+    (dict(max_len=8193), H.HATA_ERR_INVALID_ARG),
+])
+def test_sp_score_rejects_on_host(over, status):
+    assert sp_score(**over) == status
+    assert H.lib().hata_last_error().decode() != ""
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(hist_all=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(part=NULL), H.HATA_ERR_INVALID_ARG),
+    (dict(part=FAKE + 4), H.HATA_ERR_INVALID_ARG),
+    (dict(world=0), H.HATA_ERR_INVALID_ARG),
+    (dict(rank=2), H.HATA_ERR_INVALID_ARG),
+    (dict(rank=-1), H.HATA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), H.HATA_ERR_INVALID_ARG),
+    (dict(H_q=3), H.HATA_ERR_UNSUPPORTED),
+    (dict(ws=FAKE + 16), H.HATA_ERR_INVALID_ARG),
+])
+def test_sp_attend_rejects_on_host(over, status):
+    assert sp_attend(**over) == status
+
+
+def test_sp_merge_rejects_on_host():
+    L = H.lib()
+    assert L.hata_sp_merge(NULL, 2, 1, 4, FAKE, NULL) == H.HATA_ERR_INVALID_ARG
+    assert L.hata_sp_merge(FAKE, 0, 1, 4, FAKE, NULL) == H.HATA_ERR_INVALID_ARG
+    assert L.hata_sp_merge(FAKE, 2, 1, 4, FAKE + 4, NULL) == H.HATA_ERR_INVALID_ARG
+    assert L.hata_sp_merge(FAKE, 2, 4096, 32, FAKE, NULL) == H.HATA_ERR_INVALID_ARG
+
+
+def test_wide_codes_need_wider_histogram_rows():
+    """The workspace reserves 257-bin tile histogram rows, whatever r."""
+    import math
+    B, H_q, n = 1, 4, 100_000
+    tiles = math.ceil(math.ceil(n / 4096) * 4096 / 36864)
+    assert H.hata_decode_workspace_size(B, H_q, 1, n, 64) >= 4 * B * H_q * tiles * 260
 
 
 def test_hash_and_append_reject_on_host():

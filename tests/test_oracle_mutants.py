@@ -37,6 +37,12 @@ MUTANTS = {
     "bf16 cache rows strided as 4-byte elements": (
         "row * d * (dtype == ORACLE_DT_BF16 ? 2 : 4);",
         "row * d * (dtype == ORACLE_DT_BF16 ? 4 : 4);"),
+    "hamming stops at 128 bits": (
+        "for (int j = 0; j < r; ++j) {\n        uint32_t x",
+        "for (int j = 0; j < (r < 128 ? r : 128); ++j) {\n        uint32_t x"),
+    "distance 256 counted as 255": (
+        "dist += (int)((x >> (j % 32)) & 1u);\n    }\n    return dist;",
+        "dist += (int)((x >> (j % 32)) & 1u);\n    }\n    return dist > 255 ? 255 : dist;"),
 }
 
 

@@ -323,7 +323,7 @@ def test_attend_empty_set_is_zero():
 
 # ---------------------------------------------------------- decode step ---
 
-@pytest.mark.parametrize("r", [128, 64, 32])
+@pytest.mark.parametrize("r", [128, 64, 32, 256])
 def test_decode_head_matches_independent_restatement(r):
     """The composed step against an independent numpy/Python restatement
     (fp64 projection sign, unpackbits popcount, sorted() top-k, numpy
@@ -398,7 +398,7 @@ def test_narrow_code_is_prefix_of_wide_code(r):
         assert np.array_equal(bits[sure], (proj[sure] > 0).astype(np.uint8))
 
 
-@pytest.mark.parametrize("r", [32, 64])
+@pytest.mark.parametrize("r", [32, 64, 256])
 def test_narrow_hamming_range_and_brute_force(r):
     w = r // 32
     codes = RNG.integers(0, 2**32, (200, w), dtype=np.uint64).astype(np.uint32)
@@ -409,3 +409,57 @@ def test_narrow_hamming_range_and_brute_force(r):
     assert np.array_equal(d, (ub != uq[None, :]).sum(-1))
     assert oracle.hamming(q, ~q) == r and oracle.hamming(q, q) == 0
     assert d.min() >= 0 and d.max() <= r
+
+
+# ------------------------------------------------------ 256-bit codes (r) ---
+# The ablation's widest code: bit j still depends on column j of W_H alone,
+# so the 128-bit code is the first four words of the 256-bit one, and the
+# Hamming range is 0..256 (257 values, one more than a byte holds).
+
+def test_wide_code_extends_the_128_bit_code():
+    W = RNG.standard_normal((128, 256)).astype(np.float32) / math.sqrt(128)
+    for _ in range(20):
+        x = RNG.standard_normal(128).astype(np.float32)
+        wide = oracle.hash_vec(x, W)
+        assert wide.shape == (8,)
+        assert np.array_equal(wide[:4], oracle.hash_vec(x, np.ascontiguousarray(W[:, :128])))
+        proj = x.astype(np.float64) @ W.astype(np.float64)
+        bits = np.unpackbits(wide.view(np.uint8), bitorder="little")
+        sure = np.abs(proj) > 1e-4
+        assert np.array_equal(bits[sure], (proj[sure] > 0).astype(np.uint8))
+
+
+def test_topk_at_the_top_of_the_wide_range():
+    """Boundaries at 255 and 256 (the values a byte-wide row cannot tell
+    apart) against brute force."""
+    for trial in range(30):
+        n = int(RNG.integers(1, 300))
+        d = RNG.choice([250, 254, 255, 256], size=n).astype(np.int32)
+        k = int(RNG.integers(1, n + 3))
+        assert oracle.topk(d, k).tolist() == brute_topk(d.tolist(), k)
+
+
+def test_wide_decode_head_complement_codes():
+    """Keys coded as the complement of the query code sit at distance 256,
+    one flipped bit back at 255: the oracle's selection over them is the
+    brute-force one (lower distance first, then lower index)."""
+    d = 128
+    W = (RNG.standard_normal((d, 256)) / math.sqrt(d)).astype(np.float32)
+    q = RNG.standard_normal(d).astype(np.float32)
+    qc = oracle.hash_vec(q, W)
+    n = 97
+    codes = np.tile(~qc, (n, 1))
+    flip = RNG.choice(n, 20, replace=False)
+    for i in flip:  # distance 255
+        w, b = divmod(int(RNG.integers(0, 256)), 32)
+        codes[i, w] ^= np.uint32(1 << b)
+    K = bf16_round_bits(RNG.standard_normal((n, d)).astype(np.float32))
+    V = bf16_round_bits(RNG.standard_normal((n, d)).astype(np.float32))
+    for k in (5, 20, 21, 60, n, n + 4):
+        oqc, odist, oidx, oout, m = oracle.decode_head(q, W, codes, K, V, n, k, 0.1)
+        assert np.array_equal(oqc, qc)
+        want = np.full(n, 256, np.int32)
+        want[flip] = 255
+        assert np.array_equal(odist, want)
+        assert oidx.tolist() == brute_topk(want.tolist(), k)
+        assert m == min(k, n)

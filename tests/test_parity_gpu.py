@@ -84,11 +84,11 @@ def test_append_code_and_position_check():
     assert int(err.item()) == H.HATA_FLAG_POS_RANGE
 
 
-@pytest.mark.parametrize("r", [32, 64])
+@pytest.mark.parametrize("r", [32, 64, 256])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_hash_keys_narrow_codes_bit_exact(r, dtype):
-    """r = 32 / 64 bit codes (the page's ablation widths), r/32 words per
-    token, against the oracle with the same r columns."""
+    """r = 32 / 64 / 256 bit codes (the page's other ablation widths), r/32
+    words per token, against the oracle with the same r columns."""
     g = torch.Generator(device="cuda").manual_seed(13 + r)
     B, Hkv, n_cap, pos0, n = 2, 3, 3001, 5, 2990
     K = _kv(dtype, (B, Hkv, n_cap, 128), g)
@@ -108,7 +108,7 @@ def test_hash_keys_narrow_codes_bit_exact(r, dtype):
                                            device="cuda"), 0, 1)
 
 
-@pytest.mark.parametrize("r", [32, 64])
+@pytest.mark.parametrize("r", [32, 64, 256])
 def test_append_code_narrow(r):
     g = torch.Generator(device="cuda").manual_seed(14 + r)
     B, Hkv, n_cap = 2, 3, 50
@@ -191,10 +191,11 @@ NARROW = [("llama31_8b_gqa_128k", dict(N=10000, topk=156, B=2)),  # stream-K att
           ("tiny_mha_4k", dict(N=4096))]                          # fp32 K/V
 
 
-@pytest.mark.parametrize("r", [32, 64])
+@pytest.mark.parametrize("r", [32, 64, 256])
 @pytest.mark.parametrize("case", range(len(NARROW)))
 def test_decode_narrow_codes(r, case, decode_mode):
-    """The whole decode step with r = 32 / 64 bit codes (distances 0..r)."""
+    """The whole decode step with r = 32 / 64 / 256 bit codes (distances
+    0..r)."""
     name, kw = NARROW[case]
     cfg = wl.scaled(wl.CONFIGS[name], **kw)
     run_and_check(cfg, seed=wl.SEED_BASE + 40 + case, steps=2, r=r)
