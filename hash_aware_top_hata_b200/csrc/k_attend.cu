@@ -745,14 +745,15 @@ cudaError_t launch_attend(AttendArgs &a, bool bf16, cudaStream_t s)
 }
 
 // The sequence-parallel step's attention (bf16): head_split CTAs per head,
-// enough to fill one wave of CTAs and to keep each CTA's part of a list
-// within kIdxCap; a.n_split (partial slots per head) bounds head_split.
+// as many as one wave of CTAs holds (at least one), and enough to keep each
+// CTA's part of a list within kIdxCap; a.n_split (partial slots per head)
+// bounds head_split.
 cudaError_t launch_attend_split(AttendArgs &a, cudaStream_t s)
 {
     int64_t P = 0;
     if (cudaError_t e = occupancy_grid(attend_head_kernel, tc::kThreads, tc::kSmem, &P)) return e;
     const int64_t heads = int64_t(a.B) * a.H_q;
-    int64_t split = std::max(ceil_div(a.topk, tc::kIdxCap), ceil_div(P, heads));
+    int64_t split = std::max(ceil_div(a.topk, tc::kIdxCap), std::max<int64_t>(P / heads, 1));
     if (split > a.n_split) split = a.n_split;
     if (split * heads >= (int64_t(1) << 31) || ceil_div(a.topk, split) > tc::kIdxCap)
         return cudaErrorInvalidValue;

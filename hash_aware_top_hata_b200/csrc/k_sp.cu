@@ -39,8 +39,10 @@ __global__ void __launch_bounds__(32 * kSpWarps) sp_hist_kernel(const uint32_t *
         const int bin = lane + 32 * e;
         if (bin >= kSpHistWords) break;
         uint32_t v = 0;
-        if (bin < stride)
-            for (int64_t t = 0; t < n_tiles; ++t) v += __ldg(row + t * stride + bin);
+        if (bin < stride) {
+#pragma unroll 8
+            for (int64_t t = 0; t < n_tiles; ++t) v += __ldg(row + t * stride + bin);  // 8 in flight
+        }
         out[bh * kSpHistWords + bin] = v;
     }
 }
@@ -70,7 +72,8 @@ __global__ void __launch_bounds__(32 * kSpWarps) sp_quota_kernel(const uint32_t 
     uint32_t mine[kSpBPL];
 #pragma unroll
     for (int e = 0; e < kSpBPL; ++e) tot[e] = before[e] = mine[e] = 0;
-    for (int w = 0; w < world; ++w) {
+#pragma unroll 4
+    for (int w = 0; w < world; ++w) {  // the loads of 4 ranks in flight together
         const uint32_t *row = hist_all + (int64_t(w) * BH + bh) * kSpHistWords;
 #pragma unroll
         for (int e = 0; e < kSpBPL; ++e) {
@@ -128,23 +131,51 @@ __global__ void __launch_bounds__(32 * kSpWarps) sp_quota_kernel(const uint32_t 
     }
 }
 
+// One warp per head.  Rounds of 32 ranks: lane w holds rank w's m and l, so
+// the maximum and the weights come from shuffles, and all the acc loads of a
+// round are issued before any is used (one memory round trip per round of
+// ranks, not one per rank).
 __global__ void __launch_bounds__(32 * kSpWarps) sp_merge_kernel(const float *part_all, int world,
                                                                  int64_t BH, float *out)
 {
+    constexpr int kRound = 8;  // ranks whose acc loads are in flight together
     const int lane = threadIdx.x & 31;
     const int64_t bh = int64_t(blockIdx.x) * kSpWarps + (threadIdx.x >> 5);
     if (bh >= BH) return;
+    auto rec = [&](int w) { return part_all + (int64_t(w) * BH + bh) * kPartStride; };
     float M = -INFINITY;
-    for (int w = 0; w < world; ++w) M = fmaxf(M, __ldg(part_all + (int64_t(w) * BH + bh) * kPartStride));
+    for (int w0 = 0; w0 < world; w0 += 32)
+        if (w0 + lane < world) M = fmaxf(M, __ldg(rec(w0 + lane)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (M != -INFINITY) {
-        for (int w = 0; w < world; ++w) {
-            const float *pp = part_all + (int64_t(w) * BH + bh) * kPartStride;
-            const float m = __ldg(pp);
-            const float wt = m == -INFINITY ? 0.0f : exp2f(m - M);
-            L = fmaf(__ldg(pp + 1), wt, L);
+        for (int w0 = 0; w0 < world; w0 += 32) {
+            const int w = w0 + lane;
+            float wt = 0.0f, lw = 0.0f;
+            if (w < world) {
+                const float m = __ldg(rec(w));
+                wt = m == -INFINITY ? 0.0f : exp2f(m - M);
+                lw = __ldg(rec(w) + 1) * wt;
+            }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) A[i] = fmaf(__ldg(pp + 4 + lane + 32 * i), wt, A[i]);
+            for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+            L += lw;
+            const int nw = world - w0 < 32 ? world - w0 : 32;
+            for (int j0 = 0; j0 < nw; j0 += kRound) {
+                float acc[kRound][4];
+#pragma unroll
+                for (int j = 0; j < kRound; ++j)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        acc[j][i] = j0 + j < nw ? __ldg(rec(w0 + j0 + j) + 4 + lane + 32 * i) : 0.0f;
+#pragma unroll
+                for (int j = 0; j < kRound; ++j) {
+                    const float wj = __shfl_sync(0xffffffffu, wt, (j0 + j) & 31);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) A[i] = fmaf(acc[j][i], j0 + j < nw ? wj : 0.0f, A[i]);
+                }
+            }
         }
     }
 #pragma unroll

@@ -16,8 +16,8 @@
 
 namespace hata {
 
-// Byte-wise zero test of four distances (bytes of w: 0..128 or the pad
-// 255) against T4 (one value in every byte), plain integer logic: bit 7 of
+// Byte-wise equality test of four distances (any byte values) against T4
+// (one value in every byte), plain integer logic: bit 7 of
 // each byte of the result is set iff the byte equals T; the other bits are
 // zero.  x = d ^ T is zero iff equal; (x & 0x7f) + 0x7f sets bit 7 iff the
 // low seven bits of x are not all zero (no carry out).
@@ -67,17 +67,25 @@ __device__ __forceinline__ void group_masks(const uint32_t (&dw)[8], uint32_t T4
     eq_out = le & ~lb;
 }
 
-// "< T" and "== T" masks of 32 consecutive distances for any T in 0..254
-// (the 256-bit codes, whose stored distances run 0..255): per-byte unsigned
-// compares, packed like group_masks.
+// "< T" and "== T" masks of 32 consecutive distances for any T in 0..255
+// (the 256-bit codes, whose stored distances run 0..255), packed like
+// group_masks.  Per byte, unsigned x < T: t = (x | 0x80) - (T & 0x7f) never
+// borrows across bytes and its bit 7 says "low seven bits of x >= those of
+// T", so x < T iff (x7 < T7) or (x7 == T7 and not that):
+// ((~x & T) | (~(x ^ T) & ~t)) & 0x80 -- plain integer logic (the SIMD
+// byte-compare intrinsics are emulated at many instructions each).
 __device__ __forceinline__ void group_masks_any(const uint32_t (&dw)[8], uint32_t T4,
                                                 uint32_t &lt_out, uint32_t &eq_out)
 {
+    const uint32_t tlow = T4 & 0x7f7f7f7fu;
     uint32_t lb = 0, lq = 0;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-        lb = __umulhi(lb, 0x80000000u) + (__vcmpltu4(dw[w], T4) & 0x80808080u);
-        lq = __umulhi(lq, 0x80000000u) + (__vcmpeq4(dw[w], T4) & 0x80808080u);
+        const uint32_t x = dw[w];
+        const uint32_t t = (x | 0x80808080u) - tlow;
+        const uint32_t lt = ((~x & T4) | (~(x ^ T4) & ~t)) & 0x80808080u;
+        lb = __umulhi(lb, 0x80000000u) + lt;
+        lq = __umulhi(lq, 0x80000000u) + byte_eq_mask(x, T4);
     }
     lt_out = lb;
     eq_out = lq;
