@@ -563,8 +563,18 @@ def wide_code_leg(dev, name="llama31_8b_gqa_128k"):
     torch.cuda.synchronize()
     H.hata_workspace_check(ws)
     us = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
+    # per-kernel breakdown: one more (untimed) step with events between kernels
+    kev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for e in kev:  # torch creates the CUDA event on first record; the library needs handles
+        e.record(stream)
+    torch.sum(flush_buf)
+    H.hata_decode_step(w.q[warm + timed - 1], W, codes, w.K, w.V, seq[warm + timed - 1], w.n_cap,
+                       cfg.topk, 1.0 / math.sqrt(128), ws, out, events=kev)
+    torch.cuda.synchronize()
+    names = ("prep", "score", "select", "attend", "combine")
+    kernels = {n: round(kev[i].elapsed_time(kev[i + 1]) * 1e3, 2) for i, n in enumerate(names)}
     step_bytes = B * Hkv * (N + warm + timed // 2) * 32 + B * Hq * cfg.topk * 2 * 256
-    res = {"us_per_step": round(us, 2), "steps": timed, "r": 256,
+    res = {"us_per_step": round(us, 2), "steps": timed, "r": 256, "kernels_us": kernels,
            "step_roofline_bytes": step_bytes,
            "step_frac_of_measured": round(step_bytes / (us * 1e-6) / 1e9 / peak, 4),
            "shape": f"{name} with 256-bit codes: B {B}, {Hq}/{Hkv} heads, context {N}, "

@@ -314,71 +314,127 @@ cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
 }
 
 // ------------------------------------------------------- r = 256 codes --
-// One CTA per (4096-token chunk, slab, group of <= 8 query heads); thread t
-// scores tokens 4t .. 4t+3 of each 1024-token quarter of the chunk (two
-// 16-byte halves of each 32-byte code, read once for all heads of the
-// group), stores the four distances of a head as one 32-bit word (a warp
-// writes 128 consecutive bytes) and counts them in a 257-bin shared
-// histogram per head, added to the chunk's tile histogram at the end.
+// The work is the flat sequence of 1024-token pieces of all (b, h_kv, group
+// of <= 8 query heads) slabs; CTA c takes one contiguous range of about
+// U / gridDim.x pieces (one CTA range per resident CTA, so the CTAs end
+// together).  In a piece, thread t scores tokens 4t .. 4t+3: their 32-byte
+// codes arrive by 16-byte asynchronous copies into a two-piece shared ring,
+// one piece ahead (each thread reads back only what it copied, so its own
+// wait is the only synchronisation), and are read once for all heads of the
+// group.  The four distances of a head go out as one 32-bit word (a warp
+// writes 128 consecutive bytes) and into a 257-bin shared histogram per
+// head; the histograms go to the (slab, 36K-token tile) rows in global
+// memory whenever the range moves to another tile, and at its end.
 constexpr int kWideThreads = 256;
-constexpr int kWideQuarter = 4 * kWideThreads;  // tokens per pass
-static_assert(kChunk == 4 * kWideQuarter, "four passes cover a chunk");
-static_assert(kTile % kChunk == 0, "a chunk lies in one histogram tile");
+constexpr int kWidePiece = 4 * kWideThreads;                      // tokens per piece
+constexpr size_t kWideRing = 2 * size_t(kWidePiece) * 2 * 16;    // two pieces of 32-byte codes
+static_assert(kTile % kWidePiece == 0, "a piece lies in one histogram tile");
 
-__global__ void __launch_bounds__(kWideThreads) score_wide_kernel(ScoreArgs a)
+__global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a)
 {
+    extern __shared__ __align__(16) uint4 ring[];  // [2][kWidePiece * 2]
     __shared__ uint32_t hist[kScoreHeads][kHistStrideWide];
     __shared__ uint4 qs[kScoreHeads][2];
     __shared__ uint2 qd[kScoreHeads][2];
     pdl_trigger();
     const int tid = threadIdx.x;
-    const int chunk = blockIdx.x;
-    const int slab = blockIdx.y;  // (b * H_kv + h) * zgroups + z
-    const int z = slab % a.zgroups, bhk = slab / a.zgroups;
-    const int h = bhk % a.H_kv, b = bhk / a.H_kv;
-    const int g0 = z * kScoreHeads;
-    const int ng = min(kScoreHeads, a.G - g0);
-    const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);  // step input
+    const int64_t per_slab = a.dist_row / kWidePiece;
+    const int64_t U = int64_t(a.B) * a.H_kv * a.zgroups * per_slab;
+    const int64_t f_beg = int64_t(blockIdx.x) * U / gridDim.x;
+    const int64_t f_end = int64_t(blockIdx.x + 1) * U / gridDim.x;
     for (int i = tid; i < kScoreHeads * kHistStrideWide; i += kWideThreads) (&hist[0][0])[i] = 0u;
-    const int64_t bh0 = int64_t(b) * a.H_q + int64_t(h) * a.G + g0;  // first head of the group
     pdl_wait();  // query codes, the appended key code, cleared tile histograms
-    if (tid < 2 * ng) {
-        const int g = tid >> 1, half = tid & 1;
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.qcodes + (bh0 + g) * 8) + half);
-        qs[g][half] = v;
-        const uint32_t q012 = v.x ^ v.y ^ v.z;
-        qd[g][half] = make_uint2(q012, q012 ^ v.w);
-    }
-    __syncthreads();
 
-    const uint4 *code = reinterpret_cast<const uint4 *>(a.codes) +
-                        ((int64_t(b) * a.H_kv + h) * a.n_cap) * 2;
-    const int64_t t00 = int64_t(chunk) * kChunk;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int64_t t0 = t00 + pass * kWideQuarter + 4 * tid;  // this thread's first token
-        uint4 k[4][2];
+    // copy this thread's four codes of piece f into ring slot `slot`
+    // (always commits one group; zero fill past the sequence end)
+    auto issue = [&](int64_t f, int slot) {
+        asm volatile("" ::: "memory");  // earlier reads of the ring stay before the copies
+        if (f < f_end) {
+            const int64_t slab = f / per_slab, t0 = (f - slab * per_slab) * kWidePiece + 4 * tid;
+            const int bhk = int(slab / a.zgroups), h = bhk % a.H_kv, b = bhk / a.H_kv;
+            const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.codes) +
+                               ((int64_t(b) * a.H_kv + h) * a.n_cap + t0) * 2;
+            const uint32_t dst = smem_addr(ring + size_t(slot) * kWidePiece * 2 + 8 * tid);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const bool in = t0 + (j >> 1) < len;
+                cp_async16_zfill(dst + 16u * j, in ? src + j : a.codes, in ? 16u : 0u);
+            }
+        }
+        cp_async_commit();
+    };
+
+    int64_t key = -1;    // (slab, tile) of the histograms being counted
+    int ng = 0;          // heads of that slab's group
+    int64_t bh0 = 0;     // its first query head
+    int64_t len = 0;
+    auto flush = [&]() {  // the counts so far to the tile rows, then cleared
+        __syncthreads();
+        const int64_t tile = key % a.n_tiles;
+        for (int i = tid; i < ng * kBinsWide; i += kWideThreads) {
+            const int g = i / kBinsWide, t = i % kBinsWide;
+            const uint32_t v = hist[g][t];
+            if (v) {
+                atomicAdd(a.hist + ((bh0 + g) * a.n_tiles + tile) * kHistStrideWide + t, v);
+                hist[g][t] = 0u;
+            }
+        }
+    };
+    issue(f_beg, 0);
+    for (int64_t f = f_beg; f < f_end; ++f) {
+        const int slot = int((f - f_beg) & 1);
+        issue(f + 1, slot ^ 1);
+        const int64_t slab = f / per_slab, piece = f - slab * per_slab;
+        const int64_t t00 = piece * kWidePiece;
+        const int64_t k = slab * a.n_tiles + t00 / kTile;
+        if (k != key) {  // CTA-uniform
+            if (key >= 0) flush();
+            const int z = int(slab % a.zgroups), bhk = int(slab / a.zgroups);
+            const int h = bhk % a.H_kv, b = bhk / a.H_kv;
+            const int g0 = z * kScoreHeads;
+            ng = min(kScoreHeads, a.G - g0);
+            bh0 = int64_t(b) * a.H_q + int64_t(h) * a.G + g0;
+            len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);
+            __syncthreads();  // the previous slab's query codes are no longer read
+            if (tid < 2 * ng) {
+                const int g = tid >> 1, half = tid & 1;
+                const uint4 v =
+                    __ldg(reinterpret_cast<const uint4 *>(a.qcodes + (bh0 + g) * 8) + half);
+                qs[g][half] = v;
+                const uint32_t q012 = v.x ^ v.y ^ v.z;
+                qd[g][half] = make_uint2(q012, q012 ^ v.w);
+            }
+            __syncthreads();
+            key = k;
+        }
+        const int64_t t0 = t00 + 4 * tid;  // this thread's first token
+        cp_async_wait<1>();                // its copies of piece f have landed
+        const uint4 *mine = ring + size_t(slot) * kWidePiece * 2 + 8 * tid;
+        uint4 kc[4][2];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const bool in = t0 + i < len;
-            k[i][0] = in ? __ldg(code + (t0 + i) * 2) : make_uint4(0u, 0u, 0u, 0u);
-            k[i][1] = in ? __ldg(code + (t0 + i) * 2 + 1) : make_uint4(0u, 0u, 0u, 0u);
+            kc[i][0] = mine[2 * i];
+            kc[i][1] = mine[2 * i + 1];
         }
         uint32_t k012[4][2], k0123[4][2];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                k012[i][hf] = k[i][hf].x ^ k[i][hf].y ^ k[i][hf].z;
-                k0123[i][hf] = k012[i][hf] ^ k[i][hf].w;
+                k012[i][hf] = kc[i][hf].x ^ kc[i][hf].y ^ kc[i][hf].z;
+                k0123[i][hf] = k012[i][hf] ^ kc[i][hf].w;
             }
         for (int g = 0; g < ng; ++g) {
+            const uint4 q0 = qs[g][0], q1 = qs[g][1];
+            const uint2 d0 = qd[g][0], d1 = qd[g][1];
             uint32_t word = 0u;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 uint32_t byte = kDistPad;
                 if (t0 + i < len) {
-                    const int d = hamming128(k[i][0], k012[i][0], k0123[i][0], qs[g][0], qd[g][0]) +
-                                  hamming128(k[i][1], k012[i][1], k0123[i][1], qs[g][1], qd[g][1]);
+                    const int d = hamming128(kc[i][0], k012[i][0], k0123[i][0], q0, d0) +
+                                  hamming128(kc[i][1], k012[i][1], k0123[i][1], q1, d1);
                     atomicAdd(&hist[g][d], 1u);
                     byte = d < 255 ? uint32_t(d) : 255u;
                 }
@@ -387,14 +443,8 @@ __global__ void __launch_bounds__(kWideThreads) score_wide_kernel(ScoreArgs a)
             __stcg(reinterpret_cast<uint32_t *>(a.dist + (bh0 + g) * a.dist_row + t0), word);
         }
     }
-    __syncthreads();
-    // add the non-zero bins to the chunk's tile histograms
-    const int64_t tile = t00 / kTile;
-    for (int i = tid; i < ng * kBinsWide; i += kWideThreads) {
-        const int g = i / kBinsWide, t = i % kBinsWide;
-        const uint32_t v = hist[g][t];
-        if (v) atomicAdd(a.hist + ((bh0 + g) * a.n_tiles + tile) * kHistStrideWide + t, v);
-    }
+    cp_async_wait<0>();
+    if (key >= 0) flush();
 }
 
 }  // namespace
@@ -402,11 +452,20 @@ __global__ void __launch_bounds__(kWideThreads) score_wide_kernel(ScoreArgs a)
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t s)
 {
     if (a.words == 8) {
-        if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(score_wide_kernel), 0))
+        if (cudaError_t e =
+                ensure_smem_attr(reinterpret_cast<const void *>(score_wide_kernel), kWideRing))
             return e;
-        const dim3 grid(unsigned(a.dist_row / kChunk),
-                        unsigned(int64_t(a.B) * a.H_kv * a.zgroups));
-        return launch_pdl(score_wide_kernel, grid, dim3(kWideThreads), 0, s, a);
+        int dev = 0, sms = 0, per_sm = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_wide_kernel,
+                                                              kWideThreads, kWideRing);
+        if (e != cudaSuccess) return e;
+        const int64_t U = int64_t(a.B) * a.H_kv * a.zgroups * (a.dist_row / kWidePiece);
+        const int64_t wave = int64_t(per_sm > 0 ? per_sm : 1) * sms;
+        return launch_pdl(score_wide_kernel, dim3(unsigned(U < wave ? U : wave)),
+                          dim3(kWideThreads), kWideRing, s, a);
     }
     const int gb = a.G < kScoreHeads ? a.G : kScoreHeads;
     if (a.words == 4) {

@@ -131,51 +131,51 @@ __global__ void __launch_bounds__(32 * kSpWarps) sp_quota_kernel(const uint32_t 
     }
 }
 
-// One warp per head.  Rounds of 32 ranks: lane w holds rank w's m and l, so
-// the maximum and the weights come from shuffles, and all the acc loads of a
-// round are issued before any is used (one memory round trip per round of
-// ranks, not one per rank).
+// One warp per head, an online merge over rounds of kRound ranks: all loads
+// of a round (lane j < kRound: rank j's m and l; every lane: its 4 output
+// dims of each rank's acc) are issued before any is used, so a step of up to
+// kRound ranks costs one memory round trip.
 __global__ void __launch_bounds__(32 * kSpWarps) sp_merge_kernel(const float *part_all, int world,
                                                                  int64_t BH, float *out)
 {
-    constexpr int kRound = 8;  // ranks whose acc loads are in flight together
+    constexpr int kRound = 8;
     const int lane = threadIdx.x & 31;
     const int64_t bh = int64_t(blockIdx.x) * kSpWarps + (threadIdx.x >> 5);
     if (bh >= BH) return;
     auto rec = [&](int w) { return part_all + (int64_t(w) * BH + bh) * kPartStride; };
-    float M = -INFINITY;
-    for (int w0 = 0; w0 < world; w0 += 32)
-        if (w0 + lane < world) M = fmaxf(M, __ldg(rec(w0 + lane)));
+    float M = -INFINITY, L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int w0 = 0; w0 < world; w0 += kRound) {
+        const bool mine = lane < kRound && w0 + lane < world;
+        const float mc = mine ? __ldg(rec(w0 + lane)) : -INFINITY;
+        const float lc = mine ? __ldg(rec(w0 + lane) + 1) : 0.0f;
+        float acc[kRound][4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (M != -INFINITY) {
-        for (int w0 = 0; w0 < world; w0 += 32) {
-            const int w = w0 + lane;
-            float wt = 0.0f, lw = 0.0f;
-            if (w < world) {
-                const float m = __ldg(rec(w));
-                wt = m == -INFINITY ? 0.0f : exp2f(m - M);
-                lw = __ldg(rec(w) + 1) * wt;
-            }
+        for (int j = 0; j < kRound; ++j)
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-            L += lw;
-            const int nw = world - w0 < 32 ? world - w0 : 32;
-            for (int j0 = 0; j0 < nw; j0 += kRound) {
-                float acc[kRound][4];
+            for (int i = 0; i < 4; ++i)
+                acc[j][i] = w0 + j < world ? __ldg(rec(w0 + j) + 4 + lane + 32 * i) : 0.0f;
+        float mr = mc;
 #pragma unroll
-                for (int j = 0; j < kRound; ++j)
+        for (int o = 16; o > 0; o >>= 1) mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+        const float Mn = fmaxf(M, mr);
+        if (Mn == -INFINITY) continue;  // warp-uniform: no weight yet
+        if (M != Mn) {
+            const float r = M == -INFINITY ? 0.0f : exp2f(M - Mn);
+            L *= r;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        acc[j][i] = j0 + j < nw ? __ldg(rec(w0 + j0 + j) + 4 + lane + 32 * i) : 0.0f;
+            for (int i = 0; i < 4; ++i) A[i] *= r;
+            M = Mn;
+        }
+        const float wc = mc == -INFINITY ? 0.0f : exp2f(mc - M);
+        float lw = lc * wc;
 #pragma unroll
-                for (int j = 0; j < kRound; ++j) {
-                    const float wj = __shfl_sync(0xffffffffu, wt, (j0 + j) & 31);
+        for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+        L += lw;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) A[i] = fmaf(acc[j][i], j0 + j < nw ? wj : 0.0f, A[i]);
-                }
-            }
+        for (int j = 0; j < kRound; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, wc, j);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) A[i] = fmaf(acc[j][i], wj, A[i]);
         }
     }
 #pragma unroll
