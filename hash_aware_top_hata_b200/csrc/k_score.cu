@@ -359,7 +359,8 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const bool in = t0 + (j >> 1) < len;
-                cp_async16_zfill(dst + 16u * j, in ? src + j : a.codes, in ? 16u : 0u);
+                cp_async16_zfill(dst + 16u * j, in ? static_cast<const void *>(src + j) : a.codes,
+                                 in ? 16u : 0u);
             }
         }
         cp_async_commit();
