@@ -318,10 +318,9 @@ cudaError_t launch_score_t(const ScoreArgs &a, cudaStream_t s)
 // of <= 8 query heads) slabs; CTA c takes one contiguous range of about
 // U / gridDim.x pieces (one CTA range per resident CTA, so the CTAs end
 // together).  In a piece, thread t scores tokens 4t .. 4t+3: their 32-byte
-// codes arrive by 16-byte asynchronous copies into a two-piece shared ring,
-// one piece ahead (each thread reads back only what it copied, so its own
-// wait is the only synchronisation), and are read once for all heads of the
-// group.  The four distances of a head go out as one 32-bit word (a warp
+// codes arrive by coalesced 16-byte asynchronous copies (each warp copies
+// its own 4 KB) into a two-piece shared ring, one piece ahead, and are read
+// once for all heads of the group.  The four distances of a head go out as one 32-bit word (a warp
 // writes 128 consecutive bytes) and into a 257-bin shared histogram per
 // head; the histograms go to the (slab, 36K-token tile) rows in global
 // memory whenever the range moves to another tile, and at its end.
@@ -345,21 +344,29 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
     for (int i = tid; i < kScoreHeads * kHistStrideWide; i += kWideThreads) (&hist[0][0])[i] = 0u;
     pdl_wait();  // query codes, the appended key code, cleared tile histograms
 
-    // copy this thread's four codes of piece f into ring slot `slot`
-    // (always commits one group; zero fill past the sequence end)
+    // copy the warp's 128 codes of piece f (4 KB) into ring slot `slot`:
+    // lane l takes 16-byte pieces l, l + 32, ... (coalesced), piece p of the
+    // warp (token p / 2, half p % 2) lands in row p / 8 (the lane that reads
+    // it: tokens 4 row .. 4 row + 3) at column (p % 8) ^ (row % 8), so each
+    // lane's 128-byte row reads back without bank conflicts.  Always commits
+    // one group; zero fill past the sequence end.
+    const int lane = tid & 31, warp = tid >> 5;
     auto issue = [&](int64_t f, int slot) {
         asm volatile("" ::: "memory");  // earlier reads of the ring stay before the copies
         if (f < f_end) {
-            const int64_t slab = f / per_slab, t0 = (f - slab * per_slab) * kWidePiece + 4 * tid;
+            const int64_t slab = f / per_slab;
+            const int64_t tw0 = (f - slab * per_slab) * kWidePiece + 128 * warp;  // warp's tokens
             const int bhk = int(slab / a.zgroups), h = bhk % a.H_kv, b = bhk / a.H_kv;
             const int64_t len = clamp_len(__ldg(a.seq_len + b), a.max_seq_len, a.n_cap);
             const uint4 *src = reinterpret_cast<const uint4 *>(a.codes) +
-                               ((int64_t(b) * a.H_kv + h) * a.n_cap + t0) * 2;
-            const uint32_t dst = smem_addr(ring + size_t(slot) * kWidePiece * 2 + 8 * tid);
+                               ((int64_t(b) * a.H_kv + h) * a.n_cap + tw0) * 2;
+            const uint32_t base = smem_addr(ring + size_t(slot) * kWidePiece * 2 + 256 * warp);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const bool in = t0 + (j >> 1) < len;
-                cp_async16_zfill(dst + 16u * j, in ? static_cast<const void *>(src + j) : a.codes,
+                const int p = lane + 32 * j, row = p >> 3;
+                const bool in = tw0 + (p >> 1) < len;
+                cp_async16_zfill(base + uint32_t(128 * row + 16 * ((p & 7) ^ (row & 7))),
+                                 in ? static_cast<const void *>(src + p) : a.codes,
                                  in ? 16u : 0u);
             }
         }
@@ -385,6 +392,7 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
     issue(f_beg, 0);
     for (int64_t f = f_beg; f < f_end; ++f) {
         const int slot = int((f - f_beg) & 1);
+        __syncwarp();  // every lane is done reading the slot the next copies overwrite
         issue(f + 1, slot ^ 1);
         const int64_t slab = f / per_slab, piece = f - slab * per_slab;
         const int64_t t00 = piece * kWidePiece;
@@ -410,13 +418,14 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
             key = k;
         }
         const int64_t t0 = t00 + 4 * tid;  // this thread's first token
-        cp_async_wait<1>();                // its copies of piece f have landed
-        const uint4 *mine = ring + size_t(slot) * kWidePiece * 2 + 8 * tid;
+        cp_async_wait<1>();                // this lane's copies of piece f have landed
+        __syncwarp();                      // and so have the other lanes'
+        const uint4 *mine = ring + size_t(slot) * kWidePiece * 2 + 8 * tid;  // row `lane`
         uint4 kc[4][2];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            kc[i][0] = mine[2 * i];
-            kc[i][1] = mine[2 * i + 1];
+            kc[i][0] = mine[(2 * i) ^ (lane & 7)];
+            kc[i][1] = mine[(2 * i + 1) ^ (lane & 7)];
         }
         uint32_t k012[4][2], k0123[4][2];
 #pragma unroll
