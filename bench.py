@@ -246,9 +246,9 @@ def profiled_traffic(cfg, kernel: str, src: str):
     return round(float(m_traffic.group(1)) * 1e6) if now == m_hash.group(1) else None
 
 
-def config_dict(cfg, l2: str) -> dict:
+def config_dict(cfg, l2: str, rbit: int = 128) -> dict:
     return {"workload": cfg.name, "B": cfg.B, "H_q": cfg.H_q, "H_kv": cfg.H_kv,
-            "context": cfg.N, "topk": cfg.topk, "head_dim": 128, "rbit": 128,
+            "context": cfg.N, "topk": cfg.topk, "head_dim": 128, "rbit": rbit,
             "kv_dtype": cfg.kv_dtype, "tokens_appended_per_step": 1, "l2": l2}
 
 
@@ -677,8 +677,10 @@ def run_hata(args, world, rank, local):
     w = wl.make_workload(cfg, seed, device=dev, steps=total_steps)
     B, Hq, Hkv, N = cfg.B, cfg.H_q, cfg.H_kv, cfg.N
     scale = 1.0 / math.sqrt(128)
-    codes = torch.zeros((B, Hkv, w.n_cap, 4), dtype=torch.int32, device=dev)
-    H.hata_hash_keys(w.K, w.W_H, codes, 0, N)
+    r = args.rbit
+    W = wl.projection(w.W_H, r)  # r = 128: the workload's W_H itself
+    codes = torch.zeros((B, Hkv, w.n_cap, r // 32), dtype=torch.int32, device=dev)
+    H.hata_hash_keys(w.K, W, codes, 0, N)
     ws = torch.empty(H.hata_decode_workspace_size(B, Hq, Hkv, w.n_cap, cfg.topk),
                      dtype=torch.uint8, device=dev)
     out = torch.empty((B, Hq, 128), device=dev)
@@ -690,7 +692,7 @@ def run_hata(args, world, rank, local):
     kv_elt = 2 if cfg.kv_dtype == "bf16" else 4
 
     def step(t, events=None):
-        H.hata_decode_step(w.q[t], w.W_H, codes, w.K, w.V, seq[t], w.n_cap, cfg.topk, scale,
+        H.hata_decode_step(w.q[t], W, codes, w.K, w.V, seq[t], w.n_cap, cfg.topk, scale,
                            ws, out, k_new=w.k_new[t], v_new=w.v_new[t], events=events)
 
     # clocks are sampled from the warm-up on, through the timed region
@@ -756,7 +758,7 @@ def run_hata(args, world, rank, local):
     peak, peak_kind = measured_peaks()
     kv_row = 128 * kv_elt
     attend_bytes = B * Hq * cfg.topk * 2 * kv_row           # selected K and V rows
-    code_bytes = B * Hkv * (N + W_steps + K_steps // 2) * 16  # every code once per KV head
+    code_bytes = B * Hkv * (N + W_steps + K_steps // 2) * (r // 8)  # every code once per KV head
     attend_s = statistics.mean(attend_ms) / 1e3
     score_s = statistics.mean(score_ms) / 1e3
     step_bytes = attend_bytes + code_bytes
@@ -776,7 +778,7 @@ def run_hata(args, world, rank, local):
         "steps": K_steps, "warmup": W_steps, "ms_per_step": round(ms_max, 5),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian q/K/V, 2% planted keys, N(0,1/128) W_H)",
-        "config": config_dict(cfg, "flushed before every timed step (512 MiB read)"),
+        "config": config_dict(cfg, "flushed before every timed step (512 MiB read)", r),
         "roofline": {"bound": "hbm", "kernel": roof_what,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
@@ -860,6 +862,8 @@ def main():
     ap.add_argument("--context", type=int, default=0, help="override the context length")
     ap.add_argument("--batch", type=int, default=0, help="override the batch size")
     ap.add_argument("--topk", type=int, default=0, help="override the top-k budget")
+    ap.add_argument("--rbit", type=int, default=128, choices=[32, 64, 128, 256],
+                    help="hash width of the timed steps (other than 128: with --no-extras)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e, dense and CPU legs (profiling runs)")
     ap.add_argument("--no-other-configs", action="store_true",
@@ -870,6 +874,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.rbit != 128 and not args.no_extras:
+        ap.error("--rbit other than 128 runs the timed steps only: add --no-extras")
     world, rank, local = dist_setup(args)
     if args.impl == "hata":
         H.hata_set_decode_mode({"auto": H.HATA_MODE_AUTO, "fused": H.HATA_MODE_FUSED,

@@ -417,7 +417,6 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
             __syncthreads();
             key = k;
         }
-        const int64_t t0 = t00 + 4 * tid;  // this thread's first token
         cp_async_wait<1>();                // this lane's copies of piece f have landed
         __syncwarp();                      // and so have the other lanes'
         const uint4 *mine = ring + size_t(slot) * kWidePiece * 2 + 8 * tid;  // row `lane`
@@ -435,22 +434,29 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
                 k012[i][hf] = kc[i][hf].x ^ kc[i][hf].y ^ kc[i][hf].z;
                 k0123[i][hf] = k012[i][hf] ^ kc[i][hf].w;
             }
+        // this thread's first token and how many of its four hold keys (32-bit:
+        // rows are shorter than 2^31)
+        const int t0 = int(t00) + 4 * tid;
+        const int nv = int(len) - t0;
+        uint8_t *drow = a.dist + bh0 * a.dist_row + t0;  // head g: + g * dist_row
+        const uint32_t hbase = smem_addr(&hist[0][0]);
         for (int g = 0; g < ng; ++g) {
             const uint4 q0 = qs[g][0], q1 = qs[g][1];
             const uint2 d0 = qd[g][0], d1 = qd[g][1];
+            const uint32_t hb = hbase + uint32_t(g * kHistStrideWide * 4);
             uint32_t word = 0u;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint32_t byte = kDistPad;
-                if (t0 + i < len) {
-                    const int d = hamming128(kc[i][0], k012[i][0], k0123[i][0], q0, d0) +
-                                  hamming128(kc[i][1], k012[i][1], k0123[i][1], q1, d1);
-                    atomicAdd(&hist[g][d], 1u);
-                    byte = d < 255 ? uint32_t(d) : 255u;
-                }
-                word |= byte << (8 * i);
+                // zero-filled codes past the sequence end are scored too and
+                // then neither counted nor stored
+                const uint32_t d =
+                    uint32_t(hamming128(kc[i][0], k012[i][0], k0123[i][0], q0, d0) +
+                             hamming128(kc[i][1], k012[i][1], k0123[i][1], q1, d1));
+                const bool v = i < nv;
+                if (v) asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(hb + 4u * d) : "memory");
+                word |= (v ? d - (d >> 8) : uint32_t(kDistPad)) << (8 * i);  // 256 saturates to 255
             }
-            __stcg(reinterpret_cast<uint32_t *>(a.dist + (bh0 + g) * a.dist_row + t0), word);
+            __stcg(reinterpret_cast<uint32_t *>(drow + g * a.dist_row), word);
         }
     }
     cp_async_wait<0>();
