@@ -737,10 +737,13 @@ def run_hata(args, world, rank, local):
     select_ms = [e[2].elapsed_time(e[3]) for e in kevs]
     attend_ms = [e[3].elapsed_time(e[4]) for e in kevs]
     combine_ms = [e[4].elapsed_time(e[5]) for e in kevs]
-    n_launch = H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.topk, w.K.dtype)
+    n_launch = H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.H_kv, w.n_cap, cfg.topk, w.K.dtype,
+                                             r)
     fused = n_launch == 3
+    cluster = n_launch == 1
     # four launches: one CTA per head, merged in shared memory
-    attend_kernel = ("fused_select_attend_kernel" if fused else
+    attend_kernel = ("cluster_step_kernel" if cluster else
+                     "fused_select_attend_kernel" if fused else
                      "attend_head_kernel" if n_launch == 4 else "attend_tc_kernel")
     split_ms = [e[0].elapsed_time(e[5]) for e in kevs]
     ms = statistics.mean(step_ms)
@@ -763,7 +766,13 @@ def run_hata(args, world, rank, local):
     score_s = statistics.mean(score_ms) / 1e3
     step_bytes = attend_bytes + code_bytes
     fused_s = statistics.mean(select_ms) / 1e3  # fused step: the selection + attention kernel
-    if fused:
+    cluster_s = statistics.mean(prep_ms) / 1e3  # cluster step: its one kernel
+    if cluster:
+        # the one kernel of the step moves every code and the selected K/V rows
+        roof_bytes, roof_s = step_bytes, cluster_s
+        roof_src = "hash_aware_top_hata_b200/csrc/k_cluster.cu"
+        roof_what = "cluster_step_kernel (hash + score + top-k + gather + softmax)"
+    elif fused:
         # the selection + attention kernel moves the selected K/V rows
         roof_bytes, roof_s = attend_bytes, fused_s
         roof_src = "hash_aware_top_hata_b200/csrc/k_fused.cu"
@@ -787,7 +796,8 @@ def run_hata(args, world, rank, local):
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
                           "frac_of_measured": round(step_bytes / (ms / 1e3) / 1e9 / peak, 4),
                           "frac_of_8000": round(step_bytes / (ms / 1e3) / 1e9 / 8000.0, 4)},
-        "kernels_us": ({"prep": round(statistics.mean(prep_ms) * 1e3, 2),
+        "kernels_us": ({"cluster_step": round(cluster_s * 1e6, 2)} if cluster else
+                       {"prep": round(statistics.mean(prep_ms) * 1e3, 2),
                         "score": round(score_s * 1e6, 2),
                         "select_attend": round(fused_s * 1e6, 2),
                         "sum_with_events": round(statistics.mean(split_ms) * 1e3, 2),
@@ -868,7 +878,8 @@ def main():
                     help="skip the e2e, dense and CPU legs (profiling runs)")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the side measurements of the other large workloads")
-    ap.add_argument("--decode-mode", default="auto", choices=["auto", "multi_kernel", "fused"],
+    ap.add_argument("--decode-mode", default="auto",
+                    choices=["auto", "multi_kernel", "fused", "cluster"],
                     help="step implementation: auto (the library's choice), the multi-kernel "
                          "step or the fused step")
     args = ap.parse_args()
@@ -879,7 +890,8 @@ def main():
     world, rank, local = dist_setup(args)
     if args.impl == "hata":
         H.hata_set_decode_mode({"auto": H.HATA_MODE_AUTO, "fused": H.HATA_MODE_FUSED,
-                                "multi_kernel": H.HATA_MODE_MULTI_KERNEL}[args.decode_mode])
+                                "multi_kernel": H.HATA_MODE_MULTI_KERNEL,
+                                "cluster": H.HATA_MODE_CLUSTER}[args.decode_mode])
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)

@@ -20,8 +20,9 @@ thread_local char g_err[512];
 std::atomic<int> g_mode{HATA_MODE_AUTO};
 std::atomic<uint64_t> g_wait_ns{1000000000ull};
 
-// Which step HATA_MODE_AUTO picks for bf16 caches (the faster one on B200).
+// Which steps HATA_MODE_AUTO picks for bf16 caches (the faster ones on B200).
 constexpr bool kAutoFused = false;
+constexpr bool kAutoCluster = true;
 
 // The fused step serves bf16 K/V caches with codes of up to 128 bits when
 // asked for (or chosen by AUTO); fp32 caches and 256-bit codes always take
@@ -31,6 +32,15 @@ bool use_fused(hata_dtype_t kv_dtype, int r)
     const int m = g_mode.load();
     return kv_dtype == HATA_DT_BF16 && r <= kRbit &&
            (m == HATA_MODE_FUSED || (m == HATA_MODE_AUTO && kAutoFused));
+}
+
+// The cluster step serves bf16 caches with 128-bit codes when the mode asks
+// for it (or AUTO picks it) and the sizes fit (cluster_step_fits).
+bool want_cluster(hata_dtype_t kv_dtype, int r)
+{
+    const int m = g_mode.load();
+    return kv_dtype == HATA_DT_BF16 && r == kRbit &&
+           (m == HATA_MODE_CLUSTER || (m == HATA_MODE_AUTO && kAutoCluster));
 }
 
 hata_status_t fail(hata_status_t st, const char *fmt, ...)
@@ -117,7 +127,7 @@ cudaError_t ensure_smem_attr(const void *func, size_t bytes)
 
 extern "C" {
 
-int hata_abi_version(void) { return 3; }
+int hata_abi_version(void) { return 4; }
 
 const char *hata_status_string(int status)
 {
@@ -135,7 +145,8 @@ const char *hata_last_error(void) { return g_err; }
 
 hata_status_t hata_set_decode_mode(int mode)
 {
-    if (mode != HATA_MODE_AUTO && mode != HATA_MODE_MULTI_KERNEL && mode != HATA_MODE_FUSED)
+    if (mode != HATA_MODE_AUTO && mode != HATA_MODE_MULTI_KERNEL && mode != HATA_MODE_FUSED &&
+        mode != HATA_MODE_CLUSTER)
         return fail(HATA_ERR_INVALID_ARG, "decode mode %d", mode);
     g_mode.store(mode);
     return ok();
@@ -221,14 +232,24 @@ int64_t hata_dist_row_bytes(int64_t max_seq_len)
     return max_seq_len <= 0 ? 0 : ceil_div(max_seq_len, kChunk) * kChunk;
 }
 
-int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
+int hata_decode_kernel_launches(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
+                                hata_dtype_t kv_dtype, int r)
 {
-    if (B <= 0 || H_q <= 0 || topk <= 0 || !valid_dtype(kv_dtype)) {
-        fail(HATA_ERR_INVALID_ARG, "B=%d H_q=%d topk=%d kv_dtype=%d", B, H_q, topk,
-             int(kv_dtype));
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv || max_seq_len <= 0 || topk <= 0 ||
+        !valid_dtype(kv_dtype) || (r != 32 && r != 64 && r != kRbit && r != kRbitWide)) {
+        fail(HATA_ERR_INVALID_ARG, "B=%d H_q=%d H_kv=%d max_seq_len=%lld topk=%d kv_dtype=%d r=%d",
+             B, H_q, H_kv, (long long)max_seq_len, topk, int(kv_dtype), r);
         return -1;
     }
-    if (use_fused(kv_dtype, kRbit)) return 3;  // prep, score, the selection + attention kernel
+    if (use_fused(kv_dtype, r)) return 3;  // prep, score, the selection + attention kernel
+    if (want_cluster(kv_dtype, r)) {
+        ClusterPlan plan;
+        if (cudaError_t e = cluster_step_plan(B, H_q, H_kv, max_seq_len, topk, &plan)) {
+            cuda_fail(e, "cluster occupancy query");
+            return -1;
+        }
+        if (plan.kM) return 1;
+    }
     int n = 0;
     if (cudaError_t e = attend_launch_count(B, H_q, topk, kv_dtype == HATA_DT_BF16, &n)) {
         cuda_fail(e, "occupancy query");
@@ -446,13 +467,52 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const StepBufs sb = step_bufs(ws, L, q_codes, dist, dist_row_bytes, sel_idx);
     const Events ev{events, s};
+    cudaError_t e;
+    if (want_cluster(kv_dtype, r)) {
+        ClusterPlan plan;
+        if ((e = cluster_step_plan(B, H_q, H_kv, max_seq_len, topk, &plan)) != cudaSuccess)
+            return cuda_fail(e, "cluster occupancy query");
+        if (plan.kM) {
+            ClusterArgs ca{};
+            ca.q = q;
+            ca.W = W_H;
+            ca.codes = codes;
+            ca.K = K;
+            ca.V = V;
+            ca.k_new = k_new;
+            ca.v_new = v_new;
+            ca.seq_len = seq_len;
+            ca.q_out = q_codes;
+            ca.dist = dist;
+            ca.dist_row = dist_row_bytes;
+            ca.idx = sb.idx;
+            ca.out = out;
+            ca.flags = sb.flags;
+            ca.ws_header = reinterpret_cast<uint32_t *>(ws);
+            ca.n_cap = n_cap;
+            ca.max_seq_len = max_seq_len;
+            ca.B = B;
+            ca.H_q = H_q;
+            ca.H_kv = H_kv;
+            ca.G = H_q / H_kv;
+            ca.topk = topk;
+            ca.tok_per_cta = plan.tok_per_cta;
+            ca.scale_log2 = scale * 1.4426950408889634f;
+            if ((e = ev.record(0)) != cudaSuccess) return cuda_fail(e, "event record");
+            if ((e = launch_cluster_step(ca, plan, s)) != cudaSuccess)
+                return cuda_fail(e, "cluster step launch");
+            // one kernel does the work of all five: its end is recorded for each
+            for (int i = 1; i <= 5; ++i)
+                if ((e = ev.record(i)) != cudaSuccess) return cuda_fail(e, "event record");
+            return ok();
+        }
+    }
     const bool fused = use_fused(kv_dtype, r);
     uint32_t *sync = reinterpret_cast<uint32_t *>(ws + L.off_sync);
     if (hata_status_t st = enqueue_front(q, W_H, codes, K, V, kv_dtype, n_cap, seq_len,
                                          max_seq_len, k_new, v_new, B, H_q, H_kv, r, L, sb, ws,
                                          fused ? sync : nullptr, ev))
         return st;
-    cudaError_t e;
 
     if (fused) {
         FusedArgs fa{};

@@ -210,6 +210,38 @@ struct FusedArgs {
     uint64_t spin_limit_ns;  // bound of every wait
 };
 
+// The cluster step (one kernel per decode step for heads whose cache fits a
+// thread-block cluster of up to kClusterMaxC CTAs of 8192 tokens each).
+constexpr int kClusterMaxG = 4;   // query heads per KV head it serves (1, 2 or 4)
+constexpr int kClusterMaxC = 8;   // CTAs per cluster (portable cluster size)
+
+struct ClusterArgs {
+    const float *q;          // [B][H_q][128]; device or mapped host
+    const float *W;          // [H_kv][128][128]
+    uint32_t *codes;         // [B][H_kv][n_cap][4]; the new key's code is written
+    void *K, *V;             // bf16 caches; the new rows written if v_new
+    const void *k_new;       // [B][H_kv][128] bf16 or null
+    const void *v_new;       // [B][H_kv][128] bf16 or null
+    const int32_t *seq_len;
+    uint32_t *q_out;         // [B][H_q][4] or null
+    uint8_t *dist;           // caller's distance rows or null
+    int64_t dist_row;
+    int32_t *idx;            // [B][H_q][topk]
+    float *out;              // [B][H_q][128]; device or mapped host
+    uint32_t *flags;         // per-b flag words
+    uint32_t *ws_header;     // {magic, B}
+    int64_t n_cap, max_seq_len;
+    int B, H_q, H_kv, G, topk;
+    int tok_per_cta;         // tokens of a CTA's range (a multiple of 32; the plan's)
+    float scale_log2;
+};
+
+// How the cluster step covers a head: kM = 0 (it does not), else CTAs of up
+// to 8192 kM tokens, C of them per (b, h_kv), tok_per_cta tokens each.
+struct ClusterPlan {
+    int kM = 0, C = 0, tok_per_cta = 0;
+};
+
 struct DenseArgs {
     const float *q;
     const void *K, *V;
@@ -297,6 +329,11 @@ cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s);
 cudaError_t attend_launch_count(int B, int H_q, int topk, bool bf16, int *n);
 cudaError_t launch_dense(const DenseArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_fused(const FusedArgs &a, cudaStream_t s);
+// The cluster step's plan for these sizes on this device (bf16 K/V and
+// r = 128 are the caller's checks); plan->kM == 0 when it does not serve them.
+cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
+                              ClusterPlan *plan);
+cudaError_t launch_cluster_step(const ClusterArgs &a, const ClusterPlan &p, cudaStream_t s);
 // Sequence-parallel step: the attention of one shard's selected keys split
 // over several CTAs per head (bf16; fp32 caches take launch_attend with
 // a.k_head), partials merged by launch_combine into a.part_out.

@@ -1,0 +1,523 @@
+// k_cluster.cu -- the whole decode step in ONE kernel for heads whose cache
+// fits a thread-block cluster: one cluster of C <= 8 CTAs per (batch row,
+// KV head), CTA r owning tokens [8192 r, 8192 (r + 1)) of the slab.
+//
+// HATA review page (arXiv 2506.02572): "What carries the argument" (hash
+// q, XOR + popcount against every cached key code, attention over the
+// top-k keys only), Figure 2 caption (Algorithm 1: the key code cache,
+// extended by one token per decode step), referee report, major comment 1
+// (Algorithm 3: a threshold top-k over the r + 1 Hamming values; boundary
+// ties here go to the lower token index).
+//
+// Small problems (a few heads, tens of thousands of keys) are bound by the
+// latency of kernel boundaries, not by bytes: the multi-kernel step runs
+// four or five dependent kernels, each paying its launch, its first memory
+// round trip and its grid-completion flush.  Here each CTA runs every step
+// on its own tokens and the CTAs of a cluster meet twice, through
+// distributed shared memory instead of global memory:
+//
+//   1. every CTA hashes the G query heads of its KV head (the same fp32
+//      chain as the prep kernel, so codes are bit-exact) and, if its range
+//      holds the new token, appends its code and K/V rows;
+//   2. it scores its tokens against all G heads: distances stay in shared
+//      memory (copied to the caller's rows only when asked for), counts go
+//      to a shared histogram per head;
+//   3. cluster barrier; every CTA reads the C histograms of its head group
+//      from the other CTAs' shared memory: the sum gives T and #(< T), the
+//      CTAs before it the keys below T and at T it must skip -- the same
+//      placement arithmetic as the tile CTAs of the selection kernel;
+//   4. it selects its share (byte-wise masks, one block scan per head) into
+//      the head's index list, ascending;
+//   5. its warps gather and attend its selected rows (G heads side by side,
+//      8 / G warps each, the tensor-core stage of attend_common.cuh) and
+//      merge them into one partial (m, l, acc) per head, written into the
+//      shared memory of the cluster's first CTA;
+//   6. cluster barrier; the first CTA merges the C partials per head into
+//      out.
+//
+// Every CTA of a cluster is resident at once (the hardware schedules a
+// cluster as a unit), so the two barriers cannot wait on a CTA that never
+// runs.  bf16 K/V, r = 128, G in {1, 2, 4}.
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "hata_internal.cuh"
+#include "async_copy.cuh"
+#include "attend_common.cuh"
+#include "score_common.cuh"
+#include "select_common.cuh"
+
+namespace hata {
+namespace {
+
+namespace cg = cooperative_groups;
+
+constexpr int kCThreads = 256;
+constexpr int kCWarps = kCThreads / 32;
+constexpr int kCRing = 2;                    // attention stages per warp ring
+constexpr size_t kCRingBytes = size_t(kCWarps) * kCRing * tc::kStageBytes;
+
+// kM: a CTA holds up to 8192 kM tokens, 32 kM per thread in the selection
+template <int kM>
+struct ClusterSmem {
+    static constexpr int kTok = 8192 * kM;
+    uint8_t ring[kCRingBytes];                        // attention rings (phase 5)
+    uint8_t dist[kClusterMaxG][kTok];                 // this CTA's distances
+    uint32_t hist[kClusterMaxG][kHistStride];         // and their histograms
+    float q[kClusterMaxG][kD];                        // the query rows
+    float part[kCWarps][kPartStride];                 // warp partials
+    float merged[kClusterMaxC][kClusterMaxG][kPartStride];  // CTA partials (first CTA)
+    uint32_t qcode[kClusterMaxG][4];
+    int2 scan[kCWarps + 1];
+    int sel[kClusterMaxG][4];                         // T, n_less, start, count per head
+};
+
+// The fp32 chain acc = fmaf(x_i, W[i][j], acc), i = 0..127, of bit j of the
+// code of row x (shared memory) with one head's W ([128][128], global).
+__device__ __forceinline__ bool hash_bit(const float *x, const float *Wh, int j)
+{
+    float acc = 0.0f;
+#pragma unroll 16
+    for (int i = 0; i < kD; ++i) acc = __fmaf_rn(x[i], __ldg(Wh + i * kRbit + j), acc);
+    return acc > 0.0f;
+}
+
+template <int kM>
+__global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs a)
+{
+    constexpr int kCTok = ClusterSmem<kM>::kTok;  // token capacity of a CTA
+    constexpr int kCPer = kCTok / kCThreads;      // tokens per thread in the selection
+    constexpr int kGroups = kCPer / 32;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    ClusterSmem<kM> &S = *reinterpret_cast<ClusterSmem<kM> *>(smem_raw);
+    cg::cluster_group cl = cg::this_cluster();
+    const int C = int(cl.num_blocks());
+    const int rank = int(cl.block_rank());
+    const int slab_id = int(blockIdx.x) / C;  // b * H_kv + h
+    const int b = slab_id / a.H_kv, h = slab_id - b * a.H_kv;
+    const int G = a.G;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t bh0 = int64_t(b) * a.H_q + int64_t(h) * G;  // first query head
+    const int64_t slab = (int64_t(b) * a.H_kv + h) * a.n_cap;  // first K/V row and code
+    const int32_t sl = a.seq_len[b];
+    const int len = int(clamp_len(sl, a.max_seq_len, a.n_cap));
+    const int t_beg = rank * a.tok_per_cta;                    // this CTA's range of the slab
+    const int nloc = min(max(len - t_beg, 0), a.tok_per_cta);  // the tokens of it that hold keys
+    const float *Wh = a.W + size_t(h) * kD * kRbit;
+
+    // ---- 1. query rows, their codes, the append, the flags ----
+    for (int i = tid; i < G * kD; i += kCThreads)
+        S.q[i / kD][i % kD] = a.q[(bh0 + i / kD) * kD + i % kD];
+    for (int i = tid; i < G * kHistStride; i += kCThreads) (&S.hist[0][0])[i] = 0u;
+    if (a.ws_header && blockIdx.x == 0 && tid == 0) {
+        a.ws_header[0] = kWsMagic;
+        a.ws_header[1] = uint32_t(a.B);
+    }
+    if (rank == 0 && h == 0 && tid == 0) {
+        uint32_t f = 0;
+        if (sl < 0 || sl > a.max_seq_len || sl > a.n_cap) f |= HATA_FLAG_SEQ_LEN_RANGE;
+        if (a.k_new && (int64_t(sl) - 1 < 0 || int64_t(sl) - 1 >= a.n_cap)) f |= HATA_FLAG_POS_RANGE;
+        a.flags[b] = f;
+    }
+    // the new token (at seq_len - 1) belongs to the CTA whose range holds it;
+    // a position past every range (a length beyond max_seq_len) to the last
+    const int64_t pos = int64_t(sl) - 1;
+    const bool append = a.k_new && pos >= 0 && pos < a.n_cap &&
+                        min(int(pos / a.tok_per_cta), C - 1) == rank;
+    __syncthreads();
+    // 2G chains of 128 steps over the 256 threads (G <= 4: at most two each),
+    // plus the appended key's 128 in the CTA that owns it
+    {
+        const int j = tid & (kRbit - 1);
+        for (int g = tid >> 7; g < G; g += 2) {
+            const bool bit = hash_bit(S.q[g], Wh, j);
+            const uint32_t word = __ballot_sync(0xffffffffu, bit);
+            if (lane == 0) S.qcode[g][j >> 5] = word;
+        }
+    }
+    if (append) {
+        // stage k_new (bf16, widened exactly) in the merge buffer, then hash
+        float *xk = S.merged[0][0];
+        const uint16_t *kn = static_cast<const uint16_t *>(a.k_new) + (int64_t(b) * a.H_kv + h) * kD;
+        for (int i = tid; i < kD; i += kCThreads) xk[i] = __uint_as_float(uint32_t(kn[i]) << 16);
+        __syncthreads();
+        if (tid < kRbit) {
+            const bool bit = hash_bit(xk, Wh, tid);
+            const uint32_t word = __ballot_sync(0xffffffffu, bit);
+            if (lane == 0) a.codes[(slab + pos) * 4 + (tid >> 5)] = word;
+        }
+        if (a.v_new && tid >= kRbit) {  // K and V rows of the new token
+            const int e = tid - kRbit;  // 0..127
+            const uint16_t *vn =
+                static_cast<const uint16_t *>(a.v_new) + (int64_t(b) * a.H_kv + h) * kD;
+            static_cast<uint16_t *>(a.K)[(slab + pos) * kD + e] = kn[e];
+            static_cast<uint16_t *>(a.V)[(slab + pos) * kD + e] = vn[e];
+        }
+    }
+    __syncthreads();
+    if (a.q_out && rank == 0)
+        for (int i = tid; i < G * 4; i += kCThreads) a.q_out[(bh0 + i / 4) * 4 + i % 4] = S.qcode[i / 4][i % 4];
+
+    // ---- 2. scores of this CTA's tokens (token t_beg + tid + 256 m) ----
+    {
+        uint4 qv[kClusterMaxG];
+        uint2 qd[kClusterMaxG];
+#pragma unroll
+        for (int g = 0; g < kClusterMaxG; ++g) {
+            const uint32_t *c = S.qcode[g < G ? g : 0];
+            qv[g] = make_uint4(c[0], c[1], c[2], c[3]);
+            const uint32_t q012 = c[0] ^ c[1] ^ c[2];
+            qd[g] = make_uint2(q012, q012 ^ c[3]);
+        }
+        const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes) + slab + t_beg;
+        constexpr int kBatch = 8;  // tokens whose loads are in flight together
+        for (int m0 = 0; m0 < kCPer; m0 += kBatch) {
+            uint4 kv[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int t = tid + kCThreads * (m0 + u);
+                // plain loads: the appended code was written by this kernel
+                kv[u] = t < nloc ? codes[t] : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int t = tid + kCThreads * (m0 + u);
+                const uint32_t k012 = kv[u].x ^ kv[u].y ^ kv[u].z, k0123 = k012 ^ kv[u].w;
+#pragma unroll
+                for (int g = 0; g < kClusterMaxG; ++g) {
+                    if (g < G) {
+                        uint8_t byte = kDistPad;
+                        if (t < nloc) {
+                            const int d = hamming128(kv[u], k012, k0123, qv[g], qd[g]);
+                            atomicAdd(&S.hist[g][d], 1u);
+                            byte = uint8_t(d);
+                        }
+                        S.dist[g][t] = byte;
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (a.dist) {  // the caller's distance rows: this CTA's part of them (the last
+                   // CTA's up to the row's end)
+        const int64_t row_len = a.dist_row;
+        const int64_t n_out =
+            rank == C - 1 ? row_len - t_beg : min(int64_t(a.tok_per_cta), row_len - t_beg);
+        for (int g = 0; g < G; ++g) {
+            uint8_t *dst = a.dist + (bh0 + g) * row_len + t_beg;
+            // past the CTA's capacity (the last CTA, rows longer than the
+            // context): pad bytes
+            for (int64_t i = int64_t(tid) * 16; i < n_out; i += int64_t(kCThreads) * 16)
+                *reinterpret_cast<uint4 *>(dst + i) =
+                    i < kCTok ? *reinterpret_cast<const uint4 *>(&S.dist[g][i])
+                              : make_uint4(~0u, ~0u, ~0u, ~0u);
+        }
+    }
+
+    // ---- 3. the cluster's histograms: T, #(< T), this CTA's placement ----
+    cl.sync();
+    const int k_eff = min(a.topk, len);
+    if (warp < G) {
+        const int g = warp;
+        // lane l: bins 5l .. 5l+4, summed over the C CTAs; before: the CTAs
+        // ranked below this one
+        uint32_t tot[5] = {0u, 0u, 0u, 0u, 0u}, pre[5] = {0u, 0u, 0u, 0u, 0u};
+        for (int r = 0; r < C; ++r) {
+            const uint32_t *hr = cl.map_shared_rank(&S.hist[g][0], r);
+#pragma unroll
+            for (int e = 0; e < 5; ++e) {
+                const uint32_t v = lane * 5 + e < kBins ? hr[lane * 5 + e] : 0u;
+                tot[e] += v;
+                pre[e] += r < rank ? v : 0u;
+            }
+        }
+        const uint32_t run = tot[0] + tot[1] + tot[2] + tot[3] + tot[4];
+        uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
+        int Tl = -1;
+        uint32_t less_l = 0;
+#pragma unroll
+        for (int e = 0; e < 5; ++e) {
+            if (Tl < 0 && lane * 5 + e < kBins && acc + tot[e] >= uint32_t(k_eff)) {
+                Tl = lane * 5 + e;
+                less_l = acc;
+            }
+            acc += tot[e];
+        }
+        const unsigned found = __ballot_sync(0xffffffffu, Tl >= 0);
+        const int src = found ? __ffs(int(found)) - 1 : 0;
+        const int T = found ? __shfl_sync(0xffffffffu, Tl, src) : kBins - 1;
+        const int n_less = found ? __shfl_sync(0xffffffffu, int(less_l), src) : 0;
+        int l = 0, q = 0;
+#pragma unroll
+        for (int e = 0; e < 5; ++e) {
+            const int bin = lane * 5 + e;
+            l += bin < T ? int(pre[e]) : 0;
+            q += bin == T ? int(pre[e]) : 0;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            l += __shfl_xor_sync(0xffffffffu, l, o);
+            q += __shfl_xor_sync(0xffffffffu, q, o);
+        }
+        if (lane == 0) {
+            S.sel[g][0] = T;
+            S.sel[g][1] = n_less;
+            S.sel[g][2] = l;  // keys below T in the CTAs before this one
+            S.sel[g][3] = q;  // keys at T in the CTAs before this one
+        }
+    }
+    __syncthreads();
+
+    // ---- 4. this CTA's share of every head's list (tokens 32 tid ...) ----
+    for (int g = 0; g < G; ++g) {
+        const int T = S.sel[g][0], n_less = S.sel[g][1];
+        const int less_before = S.sel[g][2], ties_before = S.sel[g][3];
+        const int r_ties = k_eff - n_less;  // boundary keys over the whole head
+        const int ties_done = ties_before < r_ties ? ties_before : r_ties;
+        int32_t *idx = a.idx + (bh0 + g) * a.topk;
+        if (rank == 0)
+            for (int i = k_eff + tid; i < a.topk; i += kCThreads) idx[i] = -1;
+        uint32_t lt[kGroups], eq[kGroups];
+        int n_lt = 0, n_eq = 0;
+#pragma unroll
+        for (int m = 0; m < kGroups; ++m) {
+            lt[m] = eq[m] = 0u;
+            if (k_eff > 0) {
+                const uint8_t *dm = &S.dist[g][kCPer * tid + 32 * m];
+                const uint4 v0 = *reinterpret_cast<const uint4 *>(dm);
+                const uint4 v1 = *reinterpret_cast<const uint4 *>(dm + 16);
+                const uint32_t dw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                const uint32_t T4 = uint32_t(T) * 0x01010101u, T4p = T4 + 0x01010101u;
+                if (T < kRbit)
+                    group_masks<false>(dw, T4, T4p, lt[m], eq[m]);
+                else
+                    group_masks<true>(dw, T4, T4p, lt[m], eq[m]);
+            }
+            n_lt += __popc(lt[m]);
+            n_eq += __popc(eq[m]);
+        }
+        int tile_lt, tile_eq;
+        const int2 before =
+            block_exclusive_scan2<kCThreads>(n_lt, n_eq, S.scan, &tile_lt, &tile_eq);
+        const int room = r_ties - ties_before > 0 ? r_ties - ties_before : 0;  // ties left
+        const int take_cta = room < tile_eq ? room : tile_eq;
+        const int taken_before = before.y < take_cta ? before.y : take_cta;
+        int my_take = take_cta - before.y;
+        my_take = my_take < 0 ? 0 : (my_take > n_eq ? n_eq : my_take);
+        const int start = less_before + ties_done;  // this CTA's first list position
+        emit_selected(lt, eq, my_take, start + before.x + taken_before, t_beg + kCPer * tid,
+                      [&](int p, int tok) {
+                          if (p < a.topk) idx[p] = tok;
+                      });
+        if (tid == 0) {
+            S.sel[g][2] = start;
+            S.sel[g][3] = k_eff > 0 ? tile_lt + take_cta : 0;  // entries of this CTA
+        }
+    }
+    __syncthreads();  // the CTA's list entries (global memory) and counts are visible
+
+    // ---- 5. gather + attention over this CTA's entries, G heads side by side ----
+    {
+        using namespace tc;
+        const int wpg = kCWarps / G;  // warps per head
+        const int g = warp / wpg, sub = warp - g * wpg;
+        const int start = S.sel[g][2], cnt = S.sel[g][3];
+        const int r0 = start + int(int64_t(sub) * cnt / wpg);
+        const int r1 = start + int(int64_t(sub + 1) * cnt / wpg);
+        const int n_st = (r1 - r0 + kSub - 1) / kSub;
+        const int32_t *idx = a.idx + (bh0 + g) * a.topk;
+        const int p = lane & 15, rh = lane >> 4;
+        const uint8_t *Kp = static_cast<const uint8_t *>(a.K) + slab * kRowB + p * 16;
+        const uint8_t *Vp = static_cast<const uint8_t *>(a.V) + slab * kRowB + p * 16;
+        const uint32_t wring = smem_addr(S.ring) + uint32_t(warp * kCRing * kStageBytes);
+        uint32_t doff[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) doff[u] = swz(8 * rh + u, p);
+        auto issue = [&](int s) {
+            if (s < n_st) {
+                const uint32_t Ks = wring + uint32_t((s % kCRing) * kStageBytes);
+                const uint32_t Vs = Ks + kSub * kRowB;
+                const int x0 = r0 + s * kSub + 8 * rh;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int32_t row = x0 + u < r1 ? idx[x0 + u] : -1;
+                    // the selection never yields an index outside [0, len); the
+                    // check keeps a corrupted list from steering a copy outside
+                    // the cache.  Rows without a key are zero-filled.
+                    const bool ok = row >= 0 && row < len;
+                    const int64_t off = ok ? int64_t(row) * kRowB : 0;
+                    cp_async16_zfill(Ks + doff[u], Kp + off, ok ? 16u : 0u);
+                    cp_async16_zfill(Vs + doff[u], Vp + off, ok ? 16u : 0u);
+                }
+            }
+            cp_async_commit();
+        };
+        for (int i = 0; i < kCRing - 1; ++i) issue(i);
+        const LaneOffsets lo(lane);
+        uint32_t qb[8][2];
+        load_query<false>(S.q[g], a.scale_log2, lane, qb);
+        float O[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
+        float m_ref = -INFINITY, l_part = 0.0f;
+        for (int s = 0; s < n_st; ++s) {
+            cp_async_wait<kCRing - 2>();
+            __syncwarp();
+            issue(s + kCRing - 1);
+            const int x = r0 + s * kSub + lane;
+            const int32_t row = lane < kSub && x < r1 ? idx[x] : -1;
+            const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0 && row < len);
+            attend_stage(vmask, wring + uint32_t((s % kCRing) * kStageBytes), qb, lo, O, m_ref,
+                         l_part, lane);
+        }
+        cp_async_wait<0>();
+        for (int i = lane; i < kPartStride; i += 32) S.part[warp][i] = i == 0 ? -INFINITY : 0.0f;
+        __syncwarp();
+        if (n_st > 0) store_partial(S.part[warp], O, m_ref, l_part, lane);
+    }
+    __syncthreads();
+    // the warps of each head merged into the CTA's partial, written into the
+    // first CTA's shared memory
+    {
+        float *dst0 = cl.map_shared_rank(&S.merged[0][0][0], 0);
+        const int wpg = kCWarps / G;
+        for (int i = tid; i < G * kD; i += kCThreads) {
+            const int g = i / kD, d = i % kD;
+            float M = -INFINITY;
+            for (int w = g * wpg; w < (g + 1) * wpg; ++w) M = fmaxf(M, S.part[w][0]);
+            float L = 0.0f, A = 0.0f;
+            if (M != -INFINITY)
+                for (int w = g * wpg; w < (g + 1) * wpg; ++w) {
+                    const float wt = S.part[w][0] == -INFINITY ? 0.0f : exp2f(S.part[w][0] - M);
+                    L = fmaf(S.part[w][1], wt, L);
+                    A = fmaf(S.part[w][4 + d], wt, A);
+                }
+            float *pp = dst0 + (size_t(rank) * kClusterMaxG + g) * kPartStride;
+            if (d == 0) {
+                pp[0] = M;
+                pp[1] = L;
+            }
+            pp[4 + d] = A;
+        }
+    }
+
+    // ---- 6. the first CTA merges the C partials of each head ----
+    cl.sync();
+    if (rank != 0) return;
+    for (int i = tid; i < G * kD; i += kCThreads) {
+        const int g = i / kD, d = i % kD;
+        float M = -INFINITY;
+        for (int r = 0; r < C; ++r) M = fmaxf(M, S.merged[r][g][0]);
+        float L = 0.0f, A = 0.0f;
+        if (M != -INFINITY)
+            for (int r = 0; r < C; ++r) {
+                const float wt = S.merged[r][g][0] == -INFINITY ? 0.0f : exp2f(S.merged[r][g][0] - M);
+                L = fmaf(S.merged[r][g][1], wt, L);
+                A = fmaf(S.merged[r][g][4 + d], wt, A);
+            }
+        a.out[(bh0 + g) * kD + d] = L > 0.0f ? A / L : 0.0f;
+    }
+}
+
+// The cluster launch of instantiation kM over `ctas` CTAs in clusters of C.
+template <int kM>
+cudaLaunchConfig_t cluster_cfg(int64_t ctas, int C, cudaStream_t s, cudaLaunchAttribute *attr)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(unsigned(ctas));
+    cfg.blockDim = dim3(kCThreads);
+    cfg.dynamicSmemBytes = sizeof(ClusterSmem<kM>);
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(C);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// Clusters of C CTAs (instantiation kM) the current device holds at once;
+// queried once per (device, C) and kept.
+template <int kM>
+cudaError_t resident_clusters(int C, int *clusters)
+{
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev)) return e;
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, int> known;  // (device, C) -> clusters
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = known.find({dev, C});
+        if (it != known.end()) {
+            *clusters = it->second;
+            return cudaSuccess;
+        }
+    }
+    const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<kM>);
+    if (cudaError_t e = ensure_smem_attr(fn, sizeof(ClusterSmem<kM>))) return e;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = cluster_cfg<kM>(C, C, nullptr, attr);
+    int n = 0;
+    if (cudaError_t e = cudaOccupancyMaxActiveClusters(&n, cluster_step_kernel<kM>, &cfg)) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    known[{dev, C}] = n;
+    *clusters = n;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+// The cluster step's shape for these sizes: CTAs of up to 8192 tokens (kM
+// 1) or, if those clusters do not all fit the device at once, of up to
+// 16384 (kM 2); C = the CTAs a head needs, each taking an equal range (a
+// multiple of 32 tokens).  plan->kM = 0: the step does not serve them.
+cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
+                              ClusterPlan *plan)
+{
+    *plan = ClusterPlan{};
+    const int G = H_q / H_kv;
+    if ((G != 1 && G != 2 && G != 4) || topk <= 0 || max_seq_len <= 0) return cudaSuccess;
+    const int64_t slabs = int64_t(B) * H_kv;
+    for (int kM = 1; kM <= 2; ++kM) {
+        const int64_t C = ceil_div(max_seq_len, int64_t(8192) * kM);
+        if (C > kClusterMaxC) continue;
+        int clusters = 0;
+        cudaError_t e = kM == 1 ? resident_clusters<1>(int(C), &clusters)
+                                : resident_clusters<2>(int(C), &clusters);
+        if (e != cudaSuccess) return e;
+        if (clusters > 0 && int64_t(clusters) >= slabs) {  // one wave
+            plan->kM = kM;
+            plan->C = int(C);
+            plan->tok_per_cta = int(ceil_div(ceil_div(max_seq_len, C), 32) * 32);
+            return cudaSuccess;
+        }
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_cluster_step(const ClusterArgs &a, const ClusterPlan &p, cudaStream_t s)
+{
+    const int64_t ctas = int64_t(p.C) * a.B * a.H_kv;
+    cudaLaunchAttribute attr[1];
+    if (p.kM == 1) {
+        const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<1>);
+        if (cudaError_t e = ensure_smem_attr(fn, sizeof(ClusterSmem<1>))) return e;
+        cudaLaunchConfig_t cfg = cluster_cfg<1>(ctas, p.C, s, attr);
+        return cudaLaunchKernelEx(&cfg, cluster_step_kernel<1>, a);
+    }
+    if (p.kM == 2) {
+        const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<2>);
+        if (cudaError_t e = ensure_smem_attr(fn, sizeof(ClusterSmem<2>))) return e;
+        cudaLaunchConfig_t cfg = cluster_cfg<2>(ctas, p.C, s, attr);
+        return cudaLaunchKernelEx(&cfg, cluster_step_kernel<2>, a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace hata

@@ -32,6 +32,7 @@ HATA_NOALLOC_WORKSPACE_BYTES = 64 << 20
 HATA_MODE_AUTO = 0
 HATA_MODE_MULTI_KERNEL = 1
 HATA_MODE_FUSED = 2
+HATA_MODE_CLUSTER = 3
 HATA_SP_HIST_WORDS = 260
 HATA_SP_PART_WORDS = 132
 D = 128
@@ -55,7 +56,7 @@ _SIGS = {
     "hata_append_code": ([P, I, P, P, I64, P, I, I, I, I, P, P], I),
     "hata_decode_workspace_size": ([I, I, I, I64, I], U64),
     "hata_dist_row_bytes": ([I64], I64),
-    "hata_decode_kernel_launches": ([I, I, I, I], I),
+    "hata_decode_kernel_launches": ([I, I, I, I64, I, I, I], I),
     "hata_decode_step": ([P, P, P, P, P, I, I64, P, I64, P, P, I, I, I, I, I, I, F, P, U64, P,
                           P, P, P, I64, P, P], I),
     "hata_decode_step_noalloc": ([P, P, P, P, P, I, I64, P, I64, P, P, I, I, I, I, I, I, F, P,
@@ -208,10 +209,11 @@ def hata_dist_row_bytes(max_seq_len: int) -> int:
     return int(lib().hata_dist_row_bytes(max_seq_len))
 
 
-def hata_decode_kernel_launches(B: int, H_q: int, topk: int, kv_dtype: torch.dtype) -> int:
+def hata_decode_kernel_launches(B: int, H_q: int, H_kv: int, max_seq_len: int, topk: int,
+                                kv_dtype: torch.dtype, r: int = RBIT) -> int:
     """Kernels one decode step with these sizes launches on the current device."""
     code = HATA_DT_BF16 if kv_dtype == torch.bfloat16 else HATA_DT_F32
-    n = int(lib().hata_decode_kernel_launches(B, H_q, topk, code))
+    n = int(lib().hata_decode_kernel_launches(B, H_q, H_kv, max_seq_len, topk, code, r))
     if n < 0:
         raise HataError(HATA_ERR_INVALID_ARG, "hata_decode_kernel_launches",
                         lib().hata_last_error().decode())

@@ -130,15 +130,17 @@ size_t hata_decode_workspace_size(int B, int H_q, int H_kv, int64_t max_seq_len,
 int64_t hata_dist_row_bytes(int64_t max_seq_len);
 
 /* Number of kernels one hata_decode_step with these sizes launches on the
- * current device in the current mode (hata_set_decode_mode): 3 for the fused
- * step (prep, score, the persistent selection + attention kernel); for the
- * multi-kernel step prep, score, select, attention and, unless the heads are
- * merged inside the attention CTAs, the combine kernel: 4 or 5.  Returns -1 (hata_last_error says why) for invalid sizes or if the
- * device query fails.  Host-only; launches nothing. */
-int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype);
+ * current device in the current mode (hata_set_decode_mode): 1 for the
+ * cluster step; 3 for the fused step (prep, score, the persistent selection
+ * + attention kernel); for the multi-kernel step prep, score, select,
+ * attention and, unless the heads are merged inside the attention CTAs, the
+ * combine kernel: 4 or 5.  Returns -1 (hata_last_error says why) for
+ * invalid sizes or if a device query fails.  Host-only; launches nothing. */
+int hata_decode_kernel_launches(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
+                                hata_dtype_t kv_dtype, int r);
 
 /* ------------------------------------------------------------------------
- * Step implementation.  Two implementations give the same codes, distances
+ * Step implementation.  Three implementations give the same codes, distances
  * and indices bit for bit (outputs agree within the attention tolerance):
  *   the multi-kernel step  prep, score, select, attention and (unless every
  *                          head is merged inside its attention CTA) combine;
@@ -146,15 +148,25 @@ int hata_decode_kernel_launches(int B, int H_q, int topk, hata_dtype_t kv_dtype)
  *                          CTA per SM in which selection warps build the
  *                          index lists while attention warps already gather
  *                          and attend the heads selected so far (bf16 caches
- *                          and r <= 128 only; other steps take the
- *                          multi-kernel step).
- *   HATA_MODE_AUTO          the library's choice (default)
+ *                          and r <= 128 only);
+ *   the cluster step       ONE kernel: a thread-block cluster per (b, h_kv)
+ *                          of up to 8 CTAs of 8192 tokens each hashes,
+ *                          scores, selects and attends, the CTAs meeting
+ *                          through distributed shared memory (bf16 caches,
+ *                          r = 128, H_q / H_kv of 1, 2 or 4, max_seq_len up
+ *                          to 65536, every cluster resident at once).
+ * A step whose sizes the chosen implementation does not serve takes the
+ * multi-kernel step.
+ *   HATA_MODE_AUTO          the library's choice (default): the cluster step
+ *                           where it serves, else the multi-kernel step
  *   HATA_MODE_MULTI_KERNEL  always the multi-kernel step
- *   HATA_MODE_FUSED         the fused step for bf16 caches
+ *   HATA_MODE_FUSED         the fused step
+ *   HATA_MODE_CLUSTER       the cluster step
  * The mode is process-wide and read when a step is enqueued. */
 #define HATA_MODE_AUTO 0
 #define HATA_MODE_MULTI_KERNEL 1
 #define HATA_MODE_FUSED 2
+#define HATA_MODE_CLUSTER 3
 hata_status_t hata_set_decode_mode(int mode);
 int hata_get_decode_mode(void);
 
@@ -209,7 +221,8 @@ hata_status_t hata_set_wait_limit_ns(uint64_t ns);
  *             first kernel and after each of the five kernels (prep, score,
  *             select, attend, combine) -- a profiling hook (an event between
  *             two kernels keeps the second from starting early).  In the
- *             fused step events 2..5 are all recorded after the step kernel.
+ *             fused step events 3..5 are all recorded after the step kernel,
+ *             in the cluster step events 1..5 after its one kernel.
  */
 hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes, void *K,
                                void *V, hata_dtype_t kv_dtype, int64_t n_cap,

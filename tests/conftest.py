@@ -26,14 +26,16 @@ def pytest_collection_modifyitems(config, items):
             item.add_marker(skip)
 
 
-@pytest.fixture(params=["fused", "multi_kernel"])
+@pytest.fixture(params=["fused", "multi_kernel", "cluster"])
 def decode_mode(request):
-    """Run a decode-step test under both step implementations: the fused
-    step (selection + attention in one persistent kernel) and the
-    multi-kernel step.
+    """Run a decode-step test under each step implementation: the fused step
+    (selection + attention in one persistent kernel), the multi-kernel step
+    and the cluster step (one kernel per step where the sizes fit a
+    thread-block cluster; other sizes fall back to the multi-kernel step).
     The process-wide mode is restored afterwards."""
     from hash_aware_top_hata_b200 import hata as H
-    mode = H.HATA_MODE_FUSED if request.param == "fused" else H.HATA_MODE_MULTI_KERNEL
+    mode = {"fused": H.HATA_MODE_FUSED, "multi_kernel": H.HATA_MODE_MULTI_KERNEL,
+            "cluster": H.HATA_MODE_CLUSTER}[request.param]
     H.hata_set_decode_mode(mode)
     yield request.param
     H.hata_set_decode_mode(H.HATA_MODE_AUTO)

@@ -22,7 +22,7 @@ def test_library_exports_every_header_function():
     lib = H.lib()
     for n in names:
         assert hasattr(lib, n), n
-    assert H.hata_abi_version() == 3
+    assert H.hata_abi_version() == 4
 
 
 def test_status_strings():
@@ -202,7 +202,8 @@ def test_binding_rejects_hash_keys_views_it_cannot_pass():
 def test_decode_modes():
     assert H.hata_get_decode_mode() == H.HATA_MODE_AUTO
     assert H.lib().hata_set_decode_mode(7) == H.HATA_ERR_INVALID_ARG
-    for m in (H.HATA_MODE_MULTI_KERNEL, H.HATA_MODE_FUSED):
+    assert H.lib().hata_set_decode_mode(4) == H.HATA_ERR_INVALID_ARG
+    for m in (H.HATA_MODE_MULTI_KERNEL, H.HATA_MODE_FUSED, H.HATA_MODE_CLUSTER):
         H.hata_set_decode_mode(m)
         try:
             assert H.hata_get_decode_mode() == m
@@ -233,15 +234,20 @@ def test_workspace_check_rejects_bad_workspace():
 def test_decode_kernel_launches_host_logic():
     L = H.lib()
     # fp32 caches take the SIMT attention kernel, always followed by the combine
-    assert H.hata_decode_kernel_launches(4, 32, 2048, torch.float32) == 5
+    assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, torch.float32) == 5
     # bf16 caches in the fused step: prep, score, the selection + attention kernel
     H.hata_set_decode_mode(H.HATA_MODE_FUSED)
     try:
-        assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 3
+        assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, torch.bfloat16) == 3
+        # 256-bit codes never take the fused step
+        assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, torch.float32, 256) == 5
     finally:
         H.hata_set_decode_mode(H.HATA_MODE_AUTO)
-    for bad in ((0, 32, 2048, H.HATA_DT_BF16), (4, 0, 2048, H.HATA_DT_BF16),
-                (4, 32, 0, H.HATA_DT_BF16), (4, 32, 2048, 9)):
+    # B, H_q, H_kv, max_seq_len, topk, dtype, r
+    for bad in ((0, 32, 8, 4096, 2048, H.HATA_DT_BF16, 128), (4, 0, 8, 4096, 2048, H.HATA_DT_BF16, 128),
+                (4, 32, 0, 4096, 2048, H.HATA_DT_BF16, 128), (4, 32, 5, 4096, 2048, H.HATA_DT_BF16, 128),
+                (4, 32, 8, 0, 2048, H.HATA_DT_BF16, 128), (4, 32, 8, 4096, 0, H.HATA_DT_BF16, 128),
+                (4, 32, 8, 4096, 2048, 9, 128), (4, 32, 8, 4096, 2048, H.HATA_DT_BF16, 96)):
         assert L.hata_decode_kernel_launches(*bad) == -1
     with pytest.raises(H.HataError):
-        H.hata_decode_kernel_launches(4, 32, -1, torch.bfloat16)
+        H.hata_decode_kernel_launches(4, 32, 8, 4096, -1, torch.bfloat16)

@@ -604,21 +604,34 @@ def test_decode_many_selected_rows(decode_mode):
 
 def test_decode_kernel_launch_count():
     """Fused step: prep, score and one persistent selection + attention
-    kernel.  Multi-kernel step: 128
-    heads at topk 2048 fill about one wave of attention CTAs (merged in-CTA,
-    no combine kernel); 32 heads do not."""
+    kernel.  Multi-kernel step: 128 heads at topk 2048 fill about one wave of
+    attention CTAs (merged in-CTA, no combine kernel); 32 heads do not.
+    Cluster step: one kernel where a cluster per KV head fits (context up to
+    64K, 1, 2 or 4 query heads per KV head, every cluster resident)."""
+    bf = torch.bfloat16
     H.hata_set_decode_mode(H.HATA_MODE_FUSED)
     try:
-        assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 3
+        assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, bf) == 3
     finally:
         H.hata_set_decode_mode(H.HATA_MODE_AUTO)
     H.hata_set_decode_mode(H.HATA_MODE_MULTI_KERNEL)
     try:
-        assert H.hata_decode_kernel_launches(4, 32, 2048, torch.bfloat16) == 4
-        assert H.hata_decode_kernel_launches(1, 32, 2048, torch.bfloat16) == 5
-        assert H.hata_decode_kernel_launches(4, 32, 100, torch.bfloat16) == 5  # too few rows per warp
+        assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, bf) == 4
+        assert H.hata_decode_kernel_launches(1, 32, 8, 131072, 2048, bf) == 5
+        assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 100, bf) == 5  # too few rows per warp
     finally:
         H.hata_set_decode_mode(H.HATA_MODE_AUTO)
+    for mode in (H.HATA_MODE_CLUSTER, H.HATA_MODE_AUTO):
+        H.hata_set_decode_mode(mode)
+        try:
+            assert H.hata_decode_kernel_launches(1, 32, 32, 32769, 512, bf) == 1   # 5 CTAs a head
+            assert H.hata_decode_kernel_launches(1, 32, 8, 65536, 512, bf) == 1    # 8 CTAs, G 4
+            assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, bf) == 4  # 16 CTAs: no
+            assert H.hata_decode_kernel_launches(32, 28, 4, 32768, 512, bf) == 5   # G 7: no
+            assert H.hata_decode_kernel_launches(1, 32, 32, 32768, 512, bf, 64) == 5  # r 64: no
+            assert H.hata_decode_kernel_launches(64, 32, 32, 32768, 512, bf) == 4  # too many clusters
+        finally:
+            H.hata_set_decode_mode(H.HATA_MODE_AUTO)
 
 
 def test_one_wave_of_heads_ties_across_tiles(decode_mode):
@@ -631,8 +644,9 @@ def test_one_wave_of_heads_ties_across_tiles(decode_mode):
     heads = [(b, hq) for b in range(cfg.B) for hq in (0, 5, 31)]
     slabs = host_slabs(w, sorted({(b, hq // cfg.G) for b, hq in heads}))
     dec = GpuDecoder(w, cfg.topk)
-    assert H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.topk, torch.bfloat16) == (
-        4 if decode_mode == "multi_kernel" else 3)
+    assert H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.H_kv, dec.max_seq_len, cfg.topk,
+                                         torch.bfloat16) == (
+        {"multi_kernel": 4, "fused": 3, "cluster": 1}[decode_mode])
     lens = [cfg.N, 17001, 2999, 19999]
     got = dec.step(w.q[0], lens)
     Wn = w.W_H.cpu().numpy()
