@@ -629,7 +629,7 @@ def test_decode_kernel_launch_count():
             assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, bf) == 4  # 16 CTAs: no
             assert H.hata_decode_kernel_launches(32, 28, 4, 32768, 512, bf) == 5   # G 7: no
             assert H.hata_decode_kernel_launches(1, 32, 32, 32768, 512, bf, 64) == 5  # r 64: no
-            assert H.hata_decode_kernel_launches(64, 32, 32, 32768, 512, bf) == 4  # too many clusters
+            assert H.hata_decode_kernel_launches(64, 32, 32, 32768, 512, bf) == 5  # too many clusters
         finally:
             H.hata_set_decode_mode(H.HATA_MODE_AUTO)
 
