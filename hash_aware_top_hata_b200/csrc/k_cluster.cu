@@ -65,25 +65,50 @@ constexpr size_t kCRingBytes = size_t(kCWarps) * kCRing * tc::kStageBytes;
 template <int kM>
 struct ClusterSmem {
     static constexpr int kTok = 8192 * kM;
-    uint8_t ring[kCRingBytes];                        // attention rings (phase 5)
-    uint8_t dist[kClusterMaxG][kTok];                 // this CTA's distances
+    static constexpr int kDistBytes = kClusterMaxG * kTok > kD * kRbit * 4 ? kClusterMaxG * kTok
+                                                                          : kD * kRbit * 4;
+    uint8_t ring[kCRingBytes];                        // code chunks (phase 2), attention rings
+                                                      // (phase 5)
+    union {
+        uint8_t dist[kClusterMaxG][kTok];             // this CTA's distances (phase 2 on)
+        uint8_t w[kDistBytes];                        // W_H of the KV head (phase 1)
+    };
     uint32_t hist[kClusterMaxG][kHistStride];         // and their histograms
     float q[kClusterMaxG][kD];                        // the query rows
     float part[kCWarps][kPartStride];                 // warp partials
     float merged[kClusterMaxC][kClusterMaxG][kPartStride];  // CTA partials (first CTA)
     uint32_t qcode[kClusterMaxG][4];
+    uint32_t kcode[4];                                // the appended key's code
     int2 scan[kCWarps + 1];
     int sel[kClusterMaxG][4];                         // T, n_less, start, count per head
 };
 
 // The fp32 chain acc = fmaf(x_i, W[i][j], acc), i = 0..127, of bit j of the
-// code of row x (shared memory) with one head's W ([128][128], global).
-__device__ __forceinline__ bool hash_bit(const float *x, const float *Wh, int j)
+// code of row x with one head's W ([128][128]); both in shared memory.
+__device__ __forceinline__ bool hash_bit(const float *x, const float *Ws, int j)
 {
     float acc = 0.0f;
-#pragma unroll 16
-    for (int i = 0; i < kD; ++i) acc = __fmaf_rn(x[i], __ldg(Wh + i * kRbit + j), acc);
+#pragma unroll 4
+    for (int i = 0; i < kD; ++i) acc = __fmaf_rn(x[i], Ws[i * kRbit + j], acc);
     return acc > 0.0f;
+}
+
+constexpr int kChunk = 4096;  // tokens per code chunk (64 KB) of the scan
+
+// Copy chunk c of this CTA's key codes (thread t: tokens t + 256 j of the
+// chunk, 16 bytes each) into `dst` (64 KB of shared memory), zero-filling
+// tokens that hold no key; always commits one group.
+__device__ __forceinline__ void copy_chunk(const uint4 *codes, int c, int nloc, uint32_t dst, int tid)
+{
+    asm volatile("" ::: "memory");  // earlier reads of the slot stay before the copies
+#pragma unroll
+    for (int j = 0; j < kChunk / kCThreads; ++j) {
+        const int t = kChunk * c + tid + kCThreads * j;
+        const bool in = t < nloc;
+        cp_async16_zfill(dst + 16u * uint32_t(tid + kCThreads * j), in ? codes + t : codes,
+                         in ? 16u : 0u);
+    }
+    cp_async_commit();
 }
 
 template <int kM>
@@ -110,6 +135,23 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
     const float *Wh = a.W + size_t(h) * kD * kRbit;
 
     // ---- 1. query rows, their codes, the append, the flags ----
+    // W_H of the KV head (64 KB) goes to the distance area (written from
+    // phase 2 on), the first two code chunks (2 x 64 KB) to the attention
+    // rings (unused until phase 5): all three copies start now and overlap
+    // the query loads and the hashing
+    const uint32_t ring0 = smem_addr(S.ring);              // even chunks
+    const uint32_t ring1 = ring0 + uint32_t(kChunk * 16);  // odd chunks
+    const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes) + slab + t_beg;
+    for (int i = tid; i < kD * kRbit / 4; i += kCThreads)
+        cp_async16(S.w + 16 * i, Wh + 4 * i);
+    cp_async_commit();
+    constexpr int kChunks = kCTok / kChunk;
+    copy_chunk(codes, 0, nloc, ring0, tid);
+    if (kChunks > 1)
+        copy_chunk(codes, 1, nloc, ring1, tid);
+    else
+        cp_async_commit();
+    const float *Ws = reinterpret_cast<const float *>(S.w);
     for (int i = tid; i < G * kD; i += kCThreads)
         S.q[i / kD][i % kD] = a.q[(bh0 + i / kD) * kD + i % kD];
     for (int i = tid; i < G * kHistStride; i += kCThreads) (&S.hist[0][0])[i] = 0u;
@@ -128,13 +170,14 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
     const int64_t pos = int64_t(sl) - 1;
     const bool append = a.k_new && pos >= 0 && pos < a.n_cap &&
                         min(int(pos / a.tok_per_cta), C - 1) == rank;
+    cp_async_wait<2>();  // this thread's copies of W
     __syncthreads();
     // 2G chains of 128 steps over the 256 threads (G <= 4: at most two each),
     // plus the appended key's 128 in the CTA that owns it
     {
         const int j = tid & (kRbit - 1);
         for (int g = tid >> 7; g < G; g += 2) {
-            const bool bit = hash_bit(S.q[g], Wh, j);
+            const bool bit = hash_bit(S.q[g], Ws, j);
             const uint32_t word = __ballot_sync(0xffffffffu, bit);
             if (lane == 0) S.qcode[g][j >> 5] = word;
         }
@@ -146,9 +189,13 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
         for (int i = tid; i < kD; i += kCThreads) xk[i] = __uint_as_float(uint32_t(kn[i]) << 16);
         __syncthreads();
         if (tid < kRbit) {
-            const bool bit = hash_bit(xk, Wh, tid);
+            const bool bit = hash_bit(xk, Ws, tid);
             const uint32_t word = __ballot_sync(0xffffffffu, bit);
-            if (lane == 0) a.codes[(slab + pos) * 4 + (tid >> 5)] = word;
+            if (lane == 0) {
+                S.kcode[tid >> 5] = word;  // the scan takes it from here: the copy of
+                                           // its slot may predate this write
+                a.codes[(slab + pos) * 4 + (tid >> 5)] = word;
+            }
         }
         if (a.v_new && tid >= kRbit) {  // K and V rows of the new token
             const int e = tid - kRbit;  // 0..127
@@ -162,7 +209,8 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
     if (a.q_out && rank == 0)
         for (int i = tid; i < G * 4; i += kCThreads) a.q_out[(bh0 + i / 4) * 4 + i % 4] = S.qcode[i / 4][i % 4];
 
-    // ---- 2. scores of this CTA's tokens (token t_beg + tid + 256 m) ----
+    // ---- 2. scores of this CTA's tokens: chunks of 4096 through the rings,
+    // two chunks in flight (thread t reads back only the tokens it copied) ----
     {
         uint4 qv[kClusterMaxG];
         uint2 qd[kClusterMaxG];
@@ -173,26 +221,26 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
             const uint32_t q012 = c[0] ^ c[1] ^ c[2];
             qd[g] = make_uint2(q012, q012 ^ c[3]);
         }
-        const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes) + slab + t_beg;
-        constexpr int kBatch = 8;  // tokens whose loads are in flight together
-        for (int m0 = 0; m0 < kCPer; m0 += kBatch) {
-            uint4 kv[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int t = tid + kCThreads * (m0 + u);
-                // plain loads: the appended code was written by this kernel
-                kv[u] = t < nloc ? codes[t] : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int t = tid + kCThreads * (m0 + u);
-                const uint32_t k012 = kv[u].x ^ kv[u].y ^ kv[u].z, k0123 = k012 ^ kv[u].w;
+        // the appended token's position in this CTA's range, if it holds it
+        const int lp = append ? int(pos) - t_beg : -1;
+        const uint4 kap = append ? make_uint4(S.kcode[0], S.kcode[1], S.kcode[2], S.kcode[3])
+                                 : make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < kChunks; ++c) {
+            cp_async_wait<1>();  // this thread's copies of chunk c (chunk c + 1 may fly)
+            const uint4 *mine = reinterpret_cast<const uint4 *>(S.ring + (c & 1) * kChunk * 16);
+#pragma unroll 4
+            for (int j = 0; j < kChunk / kCThreads; ++j) {
+                const int tl = tid + kCThreads * j;     // in the chunk
+                const int t = kChunk * c + tl;          // in the CTA's range
+                uint4 kv = mine[tl];
+                if (t == lp) kv = kap;
+                const uint32_t k012 = kv.x ^ kv.y ^ kv.z, k0123 = k012 ^ kv.w;
 #pragma unroll
                 for (int g = 0; g < kClusterMaxG; ++g) {
                     if (g < G) {
                         uint8_t byte = kDistPad;
                         if (t < nloc) {
-                            const int d = hamming128(kv[u], k012, k0123, qv[g], qd[g]);
+                            const int d = hamming128(kv, k012, k0123, qv[g], qd[g]);
                             atomicAdd(&S.hist[g][d], 1u);
                             byte = uint8_t(d);
                         }
@@ -200,7 +248,14 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
                     }
                 }
             }
+            // chunk c + 2 into the slot chunk c leaves (this thread read only
+            // the tokens it copied itself)
+            if (c + 2 < kChunks)
+                copy_chunk(codes, c + 2, nloc, (c & 1) ? ring1 : ring0, tid);
+            else
+                cp_async_commit();
         }
+        cp_async_wait<0>();
     }
     __syncthreads();
     if (a.dist) {  // the caller's distance rows: this CTA's part of them (the last
