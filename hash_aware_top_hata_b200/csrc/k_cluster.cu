@@ -88,7 +88,7 @@ struct ClusterSmem {
 __device__ __forceinline__ bool hash_bit(const float *x, const float *Ws, int j)
 {
     float acc = 0.0f;
-#pragma unroll 4
+#pragma unroll 16
     for (int i = 0; i < kD; ++i) acc = __fmaf_rn(x[i], Ws[i * kRbit + j], acc);
     return acc > 0.0f;
 }
