@@ -508,6 +508,8 @@ def other_workloads(args, dev):
         us = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
         step_bytes = B * Hkv * (N + warm + timed // 2) * 16 + B * Hq * cfg.topk * 2 * 256
         entry = {"us_per_step": round(us, 2), "steps": timed,
+                 "launches_per_step": H.hata_decode_kernel_launches(B, Hq, Hkv, w.n_cap, cfg.topk,
+                                                                     w.K.dtype),
                  "step_roofline_bytes": step_bytes,
                  "step_frac_of_measured": round(step_bytes / (us * 1e-6) / 1e9 / peak, 4),
                  "shape": f"B {B}, {Hq}/{Hkv} heads, context {N}, top-{cfg.topk}"}
