@@ -1,6 +1,6 @@
 // k_cluster.cu -- the whole decode step in ONE kernel for heads whose cache
 // fits a thread-block cluster: one cluster of C <= 8 CTAs per (batch row,
-// KV head), CTA r owning tokens [8192 r, 8192 (r + 1)) of the slab.
+// KV head), CTA r owning an equal range of up to 16384 tokens of the slab.
 //
 // HATA review page (arXiv 2506.02572): "What carries the argument" (hash
 // q, XOR + popcount against every cached key code, attention over the
@@ -28,8 +28,8 @@
 //      placement arithmetic as the tile CTAs of the selection kernel;
 //   4. it selects its share (byte-wise masks, one block scan per head) into
 //      the head's index list, ascending;
-//   5. its warps gather and attend its selected rows (G heads side by side,
-//      8 / G warps each, the tensor-core stage of attend_common.cuh) and
+//   5. its first 8 warps gather and attend its selected rows (G heads side
+//      by side, 8 / G warps each, the tensor-core stage of attend_common.cuh) and
 //      merge them into one partial (m, l, acc) per head, written into the
 //      shared memory of the cluster's first CTA;
 //   6. cluster barrier; the first CTA merges the C partials per head into
@@ -37,7 +37,10 @@
 //
 // Every CTA of a cluster is resident at once (the hardware schedules a
 // cluster as a unit), so the two barriers cannot wait on a CTA that never
-// runs.  bf16 K/V, r = 128, G in {1, 2, 4}.
+// runs.  bf16 K/V, r = 128, G in {1, 2, 4}.  512 threads: all 16 warps scan
+// and select (the scan is latency-bound, so warps matter), the first 8
+// attend (their rings take the 128 KB that held W_H and the code chunks);
+// 126 registers, no spills.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
@@ -56,12 +59,14 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-constexpr int kCThreads = 256;
-constexpr int kCWarps = kCThreads / 32;
+constexpr int kCThreads = 512;
+constexpr int kCWarps = kCThreads / 32;      // 16 warps scan and select
+constexpr int kAWarps = 8;                   // the first 8 of them attend
 constexpr int kCRing = 2;                    // attention stages per warp ring
-constexpr size_t kCRingBytes = size_t(kCWarps) * kCRing * tc::kStageBytes;
+constexpr size_t kCRingBytes = size_t(kAWarps) * kCRing * tc::kStageBytes;
 
-// kM: a CTA holds up to 8192 kM tokens, 32 kM per thread in the selection
+// kM: a CTA holds up to 8192 kM tokens, 16 kM per thread in the selection
+// (the plan uses kM = 2: 32 tokens, one mask word, per thread)
 template <int kM>
 struct ClusterSmem {
     static constexpr int kTok = 8192 * kM;
@@ -75,7 +80,7 @@ struct ClusterSmem {
     };
     uint32_t hist[kClusterMaxG][kHistStride];         // and their histograms
     float q[kClusterMaxG][kD];                        // the query rows
-    float part[kCWarps][kPartStride];                 // warp partials
+    float part[kAWarps][kPartStride];                 // attention warp partials
     float merged[kClusterMaxC][kClusterMaxG][kPartStride];  // CTA partials (first CTA)
     uint32_t qcode[kClusterMaxG][4];
     uint32_t kcode[4];                                // the appended key's code
@@ -172,11 +177,11 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
                         min(int(pos / a.tok_per_cta), C - 1) == rank;
     cp_async_wait<2>();  // this thread's copies of W
     __syncthreads();
-    // 2G chains of 128 steps over the 256 threads (G <= 4: at most two each),
+    // G chains of 128 steps per bit over the 512 threads (G <= 4: one each),
     // plus the appended key's 128 in the CTA that owns it
     {
         const int j = tid & (kRbit - 1);
-        for (int g = tid >> 7; g < G; g += 2) {
+        for (int g = tid >> 7; g < G; g += kCThreads / kRbit) {
             const bool bit = hash_bit(S.q[g], Ws, j);
             const uint32_t word = __ballot_sync(0xffffffffu, bit);
             if (lane == 0) S.qcode[g][j >> 5] = word;
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
                 a.codes[(slab + pos) * 4 + (tid >> 5)] = word;
             }
         }
-        if (a.v_new && tid >= kRbit) {  // K and V rows of the new token
+        if (a.v_new && tid >= kRbit && tid < 2 * kRbit) {  // K and V rows of the new token
             const int e = tid - kRbit;  // 0..127
             const uint16_t *vn =
                 static_cast<const uint16_t *>(a.v_new) + (int64_t(b) * a.H_kv + h) * kD;
@@ -377,9 +382,9 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
     __syncthreads();  // the CTA's list entries (global memory) and counts are visible
 
     // ---- 5. gather + attention over this CTA's entries, G heads side by side ----
-    {
+    if (warp < kAWarps) {
         using namespace tc;
-        const int wpg = kCWarps / G;  // warps per head
+        const int wpg = kAWarps / G;  // warps per head
         const int g = warp / wpg, sub = warp - g * wpg;
         const int start = S.sel[g][2], cnt = S.sel[g][3];
         const int r0 = start + int(int64_t(sub) * cnt / wpg);
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
     // first CTA's shared memory
     {
         float *dst0 = cl.map_shared_rank(&S.merged[0][0][0], 0);
-        const int wpg = kCWarps / G;
+        const int wpg = kAWarps / G;
         for (int i = tid; i < G * kD; i += kCThreads) {
             const int g = i / kD, d = i % kD;
             float M = -INFINITY;
@@ -528,10 +533,10 @@ cudaError_t resident_clusters(int C, int *clusters)
 
 }  // namespace
 
-// The cluster step's shape for these sizes: CTAs of up to 8192 tokens (kM
-// 1) or, if those clusters do not all fit the device at once, of up to
-// 16384 (kM 2); C = the CTAs a head needs, each taking an equal range (a
-// multiple of 32 tokens).  plan->kM = 0: the step does not serve them.
+// The cluster step's shape for these sizes: C = the CTAs of up to 16384
+// tokens a head needs (C <= 8), each taking an equal range (a multiple of
+// 32 tokens), when every cluster fits the device at once.  plan->kM = 0:
+// the step does not serve them.
 cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
                               ClusterPlan *plan)
 {
@@ -539,12 +544,11 @@ cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int
     const int G = H_q / H_kv;
     if ((G != 1 && G != 2 && G != 4) || topk <= 0 || max_seq_len <= 0) return cudaSuccess;
     const int64_t slabs = int64_t(B) * H_kv;
-    for (int kM = 1; kM <= 2; ++kM) {
+    for (int kM = 2; kM <= 2; ++kM) {  // 16384-token CTAs: 32 tokens a thread
         const int64_t C = ceil_div(max_seq_len, int64_t(8192) * kM);
         if (C > kClusterMaxC) continue;
         int clusters = 0;
-        cudaError_t e = kM == 1 ? resident_clusters<1>(int(C), &clusters)
-                                : resident_clusters<2>(int(C), &clusters);
+        cudaError_t e = resident_clusters<2>(int(C), &clusters);
         if (e != cudaSuccess) return e;
         if (clusters > 0 && int64_t(clusters) >= slabs) {  // one wave
             plan->kM = kM;
@@ -560,12 +564,6 @@ cudaError_t launch_cluster_step(const ClusterArgs &a, const ClusterPlan &p, cuda
 {
     const int64_t ctas = int64_t(p.C) * a.B * a.H_kv;
     cudaLaunchAttribute attr[1];
-    if (p.kM == 1) {
-        const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<1>);
-        if (cudaError_t e = ensure_smem_attr(fn, sizeof(ClusterSmem<1>))) return e;
-        cudaLaunchConfig_t cfg = cluster_cfg<1>(ctas, p.C, s, attr);
-        return cudaLaunchKernelEx(&cfg, cluster_step_kernel<1>, a);
-    }
     if (p.kM == 2) {
         const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<2>);
         if (cudaError_t e = ensure_smem_attr(fn, sizeof(ClusterSmem<2>))) return e;

@@ -150,11 +150,11 @@ int hata_decode_kernel_launches(int B, int H_q, int H_kv, int64_t max_seq_len, i
  *                          and attend the heads selected so far (bf16 caches
  *                          and r <= 128 only);
  *   the cluster step       ONE kernel: a thread-block cluster per (b, h_kv)
- *                          of up to 8 CTAs of 8192 tokens each hashes,
+ *                          of up to 8 CTAs of up to 16384 tokens each hashes,
  *                          scores, selects and attends, the CTAs meeting
  *                          through distributed shared memory (bf16 caches,
  *                          r = 128, H_q / H_kv of 1, 2 or 4, max_seq_len up
- *                          to 65536, every cluster resident at once).
+ *                          to 131072, every cluster resident at once).
  * A step whose sizes the chosen implementation does not serve takes the
  * multi-kernel step.
  *   HATA_MODE_AUTO          the library's choice (default): the cluster step
