@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(kThreads, kWide ? 2 : 4) select_kernel(SelectA
     __shared__ int2 scan_s[kWarps + 1];
     __shared__ int s_thr[4];
     __shared__ __align__(16) uint8_t dist_s[kThreads * kPer];  // the tile's distances
+    __shared__ uint32_t hsum[kWarps][2][160];                   // per-warp bin sums (many tiles)
 
     if (tile == 0)
         for (int i = k_eff + tid; i < a.topk; i += kThreads) idx[i] = -1;
@@ -89,13 +90,15 @@ __global__ void __launch_bounds__(kThreads, kWide ? 2 : 4) select_kernel(SelectA
     // this thread's 128 distances (bytes past the row read as padding)
     const uint8_t *drow = a.dist + bh * a.dist_row;
     const int my0 = tile * kTile + tid * kPer;
-    // ---- warp 0 first finds T, #(dist < T) and the keys below T / at T in
-    // the tiles before this one from the head's tile histograms (one round
-    // trip to L2 per 4 tiles), ahead of its own distance loads;
-    // the other warps' distance loads are in flight meanwhile ----
-    if (tid < 32)
-        head_threshold<false, 4, kWide>(a.hist + bh * size_t(a.n_tiles) * kStride,
-                                        int(a.n_tiles), k_eff, tile, tid, s_thr);
+    // ---- T, #(dist < T) and the keys below T / at T in the tiles before
+    // this one, from the head's tile histograms.  Up to 4 tiles: warp 0, one
+    // round trip to L2, ahead of its own distance loads; more tiles: every
+    // warp sums its share of them (one round trip for up to 36 tiles) while
+    // the distance copies are in flight, and warp 0 adds the shares ----
+    const uint32_t *hrow = a.hist + bh * size_t(a.n_tiles) * kStride;
+    const bool many = !kWide && a.n_tiles > 4;  // CTA-uniform
+    if (!many && tid < 32)
+        head_threshold<false, 4, kWide>(hrow, int(a.n_tiles), k_eff, tile, tid, s_thr);
     // the warp's 4 KB arrive by coalesced 16-byte copies (lane l: bytes
     // 16l .. 16l+15 of each 512-byte block) into a swizzled shared tile,
     // piece v of thread t at t*128 + 16*(v ^ (t & 7)), so that each thread
@@ -113,13 +116,6 @@ __global__ void __launch_bounds__(kThreads, kWide ? 2 : 4) select_kernel(SelectA
 #pragma unroll
         for (int k = 0; k < kPieces; ++k)
             cp_async16_zfill((k & 1 ? d1 : d0) + 512u * k, src + 512 * k, 16u);
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncwarp();
-        const uint8_t *mine = dist_s + tid * kPer;
-#pragma unroll
-        for (int v = 0; v < kPieces; ++v)
-            dv[v] = *reinterpret_cast<const uint4 *>(mine + 16 * (v ^ (tid & 7)));
     } else {  // the row's last tile: pieces past the row read as padding
 #pragma unroll
         for (int k = 0; k < kPieces; ++k) {
@@ -130,9 +126,41 @@ __global__ void __launch_bounds__(kThreads, kWide ? 2 : 4) select_kernel(SelectA
             cp_async16_zfill(sbase + uint32_t(t * kPer + 16 * (v ^ (t & 7))), in ? drow + g : drow,
                              in ? 16u : 0u);
         }
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncwarp();
+    }
+    cp_async_commit();
+    if (many) {
+        const int warp = tid >> 5;
+        uint32_t tot[5], pre[5];
+        tile_sums(hrow, int(a.n_tiles), warp, kWarps, tile, lane, tot, pre);
+#pragma unroll
+        for (int e = 0; e < 5; ++e) {
+            hsum[warp][0][lane * 5 + e] = tot[e];
+            hsum[warp][1][lane * 5 + e] = pre[e];
+        }
+        __syncthreads();
+        if (warp == 0) {
+#pragma unroll
+            for (int e = 0; e < 5; ++e) {
+                uint32_t t = 0u, p = 0u;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) {
+                    t += hsum[w][0][lane * 5 + e];
+                    p += hsum[w][1][lane * 5 + e];
+                }
+                tot[e] = t;
+                pre[e] = p;
+            }
+            threshold_from_sums(tot, pre, k_eff, lane, s_thr);
+        }
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+    if (full) {
+        const uint8_t *mine = dist_s + tid * kPer;
+#pragma unroll
+        for (int v = 0; v < kPieces; ++v)
+            dv[v] = *reinterpret_cast<const uint4 *>(mine + 16 * (v ^ (tid & 7)));
+    } else {
 #pragma unroll
         for (int v = 0; v < kPieces; ++v)
             dv[v] = my0 + 16 * v < a.dist_row

@@ -177,6 +177,80 @@ __device__ __forceinline__ void head_threshold(const uint32_t *hrow, int n_tiles
     }
 }
 
+// Partial sums of one head's tile histograms (hrow: n_tiles rows of
+// kHistStride words) over the tiles first, first + step, ...: tot = all of
+// them, pre = those before `tile`.  Lane l: bins 5l .. 5l+4.  The loads of
+// up to 4 tiles are issued before any is summed.
+__device__ __forceinline__ void tile_sums(const uint32_t *hrow, int n_tiles, int first, int step,
+                                          int tile, int lane, uint32_t (&tot)[5],
+                                          uint32_t (&pre)[5])
+{
+#pragma unroll
+    for (int e = 0; e < 5; ++e) tot[e] = pre[e] = 0u;
+    for (int t0 = first; t0 < n_tiles; t0 += 4 * step) {
+        uint32_t rv[4][5];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int t = t0 + r * step;
+#pragma unroll
+            for (int e = 0; e < 5; ++e)
+                rv[r][e] = t < n_tiles && lane * 5 + e < kBins
+                               ? __ldg(hrow + t * kHistStride + lane * 5 + e)
+                               : 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int e = 0; e < 5; ++e) {
+                tot[e] += rv[r][e];
+                pre[e] += t0 + r * step < tile ? rv[r][e] : 0u;
+            }
+    }
+}
+
+// head_threshold's second half: T, #(< T), and the keys below / at T in
+// the tiles before this one, from the summed bins (lane l: bins 5l ..
+// 5l+4); one warp; out as head_threshold's.
+__device__ __forceinline__ void threshold_from_sums(const uint32_t (&tot)[5],
+                                                    const uint32_t (&pre)[5], int k_eff, int lane,
+                                                    int *out)
+{
+    const uint32_t run = tot[0] + tot[1] + tot[2] + tot[3] + tot[4];
+    uint32_t acc = uint32_t(warp_inclusive_scan(int(run))) - run;
+    int Tl = -1;
+    uint32_t less_l = 0;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+        if (Tl < 0 && lane * 5 + e < kBins && acc + tot[e] >= uint32_t(k_eff)) {
+            Tl = lane * 5 + e;
+            less_l = acc;
+        }
+        acc += tot[e];
+    }
+    const unsigned found = __ballot_sync(0xffffffffu, Tl >= 0);
+    const int src = found ? __ffs(int(found)) - 1 : 0;
+    const int T = found ? __shfl_sync(0xffffffffu, Tl, src) : kBins - 1;  // unreachable fallback
+    const int n_less = found ? __shfl_sync(0xffffffffu, int(less_l), src) : 0;
+    int l = 0, q = 0;
+#pragma unroll
+    for (int e = 0; e < 5; ++e) {
+        const int bin = lane * 5 + e;
+        l += bin < T ? int(pre[e]) : 0;
+        q += bin == T ? int(pre[e]) : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+        q += __shfl_xor_sync(0xffffffffu, q, o);
+    }
+    if (lane == 0) {
+        out[0] = T;
+        out[1] = n_less;
+        out[2] = l;
+        out[3] = q;
+    }
+}
+
 // Store the tokens of the set bits of sel (bit 8e + w <-> token tok + 4w + e)
 // at positions pos + (their rank in token order), without transposing the
 // word: the rank of a bit is the number of set bits of lower tokens (lower w,
