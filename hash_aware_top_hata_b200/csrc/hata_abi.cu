@@ -34,13 +34,13 @@ bool use_fused(hata_dtype_t kv_dtype, int r)
            (m == HATA_MODE_FUSED || (m == HATA_MODE_AUTO && kAutoFused));
 }
 
-// The cluster step serves bf16 caches with 128-bit codes when the mode asks
-// for it (or AUTO picks it) and the sizes fit (cluster_step_fits).
+// The cluster step serves 128-bit codes when the mode asks for it (or AUTO
+// picks it) and the sizes fit (cluster_step_plan).
 bool want_cluster(hata_dtype_t kv_dtype, int r)
 {
     const int m = g_mode.load();
-    return kv_dtype == HATA_DT_BF16 && r == kRbit &&
-           (m == HATA_MODE_CLUSTER || (m == HATA_MODE_AUTO && kAutoCluster));
+    (void)kv_dtype;
+    return r == kRbit && (m == HATA_MODE_CLUSTER || (m == HATA_MODE_AUTO && kAutoCluster));
 }
 
 hata_status_t fail(hata_status_t st, const char *fmt, ...)
@@ -244,7 +244,8 @@ int hata_decode_kernel_launches(int B, int H_q, int H_kv, int64_t max_seq_len, i
     if (use_fused(kv_dtype, r)) return 3;  // prep, score, the selection + attention kernel
     if (want_cluster(kv_dtype, r)) {
         ClusterPlan plan;
-        if (cudaError_t e = cluster_step_plan(B, H_q, H_kv, max_seq_len, topk, &plan)) {
+        if (cudaError_t e = cluster_step_plan(B, H_q, H_kv, max_seq_len, topk,
+                                              kv_dtype == HATA_DT_BF16, &plan)) {
             cuda_fail(e, "cluster occupancy query");
             return -1;
         }
@@ -470,7 +471,8 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
     cudaError_t e;
     if (want_cluster(kv_dtype, r)) {
         ClusterPlan plan;
-        if ((e = cluster_step_plan(B, H_q, H_kv, max_seq_len, topk, &plan)) != cudaSuccess)
+        if ((e = cluster_step_plan(B, H_q, H_kv, max_seq_len, topk, kv_dtype == HATA_DT_BF16,
+                                   &plan)) != cudaSuccess)
             return cuda_fail(e, "cluster occupancy query");
         if (plan.kM) {
             ClusterArgs ca{};
@@ -497,6 +499,7 @@ hata_status_t hata_decode_step(const float *q, const float *W_H, uint32_t *codes
             ca.G = H_q / H_kv;
             ca.topk = topk;
             ca.tok_per_cta = plan.tok_per_cta;
+            ca.kv_bf16 = kv_dtype == HATA_DT_BF16;
             ca.scale_log2 = scale * 1.4426950408889634f;
             if ((e = ev.record(0)) != cudaSuccess) return cuda_fail(e, "event record");
             if ((e = launch_cluster_step(ca, plan, s)) != cudaSuccess)

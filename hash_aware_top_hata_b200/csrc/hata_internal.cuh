@@ -219,9 +219,9 @@ struct ClusterArgs {
     const float *q;          // [B][H_q][128]; device or mapped host
     const float *W;          // [H_kv][128][128]
     uint32_t *codes;         // [B][H_kv][n_cap][4]; the new key's code is written
-    void *K, *V;             // bf16 caches; the new rows written if v_new
-    const void *k_new;       // [B][H_kv][128] bf16 or null
-    const void *v_new;       // [B][H_kv][128] bf16 or null
+    void *K, *V;             // bf16 or fp32 caches; the new rows written if v_new
+    const void *k_new;       // [B][H_kv][128] (cache dtype) or null
+    const void *v_new;       // [B][H_kv][128] (cache dtype) or null
     const int32_t *seq_len;
     uint32_t *q_out;         // [B][H_q][4] or null
     uint8_t *dist;           // caller's distance rows or null
@@ -233,6 +233,7 @@ struct ClusterArgs {
     int64_t n_cap, max_seq_len;
     int B, H_q, H_kv, G, topk;
     int tok_per_cta;         // tokens of a CTA's range (a multiple of 32; the plan's)
+    int kv_bf16;             // 1: bf16 caches, 0: fp32
     float scale_log2;
 };
 
@@ -329,9 +330,9 @@ cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s);
 cudaError_t attend_launch_count(int B, int H_q, int topk, bool bf16, int *n);
 cudaError_t launch_dense(const DenseArgs &a, bool bf16, cudaStream_t s);
 cudaError_t launch_fused(const FusedArgs &a, cudaStream_t s);
-// The cluster step's plan for these sizes on this device (bf16 K/V and
-// r = 128 are the caller's checks); plan->kM == 0 when it does not serve them.
-cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
+// The cluster step's plan for these sizes on this device (r = 128 is the
+// caller's check); plan->kM == 0 when it does not serve them.
+cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int topk, bool bf16,
                               ClusterPlan *plan);
 cudaError_t launch_cluster_step(const ClusterArgs &a, const ClusterPlan &p, cudaStream_t s);
 // Sequence-parallel step: the attention of one shard's selected keys split

@@ -37,7 +37,7 @@
 //
 // Every CTA of a cluster is resident at once (the hardware schedules a
 // cluster as a unit), so the two barriers cannot wait on a CTA that never
-// runs.  bf16 K/V, r = 128, G in {1, 2, 4}.  512 threads: all 16 warps scan
+// runs.  bf16 or fp32 K/V, r = 128, G in {1, 2, 4}.  512 threads: all 16 warps scan
 // and select (the scan is latency-bound, so warps matter), the first 8
 // attend (their rings take the 128 KB that held W_H and the code chunks);
 // 126 registers, no spills.
@@ -116,7 +116,7 @@ __device__ __forceinline__ void copy_chunk(const uint4 *codes, int c, int nloc, 
     cp_async_commit();
 }
 
-template <int kM>
+template <int kM, bool kBF16>
 __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs a)
 {
     constexpr int kCTok = ClusterSmem<kM>::kTok;  // token capacity of a CTA
@@ -188,10 +188,13 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
         }
     }
     if (append) {
-        // stage k_new (bf16, widened exactly) in the merge buffer, then hash
+        // stage k_new (bf16 widened exactly, or fp32) in the merge buffer,
+        // then hash
         float *xk = S.merged[0][0];
-        const uint16_t *kn = static_cast<const uint16_t *>(a.k_new) + (int64_t(b) * a.H_kv + h) * kD;
-        for (int i = tid; i < kD; i += kCThreads) xk[i] = __uint_as_float(uint32_t(kn[i]) << 16);
+        const int64_t e0 = (int64_t(b) * a.H_kv + h) * kD;
+        for (int i = tid; i < kD; i += kCThreads)
+            xk[i] = kBF16 ? __uint_as_float(uint32_t(static_cast<const uint16_t *>(a.k_new)[e0 + i]) << 16)
+                          : static_cast<const float *>(a.k_new)[e0 + i];
         __syncthreads();
         if (tid < kRbit) {
             const bool bit = hash_bit(xk, Ws, tid);
@@ -204,10 +207,16 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
         }
         if (a.v_new && tid >= kRbit && tid < 2 * kRbit) {  // K and V rows of the new token
             const int e = tid - kRbit;  // 0..127
-            const uint16_t *vn =
-                static_cast<const uint16_t *>(a.v_new) + (int64_t(b) * a.H_kv + h) * kD;
-            static_cast<uint16_t *>(a.K)[(slab + pos) * kD + e] = kn[e];
-            static_cast<uint16_t *>(a.V)[(slab + pos) * kD + e] = vn[e];
+            if (kBF16) {
+                static_cast<uint16_t *>(a.K)[(slab + pos) * kD + e] =
+                    static_cast<const uint16_t *>(a.k_new)[e0 + e];
+                static_cast<uint16_t *>(a.V)[(slab + pos) * kD + e] =
+                    static_cast<const uint16_t *>(a.v_new)[e0 + e];
+            } else {
+                static_cast<float *>(a.K)[(slab + pos) * kD + e] = xk[e];
+                static_cast<float *>(a.V)[(slab + pos) * kD + e] =
+                    static_cast<const float *>(a.v_new)[e0 + e];
+            }
         }
     }
     __syncthreads();
@@ -382,7 +391,72 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
     __syncthreads();  // the CTA's list entries (global memory) and counts are visible
 
     // ---- 5. gather + attention over this CTA's entries, G heads side by side ----
-    if (warp < kAWarps) {
+    if (!kBF16 && warp < kAWarps) {
+        // fp32 K/V: CUDA cores, 4 rows a batch (their loads first), lane l
+        // holding dims 4l .. 4l+3, scores reduced across the warp; scores in
+        // log2 units (q pre-scaled by scale_log2), as in the bf16 stage
+        const int wpg = kAWarps / G;
+        const int g = warp / wpg, sub = warp - g * wpg;
+        const int start = S.sel[g][2], cnt = S.sel[g][3];
+        const int r0 = start + int(int64_t(sub) * cnt / wpg);
+        const int r1 = start + int(int64_t(sub + 1) * cnt / wpg);
+        const int32_t *idx = a.idx + (bh0 + g) * a.topk;
+        const float4 *Kf = reinterpret_cast<const float4 *>(static_cast<const float *>(a.K) + slab * kD);
+        const float4 *Vf = reinterpret_cast<const float4 *>(static_cast<const float *>(a.V) + slab * kD);
+        float4 q4 = reinterpret_cast<const float4 *>(S.q[g])[lane];
+        q4.x *= a.scale_log2; q4.y *= a.scale_log2; q4.z *= a.scale_log2; q4.w *= a.scale_log2;
+        float m = -INFINITY, l = 0.0f, acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int x0 = r0; x0 < r1; x0 += 4) {
+            int32_t row[4];
+            float4 kr[4], vr[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                row[u] = x0 + u < r1 ? idx[x0 + u] : -1;
+                // the selection never yields an index outside [0, len)
+                if (row[u] >= len) row[u] = -1;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                kr[u] = row[u] >= 0 ? Kf[int64_t(row[u]) * (kD / 4) + lane] : z;
+                vr[u] = row[u] >= 0 ? Vf[int64_t(row[u]) * (kD / 4) + lane] : z;
+            }
+            float sc[4], mx = m;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float d = q4.x * kr[u].x;
+                d = fmaf(q4.y, kr[u].y, d);
+                d = fmaf(q4.z, kr[u].z, d);
+                d = fmaf(q4.w, kr[u].w, d);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                sc[u] = row[u] >= 0 ? d : -INFINITY;
+                mx = fmaxf(mx, sc[u]);
+            }
+            if (mx == -INFINITY) continue;  // warp-uniform
+            const float alpha = m == -INFINITY ? 0.0f : exp2f(m - mx);
+            l *= alpha;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] *= alpha;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float pu = sc[u] == -INFINITY ? 0.0f : exp2f(sc[u] - mx);
+                l += pu;
+                acc[0] = fmaf(pu, vr[u].x, acc[0]);
+                acc[1] = fmaf(pu, vr[u].y, acc[1]);
+                acc[2] = fmaf(pu, vr[u].z, acc[2]);
+                acc[3] = fmaf(pu, vr[u].w, acc[3]);
+            }
+            m = mx;
+        }
+        if (lane == 0) {
+            S.part[warp][0] = m;
+            S.part[warp][1] = l;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) S.part[warp][4 + 4 * lane + i] = acc[i];
+    }
+    if (kBF16 && warp < kAWarps) {
         using namespace tc;
         const int wpg = kAWarps / G;  // warps per head
         const int g = warp / wpg, sub = warp - g * wpg;
@@ -504,13 +578,13 @@ cudaLaunchConfig_t cluster_cfg(int64_t ctas, int C, cudaStream_t s, cudaLaunchAt
 
 // Clusters of C CTAs (instantiation kM) the current device holds at once;
 // queried once per (device, C) and kept.
-template <int kM>
+template <int kM, bool kBF16>
 cudaError_t resident_clusters(int C, int *clusters)
 {
     int dev = 0;
     if (cudaError_t e = cudaGetDevice(&dev)) return e;
     static std::mutex mu;
-    static std::map<std::pair<int, int>, int> known;  // (device, C) -> clusters
+    static std::map<std::pair<int, int>, int> known;  // (device, C) -> clusters (per kernel)
     {
         std::lock_guard<std::mutex> lock(mu);
         auto it = known.find({dev, C});
@@ -519,12 +593,13 @@ cudaError_t resident_clusters(int C, int *clusters)
             return cudaSuccess;
         }
     }
-    const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<kM>);
+    const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<kM, kBF16>);
     if (cudaError_t e = ensure_smem_attr(fn, sizeof(ClusterSmem<kM>))) return e;
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = cluster_cfg<kM>(C, C, nullptr, attr);
     int n = 0;
-    if (cudaError_t e = cudaOccupancyMaxActiveClusters(&n, cluster_step_kernel<kM>, &cfg)) return e;
+    if (cudaError_t e = cudaOccupancyMaxActiveClusters(&n, cluster_step_kernel<kM, kBF16>, &cfg))
+        return e;
     std::lock_guard<std::mutex> lock(mu);
     known[{dev, C}] = n;
     *clusters = n;
@@ -537,7 +612,7 @@ cudaError_t resident_clusters(int C, int *clusters)
 // tokens a head needs (C <= 8), each taking an equal range (a multiple of
 // 32 tokens), when every cluster fits the device at once.  plan->kM = 0:
 // the step does not serve them.
-cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int topk,
+cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int topk, bool bf16,
                               ClusterPlan *plan)
 {
     *plan = ClusterPlan{};
@@ -548,7 +623,8 @@ cudaError_t cluster_step_plan(int B, int H_q, int H_kv, int64_t max_seq_len, int
         const int64_t C = ceil_div(max_seq_len, int64_t(8192) * kM);
         if (C > kClusterMaxC) continue;
         int clusters = 0;
-        cudaError_t e = resident_clusters<2>(int(C), &clusters);
+        cudaError_t e = bf16 ? resident_clusters<2, true>(int(C), &clusters)
+                             : resident_clusters<2, false>(int(C), &clusters);
         if (e != cudaSuccess) return e;
         if (clusters > 0 && int64_t(clusters) >= slabs) {  // one wave
             plan->kM = kM;
@@ -565,10 +641,11 @@ cudaError_t launch_cluster_step(const ClusterArgs &a, const ClusterPlan &p, cuda
     const int64_t ctas = int64_t(p.C) * a.B * a.H_kv;
     cudaLaunchAttribute attr[1];
     if (p.kM == 2) {
-        const void *fn = reinterpret_cast<const void *>(cluster_step_kernel<2>);
+        auto kernel = a.kv_bf16 ? cluster_step_kernel<2, true> : cluster_step_kernel<2, false>;
+        const void *fn = reinterpret_cast<const void *>(kernel);
         if (cudaError_t e = ensure_smem_attr(fn, sizeof(ClusterSmem<2>))) return e;
         cudaLaunchConfig_t cfg = cluster_cfg<2>(ctas, p.C, s, attr);
-        return cudaLaunchKernelEx(&cfg, cluster_step_kernel<2>, a);
+        return cudaLaunchKernelEx(&cfg, kernel, a);
     }
     return cudaErrorInvalidValue;
 }

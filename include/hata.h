@@ -152,9 +152,9 @@ int hata_decode_kernel_launches(int B, int H_q, int H_kv, int64_t max_seq_len, i
  *   the cluster step       ONE kernel: a thread-block cluster per (b, h_kv)
  *                          of up to 8 CTAs of up to 16384 tokens each hashes,
  *                          scores, selects and attends, the CTAs meeting
- *                          through distributed shared memory (bf16 caches,
- *                          r = 128, H_q / H_kv of 1, 2 or 4, max_seq_len up
- *                          to 131072, every cluster resident at once).
+ *                          through distributed shared memory (r = 128,
+ *                          H_q / H_kv of 1, 2 or 4, max_seq_len up to
+ *                          131072, every cluster resident at once).
  * A step whose sizes the chosen implementation does not serve takes the
  * multi-kernel step.
  *   HATA_MODE_AUTO          the library's choice (default): the cluster step

@@ -233,8 +233,9 @@ def test_workspace_check_rejects_bad_workspace():
 
 def test_decode_kernel_launches_host_logic():
     L = H.lib()
-    # fp32 caches take the SIMT attention kernel, always followed by the combine
-    assert H.hata_decode_kernel_launches(4, 32, 8, 131072, 2048, torch.float32) == 5
+    # fp32 caches beyond the cluster step's reach (more than 8 x 16384 keys)
+    # take the SIMT attention kernel, always followed by the combine
+    assert H.hata_decode_kernel_launches(4, 32, 8, 200000, 2048, torch.float32) == 5
     # bf16 caches in the fused step: prep, score, the selection + attention kernel
     H.hata_set_decode_mode(H.HATA_MODE_FUSED)
     try:

@@ -26,7 +26,8 @@ def cluster_mode():
 
 
 def _launches(cfg, n_cap):
-    return H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.H_kv, n_cap, cfg.topk, torch.bfloat16)
+    dt = torch.bfloat16 if cfg.kv_dtype == "bf16" else torch.float32
+    return H.hata_decode_kernel_launches(cfg.B, cfg.H_q, cfg.H_kv, n_cap, cfg.topk, dt)
 
 
 CASES = {
@@ -38,6 +39,9 @@ CASES = {
     "16k_ctas_gqa4": wl.Config("c", 4, 32, 8, 40000, 1500, "bf16", 0.02, 0.3, 0, 2),
     "llama2_shape": wl.Config("c", 1, 32, 32, 32768, 512, "bf16", 0.02, 0.3, 0, 2),
     "k_above_n": wl.Config("c", 2, 4, 2, 3000, 5000, "bf16", 0.0, 0.0, 0, 2),
+    "fp32_mha": wl.Config("c", 1, 4, 4, 6000, 200, "f32", 0.02, 0.3, 0, 2),
+    "fp32_gqa2_three_ctas": wl.Config("c", 2, 8, 4, 40000, 700, "f32", 0.02, 0.3, 0, 2),
+    "tiny_shape": wl.Config("c", 1, 1, 1, 4096, 64, "f32", 0.0, 0.0, 0, 2),
 }
 
 
