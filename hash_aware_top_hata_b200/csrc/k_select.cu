@@ -1,7 +1,7 @@
 // k_select.cu -- top-k selection over the Hamming distances, no sort.
 //
 // HATA review page (arXiv 2506.02572), major comment 1 (Algorithm 3): the
-// top-k runs over Hamming scores that take only 129 values, so the boundary
+// top-k runs over Hamming scores that take only r + 1 values, so the boundary
 // usually falls inside a large bucket of equal scores; the page leaves the
 // choice inside that bucket open.  Here it goes to the lower token index, so
 // the selected set is unique:
@@ -11,10 +11,11 @@
 //           keys with dist[n] == T.
 //
 // Grid: (36K-token tile, b * H_q + h_q), 288 threads, each thread owning 128
-// consecutive distances (eight 16-byte loads, issued first).  Warp 0 sums
-// the head's tile histograms (written by the scoring kernel) while they are
-// in flight: the total gives T and r, the tiles before this one the keys
-// below T and at T already placed.
+// consecutive distances (eight 16-byte loads, issued first).  The head's
+// tile histograms (written by the scoring kernel) are summed while those
+// loads are in flight -- by warp 0 for up to 4 tiles, by every warp for a
+// share of more (one round trip to L2 either way): the total gives T and
+// r, the tiles before this one the keys below T and at T already placed.
 // Each thread turns its 128 distances into "< T" and "== T" bit masks with
 // byte-wise integer compares, ONE block scan of the two counts gives every
 // thread its output position, and the ties a thread may take follow from
