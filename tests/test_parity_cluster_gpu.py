@@ -12,7 +12,7 @@ import torch
 
 from hash_aware_top_hata_b200 import hata as H
 from hash_aware_top_hata_b200 import workloads as wl
-from tests.gpu_cases import GpuDecoder, compare_head, host_slabs, oracle_head
+from tests.gpu_cases import GpuDecoder, compare_head, host_slabs, oracle_head, to_np_codes
 from tests.test_parity_gpu import run_and_check
 
 pytestmark = pytest.mark.gpu
@@ -109,3 +109,34 @@ def test_cluster_step_is_bitwise_repeatable_and_matches_multi_kernel():
     c = dec.step(w.q[0], [cfg.N, cfg.N - 77])
     assert np.array_equal(a[1], c[1]) and np.array_equal(a[2], c[2]) and np.array_equal(a[3], c[3])
     assert np.max(np.abs(a[0] - c[0])) <= 1e-4
+
+
+def test_cluster_append_lands_in_first_and_middle_ctas():
+    """The new token's code and K/V rows are written by the CTA whose range
+    holds position seq_len - 1: here the first CTA of one row's cluster and
+    a middle CTA of another's (max_seq_len 40000: three CTAs of ~13.3K)."""
+    cfg = wl.Config("c-app", 2, 8, 4, 40000, 300, "bf16", 0.02, 0.3, 0, 1)
+    w = wl.make_workload(cfg, 98, device="cuda", steps=1)
+    dec = GpuDecoder(w, cfg.topk, max_seq_len=40000)
+    assert _launches(cfg, 40000) == 1
+    lens = [100, 20000]  # appends at 99 (CTA 0) and 19999 (CTA 1)
+    pairs = [(b, h) for b in range(2) for h in range(4)]
+    slabs = host_slabs(w, pairs)
+    kn, vn = wl.to_numpy_kv(w.k_new[0]), wl.to_numpy_kv(w.v_new[0])
+    for (b, h), sl in slabs.items():
+        sl.K[lens[b] - 1] = kn[b, h]
+        sl.V[lens[b] - 1] = vn[b, h]
+    got = dec.step(w.q[0], lens, k_new=w.k_new[0], v_new=w.v_new[0])
+    Wn = w.W_H.cpu().numpy()
+    gcodes = to_np_codes(dec.codes)
+    for b in range(2):
+        for hq in range(8):
+            h = hq // 2
+            n = lens[b]
+            want = oracle_head(slabs[(b, h)], Wn[h], w.q[0, b, hq].cpu().numpy(), n, cfg.topk)
+            assert np.array_equal(gcodes[b, h, :n], want[0]), ("key codes", b, h)
+            compare_head(got, want, b, hq, n, dec.drow)
+    for (b, h), sl in slabs.items():  # the appended rows reached the caches
+        p = lens[b] - 1
+        assert np.array_equal(wl.to_numpy_kv(w.K[b, h, p]), sl.K[p])
+        assert np.array_equal(wl.to_numpy_kv(w.V[b, h, p]), sl.V[p])
