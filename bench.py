@@ -860,6 +860,8 @@ def run_hata(args, world, rank, local):
         line["other_workloads"]["llama31_8b_gqa_128k_r256"] = wide_code_leg(dev)
         line["other_workloads"]["needle_gqa_1m_seqpar8"] = seqpar_leg(dev)
     if rank == 0:
+        from hash_aware_top_hata_b200 import build as hb
+        line["build"] = hb.build_record()  # the library that ran, and its sources
         print(json.dumps(line), flush=True)
 
 

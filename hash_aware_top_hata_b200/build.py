@@ -11,6 +11,8 @@ from __future__ import annotations
 import argparse
 import concurrent.futures as cf
 import glob
+import hashlib
+import json
 import os
 import shutil
 import subprocess
@@ -22,6 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libhata.so")
+STAMP = os.path.join(PKG, "libhata.build.json")  # what the library was built from
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
               "--expt-relaxed-constexpr"]
@@ -41,6 +44,27 @@ def _sources() -> list[str]:
 def _deps() -> list[str]:
     return (_sources() + glob.glob(os.path.join(CSRC, "*.cuh"))
             + glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)])
+
+
+def sources_sha256() -> str:
+    """Digest of every file the library is built from (names and contents)."""
+    h = hashlib.sha256()
+    for p in sorted(_deps()):
+        h.update(os.path.relpath(p, ROOT).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def build_record() -> dict:
+    """The stamp written next to the library at link time, and whether the
+    sources still match it (False: the library predates a source change)."""
+    rec = {}
+    if os.path.exists(STAMP):
+        with open(STAMP) as f:
+            rec = json.load(f)
+    rec["matches_sources"] = rec.get("sources_sha256") == sources_sha256()
+    return rec
 
 
 def up_to_date() -> bool:
@@ -78,6 +102,11 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    ver = subprocess.run([nvcc(), "--version"], capture_output=True, text=True).stdout
+    with open(STAMP, "w") as f:
+        json.dump({"sources_sha256": sources_sha256(),
+                   "nvcc": ver.strip().splitlines()[-1] if ver.strip() else "",
+                   "flags": ARCH + NVCC_FLAGS}, f)
     return LIB
 
 

@@ -252,3 +252,11 @@ def test_decode_kernel_launches_host_logic():
         assert L.hata_decode_kernel_launches(*bad) == -1
     with pytest.raises(H.HataError):
         H.hata_decode_kernel_launches(4, 32, 8, 4096, -1, torch.bfloat16)
+
+
+def test_library_build_record_matches_sources():
+    """libhata.so carries a stamp of the sources it was built from; the
+    library under test is the one these sources make."""
+    from hash_aware_top_hata_b200 import build as hb
+    rec = hb.build_record()
+    assert rec.get("sources_sha256") and rec["matches_sources"], rec
