@@ -8,30 +8,35 @@
 // The work is the flat sequence of 128-token units over all (b, h_kv, group
 // of <= 8 query heads) slabs; CTA c takes one contiguous range of about
 // U / gridDim.x units, so every CTA gets the same amount of work whatever
-// the shapes.  Within its range the CTA's eight warps take units in
-// round-robin order (warp w: units w, w+8, ...) with no block-wide barrier:
-// lane l owns tokens l, l+32, l+64, l+96 of a unit (four coalesced 16-byte
-// loads per warp instruction).  The loads are asynchronous copies
-// (cp.async) into a per-warp ring of kRing units in shared memory, issued
-// kRing-1 units ahead; every lane reads back only the bytes it copied, so a
-// lane's own wait_group is the only synchronisation, and the codes in
-// flight cost no registers.  The code stream is read from HBM exactly once
-// per KV head.  Each code is scored against every query head of the group:
+// the shapes.  Within its range the CTA's 32 warps take units in the
+// order they free up, with no block-wide barrier: lane l scores tokens
+// 4l .. 4l+3 of a unit.  The codes arrive by asynchronous copies (cp.async)
+// into a per-warp ring of kRing units in shared memory, issued kRing-1
+// units ahead: lane l copies tokens l, l+32, l+64, l+96 (coalesced 16-byte
+// pieces), each landing in the 64-byte row of the lane that scores it at a
+// column XOR-ed with the row (so both the copies and the row reads are free
+// of bank conflicts); a wait_group then a warp barrier make the unit
+// visible, and the codes in flight cost no registers.  The code stream is
+// read from HBM exactly once per KV head.  Each code is scored against every
+// query head of the group with a bitwise carry-save sum of its four XOR-ed
+// words (x_w = code_w XOR q_w):
 //
-//   x_w = code_w XOR q_w (w = 0..3)
-//   (s, c)    = full-add(x0, x1, x2)    -- bitwise carry-save adder
-//   (ones, c2) = half-add(s, x3)
-//   dist = popc(ones) + 2 popc(c XOR c2) + 4 popc(c AND c2)
+//   u = x0 ^ x1, v = x2 ^ x3                     (pair sums, weight 1)
+//   c = u ? v : x0,  e = x2 & ~v                 (their carries, weight 2)
+//   dist = popc(u ^ v) + 2 (popc(c) + popc(e))
 //
-// i.e. three population counts instead of four: POPC issues at an eighth of
-// the integer-logic rate on sm_100a, and it is what bounds the arithmetic.
-// Codes of 32 or 64 bits (the ablation widths) take 4- or 8-byte copies
-// into the same 16-byte ring slots and one or two population counts.
+// i.e. three population counts instead of four (POPC issues at an eighth
+// of the integer-logic rate on sm_100a, and it is what bounds the
+// arithmetic), and six logic operations, since u and v take the key's
+// words as k0 ^ k1 and k2 ^ k3, shared by the group's heads.  Codes of 32
+// or 64 bits (the ablation widths) take 4- or 8-byte copies into the same
+// 16-byte ring slots and one or two population counts.
 //
-// Per query head the kernel stores the u8 distance row (32 lanes write 32
-// consecutive bytes per store; the row stays L2-resident for the selection
-// kernel) and counts a 129-bin histogram per (head, 36K-token tile) in
-// shared memory; a range touches at most kMaxKeys (slab, tile) pairs.  At
+// Per query head the kernel stores the u8 distance row (a lane's four
+// distances as one 32-bit word: a warp writes the head's 128 bytes of the
+// unit at once; the row stays L2-resident for the selection kernel) and
+// counts a 129-bin histogram per (head, 36K-token tile) in shared memory;
+// a range touches at most kMaxKeys (slab, tile) pairs.  At
 // the end of its range the CTA adds the non-zero bins into the tile
 // histograms in global memory (zeroed by the prep kernel), one reduction
 // per bin, so the selection kernel finds both the boundary distance and the
@@ -51,7 +56,7 @@
 namespace hata {
 namespace {
 
-constexpr int kWarps = kScoreThreads / 32;  // 8
+constexpr int kWarps = kScoreThreads / 32;  // 32
 constexpr int kUnit = 128;                  // tokens per warp step
 constexpr int kRing = 2;                    // units per warp ring
 constexpr int kTileUnits = kTile / kUnit;   // 288
@@ -64,38 +69,37 @@ __device__ __forceinline__ void red_shared_add1(uint32_t addr)
     asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
 
-// One unit's distances against the GB query heads of its group: byte
-// g*128 + 32i of the warp's tile (base tb = tile + lane) and one count in
-// bin d of head g (base hb).  kFull: all 128 tokens hold keys; otherwise the
+// One unit's distances against the GB query heads of its group: lane l's
+// tokens 4l .. 4l+3 (codes cur[i]) as one 32-bit word per head at word l of
+// the head's row (row + g * dist_row), and one count in bin d of head g
+// (histogram base hb).  kFull: all 128 tokens hold keys; otherwise the
 // tokens from nv on get the pad byte and no count.
 template <int GB, int W, bool kFull>
 __device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *qs,
-                                           const uint2 *qd, int ng, uint32_t tb, uint32_t hb,
-                                           int lane, int nv)
+                                           const uint2 *qp, int ng, uint8_t *row,
+                                           int64_t dist_row, uint32_t hb, int lane, int nv)
 {
-    uint32_t k012[4], k0123[4];
+    uint2 kp[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        k012[i] = W == 4 ? cur[i].x ^ cur[i].y ^ cur[i].z : 0u;
-        k0123[i] = W == 4 ? k012[i] ^ cur[i].w : 0u;
-    }
+    for (int i = 0; i < 4; ++i)
+        kp[i] = W == 4 ? make_uint2(cur[i].x ^ cur[i].y, cur[i].z ^ cur[i].w) : make_uint2(0u, 0u);
 #pragma unroll
     for (int g = 0; g < GB; ++g) {
         if (g < ng) {
             const uint4 q = qs[g];
-            const uint2 qx = qd[g];
+            const uint2 qx = qp[g];
+            uint32_t word = 0u;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t d = uint32_t(hamming_w<W>(cur[i], k012[i], k0123[i], q, qx));
-                const uint32_t t = tb + uint32_t(g * kUnit + 32 * i);
-                if (kFull || lane + 32 * i < nv) {
-                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(t), "r"(d) : "memory");
+                const uint32_t d = uint32_t(hamming_w<W>(cur[i], kp[i], q, qx));
+                if (kFull || 4 * lane + i < nv) {
                     red_shared_add1(hb + uint32_t(g * kHistStride * 4) + 4u * d);
+                    word |= d << (8 * i);
                 } else {
-                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(t), "r"(uint32_t(kDistPad))
-                                 : "memory");
+                    word |= uint32_t(kDistPad) << (8 * i);
                 }
             }
+            __stcg(reinterpret_cast<uint32_t *>(row + g * dist_row) + lane, word);
         }
     }
 }
@@ -103,7 +107,7 @@ __device__ __forceinline__ void score_unit(const uint4 (&cur)[4], const uint4 *q
 // A (slab, tile) histogram key of the CTA range: where its rows live.
 struct KeyInfo {
     uint4 q[kScoreHeads];  // query codes of the slab's heads
-    uint2 qd[kScoreHeads]; // their q0 ^ q1 ^ q2 and q0 ^ q1 ^ q2 ^ q3
+    uint2 qp[kScoreHeads]; // their q0 ^ q1 and q2 ^ q3
     int64_t code0;         // first code (uint4 index) of the slab
     int64_t dist0;         // first distance byte of head 0 of the slab
     int len, ng, slab, pad;
@@ -114,7 +118,6 @@ struct ScoreSmem {
     uint4 ring[kWarps][kRing][kUnit];           // 2 KB per unit
     KeyInfo key[kMaxKeys];
     uint32_t hist[kMaxKeys][GB][kHistStride];
-    uint8_t tile[kWarps][GB < 4 ? 4 : (GB + 3) / 4 * 4][kUnit];  // a unit's distances
     uint32_t unit[kMaxRange];                   // per unit of the range: key << 28 | unit in slab
     int next;                                   // units of the range handed out
 };
@@ -178,8 +181,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
             }
         }
         S.key[kk].q[g] = v;
-        const uint32_t q012 = v.x ^ v.y ^ v.z;
-        S.key[kk].qd[g] = make_uint2(q012, q012 ^ v.w);
+        S.key[kk].qp[g] = make_uint2(v.x ^ v.y, v.z ^ v.w);
     }
     __syncthreads();
 
@@ -193,6 +195,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
         if (lane == 0) u = atomicAdd(&S.next, 1);
         return __shfl_sync(0xffffffffu, u, 0);
     };
+    // Token p of a unit lands in row p / 4 (the lane that scores it), at
+    // 16-byte column (p % 4) ^ (p / 8 % 4).  Lane l copies tokens l + 32 i,
+    // at byte 64 (l / 4) + 16 ((l % 4) ^ (l / 8 % 4)) + 512 i of the slot;
+    // it reads token 4 l + i back from column i ^ (l / 2 % 4) of row l.
+    const uint32_t copy_off = 64u * uint32_t(lane >> 2) + 16u * uint32_t((lane & 3) ^ ((lane >> 3) & 3));
     // issue the copies of unit u (range-relative) into ring slot `slot`
     auto issue = [&](int u, int slot) {
         asm volatile("" ::: "memory");  // earlier reads of the ring stay before the copies
@@ -203,7 +210,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
             const int left = K.len - uis * kUnit;
             // token t of the unit -> ring slot t (16 bytes; W words used)
             const uint32_t *src = codes + (K.code0 + int64_t(uis) * kUnit + lane) * W;
-            const uint32_t dst = smem_addr(&S.ring[warp][slot][lane]);
+            const uint32_t dst = smem_addr(&S.ring[warp][slot][0]) + copy_off;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const bool ok = lane + 32 * i < left;  // zero fill past len, no read
@@ -213,20 +220,18 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
         }
         cp_async_commit();
     };
-    // lane l stores 16 bytes of head (g0 + l / 8) of a unit: its offset in
-    // the rows
-    const int64_t lane_off = int64_t(lane >> 3) * a.dist_row + (lane & 7) * 16;
-    const uint32_t tb = smem_addr(&S.tile[warp][0][0]) + uint32_t(lane);
-
     int u_cur = grab();
     issue(u_cur, 0);
     for (int j = 0; u_cur < n_range; ++j) {
         const int u_next = grab();
+        __syncwarp();  // every lane is done reading the slot the next copies overwrite
         issue(u_next, (j + 1) % kRing);
         cp_async_wait<kRing - 1>();  // this lane's copies of the current unit have landed
+        __syncwarp();                // and so have the other lanes'
         uint4 cur[4];
+        const uint4 *mine = &S.ring[warp][j % kRing][4 * lane];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cur[i] = S.ring[warp][j % kRing][lane + 32 * i];
+        for (int i = 0; i < 4; ++i) cur[i] = mine[(i ^ (lane >> 1)) & 3];
         const uint32_t e = S.unit[u_cur];
         const int uis = int(e & 0x0fffffffu), kk = int(e >> 28);
         const KeyInfo &K = S.key[kk];
@@ -240,22 +245,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
         } else {
             const uint32_t hb = smem_addr(&S.hist[kk][0][0]);
             if (c_left >= kUnit && K.ng == GB)
-                score_unit<GB, W, true>(cur, K.q, K.qd, GB, tb, hb, lane, kUnit);
+                score_unit<GB, W, true>(cur, K.q, K.qp, GB, c_row, a.dist_row, hb, lane, kUnit);
             else if (c_left >= kUnit)
-                score_unit<GB, W, true>(cur, K.q, K.qd, K.ng, tb, hb, lane, kUnit);
+                score_unit<GB, W, true>(cur, K.q, K.qp, K.ng, c_row, a.dist_row, hb, lane, kUnit);
             else
-                score_unit<GB, W, false>(cur, K.q, K.qd, K.ng, tb, hb, lane, c_left);
-            __syncwarp();
-            // the tile to the rows: lane l stores 16 bytes of head g0 + l / 8
-#pragma unroll
-            for (int g0 = 0; g0 < GB; g0 += 4) {
-                if (g0 + (lane >> 3) < K.ng) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(
-                        &S.tile[warp][g0 + (lane >> 3)][(lane & 7) * 16]);
-                    __stcg(reinterpret_cast<uint4 *>(c_row + g0 * a.dist_row + lane_off), v);
-                }
-            }
-            __syncwarp();  // the tile is rewritten by the next unit
+                score_unit<GB, W, false>(cur, K.q, K.qp, K.ng, c_row, a.dist_row, hb, lane, c_left);
         }
         u_cur = u_next;
     }

@@ -27,13 +27,30 @@ __device__ __forceinline__ int hamming128(const uint4 &k, uint32_t k012, uint32_
     return __popc(o) + 2 * (__popc(c) + __popc(e));
 }
 
-// dist(k, q) for codes of W words (r = 32 W bits): the carry-save form for
-// W = 4, plain population counts of the XOR-ed words otherwise.
-template <int W>
-__device__ __forceinline__ int hamming_w(const uint4 &k, uint32_t k012, uint32_t k0123,
-                                         const uint4 &q, const uint2 &qd)
+// The same distance from the pair sums x0 + x1 = u + 2a and x2 + x3 = v + 2b
+// (u = x0 ^ x1, v = x2 ^ x3, a = x0 & x1, b = x2 & x3):
+//   x0 + x1 + x2 + x3 = (u ^ v) + 2 (a + b + (u & v))
+// where a and u & v never both hold, so c = a | (u & v) = (u ? v : x0), and
+// b = x2 & ~v.  u and v reach the key through k0 ^ k1 and k2 ^ k3 (k01, k23,
+// shared by every head of the group) and the query through q0 ^ q1, q2 ^ q3
+// (qp): six three-input logic operations per (key, query) instead of seven.
+__device__ __forceinline__ int hamming128_pairs(const uint4 &k, uint32_t k01, uint32_t k23,
+                                                const uint4 &q, const uint2 &qp)
 {
-    if constexpr (W == 4) return hamming128(k, k012, k0123, q, qd);
+    const uint32_t u = k01 ^ qp.x, v = k23 ^ qp.y;
+    const uint32_t c = (u & v) | (~u & (k.x ^ q.x));
+    const uint32_t e = (k.z ^ q.z) & ~v;
+    return __popc(u ^ v) + 2 * (__popc(c) + __popc(e));
+}
+
+// dist(k, q) for codes of W words (r = 32 W bits): the pair-sum carry-save
+// form for W = 4 (kp = k01, k23 and qp = q01, q23 of it), plain population
+// counts of the XOR-ed words otherwise.
+template <int W>
+__device__ __forceinline__ int hamming_w(const uint4 &k, const uint2 &kp, const uint4 &q,
+                                         const uint2 &qp)
+{
+    if constexpr (W == 4) return hamming128_pairs(k, kp.x, kp.y, q, qp);
     if constexpr (W == 2) return __popc(k.x ^ q.x) + __popc(k.y ^ q.y);
     return __popc(k.x ^ q.x);
 }
