@@ -37,6 +37,16 @@ __device__ __forceinline__ void cp_async_zfill(uint32_t dst, const void *src, ui
         asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;" ::"r"(dst), "l"(src), "n"(N),
                      "r"(bytes));
 }
+// The same copies with the whole source read (no zero fill).
+template <int N>
+__device__ __forceinline__ void cp_async_n(uint32_t dst, const void *src)
+{
+    static_assert(N == 4 || N == 8 || N == 16, "cp.async copies 4, 8 or 16 bytes");
+    if constexpr (N == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src));
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(N));
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 // Wait until at most N of this thread's committed cp.async groups are pending.
 template <int N>

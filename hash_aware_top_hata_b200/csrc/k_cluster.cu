@@ -227,13 +227,12 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
     // two chunks in flight (thread t reads back only the tokens it copied) ----
     {
         uint4 qv[kClusterMaxG];
-        uint2 qd[kClusterMaxG];
+        uint2 qp[kClusterMaxG];
 #pragma unroll
         for (int g = 0; g < kClusterMaxG; ++g) {
             const uint32_t *c = S.qcode[g < G ? g : 0];
             qv[g] = make_uint4(c[0], c[1], c[2], c[3]);
-            const uint32_t q012 = c[0] ^ c[1] ^ c[2];
-            qd[g] = make_uint2(q012, q012 ^ c[3]);
+            qp[g] = make_uint2(c[0] ^ c[1], c[2] ^ c[3]);
         }
         // the appended token's position in this CTA's range, if it holds it
         const int lp = append ? int(pos) - t_beg : -1;
@@ -248,13 +247,13 @@ __global__ void __launch_bounds__(kCThreads, 1) cluster_step_kernel(ClusterArgs 
                 const int t = kChunk * c + tl;          // in the CTA's range
                 uint4 kv = mine[tl];
                 if (t == lp) kv = kap;
-                const uint32_t k012 = kv.x ^ kv.y ^ kv.z, k0123 = k012 ^ kv.w;
+                const uint32_t k01 = kv.x ^ kv.y, k23 = kv.z ^ kv.w;
 #pragma unroll
                 for (int g = 0; g < kClusterMaxG; ++g) {
                     if (g < G) {
                         uint8_t byte = kDistPad;
                         if (t < nloc) {
-                            const int d = hamming128(kv, k012, k0123, qv[g], qd[g]);
+                            const int d = hamming128(kv, k01, k23, qv[g], qp[g]);
                             atomicAdd(&S.hist[g][d], 1u);
                             byte = uint8_t(d);
                         }

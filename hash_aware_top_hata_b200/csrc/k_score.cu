@@ -208,14 +208,19 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(ScoreArgs a)
             const int uis = int(e & 0x0fffffffu);
             const KeyInfo &K = S.key[e >> 28];
             const int left = K.len - uis * kUnit;
-            // token t of the unit -> ring slot t (16 bytes; W words used)
+            // 16 bytes per token in the ring, W words of them used
             const uint32_t *src = codes + (K.code0 + int64_t(uis) * kUnit + lane) * W;
             const uint32_t dst = smem_addr(&S.ring[warp][slot][0]) + copy_off;
+            if (left >= kUnit) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const bool ok = lane + 32 * i < left;  // zero fill past len, no read
-                cp_async_zfill<4 * W>(dst + 512u * i, ok ? src + 32 * W * i : codes,
-                                      ok ? 4u * W : 0u);
+                for (int i = 0; i < 4; ++i) cp_async_n<4 * W>(dst + 512u * i, src + 32 * W * i);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const bool ok = lane + 32 * i < left;  // zero fill past len, no read
+                    cp_async_zfill<4 * W>(dst + 512u * i, ok ? src + 32 * W * i : codes,
+                                          ok ? 4u * W : 0u);
+                }
             }
         }
         cp_async_commit();
@@ -328,7 +333,7 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
     extern __shared__ __align__(16) uint4 ring[];  // [2][kWidePiece * 2]
     __shared__ uint32_t hist[kScoreHeads][kHistStrideWide];
     __shared__ uint4 qs[kScoreHeads][2];
-    __shared__ uint2 qd[kScoreHeads][2];
+    __shared__ uint2 qp[kScoreHeads][2];
     pdl_trigger();
     const int tid = threadIdx.x;
     const int64_t per_slab = a.dist_row / kWidePiece;
@@ -405,8 +410,7 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
                 const uint4 v =
                     __ldg(reinterpret_cast<const uint4 *>(a.qcodes + (bh0 + g) * 8) + half);
                 qs[g][half] = v;
-                const uint32_t q012 = v.x ^ v.y ^ v.z;
-                qd[g][half] = make_uint2(q012, q012 ^ v.w);
+                qp[g][half] = make_uint2(v.x ^ v.y, v.z ^ v.w);
             }
             __syncthreads();
             key = k;
@@ -420,13 +424,13 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
             kc[i][0] = mine[(2 * i) ^ (lane & 7)];
             kc[i][1] = mine[(2 * i + 1) ^ (lane & 7)];
         }
-        uint32_t k012[4][2], k0123[4][2];
+        uint32_t k01[4][2], k23[4][2];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                k012[i][hf] = kc[i][hf].x ^ kc[i][hf].y ^ kc[i][hf].z;
-                k0123[i][hf] = k012[i][hf] ^ kc[i][hf].w;
+                k01[i][hf] = kc[i][hf].x ^ kc[i][hf].y;
+                k23[i][hf] = kc[i][hf].z ^ kc[i][hf].w;
             }
         // this thread's first token and how many of its four hold keys (32-bit:
         // rows are shorter than 2^31)
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
         const uint32_t hbase = smem_addr(&hist[0][0]);
         for (int g = 0; g < ng; ++g) {
             const uint4 q0 = qs[g][0], q1 = qs[g][1];
-            const uint2 d0 = qd[g][0], d1 = qd[g][1];
+            const uint2 p0 = qp[g][0], p1 = qp[g][1];
             const uint32_t hb = hbase + uint32_t(g * kHistStrideWide * 4);
             uint32_t word = 0u;
 #pragma unroll
@@ -444,8 +448,8 @@ __global__ void __launch_bounds__(kWideThreads, 3) score_wide_kernel(ScoreArgs a
                 // zero-filled codes past the sequence end are scored too and
                 // then neither counted nor stored
                 const uint32_t d =
-                    uint32_t(hamming128(kc[i][0], k012[i][0], k0123[i][0], q0, d0) +
-                             hamming128(kc[i][1], k012[i][1], k0123[i][1], q1, d1));
+                    uint32_t(hamming128(kc[i][0], k01[i][0], k23[i][0], q0, p0) +
+                             hamming128(kc[i][1], k01[i][1], k23[i][1], q1, p1));
                 const bool v = i < nv;
                 if (v) asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(hb + 4u * d) : "memory");
                 word |= (v ? d - (d >> 8) : uint32_t(kDistPad)) << (8 * i);  // 256 saturates to 255
