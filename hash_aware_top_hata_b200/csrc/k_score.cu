@@ -25,7 +25,7 @@
 //   c = u ? v : x0,  e = x2 & ~v                 (their carries, weight 2)
 //   dist = popc(u ^ v) + 2 (popc(c) + popc(e))
 //
-// i.e. three population counts instead of four (POPC issues at an eighth
+// i.e. three population counts instead of four (POPC issues at a quarter
 // of the integer-logic rate on sm_100a, and it is what bounds the
 // arithmetic), and six logic operations, since u and v take the key's
 // words as k0 ^ k1 and k2 ^ k3, shared by the group's heads.  Codes of 32
