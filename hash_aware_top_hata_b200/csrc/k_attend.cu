@@ -592,24 +592,30 @@ __global__ void __launch_bounds__(tc::kThreads, 1) attend_head_kernel(AttendArgs
 }
 
 // ------------------------------------------------------------------------
-// Combine: one warp per head merges the partials of the head's contributors
-// (workers k_first..k_last of the stream-K split) into out = acc / l.  It
-// runs as its own launch behind the attention kernel (programmatic
-// dependent launch: its CTAs are resident early and wait for the attention
-// grid to finish), so no attention worker waits for another or merges at
-// the end of its range.  The contributor count depends only on seq_len (a
-// step input), so it is known before the wait; after it, all loads of a
-// round of kCombineRound partials (lane c: m and l of contributor c; every
-// lane: its 4 output dims of each partial) are issued together, one
-// dependent memory round trip per round.
+// Combine: kWph warps per head merge the partials of the head's
+// contributors (workers k_first..k_last of the stream-K split, or the CTAs
+// of a split head) into out = acc / l.  It runs as its own launch behind the
+// attention kernel (programmatic dependent launch: its CTAs are resident
+// early and wait for the attention grid to finish), so no attention worker
+// waits for another or merges at the end of its range.  The contributor
+// count depends only on seq_len (a step input), so it is known before the
+// wait; after it, all loads of a round of kCombineRound partials (lane c: m
+// and l of contributor c; every lane: its 4 output dims of each partial)
+// are issued together, one dependent memory round trip per round.  Warp w
+// of a head takes rounds w, w + kWph, ...; with kWph = 4 the head's first 64
+// partials cost one round trip, and the warps' merged partials are merged
+// once more in shared memory.
 constexpr int kCombineWarps = 4;
 constexpr int kCombineRound = 16;
 
+template <int kWph>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(AttendArgs a)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t bh = int64_t(blockIdx.x) * kCombineWarps + (threadIdx.x >> 5);
-    const bool live = bh < int64_t(a.B) * a.H_q;
+    static_assert(kCombineWarps % kWph == 0, "whole heads per CTA");
+    __shared__ float part_s[kWph > 1 ? kCombineWarps : 1][kPartStride];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = warp % kWph;
+    const int64_t bh = int64_t(blockIdx.x) * (kCombineWarps / kWph) + warp / kWph;
+    const bool live = bh < int64_t(a.B) * a.H_q;  // uniform over the head's warps
     int n_contrib = 0;
     if (live && a.head_split > 0) {
         n_contrib = a.head_split;  // one partial per CTA of the head
@@ -622,10 +628,9 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(AttendArgs 
         n_contrib = int(owner(h0 + (keff > 0 ? keff : 1) - 1, T, NW) - owner(h0, T, NW) + 1);
     }
     pdl_wait();  // every partial is written
-    if (!live) return;
-    const float *pc = a.part + bh * a.n_split * kPartStride;
+    const float *pc = a.part + (live ? bh : 0) * a.n_split * kPartStride;
     float M = -INFINITY, L = 0.0f, A[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int c0 = 0; c0 < n_contrib; c0 += kCombineRound) {
+    for (int c0 = kCombineRound * sub; c0 < n_contrib; c0 += kCombineRound * kWph) {
         const int c = c0 + lane;
         const bool mine = lane < kCombineRound && c < n_contrib;
         const float mc = mine ? __ldcg(pc + c * kPartStride) : -INFINITY;
@@ -661,6 +666,36 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(AttendArgs 
             for (int i = 0; i < 4; ++i) A[i] = fmaf(acc[j][i], w, A[i]);
         }
     }
+    if constexpr (kWph > 1) {  // the head's warps: one more merge, in shared memory
+        const int wp = kWph > 1 ? warp : 0;
+        if (lane == 0) {
+            part_s[wp][0] = M;
+            part_s[wp][1] = L;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) part_s[wp][4 + lane + 32 * i] = A[i];
+        __syncthreads();
+        if (sub != 0) return;
+        const int w0 = wp;  // the head's first warp
+        float Mh = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWph; ++w) Mh = fmaxf(Mh, part_s[w0 + w][0]);
+        L = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) A[i] = 0.0f;
+        if (Mh != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kWph; ++w) {
+                const float mw = part_s[w0 + w][0];
+                const float wt = mw == -INFINITY ? 0.0f : exp2f(mw - Mh);
+                L = fmaf(part_s[w0 + w][1], wt, L);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) A[i] = fmaf(part_s[w0 + w][4 + lane + 32 * i], wt, A[i]);
+            }
+        }
+        M = Mh;
+    }
+    if (!live) return;
     if (a.part_out) {  // the sequence-parallel step: this shard's unnormalised partial
         float *pp = a.part_out + bh * kPartStride;
         if (lane == 0) {
@@ -770,11 +805,24 @@ cudaError_t launch_combine(const AttendArgs &a, cudaStream_t s)
 {
     if (a.head_per_cta) return cudaSuccess;  // merged inside the attention CTAs
     const int64_t heads = int64_t(a.B) * a.H_q;
+    // most partials one head can have: its CTAs when split, else the
+    // stream-K workers that can touch one head's topk rows
+    int64_t most = a.head_split;
+    if (most <= 0) {
+        const int64_t T = heads * a.topk, per = a.n_workers > 0 ? T / a.n_workers : T;
+        most = (a.topk + (per > 0 ? per : 1) - 1) / (per > 0 ? per : 1) + 1;
+    }
     // the same carveout as the attention kernel, so its CTAs can join the
     // SMs without a shared-memory reconfiguration
-    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(combine_kernel), 0))
+    if (most > kCombineRound) {  // four warps per head: up to 64 partials in one round trip
+        if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(combine_kernel<4>), 0))
+            return e;
+        return launch_pdl(combine_kernel<4>, dim3(unsigned(heads)), dim3(32 * kCombineWarps), 0, s,
+                          a);
+    }
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(combine_kernel<1>), 0))
         return e;
-    return launch_pdl(combine_kernel, dim3(unsigned(ceil_div(heads, kCombineWarps))),
+    return launch_pdl(combine_kernel<1>, dim3(unsigned(ceil_div(heads, kCombineWarps))),
                       dim3(32 * kCombineWarps), 0, s, a);
 }
 
